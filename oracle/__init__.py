@@ -1,0 +1,144 @@
+"""CPU oracle for the FP8 NT GEMM family -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference legs of ``bench.py`` may
+import this package.  It shares no code with the CUDA library and the library never calls it.
+
+The arithmetic lives in ``oracle.c`` (plain C, OpenMP over rows, double accumulation): the definition
+
+    ref[m, n] = sum_kb sfa(m, kb) * sfb(g, n // 128, kb) * sum_{k in block kb} dec(a[m, k]) * dec(b_g[n, k])
+
+("FP8 GEMM kernels with fine-grained scaling", DeepGEMM-for-PPU README, "Interfaces": the NT dense GEMM
+gemm_fp8_fp8_bf16_nt, the contiguous- and masked-layout grouped GEMMs; recipe (1, 128, 128) from the MATE
+deep_gemm wrapper API list).  This module only selects rows and marshals pointers.
+
+Grouped layouts (same README, "Grouped GEMMs (contiguous layout)" / "(masked layout)"):
+* contiguous: row m belongs to group m_indices[m]; rows with m_indices == -1 are padding and produce nothing.
+* masked: group g owns rows 0 .. masked_m[g]-1 of its [M_max, K] slab; the other rows produce nothing.
+Rows that produce nothing are returned as NaN (the "left untouched" sentinel).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        L.oracle_e4m3_decode.restype = ctypes.c_double
+        L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_decode_array.argtypes = [P, i64, P]
+        L.oracle_gemm_rows.argtypes = [P, P, P, i64, P, i64, P, i64, P, P, i64, i64, i64, P]
+        L.oracle_num_threads.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(x: np.ndarray):
+    return ctypes.c_void_p(x.ctypes.data)
+
+
+def num_threads() -> int:
+    return int(lib().oracle_num_threads())
+
+
+def decode_e4m3(codes) -> np.ndarray:
+    """OCP E4M3 codes (uint8) -> float64 values."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, np.float64)
+    lib().oracle_e4m3_decode_array(_ptr(c), c.size, _ptr(out))
+    return out
+
+
+def gemm_rows(a, sfa_row_off, sfa_kb_stride, sfa, b, sfb, rows, groups, N, K) -> np.ndarray:
+    """Raw entry: listed rows of the fine-grained-scaled product, double [len(rows), N]."""
+    a = np.ascontiguousarray(a, np.uint8)
+    sfa = np.ascontiguousarray(sfa, np.float32)
+    b = np.ascontiguousarray(b, np.uint8)
+    sfb = np.ascontiguousarray(sfb, np.float32)
+    rows = np.ascontiguousarray(rows, np.int64)
+    groups = np.ascontiguousarray(groups, np.int32)
+    off = np.ascontiguousarray(sfa_row_off, np.int64)
+    assert K % 128 == 0 and a.shape[-1] == K
+    n_rows = len(rows)
+    out = np.empty((n_rows, N), np.float64)
+    if n_rows == 0 or N == 0:
+        return out
+    G = b.shape[0] if b.ndim == 3 else 1
+    assert rows.min() >= 0 and rows.max() < a.shape[0]
+    assert groups.min() >= 0 and groups.max() < G
+    nnb = (N + 127) // 128
+    b_group_stride = N * K
+    sfb_group_stride = nnb * (K // 128)
+    assert sfb.size == G * sfb_group_stride and b.size == G * b_group_stride
+    assert off.max() + (K // 128 - 1) * sfa_kb_stride < sfa.size
+    lib().oracle_gemm_rows(_ptr(a), _ptr(sfa), _ptr(off), sfa_kb_stride, _ptr(b), b_group_stride, _ptr(sfb),
+                           sfb_group_stride, _ptr(rows), _ptr(groups), n_rows, N, K, _ptr(out))
+    return out
+
+
+def problem_rows(p, rows) -> np.ndarray:
+    """Selected global rows of a ``synth.Problem`` (rows must be rows the GEMM produces)."""
+    rows = np.asarray(rows, np.int64)
+    groups = p.row_groups(rows)
+    if p.kind == "masked":
+        Ma = p.sfa.shape[2]
+        nkb = p.sfa.shape[1]
+        g = rows // p.M
+        off = g * nkb * Ma + (rows - g * p.M)
+        kb_stride = Ma
+    else:
+        kb_stride = p.sfa.shape[1]
+        off = rows
+    return gemm_rows(p.a, off, kb_stride, p.sfa, p.b, p.sfb, rows, groups, p.N, p.K)
+
+
+def problem_full(p) -> np.ndarray:
+    """The whole output of a ``synth.Problem`` in its output shape; rows that produce nothing are NaN."""
+    rows = p.valid_rows()
+    out = np.full((p.rows, p.N), np.nan, np.float64)
+    out[rows] = problem_rows(p, rows)
+    return out.reshape(p.out_shape())
+
+
+# ----- convenience entry points in the library's own call shapes ---------------------------------------
+
+def fp8_gemm_nt(a, sfa, b, sfb):
+    """Dense: a [M,K] codes, sfa [K/128, >=M] MN-major, b [N,K] codes, sfb [ceil(N/128), K/128]."""
+    M, K = a.shape
+    N = b.shape[0]
+    rows = np.arange(M, dtype=np.int64)
+    return gemm_rows(a, rows, sfa.shape[1], sfa, b.reshape(1, N, K), sfb.reshape(1, *sfb.shape), rows,
+                     np.zeros(M, np.int32), N, K)
+
+
+def m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, m_indices):
+    """a [M_total,K], sfa [K/128, >=M_total], b [G,N,K], sfb [G, ceil(N/128), K/128], m_indices [M_total]."""
+    M, K = a.shape
+    G, N, _ = b.shape
+    rows = np.nonzero(np.asarray(m_indices) >= 0)[0].astype(np.int64)
+    out = np.full((M, N), np.nan)
+    out[rows] = gemm_rows(a, rows, sfa.shape[1], sfa, b, sfb, rows, np.asarray(m_indices)[rows], N, K)
+    return out
+
+
+def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, masked_m):
+    """a [G,M_max,K], sfa [G, K/128, >=M_max], b [G,N,K], sfb [G, ceil(N/128), K/128], masked_m [G]."""
+    G, M_max, K = a.shape
+    N = b.shape[1]
+    nkb, Ma = sfa.shape[1], sfa.shape[2]
+    rows = np.concatenate([g * M_max + np.arange(int(masked_m[g])) for g in range(G)]).astype(np.int64)
+    g = rows // M_max
+    out = np.full((G * M_max, N), np.nan)
+    out[rows] = gemm_rows(a.reshape(G * M_max, K), g * nkb * Ma + rows - g * M_max, Ma, sfa, b, sfb, rows, g, N, K)
+    return out.reshape(G, M_max, N)

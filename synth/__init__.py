@@ -1,0 +1,273 @@
+"""Seeded synthetic inputs for the FP8 NT GEMM family (dense, M-grouped contiguous, M-grouped masked).
+
+This module only *prepares inputs*: it draws fp32 N(0,1) data from ``numpy.random.default_rng(seed)``,
+quantises it to OCP e4m3 with power-of-two (UE8M0-representable) scales, and builds the grouping metadata
+(``m_indices`` / ``masked_m``).  It holds none of the GEMM arithmetic.  Both the CPU oracle and the CUDA
+path consume what it returns, and neither is imported here.
+
+Recipe (fine-grained scaling, "FP8 GEMM kernels with fine-grained scaling", DeepGEMM-for-PPU README,
+"Interfaces / Notices" and the scaling recipe (1, 128, 128) named by the MATE deep_gemm wrapper API list):
+
+* A [rows, K]: one scale per (row, 128-K block); B [N, K] per group: one scale per 128x128 block.
+* scale s = 2**e with e the smallest integer such that amax <= 448 * 2**e (= 2**ceil(log2(amax / 448))),
+  computed exactly from the binary exponent of amax; amax == 0 gives s = 1.
+* q = e4m3_RNE(x / s) (torch's fp32 -> float8_e4m3fn cast, round-to-nearest-even; |x / s| <= 448).
+* sfa is stored MN-major ("LHS scale TMA-aligned and transposed"): [K/128][align4(rows)] fp32
+  (masked: [G][K/128][align4(M_max)]).  sfb is [G][ceil(N/128)][K/128] fp32.
+* Rows that no group owns (contiguous padding, masked rows >= masked_m[g]) hold garbage: random bytes,
+  e4m3 NaN codes included, with random power-of-two scales.
+
+Draw order per problem: group sizes (or masked_m) -> A fp32 -> B fp32 (group by group) -> garbage.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional, Sequence
+
+import numpy as np
+
+E4M3_MAX = 448.0
+SCALE_BLOCK = 128  # K (and B's N) extent of one scale block
+M_ALIGNMENT = 128  # per-segment padding of the contiguous layout
+
+
+def align_up(x: int, a: int) -> int:
+    return (x + a - 1) // a * a
+
+
+def tma_aligned_rows(rows: int) -> int:
+    """Row extent of the MN-major fp32 scale array: padded to a 16-byte multiple (4 floats)."""
+    return align_up(rows, 4)
+
+
+@dataclasses.dataclass
+class Problem:
+    """One GEMM problem in the layouts the library takes.
+
+    kind       'dense' | 'contiguous' | 'masked'
+    a          uint8 e4m3 codes, [rows, K]; masked: [G * M_max, K] (= [G, M_max, K] flattened)
+    sfa        fp32, dense/contiguous [K/128, align4(rows)]; masked [G, K/128, align4(M_max)]
+    b          uint8 e4m3 codes, [G, N, K] (G = 1 for dense)
+    sfb        fp32, [G, ceil(N/128), K/128]
+    m_indices  int32 [rows] (contiguous only): group id of each row, -1 for padding rows
+    masked_m   int32 [G] (masked only): number of valid rows of each group
+    """
+
+    kind: str
+    M: int  # dense: M; contiguous: M_total (padded); masked: M_max
+    N: int
+    K: int
+    G: int
+    a: np.ndarray
+    sfa: np.ndarray
+    b: np.ndarray
+    sfb: np.ndarray
+    m_indices: Optional[np.ndarray] = None
+    masked_m: Optional[np.ndarray] = None
+    expected_m: int = 0
+    counts: Optional[np.ndarray] = None  # contiguous: valid rows per group
+    name: str = ""
+
+    @property
+    def rows(self) -> int:
+        return self.a.shape[0]
+
+    def valid_rows(self) -> np.ndarray:
+        """Global row indices (into ``a`` / the flattened output) that the GEMM must produce."""
+        if self.kind == "dense":
+            return np.arange(self.M, dtype=np.int64)
+        if self.kind == "contiguous":
+            return np.nonzero(self.m_indices >= 0)[0].astype(np.int64)
+        out = [g * self.M + np.arange(int(self.masked_m[g]), dtype=np.int64) for g in range(self.G)]
+        return np.concatenate(out) if out else np.zeros(0, np.int64)
+
+    def row_groups(self, rows: np.ndarray) -> np.ndarray:
+        if self.kind == "dense":
+            return np.zeros(len(rows), np.int32)
+        if self.kind == "contiguous":
+            return self.m_indices[rows].astype(np.int32)
+        return (rows // self.M).astype(np.int32)
+
+    def flops(self) -> int:
+        return 2 * int(len(self.valid_rows())) * self.N * self.K
+
+    def out_shape(self):
+        if self.kind == "masked":
+            return (self.G, self.M, self.N)
+        return (self.rows, self.N)
+
+
+# ----------------------------------------------------------------------------------------------
+# quantisation (input preparation)
+# ----------------------------------------------------------------------------------------------
+
+def pow2_scale_exponent(amax: np.ndarray) -> np.ndarray:
+    """Smallest integer e with amax <= 448 * 2**e, exactly (amax >= 0, fp32).  amax == 0 -> 0.
+
+    With amax = f * 2**ea (frexp, f in [0.5, 1)) and 448 = 0.875 * 2**9:
+    amax <= 0.875 * 2**(9 + e)  <=>  e >= ea - 9 when f <= 0.875, else e >= ea - 8.
+    """
+    f, ea = np.frexp(amax.astype(np.float64))
+    e = ea.astype(np.int64) - 9 + (f > 0.875).astype(np.int64)
+    return np.where(amax > 0, e, 0)
+
+
+def _to_e4m3_codes(x: np.ndarray) -> np.ndarray:
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def quantize_rows(x: np.ndarray):
+    """x fp32 [R, K] -> (codes uint8 [R, K], scales fp32 [R, K/128]) with one scale per (row, 128-K block)."""
+    R, K = x.shape
+    assert K % SCALE_BLOCK == 0
+    nkb = K // SCALE_BLOCK
+    xb = x.reshape(R, nkb, SCALE_BLOCK)
+    e = pow2_scale_exponent(np.abs(xb).max(axis=2))  # [R, nkb]
+    q = np.ldexp(xb, -e[:, :, None]).astype(np.float32)
+    codes = _to_e4m3_codes(q.reshape(R, K))
+    return codes, np.ldexp(np.ones_like(e, dtype=np.float32), e).astype(np.float32)
+
+
+def quantize_blocks(x: np.ndarray):
+    """x fp32 [N, K] -> (codes uint8 [N, K], scales fp32 [ceil(N/128), K/128]), one scale per 128x128 block."""
+    N, K = x.shape
+    assert K % SCALE_BLOCK == 0
+    nkb = K // SCALE_BLOCK
+    nnb = (N + SCALE_BLOCK - 1) // SCALE_BLOCK
+    pad = nnb * SCALE_BLOCK - N
+    xp = np.pad(x, ((0, pad), (0, 0))) if pad else x
+    xb = xp.reshape(nnb, SCALE_BLOCK, nkb, SCALE_BLOCK)
+    e = pow2_scale_exponent(np.abs(xb).max(axis=(1, 3)))  # [nnb, nkb]
+    q = np.ldexp(xb, -e[:, None, :, None]).astype(np.float32).reshape(nnb * SCALE_BLOCK, K)[:N]
+    return _to_e4m3_codes(q), np.ldexp(np.ones_like(e, dtype=np.float32), e).astype(np.float32)
+
+
+def _garbage_rows(rng: np.random.Generator, codes: np.ndarray, sfa_t: np.ndarray, rows: np.ndarray):
+    """Fill rows that no group owns with random bytes (NaN codes included) and random 2**j scales."""
+    if len(rows) == 0:
+        return
+    K = codes.shape[1]
+    junk = rng.integers(0, 256, size=(len(rows), K), dtype=np.uint8)
+    junk[:, 0] = 0x7F  # make sure every garbage row carries an e4m3 NaN code
+    codes[rows] = junk
+    nkb = sfa_t.shape[0]
+    sfa_t[:, rows] = np.ldexp(1.0, rng.integers(-10, 11, size=(nkb, len(rows)))).astype(np.float32)
+
+
+def _draw_normal(rng: np.random.Generator, shape) -> np.ndarray:
+    return rng.standard_normal(size=shape, dtype=np.float32)
+
+
+def _quantize_b(rng: np.random.Generator, G: int, N: int, K: int):
+    nkb = K // SCALE_BLOCK
+    nnb = (N + SCALE_BLOCK - 1) // SCALE_BLOCK
+    b = np.empty((G, N, K), np.uint8)
+    sfb = np.empty((G, nnb, nkb), np.float32)
+    for g in range(G):
+        b[g], sfb[g] = quantize_blocks(_draw_normal(rng, (N, K)))
+    return b, sfb
+
+
+# ----------------------------------------------------------------------------------------------
+# problem builders
+# ----------------------------------------------------------------------------------------------
+
+def make_dense(M: int, N: int, K: int, seed: int = 0, name: str = "") -> Problem:
+    rng = np.random.default_rng(seed)
+    codes, s = quantize_rows(_draw_normal(rng, (M, K)))
+    Ma = tma_aligned_rows(M)
+    sfa = np.ones((K // SCALE_BLOCK, Ma), np.float32)
+    sfa[:, :M] = s.T
+    b, sfb = _quantize_b(rng, 1, N, K)
+    return Problem("dense", M, N, K, 1, codes, sfa, b, sfb, name=name or f"dense M={M} N={N} K={K}")
+
+
+def make_contiguous(counts: Sequence[int], N: int, K: int, seed: int = 0, name: str = "",
+                    rng: Optional[np.random.Generator] = None, alignment: int = M_ALIGNMENT) -> Problem:
+    """Groups' token segments concatenated along M, each padded to ``alignment`` rows (padding: -1)."""
+    rng = rng if rng is not None else np.random.default_rng(seed)
+    counts = np.asarray(counts, np.int64)
+    G = len(counts)
+    padded = np.array([align_up(int(c), alignment) for c in counts], np.int64)
+    M_total = int(padded.sum())
+    m_indices = np.full(M_total, -1, np.int32)
+    starts = np.concatenate([[0], np.cumsum(padded)[:-1]]).astype(np.int64)
+    for g in range(G):
+        m_indices[starts[g]:starts[g] + counts[g]] = g
+    valid = np.nonzero(m_indices >= 0)[0]
+    invalid = np.nonzero(m_indices < 0)[0]
+    codes = np.zeros((M_total, K), np.uint8)
+    Ma = tma_aligned_rows(M_total)
+    sfa = np.ones((K // SCALE_BLOCK, Ma), np.float32)
+    qa, s = quantize_rows(_draw_normal(rng, (len(valid), K)))
+    codes[valid] = qa
+    sfa[:, valid] = s.T
+    b, sfb = _quantize_b(rng, G, N, K)
+    _garbage_rows(rng, codes, sfa, invalid)
+    return Problem("contiguous", M_total, N, K, G, codes, sfa, b, sfb, m_indices=m_indices,
+                   counts=counts.astype(np.int32), name=name or f"contiguous G={G} N={N} K={K}")
+
+
+def make_masked(G: int, M_max: int, N: int, K: int, masked_m: Optional[Sequence[int]] = None,
+                seed: int = 0, expected_m: int = 0, name: str = "") -> Problem:
+    """[G, M_max, K] activations; rows >= masked_m[g] of each group are garbage and must stay unwritten.
+    masked_m, when not given, is drawn uniformly from [0, M_max] (inclusive)."""
+    rng = np.random.default_rng(seed)
+    if masked_m is None:
+        masked_m = rng.integers(0, M_max, endpoint=True, size=G)
+    masked_m = np.asarray(masked_m, np.int32)
+    assert masked_m.shape == (G,) and (masked_m >= 0).all() and (masked_m <= M_max).all()
+    nkb = K // SCALE_BLOCK
+    codes, s = quantize_rows(_draw_normal(rng, (G * M_max, K)))
+    Ma = tma_aligned_rows(M_max)
+    sfa = np.ones((G, nkb, Ma), np.float32)
+    sfa[:, :, :M_max] = s.reshape(G, M_max, nkb).transpose(0, 2, 1)
+    b, sfb = _quantize_b(rng, G, N, K)
+    for g in range(G):
+        rows = np.arange(int(masked_m[g]), M_max)
+        view = codes[g * M_max:(g + 1) * M_max]
+        _garbage_rows(rng, view, sfa[g], rows)
+    return Problem("masked", M_max, N, K, G, codes, sfa, b, sfb, masked_m=masked_m,
+                   expected_m=expected_m or M_max, name=name or f"masked G={G} M_max={M_max} N={N} K={K}")
+
+
+def zipf_counts(total: int, G: int, s: float) -> np.ndarray:
+    """Deterministic Zipf(s) split of ``total`` tokens over G groups: w_g = (g+1)^-s, floor(total * w / sum w)
+    plus largest-remainder rounding so that the counts sum to ``total`` (ties go to the lower group id)."""
+    w = (np.arange(1, G + 1, dtype=np.float64)) ** (-s)
+    exact = total * w / w.sum()
+    counts = np.floor(exact).astype(np.int64)
+    rem = total - int(counts.sum())
+    order = np.argsort(-(exact - counts), kind="stable")
+    counts[order[:rem]] += 1
+    return counts
+
+
+# The five workloads (all seed 0).
+CONFIGS = {
+    1: "dense FP8 NT GEMM M=128 N=256 K=512",
+    2: "dense FP8 NT GEMM M=4096 N=7168 K=7168",
+    3: "M-grouped contiguous FP8 GEMM G=8 N=4096 K=7168, tokens U[1024,8192] per group",
+    4: "M-grouped masked FP8 GEMM G=32 M_max=256 N=7168 K=2048, masked_m U[0,256], expected_m=128",
+    5: "M-grouped contiguous FP8 GEMM G=64 N=7168 K=2048, Zipf(1.2) split of 65536 tokens",
+}
+
+
+def make_config(i: int, seed: int = 0) -> Problem:
+    if i == 1:
+        return make_dense(128, 256, 512, seed, name=CONFIGS[1])
+    if i == 2:
+        return make_dense(4096, 7168, 7168, seed, name=CONFIGS[2])
+    if i == 3:
+        rng = np.random.default_rng(seed)
+        counts = rng.integers(1024, 8192, endpoint=True, size=8)
+        return make_contiguous(counts, 4096, 7168, rng=rng, name=CONFIGS[3])
+    if i == 4:
+        return make_masked(32, 256, 7168, 2048, seed=seed, expected_m=128, name=CONFIGS[4])
+    if i == 5:
+        rng = np.random.default_rng(seed)
+        return make_contiguous(zipf_counts(65536, 64, 1.2), 7168, 2048, rng=rng, name=CONFIGS[5])
+    raise ValueError(f"unknown config {i}")

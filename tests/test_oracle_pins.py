@@ -1,0 +1,192 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+* e4m3 decode: all 256 codes against torch's float8_e4m3fn -> float32 conversion, plus the special values
+  of the OCP E4M3 format.
+* contraction: brute force on integer-valued operands against exact int64 matrix products; with unit
+  scales it reduces to numpy.matmul in float64.
+* scales: the blockwise definition equals dequantise-then-matmul, and scaling one block's scale by 2**j
+  scales exactly that block's contribution (scale linearity).
+* grouping: contiguous and masked results equal per-group dense products; rows that no group owns are
+  left untouched.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+
+def torch_decode(codes):
+    t = torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float32).double().numpy()
+
+
+def test_decode_all_codes_match_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    mine = oracle.decode_e4m3(codes)
+    ref = torch_decode(codes)
+    nan = np.isnan(ref)
+    assert (np.isnan(mine) == nan).all()
+    assert nan.sum() == 2  # S.1111.111 only
+    np.testing.assert_array_equal(mine[~nan], ref[~nan])
+    # signed zero
+    assert np.signbit(mine[0x80]) and not np.signbit(mine[0x00])
+
+
+@pytest.mark.parametrize("code,value", [
+    (0x00, 0.0), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9), (0x08, 2.0 ** -6), (0x38, 1.0),
+    (0x7E, 448.0), (0xFE, -448.0), (0x40, 2.0), (0x3C, 1.5), (0xB8, -1.0)])
+def test_decode_special_values(code, value):
+    assert oracle.decode_e4m3(np.array([code], np.uint8))[0] == value
+
+
+def test_decode_nan_codes():
+    assert np.isnan(oracle.decode_e4m3(np.array([0x7F, 0xFF], np.uint8))).all()
+
+
+def _codes_for_values(values):
+    """e4m3 codes of exactly representable values (via torch's encoder, independent of the oracle)."""
+    t = torch.tensor(values, dtype=torch.float32).to(torch.float8_e4m3fn)
+    back = t.to(torch.float32).numpy()
+    assert np.array_equal(back, np.asarray(values, np.float32))
+    return t.view(torch.uint8).numpy()
+
+
+@pytest.mark.parametrize("M,N", [(1, 1), (3, 5), (8, 8), (2, 128), (128, 7), (128, 128)])
+@pytest.mark.parametrize("K", [128, 256])
+def test_bruteforce_integer_operands(M, N, K):
+    rng = np.random.default_rng(M * 1000 + N * 10 + K)
+    ia = rng.integers(-8, 9, size=(M, K))
+    ib = rng.integers(-8, 9, size=(N, K))
+    a = _codes_for_values(ia.astype(np.float32))
+    b = _codes_for_values(ib.astype(np.float32))
+    sfa = np.ones((K // 128, synth.tma_aligned_rows(M)), np.float32)
+    sfb = np.ones(((N + 127) // 128, K // 128), np.float32)
+    got = oracle.fp8_gemm_nt(a, sfa, b, sfb)
+    exact = ia.astype(np.int64) @ ib.astype(np.int64).T
+    np.testing.assert_array_equal(got, exact.astype(np.float64))
+
+
+def _random_finite_codes(rng, shape):
+    c = rng.integers(0, 256, size=shape, dtype=np.uint8)
+    return np.where((c & 0x7F) == 0x7F, c ^ 0x01, c).astype(np.uint8)
+
+
+def test_unit_scales_reduce_to_numpy_matmul():
+    rng = np.random.default_rng(1)
+    M, N, K = 37, 200, 384
+    a = _random_finite_codes(rng, (M, K))
+    b = _random_finite_codes(rng, (N, K))
+    got = oracle.fp8_gemm_nt(a, np.ones((K // 128, 40), np.float32), b, np.ones((2, K // 128), np.float32))
+    ref = torch_decode(a) @ torch_decode(b).T
+    np.testing.assert_allclose(got, ref, rtol=1e-13, atol=0)
+
+
+def test_blockwise_definition_equals_dequantise_then_matmul():
+    """With arbitrary power-of-two scales the blockwise sum equals the matmul of the dequantised operands."""
+    rng = np.random.default_rng(2)
+    M, N, K = 19, 300, 512  # N not a multiple of 128: ragged last scale block
+    nkb = K // 128
+    a = _random_finite_codes(rng, (M, K))
+    b = _random_finite_codes(rng, (N, K))
+    sfa = np.ldexp(1.0, rng.integers(-6, 7, size=(nkb, 20))).astype(np.float32)
+    sfb = np.ldexp(1.0, rng.integers(-6, 7, size=(3, nkb))).astype(np.float32)
+    got = oracle.fp8_gemm_nt(a, sfa, b, sfb)
+    A = torch_decode(a) * np.repeat(sfa[:, :M].T, 128, axis=1)
+    sb_full = np.repeat(np.repeat(sfb, 128, axis=0)[:N], 128, axis=1)
+    B = torch_decode(b) * sb_full
+    np.testing.assert_allclose(got, A @ B.T, rtol=1e-12, atol=1e-9)
+
+
+def test_dropped_or_misindexed_scale_is_detected():
+    """Sanity of the pin above: a transposed sfb index would change the result (so the pin can fail)."""
+    rng = np.random.default_rng(3)
+    M, N, K = 4, 256, 256
+    a = _random_finite_codes(rng, (M, K))
+    b = _random_finite_codes(rng, (N, K))
+    sfa = np.ones((2, 4), np.float32)
+    sfb = np.array([[1.0, 2.0], [4.0, 8.0]], np.float32)
+    good = oracle.fp8_gemm_nt(a, sfa, b, sfb)
+    wrong = oracle.fp8_gemm_nt(a, sfa, b, np.ascontiguousarray(sfb.T))
+    assert not np.allclose(good, wrong)
+
+
+@pytest.mark.parametrize("which", ["sfa", "sfb"])
+def test_scale_linearity(which):
+    rng = np.random.default_rng(4)
+    M, N, K = 9, 256, 384
+    nkb = K // 128
+    a = _random_finite_codes(rng, (M, K))
+    b = _random_finite_codes(rng, (N, K))
+    sfa = np.ldexp(1.0, rng.integers(-3, 4, size=(nkb, 12))).astype(np.float32)
+    sfb = np.ldexp(1.0, rng.integers(-3, 4, size=(2, nkb))).astype(np.float32)
+    base = oracle.fp8_gemm_nt(a, sfa, b, sfb)
+    j, kb = 5, 1
+    Ad, Bd = torch_decode(a), torch_decode(b)
+    if which == "sfa":
+        m = 4
+        sfa2 = sfa.copy()
+        sfa2[kb, m] *= 2.0 ** j
+        got = oracle.fp8_gemm_nt(a, sfa2, b, sfb)
+        block = Ad[m, kb * 128:(kb + 1) * 128] @ Bd[:, kb * 128:(kb + 1) * 128].T  # [N]
+        contrib = sfa[kb, m] * np.repeat(sfb[:, kb], 128)[:N] * block
+        expect = base.copy()
+        expect[m] += (2.0 ** j - 1.0) * contrib
+        np.testing.assert_array_equal(np.delete(got, m, 0), np.delete(base, m, 0))
+        np.testing.assert_allclose(got, expect, rtol=1e-13, atol=1e-10)
+    else:
+        nb = 1
+        sfb2 = sfb.copy()
+        sfb2[nb, kb] *= 2.0 ** j
+        got = oracle.fp8_gemm_nt(a, sfa, b, sfb2)
+        cols = slice(nb * 128, (nb + 1) * 128)
+        block = Ad[:, kb * 128:(kb + 1) * 128] @ Bd[cols, kb * 128:(kb + 1) * 128].T  # [M, 128]
+        contrib = sfa[kb, :M][:, None] * sfb[nb, kb] * block
+        expect = base.copy()
+        expect[:, cols] += (2.0 ** j - 1.0) * contrib
+        np.testing.assert_array_equal(got[:, :128], base[:, :128])
+        np.testing.assert_allclose(got, expect, rtol=1e-13, atol=1e-10)
+
+
+def test_whole_row_power_of_two_scaling_is_exact():
+    rng = np.random.default_rng(5)
+    p = synth.make_dense(8, 128, 256, seed=5)
+    base = oracle.problem_full(p)
+    p.sfa[:, 3] *= 8.0
+    got = oracle.problem_full(p)
+    np.testing.assert_array_equal(got[3], 8.0 * base[3])
+
+
+def test_contiguous_equals_per_group_dense():
+    p = synth.make_contiguous([130, 1, 256, 0, 77], N=256, K=256, seed=6)
+    full = oracle.problem_full(p)
+    starts = np.concatenate([[0], np.cumsum([synth.align_up(int(c), 128) for c in p.counts])])
+    for g in range(p.G):
+        s, c = starts[g], int(p.counts[g])
+        dense = oracle.fp8_gemm_nt(p.a[s:s + c], np.ascontiguousarray(p.sfa[:, s:s + c + 4]), p.b[g], p.sfb[g])
+        np.testing.assert_array_equal(full[s:s + c], dense)
+        assert np.isnan(full[s + c:starts[g + 1]]).all()  # padding rows untouched
+
+
+def test_masked_equals_per_group_dense_and_leaves_rows_untouched():
+    p = synth.make_masked(G=4, M_max=136, N=128, K=256, masked_m=[0, 136, 5, 128], seed=7)
+    full = oracle.problem_full(p)
+    for g in range(p.G):
+        mm = int(p.masked_m[g])
+        rows = p.a[g * p.M:g * p.M + mm]
+        dense = oracle.fp8_gemm_nt(rows, np.ascontiguousarray(p.sfa[g][:, :synth.tma_aligned_rows(max(mm, 1))]),
+                                   p.b[g], p.sfb[g]) if mm else np.zeros((0, p.N))
+        np.testing.assert_array_equal(full[g, :mm], dense)
+        assert np.isnan(full[g, mm:]).all()
+
+
+def test_library_call_shapes_agree_with_problem_driver():
+    p = synth.make_masked(G=3, M_max=64, N=128, K=128, masked_m=[3, 64, 0], seed=8)
+    a = p.a.reshape(p.G, p.M, p.K)
+    got = oracle.m_grouped_fp8_gemm_nt_masked(a, p.sfa, p.b, p.sfb, p.masked_m)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(oracle.problem_full(p)))
+    np.testing.assert_array_equal(np.nan_to_num(got), np.nan_to_num(oracle.problem_full(p)))
+    q = synth.make_contiguous([5, 200], N=128, K=128, seed=9)
+    got = oracle.m_grouped_fp8_gemm_nt_contiguous(q.a, q.sfa, q.b, q.sfb, q.m_indices)
+    np.testing.assert_array_equal(np.nan_to_num(got), np.nan_to_num(oracle.problem_full(q)))

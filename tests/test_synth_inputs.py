@@ -1,0 +1,72 @@
+"""The seeded generator: exact power-of-two scale choice, e4m3 range, layouts and the workload facts."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+
+def test_scale_exponent_is_smallest_power_of_two_covering_amax():
+    amax = np.array([448.0, 448.0001, 447.99, 1.0, 0.875 * 2 ** -3, 3.5, 1e-30, 7e4, 0.0], np.float32)
+    e = synth.pow2_scale_exponent(amax)
+    for x, ei in zip(amax.astype(np.float64), e):
+        if x == 0:
+            assert ei == 0
+            continue
+        assert x <= 448.0 * 2.0 ** ei
+        assert x > 448.0 * 2.0 ** (ei - 1)
+
+
+def test_exact_tie_takes_the_lower_exponent():
+    # amax == 448 * 2**e exactly -> that e (ceil(log2) of an exact power of two)
+    assert list(synth.pow2_scale_exponent(np.array([448.0, 224.0, 896.0], np.float32))) == [0, -1, 1]
+
+
+def test_quantised_values_within_range_and_round_to_nearest_even():
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((64, 256), dtype=np.float32)
+    codes, s = synth.quantize_rows(x)
+    deq = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy()
+    assert np.isfinite(deq).all() and np.abs(deq).max() <= 448
+    amax_q = np.abs(deq.reshape(64, 2, 128)).max(axis=2)
+    assert (amax_q > 224 * 0.9).all()  # every block uses the top binade of e4m3
+    # each code is the nearest e4m3 value of x/s
+    xs = x / np.repeat(s, 128, axis=1)
+    err = np.abs(deq - xs)
+    assert (err <= np.abs(xs) * 2 ** -4 + 2 ** -10).all()
+
+
+def test_workload_facts():
+    rng = np.random.default_rng(0)
+    assert list(rng.integers(1024, 8192, endpoint=True, size=8)) == [7122, 5590, 4688, 2958, 3230, 1317, 1563,
+                                                                        1142]
+    rng = np.random.default_rng(0)
+    mm = rng.integers(0, 256, endpoint=True, size=32)
+    assert mm.sum() == 4319 and (mm == 0).sum() == 1 and sum((int(x) + 127) // 128 for x in mm) == 52
+    z = synth.zipf_counts(65536, 64, 1.2)
+    assert z.sum() == 65536 and z.max() == 19170 and z.min() == 130 and (np.diff(z) <= 0).all()
+    assert sum(synth.align_up(int(c), 128) for c in z) == 70016
+
+
+def test_contiguous_layout():
+    p = synth.make_contiguous([3, 128, 129], N=128, K=128, seed=1)
+    assert p.rows == 128 + 128 + 256
+    mi = p.m_indices
+    assert (mi[:3] == 0).all() and (mi[3:128] == -1).all() and (mi[128:256] == 1).all()
+    assert (mi[256:385] == 2).all() and (mi[385:] == -1).all()
+    assert p.sfa.shape == (1, 512) and p.sfb.shape == (3, 1, 1)
+    # garbage rows carry NaN codes
+    assert (p.a[3:128, 0] == 0x7F).all()
+
+
+def test_masked_layout():
+    p = synth.make_masked(G=2, M_max=10, N=128, K=256, masked_m=[0, 10], seed=1)
+    assert p.a.shape == (20, 256) and p.sfa.shape == (2, 2, 12) and p.sfb.shape == (2, 1, 2)
+    assert (p.a[:10, 0] == 0x7F).all()
+    assert len(p.valid_rows()) == 10 and p.flops() == 2 * 10 * 128 * 256
+
+
+def test_seeded_determinism():
+    a = synth.make_dense(16, 128, 256, seed=3)
+    b = synth.make_dense(16, 128, 256, seed=3)
+    assert np.array_equal(a.a, b.a) and np.array_equal(a.b, b.b) and np.array_equal(a.sfa, b.sfa)
