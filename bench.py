@@ -1,0 +1,365 @@
+#!/usr/bin/env python
+"""Benchmark: FP8 NT GEMM with fine-grained scaling on B200 (one process per GPU).
+
+One step = one call of the library's dense FP8 GEMM on the workload M=4096, N=7168, K=7168 (A and B e4m3
+with power-of-two 1x128 / 128x128 scales, bf16 out; seeded synthetic inputs), the configuration the
+headline metric is quoted on.  Other workloads can be timed with --workload (contiguous / masked grouped
+shapes) for reference; the default line is the contract line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 2]
+
+Timing: inputs resident in HBM; each step is bracketed by CUDA events on the launching stream; between
+steps a 512 MB buffer is rewritten to flush the 126 MB L2 (outside the events).  The timed loop is
+bracketed by a barrier and a device synchronise, and the per-step time is the max over ranks.  N > 1 runs
+N independent replicas (weak scaling; the GEMM has no exchange step).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio (4.5 / 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["moe_grouped_gemm_03_b200/csrc/gemm_kernel.cuh", "moe_grouped_gemm_03_b200/csrc/ptx.cuh",
+                  "moe_grouped_gemm_03_b200/csrc/dg_api.cu"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    rec = d.get(str(workload))
+    if not rec or rec.get("kernel_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for n, bit in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def call_library(p, t, out):
+    import moe_grouped_gemm_03_b200 as dg
+
+    if p.kind == "dense":
+        dg.fp8_gemm_nt((t["a"], t["sfa"]), (t["b"], t["sfb"]), out)
+    elif p.kind == "contiguous":
+        dg.m_grouped_fp8_gemm_nt_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["m_indices"])
+    else:
+        dg.m_grouped_fp8_gemm_nt_masked((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["masked_m"], p.expected_m)
+
+
+def algorithmic_bytes(p):
+    """Each valid A row once, each active group's B once, the scales of those, each valid D row once."""
+    import numpy as np
+
+    rows = p.valid_rows()
+    nkb = p.K // 128
+    groups = np.unique(p.row_groups(rows)) if len(rows) else []
+    nnb = (p.N + 127) // 128
+    return int(len(rows) * p.K + len(groups) * p.N * p.K + len(rows) * nkb * 4 + len(groups) * nnb * nkb * 4
+               + len(rows) * p.N * 2)
+
+
+def oracle_sample(p, seconds, rng_seed=0):
+    """Time the oracle on a bounded random sample of valid rows (about `seconds` of CPU time)."""
+    import numpy as np
+
+    import oracle
+
+    valid = p.valid_rows()
+    rng = np.random.default_rng(rng_seed)
+    n = min(len(valid), 4)
+    t0 = time.perf_counter()
+    oracle.problem_rows(p, np.sort(rng.choice(valid, n, replace=False)))
+    dt = max(time.perf_counter() - t0, 1e-6)
+    n = int(min(len(valid), max(n, n * seconds / dt)))
+    rows = np.sort(rng.choice(valid, n, replace=False))
+    t0 = time.perf_counter()
+    oracle.problem_rows(p, rows)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * n * p.N * p.K
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} random valid rows x all {p.N} columns of the workload (seed {rng_seed}); "
+                      f"{dt:.2f} s wall for {flops / 1e9:.1f} GFLOP in fp64"}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle, as it stands, on bounded samples of the same workload."""
+    import synth
+
+    if rank != 0:
+        return
+    p = synth.make_config(args.workload)
+    import numpy as np
+
+    import oracle
+
+    valid = p.valid_rows()
+    rng = np.random.default_rng(1)
+    probe = time.perf_counter()
+    oracle.problem_rows(p, np.sort(rng.choice(valid, 2, replace=False)))
+    per_row = (time.perf_counter() - probe) / 2
+    rows_per_step = int(max(1, min(len(valid), 3.0 / max(per_row, 1e-9))))  # ~3 s per step
+    steps = max(1, min(args.steps, 10))
+    warm = min(args.warmup, 1)
+    for _ in range(warm):
+        oracle.problem_rows(p, np.sort(rng.choice(valid, rows_per_step, replace=False)))
+    times = []
+    for _ in range(steps):
+        rows = np.sort(rng.choice(valid, rows_per_step, replace=False))
+        t0 = time.perf_counter()
+        oracle.problem_rows(p, rows)
+        times.append(time.perf_counter() - t0)
+    flops = 2.0 * rows_per_step * p.N * p.K
+    value = flops / statistics.mean(times) / 1e12
+    line = {
+        "impl": "reference", "metric": "FP8 GEMM TFLOPS (dense and M-grouped)", "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": warm, "ms_per_step": 1e3 * statistics.mean(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "G": p.G},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"{rows_per_step} random valid rows x all {p.N} columns per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import moe_grouped_gemm_03_b200 as dg
+    import synth
+
+    p = synth.make_config(args.workload)
+    t = synth.to_torch(p, f"cuda:{local}")
+    out = torch.empty(p.out_shape(), dtype=torch.bfloat16, device=f"cuda:{local}")
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.int32, device=f"cuda:{local}")
+    stream = torch.cuda.current_stream()
+    flops = p.flops()
+
+    for _ in range(max(args.warmup, 3)):
+        call_library(p, t, out)
+    torch.cuda.synchronize()
+    dg.check_device_error()
+
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier(world)
+    torch.cuda.synchronize()
+    with clocks:
+        for i in range(K):
+            flush.fill_(i)
+            starts[i].record(stream)
+            call_library(p, t, out)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    dg.check_device_error()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = max_over_ranks(statistics.mean(step_ms), world)
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # end to end through the public API: pinned host inputs -> device, GEMM, result -> pinned host
+    host = {k: v.cpu().pin_memory() for k, v in t.items()}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = host_out.numel() * host_out.element_size()
+    e2e_steps = max(3, min(K, 20))
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(e2e_steps + 2):
+        if i == 2:
+            barrier(world)
+            torch.cuda.synchronize()
+            e_start.record(stream)
+        for k in t:
+            t[k].copy_(host[k], non_blocking=True)
+        call_library(p, t, out)
+        host_out.copy_(out, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / e2e_steps, world)
+
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    achieved = flops / (statistics.mean(step_ms) * 1e-3) / 1e12
+    nbytes = algorithmic_bytes(p)
+    traffic = recorded_traffic(args.workload)
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp8_peak, "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x nominal fp8/bf16 ratio 2",
+                "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": nbytes,
+                "hbm_gbs_achieved": nbytes / (statistics.mean(step_ms) * 1e-3) / 1e9, "hbm_peak_gbs": peaks["hbm_gbs"]}
+    if p.kind == "masked":
+        roofline.update(bound="hbm", achieved=roofline["hbm_gbs_achieved"], peak=peaks["hbm_gbs"], unit="GB/s",
+                        frac=roofline["hbm_gbs_achieved"] / peaks["hbm_gbs"])
+    line = {
+        "metric": "FP8 GEMM TFLOPS (dense and M-grouped)", "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3", "data": "synthetic",
+        "config": {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "G": p.G,
+                   "block_n": dg.select_block_n(
+                       p.G * ((p.expected_m + 127) // 128) if p.kind == "masked" else (p.rows + 127) // 128,
+                       p.N, dg.get_num_sms()),
+                   "l2": "flushed between steps (512 MB write outside the timed events)",
+                   "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU",
+                   "tflops_frac_of_fp8_peak": achieved / fp8_peak},
+        "roofline": roofline,
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": K,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = oracle_sample(p, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args) if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if args.impl == "ours" and world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

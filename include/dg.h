@@ -1,0 +1,116 @@
+/*
+ * dg.h -- C ABI of the B200 (sm_100a) FP8 NT GEMM library with fine-grained scaling.
+ *
+ * The operation ("FP8 GEMM kernels with fine-grained scaling", DeepGEMM-for-PPU README, "Interfaces"):
+ *
+ *     D[m][n] = bf16_RNE( sum_kb sfa(m, kb) * sfb(g, n/128, kb) * sum_{k in block kb} A[m][k] * B_g[n][k] )
+ *
+ * A and B are OCP e4m3 ("e4m3fn") codes, one byte per element.  A has one scale per (row, 128-K block)
+ * and B one scale per 128x128 block (the (1, 128, 128) recipe of the MATE deep_gemm wrapper API list).
+ * Only the NT form exists: A is [M, K] and B is [N, K], both K-major ("non-transposed LHS, transposed
+ * RHS", README "Notices").  Accumulation is fp32 on the tensor cores.
+ *
+ * Scale layouts (README "Notices": the LHS scale is TMA-aligned and transposed):
+ *   sfa  fp32, MN-major: [K/128][ld] with ld = dg_get_tma_aligned_size(rows, 4) (rows rounded up to a
+ *        multiple of 4 so every K block's column starts on 16 bytes).  Masked layout: [G][K/128][ld(M_max)].
+ *   sfb  fp32, [G][ceil(N/128)][K/128] (G = 1 for the dense call).
+ * Every scale must be a positive power of two in [2^-127, 2^127] (a UE8M0 value): the tensor cores apply
+ * the scales as exponents.  Other values give wrong results; the library does not check them.
+ *
+ * Common conventions
+ *   - All array arguments are device pointers owned by the caller.  The library allocates nothing per
+ *     call and keeps no reference after the call returns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).  m_indices and
+ *     masked_m are read only on the device, so the host never synchronises.
+ *   - Arguments are validated before anything is launched; a bad argument returns a negative dg_status,
+ *     launches nothing and sets the message returned by dg_last_error().
+ *   - Rows the GEMM does not own are never written: contiguous rows with m_indices == -1, masked rows
+ *     with index >= masked_m[g] (all of D[g] when masked_m[g] == 0).
+ *   - Pointer alignment: a, b, d, sfa, sfb 16-byte aligned; m_indices, masked_m 4-byte aligned.
+ *   - Shapes: K % 128 == 0, N % 16 == 0, N, K > 0, all extents below 2^31 elements per dimension.
+ *   - Device-side faults are not expected.  Every wait inside the kernel is bounded; a kernel that gives
+ *     up records a code that dg_check_device_error() returns (DG_ERR_DEVICE_TIMEOUT or DG_ERR_BAD_GROUP).
+ */
+#ifndef DG_H_
+#define DG_H_
+
+#if defined(__GNUC__)
+#define DG_EXPORT __attribute__((visibility("default")))
+#else
+#define DG_EXPORT
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *dg_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    DG_OK = 0,
+    DG_ERR_INVALID_ARG = -1,   /* null pointer, bad extent, bad group count */
+    DG_ERR_ALIGNMENT = -2,     /* pointer or extent not aligned as required */
+    DG_ERR_UNSUPPORTED = -3,   /* device is not sm_100, or a shape outside the supported set */
+    DG_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed */
+    DG_ERR_DEVICE_TIMEOUT = -5,/* (device error word) a bounded wait inside the kernel ran out */
+    DG_ERR_BAD_GROUP = -6      /* (device error word) a group id outside [-1, G) or masked_m outside [0, M_max] */
+} dg_status;
+
+/* Per-segment M padding of the contiguous layout: each group's rows start on a multiple of this (128).
+ * README "Grouped GEMMs (contiguous layout)": segments are aligned to the GEMM M block size. */
+DG_EXPORT int dg_get_m_alignment_for_contiguous_layout(void);
+
+/* Rows rounded up so that `mn` elements of `elem_bytes` bytes fill whole 16-byte units (README
+ * "Utilities": get_tma_aligned_size).  Returns -1 for a non-positive elem_bytes. */
+DG_EXPORT int dg_get_tma_aligned_size(int mn, int elem_bytes);
+
+/* Cap on the persistent grid (README "Utilities": set_num_sms / get_num_sms).  n <= 0 restores the
+ * default (every SM of the current device).  Returns the value now in force, or a negative status. */
+DG_EXPORT int dg_set_num_sms(int n);
+DG_EXPORT int dg_get_num_sms(void);
+
+/* Output tiles of an M x N problem with block_m x block_n tiles: ceil(M/block_m) * ceil(N/block_n).
+ * README "Unaligned block sizes": M=256, N=7168 gives 112 tiles at 128x128 and 128 tiles at 128x112. */
+DG_EXPORT long long dg_num_tiles(long long M, long long N, int block_m, int block_n);
+
+/* The N tile the library picks for `num_m_blocks` 128-row blocks of an N-wide output on `num_sms` SMs:
+ * the candidate with the fewest SM-waves weighted by tile width (README "Unaligned block sizes"). */
+DG_EXPORT int dg_select_block_n(long long num_m_blocks, int N, int num_sms);
+
+/* Dense NT GEMM (README "Normal dense GEMMs", gemm_fp8_fp8_bf16_nt).
+ *   a [M][K] e4m3, sfa [K/128][ld(M)] fp32, b [N][K] e4m3, sfb [ceil(N/128)][K/128] fp32,
+ *   d [M][N] bf16 row-major (written in full).  M == 0 is a no-op. */
+DG_EXPORT int dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
+                   int M, int N, int K, dg_stream_t stream);
+
+/* M-grouped GEMM, contiguous layout (README "Grouped GEMMs (contiguous layout)").
+ *   a [M_total][K] e4m3 (group segments concatenated, each padded to dg_get_m_alignment...()),
+ *   sfa [K/128][ld(M_total)], b [G][N][K] e4m3, sfb [G][ceil(N/128)][K/128],
+ *   m_indices int32 [M_total] on the device: the group of each row, -1 for a padding row.  Every
+ *   128-row block must hold one group (its first row decides; a block whose first row is -1 is skipped),
+ *   d [M_total][N] bf16: rows with m_indices == -1 are left untouched.  M_total % 128 == 0. */
+DG_EXPORT int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
+                                        void *d, const int *m_indices, int M_total, int N, int K, int G,
+                                        dg_stream_t stream);
+
+/* M-grouped GEMM, masked layout (README "Grouped GEMMs (masked layout)").
+ *   a [G][M_max][K] e4m3, sfa [G][K/128][ld(M_max)], b [G][N][K] e4m3, sfb [G][ceil(N/128)][K/128],
+ *   masked_m int32 [G] on the device: rows 0..masked_m[g]-1 of group g are computed,
+ *   d [G][M_max][N] bf16: rows >= masked_m[g] are left untouched.
+ *   expected_m: the caller's guess of a typical masked_m, used only to pick the tile shape; results do
+ *   not depend on it.  1 <= G <= 1024. */
+DG_EXPORT int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const void *b, const float *sfb,
+                                    void *d, const int *masked_m, int G, int M_max, int N, int K,
+                                    int expected_m, dg_stream_t stream);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+DG_EXPORT const char *dg_last_error(void);
+
+/* Synchronises `stream`, then returns and clears the device error word of the current device:
+ * DG_OK, DG_ERR_DEVICE_TIMEOUT or DG_ERR_BAD_GROUP (DG_ERR_CUDA if the synchronisation failed). */
+DG_EXPORT int dg_check_device_error(dg_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DG_H_ */

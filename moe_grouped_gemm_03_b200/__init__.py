@@ -1,0 +1,202 @@
+"""B200 (sm_100a) FP8 NT GEMM with fine-grained scaling: dense, M-grouped contiguous and M-grouped masked.
+
+Thin ctypes binding over ``libdg.so`` (the C ABI in ``include/dg.h``).  This module only marshals
+arguments: it checks dtypes/shapes of the torch tensors, passes raw device pointers and the current CUDA
+stream, and turns a negative status into ``DGError``.  Every step of the GEMM runs in the library's CUDA
+kernels; there is no fallback of any kind.
+
+Operands follow the NT convention of the DeepGEMM family ("Interfaces / Notices" of the DeepGEMM-for-PPU
+README): ``lhs = (a, sfa)`` with ``a`` [M, K] e4m3 and ``sfa`` fp32 [K/128, tma_aligned(M)] (MN-major, one
+scale per row and 128-K block); ``rhs = (b, sfb)`` with ``b`` [N, K] e4m3 (grouped: [G, N, K]) and ``sfb``
+fp32 [ceil(N/128), K/128] (grouped: [G, ...]), one scale per 128x128 block.  Scales must be powers of two.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdg.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "dg.h")
+
+DG_OK = 0
+STATUS_NAMES = {0: "DG_OK", -1: "DG_ERR_INVALID_ARG", -2: "DG_ERR_ALIGNMENT", -3: "DG_ERR_UNSUPPORTED",
+                -4: "DG_ERR_CUDA", -5: "DG_ERR_DEVICE_TIMEOUT", -6: "DG_ERR_BAD_GROUP"}
+
+
+class DGError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m moe_grouped_gemm_03_b200.build` "
+                      "(or __graft_entry__.build()); there is no non-CUDA implementation")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_LL = ctypes.c_longlong
+
+_SIGNATURES = {
+    "dg_get_m_alignment_for_contiguous_layout": (_I, []),
+    "dg_get_tma_aligned_size": (_I, [_I, _I]),
+    "dg_set_num_sms": (_I, [_I]),
+    "dg_get_num_sms": (_I, []),
+    "dg_num_tiles": (_LL, [_LL, _LL, _I, _I]),
+    "dg_select_block_n": (_I, [_LL, _I, _I]),
+    "dg_fp8_gemm_nt": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "dg_m_grouped_fp8_gemm_nt_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "dg_m_grouped_fp8_gemm_nt_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "dg_last_error": (ctypes.c_char_p, []),
+    "dg_check_device_error": (_I, [_P]),
+}
+for _name, (_res, _args) in _SIGNATURES.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raw entry points with the names of include/dg.h)."""
+    return _lib
+
+
+def header_symbols():
+    """Names of the functions include/dg.h declares."""
+    with open(HEADER_PATH) as f:
+        return re.findall(r"^DG_EXPORT[^(]*?\b(dg_\w+)\(", f.read(), flags=re.M)
+
+
+def last_error() -> str:
+    return _lib.dg_last_error().decode()
+
+
+def _check(status: int):
+    if status != DG_OK:
+        raise DGError(status, last_error())
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+_FP8_TYPES = (torch.uint8, torch.float8_e4m3fn)
+
+
+def _need(cond: bool, what: str):
+    if not cond:
+        raise DGError(-1, what)
+
+
+def _check_operand(name, t, dims, dtypes):
+    _need(isinstance(t, torch.Tensor), f"{name} must be a torch.Tensor")
+    _need(t.dim() == dims, f"{name} must have {dims} dims, got {tuple(t.shape)}")
+    _need(t.dtype in dtypes, f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    _need(t.is_contiguous(), f"{name} must be contiguous")
+    _need(t.is_cuda, f"{name} must be a CUDA tensor")
+
+
+# ------------------------------------------------------------------------------------------------ utilities
+def get_m_alignment_for_contiguous_layout() -> int:
+    return _lib.dg_get_m_alignment_for_contiguous_layout()
+
+
+def get_tma_aligned_size(mn: int, element_size: int) -> int:
+    return _lib.dg_get_tma_aligned_size(mn, element_size)
+
+
+def set_num_sms(n: int) -> int:
+    return _lib.dg_set_num_sms(n)
+
+
+def get_num_sms() -> int:
+    return _lib.dg_get_num_sms()
+
+
+def num_tiles(M: int, N: int, block_m: int, block_n: int) -> int:
+    return _lib.dg_num_tiles(M, N, block_m, block_n)
+
+
+def select_block_n(num_m_blocks: int, N: int, num_sms: int) -> int:
+    return _lib.dg_select_block_n(num_m_blocks, N, num_sms)
+
+
+def check_device_error(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel recorded a device-side error since the last check."""
+    s = _stream() if stream is None else stream
+    _check(_lib.dg_check_device_error(s))
+
+
+# ------------------------------------------------------------------------------------------------ GEMMs
+def fp8_gemm_nt(lhs: Tuple[torch.Tensor, torch.Tensor], rhs: Tuple[torch.Tensor, torch.Tensor],
+                out: torch.Tensor) -> None:
+    """out[M, N] = bf16(lhs @ rhs^T) with fine-grained scales (dense)."""
+    a, sfa = lhs
+    b, sfb = rhs
+    _check_operand("a", a, 2, _FP8_TYPES)
+    _check_operand("b", b, 2, _FP8_TYPES)
+    _check_operand("sfa", sfa, 2, (torch.float32,))
+    _check_operand("sfb", sfb, 2, (torch.float32,))
+    _check_operand("out", out, 2, (torch.bfloat16,))
+    M, K = a.shape
+    N = b.shape[0]
+    _need(b.shape[1] == K and tuple(out.shape) == (M, N), "shape mismatch between a, b and out")
+    _need(sfa.shape == (K // 128, get_tma_aligned_size(M, 4)), f"sfa must be [{K // 128}, {get_tma_aligned_size(M, 4)}]")
+    _need(sfb.shape == ((N + 127) // 128, K // 128), "sfb must be [ceil(N/128), K/128]")
+    _check(_lib.dg_fp8_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(out), M, N, K, _stream()))
+
+
+def m_grouped_fp8_gemm_nt_contiguous(lhs, rhs, out: torch.Tensor, m_indices: torch.Tensor) -> None:
+    """Contiguous layout: out[m] = lhs[m] @ rhs[m_indices[m]]^T; rows with m_indices == -1 are untouched."""
+    a, sfa = lhs
+    b, sfb = rhs
+    _check_operand("a", a, 2, _FP8_TYPES)
+    _check_operand("b", b, 3, _FP8_TYPES)
+    _check_operand("sfa", sfa, 2, (torch.float32,))
+    _check_operand("sfb", sfb, 3, (torch.float32,))
+    _check_operand("out", out, 2, (torch.bfloat16,))
+    _check_operand("m_indices", m_indices, 1, (torch.int32,))
+    M, K = a.shape
+    G, N, _ = b.shape
+    _need(b.shape[2] == K and tuple(out.shape) == (M, N) and m_indices.shape[0] == M, "shape mismatch")
+    _need(sfa.shape == (K // 128, get_tma_aligned_size(M, 4)), "sfa must be [K/128, tma_aligned(M)]")
+    _need(sfb.shape == (G, (N + 127) // 128, K // 128), "sfb must be [G, ceil(N/128), K/128]")
+    _check(_lib.dg_m_grouped_fp8_gemm_nt_contiguous(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(out),
+                                                    _ptr(m_indices), M, N, K, G, _stream()))
+
+
+def m_grouped_fp8_gemm_nt_masked(lhs, rhs, out: torch.Tensor, masked_m: torch.Tensor, expected_m: int) -> None:
+    """Masked layout: out[g, :masked_m[g]] = lhs[g, :masked_m[g]] @ rhs[g]^T; other rows are untouched."""
+    a, sfa = lhs
+    b, sfb = rhs
+    _check_operand("a", a, 3, _FP8_TYPES)
+    _check_operand("b", b, 3, _FP8_TYPES)
+    _check_operand("sfa", sfa, 3, (torch.float32,))
+    _check_operand("sfb", sfb, 3, (torch.float32,))
+    _check_operand("out", out, 3, (torch.bfloat16,))
+    _check_operand("masked_m", masked_m, 1, (torch.int32,))
+    G, M_max, K = a.shape
+    N = b.shape[1]
+    _need(b.shape[0] == G and b.shape[2] == K and tuple(out.shape) == (G, M_max, N) and masked_m.shape[0] == G,
+          "shape mismatch")
+    _need(sfa.shape == (G, K // 128, get_tma_aligned_size(M_max, 4)), "sfa must be [G, K/128, tma_aligned(M_max)]")
+    _need(sfb.shape == (G, (N + 127) // 128, K // 128), "sfb must be [G, ceil(N/128), K/128]")
+    _check(_lib.dg_m_grouped_fp8_gemm_nt_masked(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(out), _ptr(masked_m),
+                                                G, M_max, N, K, int(expected_m), _stream()))
+
+
+__all__ = [
+    "DGError", "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
+    "get_m_alignment_for_contiguous_layout", "get_tma_aligned_size", "set_num_sms", "get_num_sms", "num_tiles",
+    "select_block_n", "check_device_error", "lib", "header_symbols", "last_error",
+]

@@ -1,0 +1,305 @@
+// Host side of the C ABI declared in include/dg.h: argument validation, tile-shape choice, TMA
+// descriptors and the launch of the persistent sm_100a kernel on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <string>
+
+#include "dg.h"
+#include "gemm_kernel.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+int g_num_sms_cap = 0;  // 0: every SM of the device
+
+__device__ unsigned g_device_error_word;  // first device-side error code since the last check
+
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(DG_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+struct DeviceInfo {
+    int device = -1;
+    int num_sms = 0;
+    int major = 0, minor = 0;
+};
+
+int device_info(DeviceInfo &info) {
+    cudaError_t e = cudaGetDevice(&info.device);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if ((e = cudaDeviceGetAttribute(&info.num_sms, cudaDevAttrMultiProcessorCount, info.device)) != cudaSuccess)
+        return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+    if ((e = cudaDeviceGetAttribute(&info.major, cudaDevAttrComputeCapabilityMajor, info.device)) != cudaSuccess)
+        return cuda_fail(e, "cudaDeviceGetAttribute(major)");
+    if ((e = cudaDeviceGetAttribute(&info.minor, cudaDevAttrComputeCapabilityMinor, info.device)) != cudaSuccess)
+        return cuda_fail(e, "cudaDeviceGetAttribute(minor)");
+    if (info.major != 10 || info.minor != 0)
+        return fail(DG_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a only", info.device,
+                    info.major, info.minor);
+    return DG_OK;
+}
+
+int effective_sms(const DeviceInfo &info) {
+    return (g_num_sms_cap > 0 && g_num_sms_cap < info.num_sms) ? g_num_sms_cap : info.num_sms;
+}
+
+// ----------------------------------------------------------------------------------------------- TMA
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int get_encode_fn(EncodeTiledFn &fn) {
+    static EncodeTiledFn cached = nullptr;
+    if (!cached) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
+            return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+        cached = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    fn = cached;
+    return DG_OK;
+}
+
+// Row-major byte matrix [rows][K] (K-major e4m3 operand), boxes of box_rows x 128 bytes, 128-byte swizzle.
+int make_operand_map(CUtensorMap &map, const void *base, long long rows, int K, int box_rows) {
+    EncodeTiledFn encode;
+    if (int rc = get_encode_fn(encode)) return rc;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(dg::BLOCK_K), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return DG_OK;
+}
+
+// ----------------------------------------------------------------------------------------------- launch
+template <int BN, int STAGES>
+int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows, dg::GemmParams p, int grid,
+               cudaStream_t stream) {
+    using C = dg::Cfg<BN, STAGES>;
+    CUtensorMap ta, tb;
+    if (int rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M)) return rc;
+    if (int rc = make_operand_map(tb, b, b_rows, p.K, BN)) return rc;
+    auto kernel = dg::fp8_gemm_kernel<C>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    kernel<<<grid, dg::NUM_THREADS, C::SMEM_BYTES, stream>>>(ta, tb, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return DG_OK;
+}
+
+// Tile widths the library is built with, with the pipeline depth each fits in 227 KB of shared memory
+// and 512 TMEM columns (two BN-wide accumulators plus one scale slot per stage).
+constexpr int kCandidateBN[] = {224, 192, 160, 128};
+
+int launch_bn(int bn, const void *a, long long a_rows, const void *b, long long b_rows, const dg::GemmParams &p,
+              int grid, cudaStream_t stream) {
+    switch (bn) {
+        case 224: return launch_cfg<224, 4>(a, a_rows, b, b_rows, p, grid, stream);
+        case 192: return launch_cfg<192, 5>(a, a_rows, b, b_rows, p, grid, stream);
+        case 160: return launch_cfg<160, 5>(a, a_rows, b, b_rows, p, grid, stream);
+        case 128: return launch_cfg<128, 6>(a, a_rows, b, b_rows, p, grid, stream);
+        default: return fail(DG_ERR_UNSUPPORTED, "no kernel instantiated for BN=%d", bn);
+    }
+}
+
+int block_n_for(long long num_m_blocks, int N, int num_sms) { return dg_select_block_n(num_m_blocks, N, num_sms); }
+
+unsigned *device_error_word() {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
+    return static_cast<unsigned *>(p);
+}
+
+int check_common(const void *a, const float *sfa, const void *b, const float *sfb, const void *d, long long N,
+                 long long K) {
+    if (!a || !sfa || !b || !sfb || !d) return fail(DG_ERR_INVALID_ARG, "null pointer argument");
+    if (N <= 0 || K <= 0) return fail(DG_ERR_INVALID_ARG, "N=%lld and K=%lld must be positive", N, K);
+    if (K % 128) return fail(DG_ERR_ALIGNMENT, "K=%lld must be a multiple of 128", K);
+    if (N % 16) return fail(DG_ERR_ALIGNMENT, "N=%lld must be a multiple of 16", N);
+    if (!aligned(a, 16) || !aligned(b, 16) || !aligned(d, 16) || !aligned(sfa, 16) || !aligned(sfb, 16))
+        return fail(DG_ERR_ALIGNMENT, "a, b, d, sfa and sfb must be 16-byte aligned");
+    return DG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dg_get_m_alignment_for_contiguous_layout(void) { return dg::BLOCK_M; }
+
+int dg_get_tma_aligned_size(int mn, int elem_bytes) {
+    if (elem_bytes <= 0) return -1;
+    const int per16 = 16 / elem_bytes > 0 ? 16 / elem_bytes : 1;
+    return (mn + per16 - 1) / per16 * per16;
+}
+
+int dg_set_num_sms(int n) {
+    g_num_sms_cap = n > 0 ? n : 0;
+    return dg_get_num_sms();
+}
+
+int dg_get_num_sms(void) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return g_num_sms_cap;  // no device: report the cap alone
+    }
+    return (g_num_sms_cap > 0 && g_num_sms_cap < sms) ? g_num_sms_cap : sms;
+}
+
+long long dg_num_tiles(long long M, long long N, int block_m, int block_n) {
+    if (M <= 0 || N <= 0 || block_m <= 0 || block_n <= 0) return 0;
+    return ((M + block_m - 1) / block_m) * ((N + block_n - 1) / block_n);
+}
+
+int dg_select_block_n(long long num_m_blocks, int N, int num_sms) {
+    if (num_sms <= 0) num_sms = 1;
+    if (num_m_blocks <= 0) num_m_blocks = 1;
+    // Time of a persistent pass ~ waves x per-tile time; a tile's time grows with its width plus a fixed
+    // cost (prologue, epilogue drain) worth about 32 columns.
+    int best = kCandidateBN[0];
+    long long best_cost = -1;
+    for (int bn : kCandidateBN) {
+        const long long tiles = num_m_blocks * ((N + bn - 1) / bn);
+        const long long waves = (tiles + num_sms - 1) / num_sms;
+        const long long cost = waves * (bn + 32);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
+}
+
+const char *dg_last_error(void) { return g_last_error.c_str(); }
+
+int dg_check_device_error(dg_stream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned word = 0, zero = 0;
+    if ((e = cudaMemcpyFromSymbol(&word, g_device_error_word, sizeof(word))) != cudaSuccess)
+        return cuda_fail(e, "reading the device error word");
+    if ((e = cudaMemcpyToSymbol(g_device_error_word, &zero, sizeof(zero))) != cudaSuccess)
+        return cuda_fail(e, "clearing the device error word");
+    if (word == dg::ERR_TIMEOUT) return fail(DG_ERR_DEVICE_TIMEOUT, "a bounded wait inside the kernel ran out");
+    if (word == dg::ERR_BAD_GROUP)
+        return fail(DG_ERR_BAD_GROUP, "a group id or masked_m value was out of range; those rows were skipped");
+    if (word != 0) return fail(DG_ERR_CUDA, "unknown device error word %u", word);
+    return DG_OK;
+}
+
+int dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const float *sfb, void *d, int M, int N, int K,
+                   dg_stream_t stream) {
+    if (M < 0) return fail(DG_ERR_INVALID_ARG, "M=%d must be non-negative", M);
+    if (int rc = check_common(a, sfa, b, sfb, d, N, K)) return rc;
+    if (M == 0) return DG_OK;
+    DeviceInfo info;
+    if (int rc = device_info(info)) return rc;
+    dg::GemmParams p{};
+    p.mode = dg::MODE_DENSE;
+    p.M = M; p.N = N; p.K = K; p.G = 1;
+    p.num_m_blocks = (M + dg::BLOCK_M - 1) / dg::BLOCK_M;
+    p.sfa_ld = dg_get_tma_aligned_size(M, 4);
+    p.sfa = sfa; p.sfb = sfb;
+    p.d = static_cast<__nv_bfloat16 *>(d);
+    p.err = device_error_word();
+    if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
+    const int sms = effective_sms(info);
+    const int bn = block_n_for(p.num_m_blocks, N, sms);
+    p.num_n_blocks = (N + bn - 1) / bn;
+    const long long tiles = static_cast<long long>(p.num_m_blocks) * p.num_n_blocks;
+    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+    return launch_bn(bn, a, M, b, N, p, grid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
+                                        const int *m_indices, int M_total, int N, int K, int G, dg_stream_t stream) {
+    if (int rc = check_common(a, sfa, b, sfb, d, N, K)) return rc;
+    if (!m_indices) return fail(DG_ERR_INVALID_ARG, "m_indices is null");
+    if (!aligned(m_indices, 4)) return fail(DG_ERR_ALIGNMENT, "m_indices must be 4-byte aligned");
+    if (G < 1) return fail(DG_ERR_INVALID_ARG, "G=%d must be at least 1", G);
+    if (M_total < 0) return fail(DG_ERR_INVALID_ARG, "M_total=%d must be non-negative", M_total);
+    if (M_total % dg::BLOCK_M)
+        return fail(DG_ERR_ALIGNMENT, "M_total=%d must be a multiple of %d", M_total, dg::BLOCK_M);
+    if (static_cast<long long>(G) * N > 0x7fffffffLL) return fail(DG_ERR_INVALID_ARG, "G*N exceeds 2^31");
+    if (M_total == 0) return DG_OK;
+    DeviceInfo info;
+    if (int rc = device_info(info)) return rc;
+    dg::GemmParams p{};
+    p.mode = dg::MODE_CONTIGUOUS;
+    p.M = M_total; p.N = N; p.K = K; p.G = G;
+    p.num_m_blocks = M_total / dg::BLOCK_M;
+    p.sfa_ld = dg_get_tma_aligned_size(M_total, 4);
+    p.sfa = sfa; p.sfb = sfb;
+    p.d = static_cast<__nv_bfloat16 *>(d);
+    p.m_indices = m_indices;
+    p.err = device_error_word();
+    if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
+    const int sms = effective_sms(info);
+    const int bn = block_n_for(p.num_m_blocks, N, sms);
+    p.num_n_blocks = (N + bn - 1) / bn;
+    const long long tiles = static_cast<long long>(p.num_m_blocks) * p.num_n_blocks;
+    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+    return launch_bn(bn, a, M_total, b, static_cast<long long>(G) * N, p, grid,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
+                                    const int *masked_m, int G, int M_max, int N, int K, int expected_m,
+                                    dg_stream_t stream) {
+    if (int rc = check_common(a, sfa, b, sfb, d, N, K)) return rc;
+    if (!masked_m) return fail(DG_ERR_INVALID_ARG, "masked_m is null");
+    if (!aligned(masked_m, 4)) return fail(DG_ERR_ALIGNMENT, "masked_m must be 4-byte aligned");
+    if (G < 1 || G > dg::MAX_MASKED_GROUPS)
+        return fail(DG_ERR_INVALID_ARG, "G=%d must be in [1, %d]", G, dg::MAX_MASKED_GROUPS);
+    if (M_max < 1) return fail(DG_ERR_INVALID_ARG, "M_max=%d must be positive", M_max);
+    if (static_cast<long long>(G) * M_max > 0x7fffffffLL || static_cast<long long>(G) * N > 0x7fffffffLL)
+        return fail(DG_ERR_INVALID_ARG, "G*M_max or G*N exceeds 2^31");
+    DeviceInfo info;
+    if (int rc = device_info(info)) return rc;
+    dg::GemmParams p{};
+    p.mode = dg::MODE_MASKED;
+    p.M = M_max; p.N = N; p.K = K; p.G = G;
+    p.num_m_blocks = (M_max + dg::BLOCK_M - 1) / dg::BLOCK_M;
+    p.sfa_ld = dg_get_tma_aligned_size(M_max, 4);
+    p.sfa = sfa; p.sfb = sfb;
+    p.d = static_cast<__nv_bfloat16 *>(d);
+    p.masked_m = masked_m;
+    p.err = device_error_word();
+    if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
+    const int sms = effective_sms(info);
+    const int hint = expected_m > 0 && expected_m < M_max ? expected_m : M_max;
+    const long long hint_blocks = static_cast<long long>(G) * ((hint + dg::BLOCK_M - 1) / dg::BLOCK_M);
+    const int bn = block_n_for(hint_blocks, N, sms);
+    p.num_n_blocks = (N + bn - 1) / bn;
+    const long long max_tiles = static_cast<long long>(G) * p.num_m_blocks * p.num_n_blocks;
+    const int grid = static_cast<int>(max_tiles < sms ? max_tiles : sms);
+    return launch_bn(bn, a, static_cast<long long>(G) * M_max, b, static_cast<long long>(G) * N, p, grid,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -271,3 +271,22 @@ def make_config(i: int, seed: int = 0) -> Problem:
         rng = np.random.default_rng(seed)
         return make_contiguous(zipf_counts(65536, 64, 1.2), 7168, 2048, rng=rng, name=CONFIGS[5])
     raise ValueError(f"unknown config {i}")
+
+
+def to_torch(p: Problem, device="cuda"):
+    """Device copies of a problem's arrays in the library's call layout (no arithmetic)."""
+    import torch
+
+    def t(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).to(device)
+
+    out = {"a": t(p.a), "sfa": t(p.sfa), "b": t(p.b), "sfb": t(p.sfb)}
+    if p.kind == "dense":
+        out["b"] = out["b"].view(p.N, p.K)
+        out["sfb"] = out["sfb"].view(p.sfb.shape[1], p.sfb.shape[2])
+    if p.kind == "masked":
+        out["a"] = out["a"].view(p.G, p.M, p.K)
+        out["masked_m"] = t(p.masked_m)
+    if p.kind == "contiguous":
+        out["m_indices"] = t(p.m_indices)
+    return out

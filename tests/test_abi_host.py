@@ -1,0 +1,97 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared symbol, its host arithmetic
+matches the pages' worked example, and bad arguments return error codes before anything is launched."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import moe_grouped_gemm_03_b200 as dg
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+L = dg.lib()
+
+
+def test_every_declared_symbol_is_exported():
+    names = dg.header_symbols()
+    assert len(names) >= 11
+    out = subprocess.run(["nm", "-D", "--defined-only", dg.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        getattr(L, n)  # resolvable through ctypes
+
+
+def test_alignment_and_tma_size():
+    assert dg.get_m_alignment_for_contiguous_layout() == 128
+    assert dg.get_tma_aligned_size(1, 4) == 4
+    assert dg.get_tma_aligned_size(4096, 4) == 4096
+    assert dg.get_tma_aligned_size(4319, 4) == 4320
+    assert dg.get_tma_aligned_size(17, 1) == 32
+    assert dg.get_tma_aligned_size(5, 0) == -1
+
+
+def test_tile_count_worked_example():
+    rows = [ln.split() for ln in open(os.path.join(HERE, "golden", "sm_utilisation_example.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    assert rows
+    for M, N, bm, bn, tiles in rows:
+        assert dg.num_tiles(int(M), int(N), int(bm), int(bn)) == int(tiles)
+
+
+def test_block_n_choice_avoids_wave_quantisation_on_148_sms():
+    # dense 4096 x 7168: 32 M blocks; 224-wide tiles give 1024 tiles = 6.92 waves of 148
+    assert dg.select_block_n(32, 7168, 148) == 224
+    # a single 128-row block of a 256-wide output: two 128-wide tiles beat one ragged 224 + 32
+    assert dg.select_block_n(1, 256, 148) == 128
+    for mb, n in [(1, 16), (7, 4096), (547, 7168), (220, 4096)]:
+        assert dg.select_block_n(mb, n, 148) in (128, 160, 192, 224)
+
+
+def test_num_sms_cap_roundtrip():
+    try:
+        dg.set_num_sms(100)
+        assert dg.get_num_sms() in (100,) or dg.get_num_sms() < 100
+    finally:
+        dg.set_num_sms(0)
+
+
+def _call_dense(a=1, sfa=1, b=1, sfb=1, d=1, M=128, N=256, K=512):
+    P = ctypes.c_void_p
+    return L.dg_fp8_gemm_nt(P(a * 256), P(sfa * 256), P(b * 256), P(sfb * 256), P(d * 256), M, N, K, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(a=0), -1), (dict(d=0), -1), (dict(K=100), -2), (dict(K=0), -1), (dict(N=8), -2), (dict(N=0), -1),
+    (dict(M=-1), -1)])
+def test_dense_validation(kw, code):
+    assert _call_dense(**kw) == code
+    assert dg.last_error()
+
+
+def test_dense_misaligned_pointer():
+    P = ctypes.c_void_p
+    assert L.dg_fp8_gemm_nt(P(256 + 8), P(256), P(256), P(256), P(256), 128, 256, 512, None) == -2
+
+
+def test_dense_empty_is_noop_without_device():
+    assert _call_dense(M=0) == 0
+
+
+def test_grouped_validation():
+    P = ctypes.c_void_p
+    ok = dict(a=P(256), sfa=P(256), b=P(256), sfb=P(256), d=P(256))
+    # contiguous: G < 1, M_total not a multiple of 128, null m_indices
+    assert L.dg_m_grouped_fp8_gemm_nt_contiguous(*ok.values(), P(256), 256, 256, 512, 0, None) == -1
+    assert L.dg_m_grouped_fp8_gemm_nt_contiguous(*ok.values(), P(256), 200, 256, 512, 2, None) == -2
+    assert L.dg_m_grouped_fp8_gemm_nt_contiguous(*ok.values(), None, 256, 256, 512, 2, None) == -1
+    assert L.dg_m_grouped_fp8_gemm_nt_contiguous(*ok.values(), P(258), 256, 256, 512, 2, None) == -2
+    assert L.dg_m_grouped_fp8_gemm_nt_contiguous(*ok.values(), P(256), 0, 256, 512, 2, None) == 0
+    # masked: G out of range, M_max < 1, null masked_m
+    assert L.dg_m_grouped_fp8_gemm_nt_masked(*ok.values(), P(256), 0, 256, 256, 512, 128, None) == -1
+    assert L.dg_m_grouped_fp8_gemm_nt_masked(*ok.values(), P(256), 1025, 256, 256, 512, 128, None) == -1
+    assert L.dg_m_grouped_fp8_gemm_nt_masked(*ok.values(), P(256), 4, 0, 256, 512, 128, None) == -1
+    assert L.dg_m_grouped_fp8_gemm_nt_masked(*ok.values(), None, 4, 256, 256, 512, 128, None) == -1
+    assert L.dg_m_grouped_fp8_gemm_nt_masked(*ok.values(), P(256), 4, 256, 250, 512, 128, None) == -2
