@@ -93,18 +93,36 @@ int make_operand_map(CUtensorMap &map, const void *base, long long rows, int K, 
     return DG_OK;
 }
 
+// MN-major fp32 scales [outer][ld] (outer = K blocks, times G for the masked layout): boxes of 128 rows x
+// one K block, no swizzle.
+int make_sfa_map(CUtensorMap &map, const float *base, int ld, long long outer) {
+    EncodeTiledFn encode;
+    if (int rc = get_encode_fn(encode)) return rc;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(ld), static_cast<cuuint64_t>(outer)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(dg::BLOCK_M), 1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", static_cast<int>(r));
+    return DG_OK;
+}
+
 // ----------------------------------------------------------------------------------------------- launch
 template <int BN, int STAGES>
 int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows, dg::GemmParams p, int grid,
                cudaStream_t stream) {
     using C = dg::Cfg<BN, STAGES>;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, tsfa;
     if (int rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M)) return rc;
     if (int rc = make_operand_map(tb, b, b_rows, p.K, BN)) return rc;
+    const long long sfa_rows = static_cast<long long>(p.K / dg::BLOCK_K) * (p.mode == dg::MODE_MASKED ? p.G : 1);
+    if (int rc = make_sfa_map(tsfa, p.sfa, p.sfa_ld, sfa_rows)) return rc;
     auto kernel = dg::fp8_gemm_kernel<C>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-    kernel<<<grid, dg::NUM_THREADS, C::SMEM_BYTES, stream>>>(ta, tb, p);
+    kernel<<<grid, dg::NUM_THREADS, C::SMEM_BYTES, stream>>>(ta, tb, tsfa, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return DG_OK;

@@ -43,6 +43,7 @@ constexpr int BLOCK_K = 128;  // = the scale block along K
 constexpr int MMA_K = 32;     // K of one kind::mxf8f6f4 MMA
 constexpr int NUM_THREADS = 256;
 constexpr int MAX_MASKED_GROUPS = 1024;
+constexpr int SFB_KB_REGS = 4;  // K blocks of SFB held per lane: K <= 32 * 4 * 128 = 16384 on the fast path
 constexpr int TMEM_COLS = 512;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s for any single wait
 constexpr int SMEM_LIMIT = 232448;                  // 227 KB of dynamic shared memory per CTA
@@ -74,13 +75,15 @@ struct Cfg {
     static constexpr int A_BYTES = BLOCK_M * BLOCK_K;             // e4m3: 1 byte per element
     static constexpr int B_BYTES = BN * BLOCK_K;
     static constexpr int SF_WORDS = 128 + 128 * SFB_ATOMS;        // 32-bit words per stage (SFA, then SFB)
+    static constexpr int SFA_RAW_BYTES = BLOCK_M * 4;             // fp32 SFA slice of a stage, by TMA
     static constexpr int SF_COLS = 4 + 4 * SFB_ATOMS;             // TMEM columns per stage's scales
     static constexpr int SF_TMEM_BASE = 2 * BN;                   // after the two accumulators
     static constexpr int NUM_BARRIERS = 3 * STAGES + 5;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;
-    static constexpr int OFF_BAR = OFF_SF + STAGES * SF_WORDS * 4;
+    static constexpr int OFF_SFA_RAW = OFF_SF + STAGES * SF_WORDS * 4;
+    static constexpr int OFF_BAR = OFF_SFA_RAW + STAGES * SFA_RAW_BYTES;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARRIERS * 8;   // tmem base, abort flag
     static constexpr int OFF_PREFIX = OFF_MISC + 16;               // masked: int[G+1] block prefix
     static constexpr int OFF_MM = OFF_PREFIX + 4 * (MAX_MASKED_GROUPS + 1);  // masked: clamped masked_m
@@ -179,7 +182,7 @@ __device__ __forceinline__ uint32_t ue8m0_x4(float s) {
 template <class C>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                    const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmap_sfa, const GemmParams p) {
     constexpr int BN = C::BN;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -187,6 +190,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint8_t *sA = smem + C::OFF_A;
     uint8_t *sB = smem + C::OFF_B;
     uint32_t *sSF = reinterpret_cast<uint32_t *>(smem + C::OFF_SF);
+    float *sSFA_raw = reinterpret_cast<float *>(smem + C::OFF_SFA_RAW);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *full_tma = bars;
     uint64_t *full_sf = bars + STAGES;
@@ -218,6 +222,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fence_proxy_async_smem();
         tma_prefetch_desc(&tmap_a);
         tma_prefetch_desc(&tmap_b);
+        tma_prefetch_desc(&tmap_sfa);
     }
     if (warp == 1) {
         tmem_alloc(s_tmem_base, TMEM_COLS);
@@ -270,11 +275,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 Tile ti;
                 if (!decode_tile<BN>(p, ctl, t, ti)) continue;
                 const int brow = ti.g * p.N + ti.n0;
+                const int sfa_row = p.mode == MODE_MASKED ? ti.g * nkb : 0;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!wait_bounded(&empty[s], ph ^ 1u, s_abort, p.err)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&full_tma[s], C::A_BYTES + C::B_BYTES);
+                    mbar_arrive_expect_tx(&full_tma[s], C::A_BYTES + C::B_BYTES + C::SFA_RAW_BYTES);
                     tma_load_2d(sA + s * C::A_BYTES, &tmap_a, &full_tma[s], kb * BLOCK_K, ti.row0);
                     tma_load_2d(sB + s * C::B_BYTES, &tmap_b, &full_tma[s], kb * BLOCK_K, brow);
+                    tma_load_2d(sSFA_raw + s * BLOCK_M, &tmap_sfa, &full_tma[s], ti.local_row0, sfa_row + kb);
                     armed |= 1u << s;
                     armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -342,46 +349,88 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else if (warp == 2) {
         // ---------------------------------------------------------------- scale-factor packer
+        // SFA arrives with the stage (fp32 slice by TMA).  SFB: the tile's <= 3 scale rows x K blocks are
+        // held in registers (lane l holds K blocks l, l+32, ...), loaded one tile ahead so the global
+        // latency hides behind the current tile.
         int s = 0;
         uint32_t ph = 0;
         const int nnb128 = (p.N + 127) / 128;
-        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-            Tile ti;
-            if (!decode_tile<BN>(p, ctl, t, ti)) continue;
-            const float *sfa_g = p.sfa + (p.mode == MODE_MASKED ? static_cast<size_t>(ti.g) * nkb * p.sfa_ld : 0);
+        const bool sfb_in_regs = nkb <= 32 * SFB_KB_REGS;
+        float cur[3][SFB_KB_REGS], nxt[3][SFB_KB_REGS];
+        auto load_sfb = [&](const Tile &ti, float (&v)[3][SFB_KB_REGS]) {
             const float *sfb_g = p.sfb + static_cast<size_t>(ti.g) * nnb128 * nkb;
-            const int r0 = 4 * lane;
-            const int mrow = ti.local_row0 + r0;
-            bool ok = true;
-            for (int kb = 0; kb < nkb; ++kb) {
-                // load before waiting: the loads do not touch the ring
-                float4 va = make_float4(1.f, 1.f, 1.f, 1.f);
-                if (mrow < p.sfa_ld)
-                    va = __ldg(reinterpret_cast<const float4 *>(sfa_g + static_cast<size_t>(kb) * p.sfa_ld + mrow));
-                float vb[C::SFB_ATOMS * 4];
+            const int nb0 = ti.n0 >> 7;
 #pragma unroll
-                for (int j = 0; j < C::SFB_ATOMS * 4; ++j) {
-                    const int n = ti.n0 + lane + 32 * j;
-                    vb[j] = n < p.N ? __ldg(sfb_g + (n >> 7) * nkb + kb) : 1.f;
+            for (int j = 0; j < 3; ++j)
+#pragma unroll
+                for (int i = 0; i < SFB_KB_REGS; ++i) {
+                    const int kb = lane + 32 * i;
+                    v[j][i] = (nb0 + j < nnb128 && kb < nkb) ? __ldg(sfb_g + (nb0 + j) * nkb + kb) : 1.f;
                 }
-                if (!warp_wait_bounded(&empty[s], ph ^ 1u, s_abort, p.err, lane)) { ok = false; break; }
+        };
+        auto next_valid = [&](int &t, Tile &ti) {
+            for (; t < total_tiles; t += gridDim.x)
+                if (decode_tile<BN>(p, ctl, t, ti)) return true;
+            return false;
+        };
+        int t = blockIdx.x;
+        Tile ti;
+        bool have = next_valid(t, ti);
+        if (have && sfb_in_regs) load_sfb(ti, cur);
+        bool ok = true;
+        while (have && ok) {
+            int t2 = t + gridDim.x;
+            Tile tn;
+            const bool have2 = next_valid(t2, tn);
+            if (have2 && sfb_in_regs) load_sfb(tn, nxt);
+            const float *sfb_g = p.sfb + static_cast<size_t>(ti.g) * nnb128 * nkb;
+            const int nb0 = ti.n0 >> 7;
+            for (int kb = 0; kb < nkb; ++kb) {
+                float sb[3];
+                if (sfb_in_regs) {
+                    const int reg = kb >> 5, src = kb & 31;
+#pragma unroll
+                    for (int j = 0; j < 3; ++j) {
+                        float x = cur[j][0];
+#pragma unroll
+                        for (int i = 1; i < SFB_KB_REGS; ++i) x = reg == i ? cur[j][i] : x;
+                        sb[j] = __shfl_sync(0xffffffffu, x, src);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 3; ++j)
+                        sb[j] = nb0 + j < nnb128 ? __ldg(sfb_g + (nb0 + j) * nkb + kb) : 1.f;
+                }
+                if (!warp_wait_bounded(&full_tma[s], ph, s_abort, p.err, lane)) { ok = false; break; }
+                const float4 va = reinterpret_cast<const float4 *>(sSFA_raw + s * BLOCK_M)[lane];
                 uint32_t *w = sSF + s * C::SF_WORDS;
                 // tcgen05.cp 32x128b source: word (r % 32) * 4 + r / 32 holds row r of a 128-row atom
+                const int r0 = 4 * lane;
                 w[((r0 + 0) & 31) * 4 + ((r0 + 0) >> 5)] = ue8m0_x4(va.x);
                 w[((r0 + 1) & 31) * 4 + ((r0 + 1) >> 5)] = ue8m0_x4(va.y);
                 w[((r0 + 2) & 31) * 4 + ((r0 + 2) >> 5)] = ue8m0_x4(va.z);
                 w[((r0 + 3) & 31) * 4 + ((r0 + 3) >> 5)] = ue8m0_x4(va.w);
 #pragma unroll
                 for (int j = 0; j < C::SFB_ATOMS * 4; ++j) {
-                    const int r = lane + 32 * j;  // row inside the BN tile
-                    w[128 + (r >> 7) * 128 + (r & 31) * 4 + ((r >> 5) & 3)] = ue8m0_x4(vb[j]);
+                    const int r = lane + 32 * j;                        // row inside the BN tile
+                    const int which = ((ti.n0 + r) >> 7) - nb0;         // 0, 1 or 2
+                    const float v = which == 0 ? sb[0] : (which == 1 ? sb[1] : sb[2]);
+                    w[128 + (r >> 7) * 128 + (r & 31) * 4 + ((r >> 5) & 3)] = ue8m0_x4(v);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full_sf[s]);
                 if (++s == STAGES) { s = 0; ph ^= 1u; }
             }
-            if (!ok) break;
+            if (sfb_in_regs) {
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+#pragma unroll
+                    for (int i = 0; i < SFB_KB_REGS; ++i) cur[j][i] = nxt[j][i];
+            }
+            ti = tn;
+            t = t2;
+            have = have2;
         }
     } else if (warp >= 4) {
         // ---------------------------------------------------------------- epilogue
