@@ -103,6 +103,13 @@ DG_EXPORT int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, c
                                     void *d, const int *masked_m, int G, int M_max, int N, int K,
                                     int expected_m, dg_stream_t stream);
 
+/* Tile-shape policy for the next calls on any thread: -1 (default) lets the library choose between one
+ * CTA per 128-row tile and CTA pairs (2-CTA clusters, tcgen05 cta_group::2) computing 256-row tiles;
+ * 0 forces single CTAs; 1 uses pairs wherever the layout allows.  Results agree within the tolerance of
+ * fp32 accumulation either way.  Returns the policy now in force.  (README "Optimizations": larger block
+ * sizes up to 256x256.) */
+DG_EXPORT int dg_set_cta_pair_policy(int policy);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 DG_EXPORT const char *dg_last_error(void);
 

@@ -53,6 +53,7 @@ _SIGNATURES = {
     "dg_fp8_gemm_nt": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_gemm_nt_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_gemm_nt_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "dg_set_cta_pair_policy": (_I, [_I]),
     "dg_last_error": (ctypes.c_char_p, []),
     "dg_check_device_error": (_I, [_P]),
 }
@@ -131,6 +132,11 @@ def select_block_n(num_m_blocks: int, N: int, num_sms: int) -> int:
     return _lib.dg_select_block_n(num_m_blocks, N, num_sms)
 
 
+def set_cta_pair_policy(policy: int) -> int:
+    """-1: library decides; 0: single-CTA 128-row tiles only; 1: 2-CTA 256-row tiles wherever possible."""
+    return _lib.dg_set_cta_pair_policy(policy)
+
+
 def check_device_error(stream=None) -> None:
     """Synchronise the stream and raise if a kernel recorded a device-side error since the last check."""
     s = _stream() if stream is None else stream
@@ -198,5 +204,5 @@ def m_grouped_fp8_gemm_nt_masked(lhs, rhs, out: torch.Tensor, masked_m: torch.Te
 __all__ = [
     "DGError", "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
     "get_m_alignment_for_contiguous_layout", "get_tma_aligned_size", "set_num_sms", "get_num_sms", "num_tiles",
-    "select_block_n", "check_device_error", "lib", "header_symbols", "last_error",
+    "select_block_n", "set_cta_pair_policy", "check_device_error", "lib", "header_symbols", "last_error",
 ]

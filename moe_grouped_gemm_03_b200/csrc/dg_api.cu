@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <string>
 
 #include "dg.h"
@@ -93,14 +94,14 @@ int make_operand_map(CUtensorMap &map, const void *base, long long rows, int K, 
     return DG_OK;
 }
 
-// MN-major fp32 scales [outer][ld] (outer = K blocks, times G for the masked layout): boxes of 128 rows x
-// one K block, no swizzle.
-int make_sfa_map(CUtensorMap &map, const float *base, int ld, long long outer) {
+// MN-major fp32 scales [outer][ld] (outer = K blocks, times G for the masked layout): boxes of one tile's
+// rows (128 or 256) x four K blocks, no swizzle.
+int make_sfa_map(CUtensorMap &map, const float *base, int ld, long long outer, int box_rows) {
     EncodeTiledFn encode;
     if (int rc = get_encode_fn(encode)) return rc;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(ld), static_cast<cuuint64_t>(outer)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(dg::BLOCK_M), 1};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(dg::SF_GROUP)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -110,40 +111,111 @@ int make_sfa_map(CUtensorMap &map, const float *base, int ld, long long outer) {
 }
 
 // ----------------------------------------------------------------------------------------------- launch
-template <int BN, int STAGES>
+int g_pair_policy = -1;  // -1: library decides; 0: single CTAs only; 1: CTA pairs whenever supported
+
+template <int BN, int CTAS, int KPS>
 int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows, dg::GemmParams p, int grid,
                cudaStream_t stream) {
-    using C = dg::Cfg<BN, STAGES>;
+    using C = dg::Cfg<BN, CTAS, KPS>;
     CUtensorMap ta, tb, tsfa;
     if (int rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M)) return rc;
-    if (int rc = make_operand_map(tb, b, b_rows, p.K, BN)) return rc;
+    if (int rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS)) return rc;
     const long long sfa_rows = static_cast<long long>(p.K / dg::BLOCK_K) * (p.mode == dg::MODE_MASKED ? p.G : 1);
-    if (int rc = make_sfa_map(tsfa, p.sfa, p.sfa_ld, sfa_rows)) return rc;
+    if (int rc = make_sfa_map(tsfa, p.sfa, p.sfa_ld, sfa_rows, C::TILE_M)) return rc;
     auto kernel = dg::fp8_gemm_kernel<C>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-    kernel<<<grid, dg::NUM_THREADS, C::SMEM_BYTES, stream>>>(ta, tb, tsfa, p);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid * CTAS), 1, 1);
+    cfg.blockDim = dim3(dg::NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CTAS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (CTAS > 1) {
+        // a persistent grid larger than the co-resident clusters would only queue behind itself
+        static int max_clusters[64] = {0};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        int &cached = max_clusters[dev & 63];
+        if (cached == 0) {
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+                cudaGetLastError();
+                n = grid;
+            }
+            cached = n;
+        }
+        if (grid > cached) cfg.gridDim.x = static_cast<unsigned>(cached * CTAS);
+    }
+    static const bool debug = getenv("DG_DEBUG") && getenv("DG_DEBUG")[0] == '1';
+    if (debug)
+        fprintf(stderr, "[dg] mode=%d M=%d N=%d K=%d G=%d BN=%d stages=%d x %d ctas=%d grid=%u smem=%d windows=%d\n", p.mode,
+                p.M, p.N, p.K, p.G, BN, C::STAGES, KPS, CTAS, cfg.gridDim.x, C::SMEM_BYTES, p.num_windows);
+    e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, p);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return DG_OK;
 }
 
-// Tile widths the library is built with, with the pipeline depth each fits in 227 KB of shared memory
-// and 512 TMEM columns (two BN-wide accumulators plus one scale slot per stage).
+// Tile widths the library is built with, and the pipeline depth each fits in 227 KB of shared memory and
+// 512 TMEM columns (two BN-wide accumulators plus one scale slot per stage).
 constexpr int kCandidateBN[] = {224, 192, 160, 128};
 
-int launch_bn(int bn, const void *a, long long a_rows, const void *b, long long b_rows, const dg::GemmParams &p,
-              int grid, cudaStream_t stream) {
-    switch (bn) {
-        case 224: return launch_cfg<224, 4>(a, a_rows, b, b_rows, p, grid, stream);
-        case 192: return launch_cfg<192, 5>(a, a_rows, b, b_rows, p, grid, stream);
-        case 160: return launch_cfg<160, 5>(a, a_rows, b, b_rows, p, grid, stream);
-        case 128: return launch_cfg<128, 6>(a, a_rows, b, b_rows, p, grid, stream);
-        default: return fail(DG_ERR_UNSUPPORTED, "no kernel instantiated for BN=%d", bn);
+int launch_bn(int bn, int ctas, const void *a, long long a_rows, const void *b, long long b_rows,
+              const dg::GemmParams &p, int grid, cudaStream_t stream) {
+    if (ctas == 2) {
+        switch (bn) {
+            case 224: return launch_cfg<224, 2, 2>(a, a_rows, b, b_rows, p, grid, stream);
+            case 192: return launch_cfg<192, 2, 2>(a, a_rows, b, b_rows, p, grid, stream);
+            case 160: return launch_cfg<160, 2, 2>(a, a_rows, b, b_rows, p, grid, stream);
+            case 128: return launch_cfg<128, 2, 2>(a, a_rows, b, b_rows, p, grid, stream);
+            default: break;
+        }
+    } else {
+        switch (bn) {
+            case 224: return launch_cfg<224, 1, 1>(a, a_rows, b, b_rows, p, grid, stream);
+            case 192: return launch_cfg<192, 1, 1>(a, a_rows, b, b_rows, p, grid, stream);
+            case 160: return launch_cfg<160, 1, 1>(a, a_rows, b, b_rows, p, grid, stream);
+            case 128: return launch_cfg<128, 1, 1>(a, a_rows, b, b_rows, p, grid, stream);
+            default: break;
+        }
     }
+    return fail(DG_ERR_UNSUPPORTED, "no kernel instantiated for BN=%d with %d CTA(s) per tile", bn, ctas);
 }
 
-int block_n_for(long long num_m_blocks, int N, int num_sms) { return dg_select_block_n(num_m_blocks, N, num_sms); }
+// Shape and launch: picks single CTAs or CTA pairs, the tile width, and the persistent grid.
+//   sel1 / sel2:     128-row / 256-row windows the tile shape is chosen for (a hint for the masked layout)
+//   bound1 / bound2: the most 128-row / 256-row tiles the device may find (sizes the grid)
+//   windows1/2:      the kernel's window count (dense, contiguous); unused for the masked layout
+struct Plan {
+    long long sel1, sel2, bound1, bound2, windows1, windows2;
+    bool pair_supported;
+};
+
+int plan_and_launch(dg::GemmParams p, const DeviceInfo &info, const Plan &plan, const void *a, long long a_rows,
+                    const void *b, long long b_rows, cudaStream_t stream) {
+    const int sms = effective_sms(info);
+    bool pair = plan.pair_supported && sms >= 2;
+    if (g_pair_policy == 0) pair = false;
+    if (g_pair_policy < 0 && pair) {
+        // pairs pay once there is at least a wave of them
+        const int bn = dg_select_block_n(plan.sel2, p.N, sms / 2);
+        pair = plan.sel2 * ((p.N + bn - 1) / bn) >= sms / 2;
+    }
+    const int units = pair ? sms / 2 : sms;
+    const int bn = dg_select_block_n(pair ? plan.sel2 : plan.sel1, p.N, units);
+    p.num_n_blocks = (p.N + bn - 1) / bn;
+    p.num_windows = static_cast<int>(p.mode == dg::MODE_MASKED ? 0 : (pair ? plan.windows2 : plan.windows1));
+    const long long tiles = (pair ? plan.bound2 : plan.bound1) * p.num_n_blocks;
+    const int grid = static_cast<int>(tiles < units ? tiles : units);
+    if (grid <= 0) return DG_OK;
+    return launch_bn(bn, pair ? 2 : 1, a, a_rows, b, b_rows, p, grid, stream);
+}
 
 unsigned *device_error_word() {
     void *p = nullptr;
@@ -240,18 +312,14 @@ int dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const float *
     dg::GemmParams p{};
     p.mode = dg::MODE_DENSE;
     p.M = M; p.N = N; p.K = K; p.G = 1;
-    p.num_m_blocks = (M + dg::BLOCK_M - 1) / dg::BLOCK_M;
     p.sfa_ld = dg_get_tma_aligned_size(M, 4);
     p.sfa = sfa; p.sfb = sfb;
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.err = device_error_word();
     if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
-    const int sms = effective_sms(info);
-    const int bn = block_n_for(p.num_m_blocks, N, sms);
-    p.num_n_blocks = (N + bn - 1) / bn;
-    const long long tiles = static_cast<long long>(p.num_m_blocks) * p.num_n_blocks;
-    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-    return launch_bn(bn, a, M, b, N, p, grid, reinterpret_cast<cudaStream_t>(stream));
+    const long long w1 = (M + dg::BLOCK_M - 1) / dg::BLOCK_M, w2 = (M + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M);
+    const Plan plan{w1, w2, w1, w2, w1, w2, true};
+    return plan_and_launch(p, info, plan, a, M, b, N, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
@@ -270,20 +338,18 @@ int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const v
     dg::GemmParams p{};
     p.mode = dg::MODE_CONTIGUOUS;
     p.M = M_total; p.N = N; p.K = K; p.G = G;
-    p.num_m_blocks = M_total / dg::BLOCK_M;
     p.sfa_ld = dg_get_tma_aligned_size(M_total, 4);
     p.sfa = sfa; p.sfb = sfb;
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.m_indices = m_indices;
     p.err = device_error_word();
     if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
-    const int sms = effective_sms(info);
-    const int bn = block_n_for(p.num_m_blocks, N, sms);
-    p.num_n_blocks = (N + bn - 1) / bn;
-    const long long tiles = static_cast<long long>(p.num_m_blocks) * p.num_n_blocks;
-    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-    return launch_bn(bn, a, M_total, b, static_cast<long long>(G) * N, p, grid,
-                     reinterpret_cast<cudaStream_t>(stream));
+    const long long w1 = M_total / dg::BLOCK_M, w2 = (w1 + 1) / 2;
+    // a 256-row window holds at most two tiles (its halves may belong to two groups)
+    const long long bound = w2 + (w2 < G ? w2 : G);
+    const Plan plan{w1, w2, w1, bound, w1, w2, w2 <= dg::MAX_PAIR_WINDOWS};
+    return plan_and_launch(p, info, plan, a, M_total, b, static_cast<long long>(G) * N,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
@@ -302,22 +368,26 @@ int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const void 
     dg::GemmParams p{};
     p.mode = dg::MODE_MASKED;
     p.M = M_max; p.N = N; p.K = K; p.G = G;
-    p.num_m_blocks = (M_max + dg::BLOCK_M - 1) / dg::BLOCK_M;
     p.sfa_ld = dg_get_tma_aligned_size(M_max, 4);
     p.sfa = sfa; p.sfb = sfb;
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.masked_m = masked_m;
     p.err = device_error_word();
     if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
-    const int sms = effective_sms(info);
+    // tile shape from the caller's hint; the grid from the most tiles masked_m could ask for
     const int hint = expected_m > 0 && expected_m < M_max ? expected_m : M_max;
-    const long long hint_blocks = static_cast<long long>(G) * ((hint + dg::BLOCK_M - 1) / dg::BLOCK_M);
-    const int bn = block_n_for(hint_blocks, N, sms);
-    p.num_n_blocks = (N + bn - 1) / bn;
-    const long long max_tiles = static_cast<long long>(G) * p.num_m_blocks * p.num_n_blocks;
-    const int grid = static_cast<int>(max_tiles < sms ? max_tiles : sms);
-    return launch_bn(bn, a, static_cast<long long>(G) * M_max, b, static_cast<long long>(G) * N, p, grid,
-                     reinterpret_cast<cudaStream_t>(stream));
+    const long long h1 = static_cast<long long>(G) * ((hint + dg::BLOCK_M - 1) / dg::BLOCK_M);
+    const long long h2 = static_cast<long long>(G) * ((hint + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M));
+    const long long max1 = static_cast<long long>(G) * ((M_max + dg::BLOCK_M - 1) / dg::BLOCK_M);
+    const long long max2 = static_cast<long long>(G) * ((M_max + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M));
+    const Plan plan{h1, h2, max1, max2, 0, 0, true};
+    return plan_and_launch(p, info, plan, a, static_cast<long long>(G) * M_max, b, static_cast<long long>(G) * N,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dg_set_cta_pair_policy(int policy) {
+    g_pair_policy = policy < 0 ? -1 : (policy > 0 ? 1 : 0);
+    return g_pair_policy;
 }
 
 }  // extern "C"

@@ -3,32 +3,45 @@
 //   D[m][n] = bf16( sum_kb sfa(m,kb) * sfb(g, n/128, kb) * sum_{k in kb} A[m][k] * B_g[n][k] )
 //
 // ("FP8 GEMM kernels with fine-grained scaling", DeepGEMM-for-PPU README: "Interfaces" for the three
-// call shapes, "Optimizations" for persistent warp specialisation and the unified block scheduler.)
+// call shapes, "Optimizations" for persistent warp specialisation, the unified block scheduler, larger
+// blocks and unaligned block sizes.)
 //
-// One CTA per SM, 256 threads:
-//   warp 0      TMA producer: A tile [128 x 128 B] and B tile [BN x 128 B] per 128-K block into a
-//               STAGES-deep shared-memory ring (128-byte swizzle).
-//   warp 1      TMEM owner and MMA issuer (one thread): per 128-K block, copies the block's scale factors
-//               shared -> TMEM (tcgen05.cp) and issues four tcgen05.mma kind::mxf8f6f4 (K = 32 each) into
-//               one of two TMEM accumulators (128 lanes x BN fp32 columns).
-//   warp 2      scale-factor packer: turns the fp32 power-of-two scales of the block into UE8M0 bytes
-//               (the fp32 exponent field) laid out the way tcgen05.cp / the block-scaled MMA read them.
-//               The 128-K scale is repeated in the four byte slots of each 32-bit word, i.e. once per
-//               32-wide K sub-block, so the MMA's per-32 scaling applies the 1x128 / 128x128 recipe
-//               exactly and the per-K-block promotion happens inside the tensor core.
-//   warps 4..7  epilogue: TMEM -> registers -> bf16 (RNE) -> global, only for rows the GEMM owns, while
-//               the MMA warp already fills the other accumulator with the next tile.
+// CTAS = 1: one CTA computes a 128 x BN output tile.  CTAS = 2: a cluster of two CTAs (a CTA pair) computes
+// a 256 x BN tile with tcgen05.mma.cta_group::2: each CTA loads its own 128 rows of A and its own BN/2 rows
+// of B (no multicast), the leader CTA issues the MMAs, and each CTA's TMEM holds its 128 rows of D.  The
+// pair halves the B bytes each SM pulls from L2 per FLOP.
 //
-// Tile scheduler (all roles walk the same sequence): tiles are 128-row M blocks x BN-column N blocks,
-// N fastest, handed round-robin to the persistent CTAs.
-//   dense       ceil(M/128) M blocks.
-//   contiguous  M_total/128 M blocks; the group of a block is m_indices[first row]; -1 skips the block.
-//   masked      per group ceil(masked_m[g]/128) M blocks, counted on the device (prefix in shared memory),
-//               so the host never needs masked_m.
+// Per CTA, 256 threads:
+//   warp 0      TMA producer: A [128 x 128 B] and B [BN/CTAS x 128 B] per 128-K block, KPS K blocks per
+//               stage of a STAGES-deep ring (128-byte swizzle; one barrier wait and one commit per stage).
+//   warp 1      TMEM owner (both CTAs) and MMA issuer (one thread of the leader CTA): per group of four
+//               128-K blocks it copies the group's scale factors shared -> TMEM (tcgen05.cp); per 128-K
+//               block it issues four tcgen05.mma kind::mxf8f6f4 (K = 32 each) into one of two TMEM
+//               accumulators (BN fp32 columns).
+//   warp 2      scale-factor packer, one group of four 128-K blocks at a time: prefetches the groups' fp32
+//               SFA [4 x 128] by TMA into its own ring (RAW_SLOTS groups ahead), turns the power-of-two
+//               scales into UE8M0 bytes (the fp32 exponent field) and packs the four K blocks' bytes of a
+//               row into one 32-bit word in the layout tcgen05.cp / the block-scaled MMA read.  The MMAs of
+//               K block kb select byte kb % 4 through the scale-factor ids of the instruction descriptor,
+//               for all four 32-wide K sub-blocks, so the per-32 scaling of the MMA applies the 1x128 /
+//               128x128 recipe exactly and the per-K-block promotion happens inside the tensor core.  SFB
+//               rows of the tile are kept in registers, prefetched one tile ahead.
+//   warps 4..7  epilogue: TMEM -> registers -> bf16 (RNE) -> global, only for rows the GEMM owns, while the
+//               MMA already fills the other accumulator with the next tile.
+//
+// Tile scheduler (every role walks the same sequence): windows of 128*CTAS rows x BN columns, N fastest,
+// handed round-robin to the persistent CTAs (pairs).
+//   dense       ceil(M / 128*CTAS) windows.
+//   contiguous  CTAS = 1: M_total/128 blocks, group = m_indices[first row], -1 skips the block.
+//               CTAS = 2: 256-row windows over the 128-aligned segments; a window whose two halves belong to
+//               different groups becomes two tiles (one per group, each storing only its own rows).  The
+//               window table (tiles per window, prefix) is built on the device at kernel start.
+//   masked      per group ceil(masked_m[g] / 128*CTAS) windows, counted on the device, so the host never
+//               needs masked_m.
 //
 // Every mbarrier wait is bounded: after WAIT_LIMIT_NS the waiting thread raises a CTA-wide abort flag and
-// records ERR_TIMEOUT in the device error word; all roles then leave their loops, the MMA warp waits (again
-// bounded) for its tensor-core work to drain, and TMEM is freed before the CTA exits.
+// records ERR_TIMEOUT in the device error word; every role then leaves its loop, the producer waits (bounded)
+// for its loads in flight, the MMA thread waits (bounded) for its tensor-core work, and TMEM is released.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -38,12 +51,16 @@ namespace dg {
 
 enum : int { MODE_DENSE = 0, MODE_CONTIGUOUS = 1, MODE_MASKED = 2 };
 
-constexpr int BLOCK_M = 128;
+constexpr int BLOCK_M = 128;  // rows per CTA
 constexpr int BLOCK_K = 128;  // = the scale block along K
 constexpr int MMA_K = 32;     // K of one kind::mxf8f6f4 MMA
 constexpr int NUM_THREADS = 256;
 constexpr int MAX_MASKED_GROUPS = 1024;
-constexpr int SFB_KB_REGS = 4;  // K blocks of SFB held per lane: K <= 32 * 4 * 128 = 16384 on the fast path
+constexpr int MAX_PAIR_WINDOWS = 4096;  // contiguous layout with CTA pairs: M_total <= 4096 * 256
+constexpr int SFB_KB_REGS = 4;          // K blocks of SFB held per lane: K <= 32 * 4 * 128 = 16384 fast path
+constexpr int SF_GROUP = 4;             // 128-K blocks whose scales share one 32-bit word (one byte each)
+constexpr int SF_SLOTS = 3;             // packed scale groups in flight (shared memory and TMEM slots)
+constexpr int RAW_SLOTS = 4;            // fp32 SFA groups the scale-factor warp prefetches ahead
 constexpr int TMEM_COLS = 512;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s for any single wait
 constexpr int SMEM_LIMIT = 232448;                  // 227 KB of dynamic shared memory per CTA
@@ -56,7 +73,7 @@ struct GemmParams {
     int mode;
     int M;             // dense: M; contiguous: M_total; masked: M_max
     int N, K, G;
-    int num_m_blocks;  // dense / contiguous: total; masked: per group (ceil(M_max/128))
+    int num_windows;   // dense / contiguous(single): total; masked: per group; contiguous(pair): windows
     int num_n_blocks;
     int sfa_ld;        // sfa floats per K block (the MN-major row extent)
     const float *sfa;
@@ -67,36 +84,51 @@ struct GemmParams {
     unsigned *err;
 };
 
-template <int BN_, int STAGES_>
+template <int BN_, int CTAS_, int KPS_>
 struct Cfg {
     static constexpr int BN = BN_;
-    static constexpr int STAGES = STAGES_;
+    static constexpr int CTAS = CTAS_;
+    static constexpr int KPS = KPS_;                              // 128-K blocks per pipeline stage
+    static constexpr int TILE_M = BLOCK_M * CTAS;
+    static constexpr int B_ROWS = BN / CTAS;                      // B rows this CTA loads
     static constexpr int SFB_ATOMS = (BN + 127) / 128;            // 128-row scale atoms covering BN rows
-    static constexpr int A_BYTES = BLOCK_M * BLOCK_K;             // e4m3: 1 byte per element
-    static constexpr int B_BYTES = BN * BLOCK_K;
-    static constexpr int SF_WORDS = 128 + 128 * SFB_ATOMS;        // 32-bit words per stage (SFA, then SFB)
-    static constexpr int SFA_RAW_BYTES = BLOCK_M * 4;             // fp32 SFA slice of a stage, by TMA
-    static constexpr int SF_COLS = 4 + 4 * SFB_ATOMS;             // TMEM columns per stage's scales
+    static constexpr int A_BYTES1 = BLOCK_M * BLOCK_K;            // one K block of A (e4m3: 1 byte each)
+    static constexpr int B_BYTES1 = B_ROWS * BLOCK_K;             // one K block of this CTA's B rows
+    static constexpr int A_BYTES = KPS * A_BYTES1;                // per stage
+    static constexpr int B_BYTES = KPS * B_BYTES1;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int SF_WORDS = 128 + 128 * SFB_ATOMS;        // packed 32-bit words per slot (SFA, then SFB)
+    static constexpr int SFA_RAW_BYTES = SF_GROUP * TILE_M * 4;   // fp32 SFA [4 K blocks][TILE_M rows], by TMA
+    static constexpr int SF_COLS = 4 + 4 * SFB_ATOMS;             // TMEM columns per slot
     static constexpr int SF_TMEM_BASE = 2 * BN;                   // after the two accumulators
-    static constexpr int NUM_BARRIERS = 3 * STAGES + 5;
+    static constexpr int TABLE_INTS = (CTAS == 2 ? MAX_PAIR_WINDOWS : MAX_MASKED_GROUPS) + 1;
+    static constexpr int FIXED_BYTES = SF_SLOTS * SF_WORDS * 4 + RAW_SLOTS * SFA_RAW_BYTES + 8 * (2 * SF_SLOTS + RAW_SLOTS + 5) + 16 +
+                                       4 * TABLE_INTS + 4 * MAX_MASKED_GROUPS + 1024 + 8 * 2 * 8;
+    static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+    static constexpr int NUM_BARRIERS = 2 * STAGES + 2 * SF_SLOTS + RAW_SLOTS + 5;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;
-    static constexpr int OFF_SFA_RAW = OFF_SF + STAGES * SF_WORDS * 4;
-    static constexpr int OFF_BAR = OFF_SFA_RAW + STAGES * SFA_RAW_BYTES;
+    static constexpr int OFF_SFA_RAW = OFF_SF + SF_SLOTS * SF_WORDS * 4;
+    static constexpr int OFF_BAR = OFF_SFA_RAW + RAW_SLOTS * SFA_RAW_BYTES;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARRIERS * 8;   // tmem base, abort flag
-    static constexpr int OFF_PREFIX = OFF_MISC + 16;               // masked: int[G+1] block prefix
-    static constexpr int OFF_MM = OFF_PREFIX + 4 * (MAX_MASKED_GROUPS + 1);  // masked: clamped masked_m
+    static constexpr int OFF_PREFIX = OFF_MISC + 16;               // int[TABLE_INTS]
+    static constexpr int OFF_MM = OFF_PREFIX + 4 * TABLE_INTS;     // masked: clamped masked_m
     static constexpr int SMEM_BYTES = OFF_MM + 4 * MAX_MASKED_GROUPS + 1024;  // + alignment slack
+    static_assert(CTAS == 1 || CTAS == 2, "single CTA or CTA pair");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32, 256]");
-    static_assert(SF_TMEM_BASE + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
+    static_assert(B_ROWS % 8 == 0, "B tile rows must fill whole 8-row swizzle atoms");
+    static_assert(STAGES >= 3, "pipeline too shallow");
+    static_assert(SF_TMEM_BASE + SF_SLOTS * SF_COLS <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
-    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+    static_assert(A_BYTES1 % 1024 == 0 && B_BYTES1 % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+    static_assert(SF_GROUP % KPS == 0, "a stage must not straddle a scale group");
 };
 
 struct Tile {
-    int row0;        // first row in A / D (flattened [rows, K] / [rows, N])
-    int local_row0;  // first row inside its group (masked) or = row0
+    int row0;        // first row of the window in A / D (flattened [rows, K] / [rows, N])
+    int local_row0;  // first row of the window inside its group (masked) or = row0
     int n0;
     int g;
 };
@@ -113,8 +145,8 @@ __device__ __forceinline__ void raise_error(unsigned *err, unsigned code) { atom
 __device__ __noinline__ bool wait_bounded_slow(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 15u) == 0) {
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+        if ((it & 3u) == 0) {
             if (*abort) return false;
             if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
                 *abort = 1;
@@ -131,7 +163,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
 }
 
 // Whole-warp wait: lane 0 waits, the verdict is broadcast, and the warp leaves converged (the callers
-// follow with .sync.aligned tcgen05 instructions or shared-memory writes guarded by the barrier).
+// follow with .sync.aligned tcgen05 instructions or shared-memory accesses guarded by the barrier).
 __device__ __forceinline__ bool warp_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort,
                                                   unsigned *err, int lane) {
     int ok = 1;
@@ -141,42 +173,104 @@ __device__ __forceinline__ bool warp_wait_bounded(uint64_t *bar, uint32_t parity
     return ok != 0;
 }
 
-template <int BN>
+__device__ __forceinline__ int group_of_block(const GemmParams &p, int block) {
+    const int row = block * BLOCK_M;
+    if (row >= p.M) return -1;
+    const int g = __ldg(p.m_indices + row);
+    if (g >= p.G) {
+        raise_error(p.err, ERR_BAD_GROUP);
+        return -1;
+    }
+    return g < 0 ? -1 : g;
+}
+
+// largest i in [0, n) with table[i] <= v, given table[0] <= v < table[n]
+__device__ __forceinline__ int upper_index(const int *table, int n, int v) {
+    int lo = 0, hi = n;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (table[mid] <= v) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+template <class C>
 __device__ __forceinline__ bool decode_tile(const GemmParams &p, const SharedCtl &ctl, int t, Tile &ti) {
-    const int mb_lin = t / p.num_n_blocks;
-    const int nb = t - mb_lin * p.num_n_blocks;
-    ti.n0 = nb * BN;
+    const int w = t / p.num_n_blocks;  // window-tile index
+    const int nb = t - w * p.num_n_blocks;
+    ti.n0 = nb * C::BN;
     if (p.mode == MODE_DENSE) {
         ti.g = 0;
-        ti.row0 = ti.local_row0 = mb_lin * BLOCK_M;
+        ti.row0 = ti.local_row0 = w * C::TILE_M;
         return true;
     }
     if (p.mode == MODE_CONTIGUOUS) {
-        ti.row0 = ti.local_row0 = mb_lin * BLOCK_M;
-        const int g = __ldg(p.m_indices + ti.row0);
-        if (g < 0) return false;
-        if (g >= p.G) {
-            raise_error(p.err, ERR_BAD_GROUP);
-            return false;
+        if constexpr (C::CTAS == 1) {
+            ti.row0 = ti.local_row0 = w * BLOCK_M;
+            ti.g = group_of_block(p, w);
+            return ti.g >= 0;
+        } else {
+            const int j = upper_index(ctl.prefix, p.num_windows, w);
+            const int k = w - ctl.prefix[j];
+            const int ga = group_of_block(p, 2 * j), gb = group_of_block(p, 2 * j + 1);
+            ti.row0 = ti.local_row0 = j * C::TILE_M;
+            ti.g = (k == 0 && ga >= 0) ? ga : gb;
+            return ti.g >= 0;
         }
-        ti.g = g;
-        return true;
     }
-    // masked: largest g with prefix[g] <= mb_lin (prefix[G] > mb_lin by construction)
-    int lo = 0, hi = p.G;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (ctl.prefix[mid] <= mb_lin) lo = mid; else hi = mid;
-    }
-    ti.g = lo;
-    ti.local_row0 = (mb_lin - ctl.prefix[lo]) * BLOCK_M;
-    ti.row0 = lo * p.M + ti.local_row0;
+    const int g = upper_index(ctl.prefix, p.G, w);
+    ti.g = g;
+    ti.local_row0 = (w - ctl.prefix[g]) * C::TILE_M;
+    ti.row0 = g * p.M + ti.local_row0;
     return true;
 }
 
-__device__ __forceinline__ uint32_t ue8m0_x4(float s) {
-    // the biased exponent of a power-of-two fp32 is its UE8M0 code; repeat it in all four byte slots
-    return ((__float_as_uint(s) >> 23) & 0xFFu) * 0x01010101u;
+__device__ __forceinline__ uint32_t ue8m0(float s) {
+    // the biased exponent of a power-of-two fp32 is its UE8M0 code
+    return (__float_as_uint(s) >> 23) & 0xFFu;
+}
+
+// Builds the scheduler table in shared memory (one warp).
+//   masked: mm[g] = clamp(masked_m[g]); prefix[g] = sum_{h<g} ceil(mm[h] / TILE_M); prefix[G] = total.
+//   contiguous, CTA pair: prefix[j] = tiles in windows before j (a window holds 0, 1 or 2 tiles).
+template <class C>
+__device__ void build_schedule_table(const GemmParams &p, int *prefix, int *mm, int lane) {
+    const bool masked = p.mode == MODE_MASKED;
+    const int n = masked ? p.G : p.num_windows;
+    const int chunk = (n + 31) / 32;
+    const int begin = min(lane * chunk, n), end = min(begin + chunk, n);
+    auto count = [&](int i) {
+        if (masked) {
+            int m = __ldg(p.masked_m + i);
+            if (m < 0 || m > p.M) {
+                raise_error(p.err, ERR_BAD_GROUP);
+                m = m < 0 ? 0 : p.M;
+            }
+            mm[i] = m;
+            return (m + C::TILE_M - 1) / C::TILE_M;
+        }
+        const int ga = group_of_block(p, 2 * i), gb = group_of_block(p, 2 * i + 1);
+        return (ga >= 0 ? 1 : 0) + (gb >= 0 && gb != ga ? 1 : 0);
+    };
+    int local = 0;
+    for (int i = begin; i < end; ++i) {
+        const int c = count(i);
+        prefix[i] = c;  // per-entry count for now
+        local += c;
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    int run = incl - local;
+    for (int i = begin; i < end; ++i) {
+        const int c = prefix[i];
+        prefix[i] = run;
+        run += c;
+    }
+    if (lane == 31) prefix[n] = incl;
 }
 
 template <class C>
@@ -185,6 +279,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const __grid_constant__ CUtensorMap tmap_sfa, const GemmParams p) {
     constexpr int BN = C::BN;
     constexpr int STAGES = C::STAGES;
+    constexpr int CTAS = C::CTAS;
+    constexpr bool PAIR = CTAS == 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem + C::OFF_A;
@@ -192,12 +288,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t *sSF = reinterpret_cast<uint32_t *>(smem + C::OFF_SF);
     float *sSFA_raw = reinterpret_cast<float *>(smem + C::OFF_SFA_RAW);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *full_tma = bars;
-    uint64_t *full_sf = bars + STAGES;
-    uint64_t *empty = bars + 2 * STAGES;
-    uint64_t *tmem_full = bars + 3 * STAGES;   // [2]
-    uint64_t *tmem_empty = tmem_full + 2;      // [2]
-    uint64_t *drain = tmem_empty + 2;          // [1]
+    uint64_t *full = bars;                       // [STAGES] A + B landed (the leader's counts both CTAs' bytes)
+    uint64_t *empty = bars + STAGES;             // [STAGES] MMAs done with the stage (both CTAs, by commit)
+    uint64_t *raw_full = bars + 2 * STAGES;      // [RAW_SLOTS] this CTA's fp32 SFA group landed
+    uint64_t *sf_full = raw_full + RAW_SLOTS;    // [SF_SLOTS] packed scales of the whole tile ready
+    uint64_t *sf_empty = sf_full + SF_SLOTS;     // [SF_SLOTS] MMAs done with the slot (both CTAs, by commit)
+    uint64_t *tmem_full = sf_empty + SF_SLOTS;   // [2]
+    uint64_t *tmem_empty = tmem_full + 2;        // [2] (the leader's counts the epilogue warps of both CTAs)
+    uint64_t *drain = tmem_empty + 2;            // [1]
     uint32_t *s_tmem_base = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     int *s_prefix = reinterpret_cast<int *>(smem + C::OFF_PREFIX);
@@ -205,16 +303,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = PAIR ? cluster_cta_rank() : 0u;
+    const int cluster_id = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int num_clusters = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full_tma[s], 1);
-            mbar_init(&full_sf[s], 1);
+            mbar_init(&full[s], 1);  // the leader's producer arms it with both CTAs' bytes
             mbar_init(&empty[s], 1);
         }
+        for (int j = 0; j < SF_SLOTS; ++j) {
+            mbar_init(&sf_full[j], 1);
+            mbar_init(&sf_empty[j], 1);
+        }
+        for (int j = 0; j < RAW_SLOTS; ++j) mbar_init(&raw_full[j], 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tmem_full[i], 1);
-            mbar_init(&tmem_empty[i], 4);  // one arrival per epilogue warp
+            mbar_init(&tmem_empty[i], 4 * CTAS);  // one arrival per epilogue warp of each CTA
         }
         mbar_init(drain, 1);
         *s_abort = 0;
@@ -225,44 +330,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tma_prefetch_desc(&tmap_sfa);
     }
     if (warp == 1) {
-        tmem_alloc(s_tmem_base, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc<CTAS>(s_tmem_base, TMEM_COLS);
+        tmem_relinquish<CTAS>();
     }
-    if (warp == 2 && p.mode == MODE_MASKED) {
-        // per-group M-block counts and their exclusive prefix; lane l owns groups [l*chunk, (l+1)*chunk)
-        const int chunk = (p.G + 31) / 32;
-        const int g_begin = min(lane * chunk, p.G), g_end = min(g_begin + chunk, p.G);
-        int local = 0;
-        for (int g = g_begin; g < g_end; ++g) {
-            int m = __ldg(p.masked_m + g);
-            if (m < 0 || m > p.M) {
-                raise_error(p.err, ERR_BAD_GROUP);
-                m = m < 0 ? 0 : p.M;
-            }
-            s_mm[g] = m;
-            local += (m + BLOCK_M - 1) / BLOCK_M;
-        }
-        int incl = local;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += v;
-        }
-        int run = incl - local;
-        for (int g = g_begin; g < g_end; ++g) {
-            s_prefix[g] = run;
-            run += (s_mm[g] + BLOCK_M - 1) / BLOCK_M;
-        }
-        if (lane == 31) s_prefix[p.G] = incl;
-    }
+    if (warp == 2 && (p.mode == MODE_MASKED || (PAIR && p.mode == MODE_CONTIGUOUS)))
+        build_schedule_table<C>(p, s_prefix, s_mm, lane);
     tc_fence_before_sync();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();  // the peer's barriers exist before any cross-CTA signal
     tc_fence_after_sync();
     const uint32_t tmem_base = *s_tmem_base;
 
     const SharedCtl ctl{s_abort, s_prefix, s_mm};
     const int nkb = p.K / BLOCK_K;
-    const int total_tiles = (p.mode == MODE_MASKED ? s_prefix[p.G] : p.num_m_blocks) * p.num_n_blocks;
+    int total_windows;
+    if (p.mode == MODE_MASKED)
+        total_windows = s_prefix[p.G];
+    else if (PAIR && p.mode == MODE_CONTIGUOUS)
+        total_windows = s_prefix[p.num_windows];
+    else
+        total_windows = p.num_windows;
+    const int total_tiles = total_windows * p.num_n_blocks;
+    const int my_rows = BLOCK_M * static_cast<int>(rank);  // offset of this CTA's rows inside the window
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
@@ -271,91 +360,169 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t ph = 0;
             uint32_t armed = 0, armed_ph = 0;  // stages armed at least once / parity of their last arming
             bool ok = true;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            for (int t = cluster_id; t < total_tiles && ok; t += num_clusters) {
                 Tile ti;
-                if (!decode_tile<BN>(p, ctl, t, ti)) continue;
-                const int brow = ti.g * p.N + ti.n0;
-                const int sfa_row = p.mode == MODE_MASKED ? ti.g * nkb : 0;
-                for (int kb = 0; kb < nkb; ++kb) {
+                if (!decode_tile<C>(p, ctl, t, ti)) continue;
+                const int arow = ti.row0 + my_rows;
+                const int brow = ti.g * p.N + ti.n0 + static_cast<int>(rank) * C::B_ROWS;
+                for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
+                    const int nk = min(C::KPS, nkb - kb0);  // K blocks in this stage
                     if (!wait_bounded(&empty[s], ph ^ 1u, s_abort, p.err)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&full_tma[s], C::A_BYTES + C::B_BYTES + C::SFA_RAW_BYTES);
-                    tma_load_2d(sA + s * C::A_BYTES, &tmap_a, &full_tma[s], kb * BLOCK_K, ti.row0);
-                    tma_load_2d(sB + s * C::B_BYTES, &tmap_b, &full_tma[s], kb * BLOCK_K, brow);
-                    tma_load_2d(sSFA_raw + s * BLOCK_M, &tmap_sfa, &full_tma[s], ti.local_row0, sfa_row + kb);
+                    uint8_t *a_dst = sA + s * C::A_BYTES;
+                    uint8_t *b_dst = sB + s * C::B_BYTES;
+                    const uint32_t bytes = static_cast<uint32_t>(nk * (C::A_BYTES1 + C::B_BYTES1));
+                    if constexpr (PAIR) {
+                        // Only the leader arrives (with both CTAs' bytes); the peer's loads just count their
+                        // bytes on the leader's barrier.  A peer load may land before the leader arms the
+                        // phase: the transaction count dips below zero but the phase cannot complete before
+                        // the leader's arrival.  (No cross-CTA release in this loop: it would wait for this
+                        // thread's loads in flight.)
+                        const uint32_t leader_full = map_shared_rank(smem_u32(&full[s]), 0);
+                        if (rank == 0) mbar_arrive_expect_tx(&full[s], CTAS * bytes);
+                        for (int i = 0; i < nk; ++i) {
+                            tma_load_2d_pair(a_dst + i * C::A_BYTES1, &tmap_a, leader_full, (kb0 + i) * BLOCK_K, arow);
+                            tma_load_2d_pair(b_dst + i * C::B_BYTES1, &tmap_b, leader_full, (kb0 + i) * BLOCK_K, brow);
+                        }
+                    } else {
+                        mbar_arrive_expect_tx(&full[s], bytes);
+                        for (int i = 0; i < nk; ++i) {
+                            tma_load_2d(a_dst + i * C::A_BYTES1, &tmap_a, &full[s], (kb0 + i) * BLOCK_K, arow);
+                            tma_load_2d(b_dst + i * C::B_BYTES1, &tmap_b, &full[s], (kb0 + i) * BLOCK_K, brow);
+                        }
+                    }
                     armed |= 1u << s;
                     armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
             }
             if (!ok) {
-                // let every load still in flight land before the CTA's shared memory goes away
+                // let the loads still in flight land before shared memory goes away (in a pair the A/B
+                // bytes of both CTAs are counted on the leader's barrier)
                 for (int i = 0; i < STAGES; ++i) {
                     if (!(armed >> i & 1u)) continue;
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(&full_tma[i], (armed_ph >> i) & 1u) &&
-                           global_timer_ns() - t0 < WAIT_LIMIT_NS) {
+                    if (!PAIR || rank == 0) {
+                        const uint64_t t1 = global_timer_ns();
+                        while (!mbar_try_wait(&full[i], (armed_ph >> i) & 1u) &&
+                               global_timer_ns() - t1 < WAIT_LIMIT_NS) {
+                        }
                     }
                 }
             }
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t IDESC = idesc_mxf8_e4m3(BLOCK_M, BN);
+        // ---------------------------------------------------------------- MMA issuer (leader CTA)
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t IDESC = idesc_mxf8_e4m3(C::TILE_M, BN);
             int s = 0;
             uint32_t ph = 0;
+            int slot = 0;
+            uint32_t slot_ph = 0;
             int acc = 0;
             uint32_t acc_ph = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            for (int t = cluster_id; t < total_tiles && ok; t += num_clusters) {
                 Tile ti;
-                if (!decode_tile<BN>(p, ctl, t, ti)) continue;
+                if (!decode_tile<C>(p, ctl, t, ti)) continue;
                 if (!wait_bounded(&tmem_empty[acc], acc_ph ^ 1u, s_abort, p.err)) break;
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!wait_bounded(&full_tma[s], ph, s_abort, p.err) ||
-                        !wait_bounded(&full_sf[s], ph, s_abort, p.err)) {
-                        ok = false;
-                        break;
+                uint32_t sf_tmem = 0;
+                for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
+                    const int nk = min(C::KPS, nkb - kb0);
+                    if (kb0 % SF_GROUP == 0) {
+                        if (!wait_bounded(&sf_full[slot], slot_ph, s_abort, p.err)) { ok = false; break; }
+                        tc_fence_after_sync();
+                        sf_tmem = tmem_base + static_cast<uint32_t>(C::SF_TMEM_BASE + slot * C::SF_COLS);
+                        const uint32_t sf_smem = smem_u32(sSF + slot * C::SF_WORDS);
+                        tc_cp_32x128b_warpx4<CTAS>(sf_tmem, sdesc_rows16_noswizzle(sf_smem));
+#pragma unroll
+                        for (int a = 0; a < C::SFB_ATOMS; ++a)
+                            tc_cp_32x128b_warpx4<CTAS>(sf_tmem + 4 + 4 * a,
+                                                       sdesc_rows16_noswizzle(sf_smem + 512 + 512 * a));
                     }
+                    if (!wait_bounded(&full[s], ph, s_abort, p.err)) { ok = false; break; }
                     tc_fence_after_sync();
-                    const uint32_t sf_tmem = tmem_base + static_cast<uint32_t>(C::SF_TMEM_BASE + s * C::SF_COLS);
-                    const uint32_t sf_smem = smem_u32(sSF + s * C::SF_WORDS);
-                    tc_cp_32x128b_warpx4(sf_tmem, sdesc_rows16_noswizzle(sf_smem));
+                    const uint32_t a_stage = smem_u32(sA + s * C::A_BYTES);
+                    const uint32_t b_stage = smem_u32(sB + s * C::B_BYTES);
+                    for (int i = 0; i < nk; ++i) {
+                        const int kb = kb0 + i;
+                        const uint32_t sub = static_cast<uint32_t>(kb % SF_GROUP);  // byte of the packed scales
+                        const uint32_t idesc = IDESC | (sub << 29) | (sub << 4);
+                        const uint32_t a_base = a_stage + i * C::A_BYTES1;
+                        const uint32_t b_base = b_stage + i * C::B_BYTES1;
 #pragma unroll
-                    for (int a = 0; a < C::SFB_ATOMS; ++a)
-                        tc_cp_32x128b_warpx4(sf_tmem + 4 + 4 * a, sdesc_rows16_noswizzle(sf_smem + 512 + 512 * a));
-                    const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
-                    const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
-#pragma unroll
-                    for (int k = 0; k < BLOCK_K / MMA_K; ++k) {
-                        tc_mma_mxf8(d_tmem, sdesc_kmajor_sw128(a_base + k * MMA_K), sdesc_kmajor_sw128(b_base + k * MMA_K),
-                                    IDESC, sf_tmem, sf_tmem + 4, (kb | k) != 0);
+                        for (int k = 0; k < BLOCK_K / MMA_K; ++k) {
+                            tc_mma_mxf8<CTAS>(d_tmem, sdesc_kmajor_sw128(a_base + k * MMA_K),
+                                              sdesc_kmajor_sw128(b_base + k * MMA_K), idesc, sf_tmem, sf_tmem + 4,
+                                              (kb | k) != 0);
+                        }
                     }
-                    tc_commit(&empty[s]);
+                    tc_commit<CTAS>(&empty[s]);
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
+                    const int last = kb0 + nk - 1;
+                    if (last % SF_GROUP == SF_GROUP - 1 || last == nkb - 1) {
+                        tc_commit<CTAS>(&sf_empty[slot]);
+                        if (++slot == SF_SLOTS) { slot = 0; slot_ph ^= 1u; }
+                    }
                 }
                 if (!ok) break;
-                tc_commit(&tmem_full[acc]);
+                tc_commit<CTAS>(&tmem_full[acc]);
                 acc ^= 1;
                 if (acc == 0) acc_ph ^= 1u;
             }
-            // all tensor-core work of this CTA must be complete before TMEM is released
-            tc_commit(drain);
+            // all tensor-core work of the pair must be complete before TMEM is released
+            tc_commit<CTAS>(drain);
             const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < WAIT_LIMIT_NS) {
             }
         }
-    } else if (warp == 2) {
-        // ---------------------------------------------------------------- scale-factor packer
-        // SFA arrives with the stage (fp32 slice by TMA).  SFB: the tile's <= 3 scale rows x K blocks are
-        // held in registers (lane l holds K blocks l, l+32, ...), loaded one tile ahead so the global
-        // latency hides behind the current tile.
-        int s = 0;
-        uint32_t ph = 0;
+    } else if (warp == 2 && rank == 0) {
+        // ---------------------------------------------------------------- scale-factor packer (leader CTA)
+        // In a pair the leader packs the scales of both CTAs' rows and stores the peer's words straight into
+        // the peer's shared memory (same offsets), so the MMA thread waits on one local barrier.
+        // Two cursors walk this CTA's (tile, group-of-4-K-blocks) sequence: the prefetch cursor keeps up to
+        // RAW_SLOTS groups of fp32 SFA in flight (TMA into this warp's own ring, which depends on nothing but
+        // this warp's progress), the consume cursor packs one group at a time into a slot the MMAs released.
         const int nnb128 = (p.N + 127) / 128;
         const bool sfb_in_regs = nkb <= 32 * SFB_KB_REGS;
+        const uint32_t sf_peer0 = PAIR ? map_shared_rank(smem_u32(sSF), 1) : 0u;  // the peer's packed words
+        auto next_valid = [&](int &t, Tile &ti) {
+            for (; t < total_tiles; t += num_clusters)
+                if (decode_tile<C>(p, ctl, t, ti)) return true;
+            return false;
+        };
+        struct Cursor {
+            int t;
+            Tile ti;
+            int kb0;
+            bool have;
+        };
+        auto advance = [&](Cursor &c) {
+            c.kb0 += SF_GROUP;
+            if (c.kb0 >= nkb) {
+                c.kb0 = 0;
+                c.t += num_clusters;
+                c.have = next_valid(c.t, c.ti);
+            }
+        };
+        Cursor pf{cluster_id, Tile{}, 0, false};
+        pf.have = next_valid(pf.t, pf.ti);
+        Cursor cs = pf;
+        uint32_t issued = 0, consumed = 0;
+        auto prefetch = [&]() {
+            while (pf.have && issued - consumed < static_cast<uint32_t>(RAW_SLOTS)) {
+                if (lane == 0) {
+                    const int rs = static_cast<int>(issued % RAW_SLOTS);
+                    const int x = pf.ti.local_row0;
+                    const int y = (p.mode == MODE_MASKED ? pf.ti.g * nkb : 0) + pf.kb0;
+                    mbar_arrive_expect_tx(&raw_full[rs], C::SFA_RAW_BYTES);
+                    tma_load_2d(sSFA_raw + rs * SF_GROUP * C::TILE_M, &tmap_sfa, &raw_full[rs], x, y);
+                }
+                ++issued;
+                advance(pf);
+            }
+        };
+        // SFB of the consume cursor's tile (cur) and of the next tile (nxt), in registers
         float cur[3][SFB_KB_REGS], nxt[3][SFB_KB_REGS];
         auto load_sfb = [&](const Tile &ti, float (&v)[3][SFB_KB_REGS]) {
             const float *sfb_g = p.sfb + static_cast<size_t>(ti.g) * nnb128 * nkb;
@@ -368,87 +535,140 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     v[j][i] = (nb0 + j < nnb128 && kb < nkb) ? __ldg(sfb_g + (nb0 + j) * nkb + kb) : 1.f;
                 }
         };
-        auto next_valid = [&](int &t, Tile &ti) {
-            for (; t < total_tiles; t += gridDim.x)
-                if (decode_tile<BN>(p, ctl, t, ti)) return true;
-            return false;
-        };
-        int t = blockIdx.x;
-        Tile ti;
-        bool have = next_valid(t, ti);
-        if (have && sfb_in_regs) load_sfb(ti, cur);
+        int t_next = cs.t + num_clusters;
+        Tile ti_next;
+        bool have_next = cs.have && next_valid(t_next, ti_next);
+        if (cs.have && sfb_in_regs) load_sfb(cs.ti, cur);
+        if (have_next && sfb_in_regs) load_sfb(ti_next, nxt);
+        int slot = 0;
+        uint32_t slot_ph = 0;
         bool ok = true;
-        while (have && ok) {
-            int t2 = t + gridDim.x;
-            Tile tn;
-            const bool have2 = next_valid(t2, tn);
-            if (have2 && sfb_in_regs) load_sfb(tn, nxt);
-            const float *sfb_g = p.sfb + static_cast<size_t>(ti.g) * nnb128 * nkb;
+        while (cs.have) {
+            prefetch();
+            const Tile &ti = cs.ti;
+            const int kb0 = cs.kb0;
             const int nb0 = ti.n0 >> 7;
-            for (int kb = 0; kb < nkb; ++kb) {
-                float sb[3];
-                if (sfb_in_regs) {
-                    const int reg = kb >> 5, src = kb & 31;
+            // packed SFB word of each of the tile's (up to) three 128-row scale blocks
+            const float *sfb_g = p.sfb + static_cast<size_t>(ti.g) * nnb128 * nkb;
+            uint32_t wb[3];
 #pragma unroll
-                    for (int j = 0; j < 3; ++j) {
+            for (int j = 0; j < 3; ++j) {
+                uint32_t word = 0;
+#pragma unroll
+                for (int i = 0; i < SF_GROUP; ++i) {
+                    const int kb = kb0 + i;
+                    float v;
+                    if (sfb_in_regs) {
+                        const int reg = kb >> 5;
                         float x = cur[j][0];
 #pragma unroll
-                        for (int i = 1; i < SFB_KB_REGS; ++i) x = reg == i ? cur[j][i] : x;
-                        sb[j] = __shfl_sync(0xffffffffu, x, src);
+                        for (int r = 1; r < SFB_KB_REGS; ++r) x = reg == r ? cur[j][r] : x;
+                        v = __shfl_sync(0xffffffffu, x, kb & 31);
+                    } else {
+                        v = (nb0 + j < nnb128 && kb < nkb) ? __ldg(sfb_g + (nb0 + j) * nkb + kb) : 1.f;
                     }
-                } else {
+                    word |= ue8m0(v) << (8 * i);
+                }
+                wb[j] = word;
+            }
+            // the group's fp32 SFA -> one packed word per row (byte i = K block kb0 + i)
+            const int rs = static_cast<int>(consumed % RAW_SLOTS);
+            if (!warp_wait_bounded(&raw_full[rs], (consumed / RAW_SLOTS) & 1u, s_abort, p.err, lane)) {
+                ok = false;
+                break;
+            }
+            const float *raw = sSFA_raw + rs * SF_GROUP * C::TILE_M;
+            uint32_t wa[CTAS][4];
+#pragma unroll
+            for (int c = 0; c < CTAS; ++c) {
+                wa[c][0] = wa[c][1] = wa[c][2] = wa[c][3] = 0u;
+#pragma unroll
+                for (int i = 0; i < SF_GROUP; ++i) {
+                    const float4 v = reinterpret_cast<const float4 *>(raw + i * C::TILE_M + c * BLOCK_M)[lane];
+                    wa[c][0] |= ue8m0(v.x) << (8 * i);
+                    wa[c][1] |= ue8m0(v.y) << (8 * i);
+                    wa[c][2] |= ue8m0(v.z) << (8 * i);
+                    wa[c][3] |= ue8m0(v.w) << (8 * i);
+                }
+            }
+            fence_proxy_async_smem();  // the raw slot's next TMA write comes after these reads
+            __syncwarp();
+            ++consumed;
+            prefetch();
+            if (!warp_wait_bounded(&sf_empty[slot], slot_ph ^ 1u, s_abort, p.err, lane)) { ok = false; break; }
+            uint32_t *w = sSF + slot * C::SF_WORDS;
+            const uint32_t w_peer = sf_peer0 + 4u * static_cast<uint32_t>(slot * C::SF_WORDS);
+            // tcgen05.cp 32x128b source: word (r % 32) * 4 + r / 32 holds row r of a 128-row atom
+            const int r0 = 4 * lane;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int idx = ((r0 + i) & 31) * 4 + ((r0 + i) >> 5);
+                w[idx] = wa[0][i];
+                if constexpr (PAIR) st_shared_cluster(w_peer + 4u * idx, wa[CTAS - 1][i]);
+            }
+#pragma unroll
+            for (int j = 0; j < C::SFB_ATOMS * 4; ++j) {
+                const int r = lane + 32 * j;                        // row inside the BN tile
+                const int which = ((ti.n0 + r) >> 7) - nb0;         // 0, 1 or 2
+                const int idx = 128 + (r >> 7) * 128 + (r & 31) * 4 + ((r >> 5) & 3);
+                const uint32_t v = which == 0 ? wb[0] : (which == 1 ? wb[1] : wb[2]);
+                w[idx] = v;
+                if constexpr (PAIR) st_shared_cluster(w_peer + 4u * idx, v);
+            }
+            if constexpr (PAIR) fence_proxy_async_all(); else fence_proxy_async_smem();
+            __syncwarp();
+            // lane 1 signals: lane 0 issues this warp's TMA loads, and a release by the thread that issued
+            // them could wait for them to land
+            if (lane == 1) {
+                if constexpr (PAIR)
+                    mbar_arrive_cluster(map_shared_rank(smem_u32(&sf_full[slot]), 0));
+                else
+                    mbar_arrive(&sf_full[slot]);
+            }
+            if (++slot == SF_SLOTS) { slot = 0; slot_ph ^= 1u; }
+            const int t_before = cs.t;
+            advance(cs);
+            if (cs.have && cs.t != t_before) {
+                // moved to the next tile: its SFB is in nxt; fetch the one after
+                if (sfb_in_regs) {
 #pragma unroll
                     for (int j = 0; j < 3; ++j)
-                        sb[j] = nb0 + j < nnb128 ? __ldg(sfb_g + (nb0 + j) * nkb + kb) : 1.f;
+#pragma unroll
+                        for (int i = 0; i < SFB_KB_REGS; ++i) cur[j][i] = nxt[j][i];
                 }
-                if (!warp_wait_bounded(&full_tma[s], ph, s_abort, p.err, lane)) { ok = false; break; }
-                const float4 va = reinterpret_cast<const float4 *>(sSFA_raw + s * BLOCK_M)[lane];
-                uint32_t *w = sSF + s * C::SF_WORDS;
-                // tcgen05.cp 32x128b source: word (r % 32) * 4 + r / 32 holds row r of a 128-row atom
-                const int r0 = 4 * lane;
-                w[((r0 + 0) & 31) * 4 + ((r0 + 0) >> 5)] = ue8m0_x4(va.x);
-                w[((r0 + 1) & 31) * 4 + ((r0 + 1) >> 5)] = ue8m0_x4(va.y);
-                w[((r0 + 2) & 31) * 4 + ((r0 + 2) >> 5)] = ue8m0_x4(va.z);
-                w[((r0 + 3) & 31) * 4 + ((r0 + 3) >> 5)] = ue8m0_x4(va.w);
-#pragma unroll
-                for (int j = 0; j < C::SFB_ATOMS * 4; ++j) {
-                    const int r = lane + 32 * j;                        // row inside the BN tile
-                    const int which = ((ti.n0 + r) >> 7) - nb0;         // 0, 1 or 2
-                    const float v = which == 0 ? sb[0] : (which == 1 ? sb[1] : sb[2]);
-                    w[128 + (r >> 7) * 128 + (r & 31) * 4 + ((r >> 5) & 3)] = ue8m0_x4(v);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&full_sf[s]);
-                if (++s == STAGES) { s = 0; ph ^= 1u; }
+                t_next = cs.t + num_clusters;
+                have_next = next_valid(t_next, ti_next);
+                if (have_next && sfb_in_regs) load_sfb(ti_next, nxt);
             }
-            if (sfb_in_regs) {
-#pragma unroll
-                for (int j = 0; j < 3; ++j)
-#pragma unroll
-                    for (int i = 0; i < SFB_KB_REGS; ++i) cur[j][i] = nxt[j][i];
-            }
-            ti = tn;
-            t = t2;
-            have = have2;
         }
+        if (!ok && lane == 0) {
+            // let this warp's loads still in flight land before shared memory goes away
+            for (uint32_t q = consumed; q != issued; ++q) {
+                const uint64_t t0 = global_timer_ns();
+                while (!mbar_try_wait(&raw_full[q % RAW_SLOTS], (q / RAW_SLOTS) & 1u) &&
+                       global_timer_ns() - t0 < WAIT_LIMIT_NS) {
+                }
+            }
+        }
+        __syncwarp();
     } else if (warp >= 4) {
         // ---------------------------------------------------------------- epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const uint32_t tmem_empty_leader0 = PAIR ? map_shared_rank(smem_u32(&tmem_empty[0]), 0) : 0u;
         int acc = 0;
         uint32_t acc_ph = 0;
-        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        for (int t = cluster_id; t < total_tiles; t += num_clusters) {
             Tile ti;
-            if (!decode_tile<BN>(p, ctl, t, ti)) continue;
+            if (!decode_tile<C>(p, ctl, t, ti)) continue;
             if (!warp_wait_bounded(&tmem_full[acc], acc_ph, s_abort, p.err, lane)) break;
             tc_fence_after_sync();
-            const int r_local = 32 * q + lane;
+            const int r_local = my_rows + 32 * q + lane;
             const int row = ti.row0 + r_local;
             bool valid;
             if (p.mode == MODE_DENSE)
                 valid = row < p.M;
             else if (p.mode == MODE_CONTIGUOUS)
-                valid = __ldg(p.m_indices + row) >= 0;
+                valid = row < p.M && __ldg(p.m_indices + row) == ti.g;
             else
                 valid = ti.local_row0 + r_local < ctl.mm[ti.g];
             __nv_bfloat16 *out = p.d + static_cast<size_t>(row) * p.N + ti.n0;
@@ -479,7 +699,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tmem_empty[acc]);
+            if (lane == 0) {
+                if constexpr (PAIR)
+                    mbar_arrive_cluster(tmem_empty_leader0 + 8u * static_cast<uint32_t>(acc));
+                else
+                    mbar_arrive(&tmem_empty[acc]);
+            }
             acc ^= 1;
             if (acc == 0) acc_ph ^= 1u;
         }
@@ -487,10 +712,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     tc_fence_before_sync();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();  // neither CTA leaves while the pair may still touch its memory
     if (warp == 1) {
         __syncwarp();
         tc_fence_after_sync();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        tmem_dealloc<CTAS>(tmem_base, TMEM_COLS);
     }
 }
 

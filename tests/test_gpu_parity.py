@@ -15,6 +15,15 @@ from _helpers import assert_close, bf16_to_f64, run_problem, untouched_rows_ok
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(params=[0, 1], ids=["single_cta", "cta_pair"])
+def policy(request):
+    import moe_grouped_gemm_03_b200 as dg
+
+    dg.set_cta_pair_policy(request.param)
+    yield request.param
+    dg.set_cta_pair_policy(-1)
+
+
 def _full_check(p):
     out = run_problem(p)
     import moe_grouped_gemm_03_b200 as dg
@@ -26,6 +35,22 @@ def _full_check(p):
     assert_close(got[valid], ref[valid], p.name)
     assert untouched_rows_ok(out, valid), "rows outside the groups were written"
     return out
+
+
+def test_pair_and_single_paths_agree():
+    """Single-CTA 128-row tiles and 2-CTA 256-row tiles give the same products (within fp32 ordering)."""
+    import moe_grouped_gemm_03_b200 as dg
+
+    p = synth.make_contiguous([300, 129, 640, 1], 1024, 1024, seed=21)
+    outs = []
+    for pol in (0, 1):
+        dg.set_cta_pair_policy(pol)
+        outs.append(run_problem(p).clone())
+    dg.set_cta_pair_policy(-1)
+    valid = np.zeros(p.rows, bool)
+    valid[p.valid_rows()] = True
+    sel = torch.from_numpy(valid).cuda()
+    assert_close(bf16_to_f64(outs[1][sel]), bf16_to_f64(outs[0][sel]), "pair vs single")
 
 
 def test_config1_dense_small():
@@ -40,7 +65,7 @@ def test_config1_dense_small():
     (1000, 2048, 1024),  # several waves of tiles
     (64, 7168, 512),     # N=7168 (224-wide tiles)
 ])
-def test_dense_shapes(M, N, K):
+def test_dense_shapes(M, N, K, policy):
     _full_check(synth.make_dense(M, N, K, seed=M + N + K))
 
 
@@ -48,8 +73,10 @@ def test_dense_shapes(M, N, K):
     ([0, 1, 127, 128, 129, 300], 512, 256),
     ([513, 7, 260], 4096, 384),
     ([1], 16, 128),
+    ([129, 1, 130, 255, 256, 257, 3], 640, 256),  # odd block counts: 256-row windows straddle groups
+    ([128] * 9, 256, 128),                        # nine one-block groups: every pair window holds two groups
 ])
-def test_contiguous_shapes(counts, N, K):
+def test_contiguous_shapes(counts, N, K, policy):
     _full_check(synth.make_contiguous(counts, N, K, seed=sum(counts) + N))
 
 
@@ -59,17 +86,17 @@ def test_contiguous_shapes(counts, N, K):
     (4, 64, 160, 128, [64, 63, 0, 1]),
     (40, 128, 384, 256, None),
 ])
-def test_masked_shapes(G, M_max, N, K, mm):
+def test_masked_shapes(G, M_max, N, K, mm, policy):
     _full_check(synth.make_masked(G, M_max, N, K, masked_m=mm, seed=G + M_max, expected_m=M_max // 2))
 
 
-def test_masked_all_groups_empty_writes_nothing():
+def test_masked_all_groups_empty_writes_nothing(policy):
     p = synth.make_masked(3, 128, 256, 256, masked_m=[0, 0, 0], seed=1)
     out = run_problem(p)
     assert untouched_rows_ok(out, np.zeros(3 * 128, bool))
 
 
-def test_row_power_of_two_scaling_is_bitwise():
+def test_row_power_of_two_scaling_is_bitwise(policy):
     """D(2^j sfa[row]) == 2^j D(sfa[row]) bit for bit (power-of-two scaling is exact in fp32 and bf16)."""
     p = synth.make_dense(256, 512, 512, seed=11)
     base = run_problem(p).clone()
@@ -81,7 +108,7 @@ def test_row_power_of_two_scaling_is_bitwise():
     assert torch.equal(got[other], base[other])
 
 
-def test_contiguous_groups_equal_dense_calls():
+def test_contiguous_groups_equal_dense_calls(policy):
     p = synth.make_contiguous([200, 77, 384], 1024, 512, seed=12)
     out = run_problem(p)
     import moe_grouped_gemm_03_b200 as dg
@@ -100,7 +127,7 @@ def test_contiguous_groups_equal_dense_calls():
         start += seg
 
 
-def test_bad_group_id_is_reported_and_skipped():
+def test_bad_group_id_is_reported_and_skipped(policy):
     import moe_grouped_gemm_03_b200 as dg
 
     p = synth.make_contiguous([128, 128], 256, 256, seed=13)
