@@ -7,10 +7,12 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
+#include <mutex>
 #include <string>
 
 #include "dg.h"
 #include "gemm_kernel.cuh"
+#include "scale_pack.cuh"
 
 namespace {
 
@@ -94,72 +96,150 @@ int make_operand_map(CUtensorMap &map, const void *base, long long rows, int K, 
     return DG_OK;
 }
 
-// MN-major fp32 scales [outer][ld] (outer = K blocks, times G for the masked layout): boxes of one tile's
-// rows (128 or 256) x four K blocks, no swizzle.
-int make_sfa_map(CUtensorMap &map, const float *base, int ld, long long outer, int box_rows) {
+// Packed scale atoms: rows of 128 32-bit words (512 bytes), boxes of `box_rows` atoms, no swizzle.
+int make_atom_map(CUtensorMap &map, const uint32_t *base, long long atoms, int box_rows) {
     EncodeTiledFn encode;
     if (int rc = get_encode_fn(encode)) return rc;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(ld), static_cast<cuuint64_t>(outer)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(dg::SF_GROUP)};
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(dg::SF_ATOM_WORDS), static_cast<cuuint64_t>(atoms)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(dg::SF_ATOM_WORDS) * 4};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(dg::SF_ATOM_WORDS), static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box, estr,
+    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", static_cast<int>(r));
     return DG_OK;
 }
 
+// Stream-ordered scratch for the packed scales, from a pool this library owns (one per device) that keeps
+// freed memory for reuse, so steady-state calls do not reach the driver's allocator.
+int scratch_pool(int device, cudaMemPool_t &pool) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (device < 0 || device >= 64) return fail(DG_ERR_UNSUPPORTED, "device index %d out of range", device);
+    if (!pools[device]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = device;
+        cudaError_t e = cudaMemPoolCreate(&pools[device], &props);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemPoolCreate");
+        uint64_t keep = ~0ull;
+        cudaMemPoolSetAttribute(pools[device], cudaMemPoolAttrReleaseThreshold, &keep);
+    }
+    pool = pools[device];
+    return DG_OK;
+}
+
 // ----------------------------------------------------------------------------------------------- launch
 int g_pair_policy = -1;  // -1: library decides; 0: single CTAs only; 1: CTA pairs whenever supported
 
+struct ScaleArgs {
+    const float *sfa;
+    int sfa_ld;
+    const float *sfb;
+};
+
 template <int BN, int CTAS, int KPS>
-int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows, dg::GemmParams p, int grid,
-               cudaStream_t stream) {
+int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows, const ScaleArgs &sc, dg::GemmParams p,
+               int grid, int device, cudaStream_t stream) {
     using C = dg::Cfg<BN, CTAS, KPS>;
-    CUtensorMap ta, tb, tsfa;
-    if (int rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M)) return rc;
-    if (int rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS)) return rc;
-    const long long sfa_rows = static_cast<long long>(p.K / dg::BLOCK_K) * (p.mode == dg::MODE_MASKED ? p.G : 1);
-    if (int rc = make_sfa_map(tsfa, p.sfa, p.sfa_ld, sfa_rows, C::TILE_M)) return rc;
-    auto kernel = dg::fp8_gemm_kernel<C>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(grid * CTAS), 1, 1);
-    cfg.blockDim = dim3(dg::NUM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CTAS;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (CTAS > 1) {
-        // a persistent grid larger than the co-resident clusters would only queue behind itself
-        static int max_clusters[64] = {0};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        int &cached = max_clusters[dev & 63];
-        if (cached == 0) {
-            int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
-                cudaGetLastError();
-                n = grid;
-            }
-            cached = n;
-        }
-        if (grid > cached) cfg.gridDim.x = static_cast<unsigned>(cached * CTAS);
+    // ---- packed scale atoms (pre-pass)
+    const int nkb = p.K / dg::BLOCK_K;
+    dg::PackParams pk{};
+    pk.sfa = sc.sfa;
+    pk.sfa_ld = sc.sfa_ld;
+    pk.sfb = sc.sfb;
+    pk.N = p.N;
+    pk.G = p.G;
+    pk.bn = BN;
+    pk.n_tiles = p.num_n_blocks;
+    pk.sfb_atoms = C::SFB_ATOMS;
+    pk.nkb = nkb;
+    pk.num_sf_groups = p.num_sf_groups;
+    if (p.mode == dg::MODE_MASKED) {
+        pk.rows_per_group = p.M;
+        pk.blocks_per_group = p.sfa_blocks;
+        pk.sfa_groups = p.G;
+    } else {
+        pk.rows_per_group = p.M;
+        pk.blocks_per_group = (p.M + dg::BLOCK_M - 1) / dg::BLOCK_M;
+        pk.sfa_groups = 1;
     }
-    static const bool debug = getenv("DG_DEBUG") && getenv("DG_DEBUG")[0] == '1';
-    if (debug)
-        fprintf(stderr, "[dg] mode=%d M=%d N=%d K=%d G=%d BN=%d stages=%d x %d ctas=%d grid=%u smem=%d windows=%d\n", p.mode,
-                p.M, p.N, p.K, p.G, BN, C::STAGES, KPS, CTAS, cfg.gridDim.x, C::SMEM_BYTES, p.num_windows);
-    e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, p);
-    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
-    return DG_OK;
+    const long long sfa_atoms = static_cast<long long>(pk.sfa_groups) * pk.blocks_per_group * p.num_sf_groups;
+    const long long sfb_atoms = static_cast<long long>(p.G) * p.num_n_blocks * p.num_sf_groups * C::SFB_ATOMS;
+    pk.sfa_words = sfa_atoms * dg::SF_ATOM_WORDS;
+    pk.sfb_words = sfb_atoms * dg::SF_ATOM_WORDS;
+    cudaMemPool_t pool;
+    if (int rc = scratch_pool(device, pool)) return rc;
+    void *scratch = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(&scratch, static_cast<size_t>(pk.sfa_words + pk.sfb_words) * 4, pool, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync (packed scales)");
+    pk.sfa_out = static_cast<uint32_t *>(scratch);
+    pk.sfb_out = pk.sfa_out + pk.sfa_words;
+    int rc = DG_OK;
+    do {
+        const long long total = pk.sfa_words + pk.sfb_words;
+        long long blocks = (total + 255) / 256;
+        if (blocks > 4096) blocks = 4096;
+        dg::pack_scales_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(pk);
+        if ((e = cudaGetLastError()) != cudaSuccess) { rc = cuda_fail(e, "scale pack launch"); break; }
+        // ---- tensor maps
+        CUtensorMap ta, tb, tsfa, tsfb;
+        if ((rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M))) break;
+        if ((rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS))) break;
+        if ((rc = make_atom_map(tsfa, pk.sfa_out, sfa_atoms, 1))) break;
+        if ((rc = make_atom_map(tsfb, pk.sfb_out, sfb_atoms, C::SFB_ATOMS))) break;
+        // ---- the GEMM, as a programmatic dependent of the pre-pass
+        auto kernel = dg::fp8_gemm_kernel<C>;
+        if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) !=
+            cudaSuccess) {
+            rc = cuda_fail(e, "cudaFuncSetAttribute");
+            break;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid * CTAS), 1, 1);
+        cfg.blockDim = dim3(dg::NUM_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = CTAS;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        if (CTAS > 1) {
+            // a persistent grid larger than the co-resident clusters would only queue behind itself
+            static int max_clusters[64] = {0};
+            int &cached = max_clusters[device & 63];
+            if (cached == 0) {
+                int n = 0;
+                if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+                    cudaGetLastError();
+                    n = grid;
+                }
+                cached = n;
+            }
+            if (grid > cached) cfg.gridDim.x = static_cast<unsigned>(cached * CTAS);
+        }
+        static const bool debug = getenv("DG_DEBUG") && getenv("DG_DEBUG")[0] == '1';
+        if (debug)
+            fprintf(stderr, "[dg] mode=%d M=%d N=%d K=%d G=%d BN=%d stages=%d x %d ctas=%d grid=%u smem=%d windows=%d"
+                            " scratch=%lld B\n",
+                    p.mode, p.M, p.N, p.K, p.G, BN, C::STAGES, KPS, CTAS, cfg.gridDim.x, C::SMEM_BYTES, p.num_windows,
+                    (pk.sfa_words + pk.sfb_words) * 4);
+        if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, tsfb, p)) != cudaSuccess) {
+            rc = cuda_fail(e, "kernel launch");
+            break;
+        }
+    } while (false);
+    cudaError_t ef = cudaFreeAsync(scratch, stream);
+    if (rc == DG_OK && ef != cudaSuccess) rc = cuda_fail(ef, "cudaFreeAsync (packed scales)");
+    return rc;
 }
 
 // Tile widths the library is built with, and the pipeline depth each fits in 227 KB of shared memory and
@@ -167,21 +247,21 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
 constexpr int kCandidateBN[] = {224, 192, 160, 128};
 
 int launch_bn(int bn, int ctas, const void *a, long long a_rows, const void *b, long long b_rows,
-              const dg::GemmParams &p, int grid, cudaStream_t stream) {
+              const ScaleArgs &sc, const dg::GemmParams &p, int grid, int device, cudaStream_t stream) {
     if (ctas == 2) {
         switch (bn) {
-            case 224: return launch_cfg<224, 2, 2>(a, a_rows, b, b_rows, p, grid, stream);
-            case 192: return launch_cfg<192, 2, 2>(a, a_rows, b, b_rows, p, grid, stream);
-            case 160: return launch_cfg<160, 2, 2>(a, a_rows, b, b_rows, p, grid, stream);
-            case 128: return launch_cfg<128, 2, 2>(a, a_rows, b, b_rows, p, grid, stream);
+            case 224: return launch_cfg<224, 2, 2>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 192: return launch_cfg<192, 2, 2>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 160: return launch_cfg<160, 2, 2>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 128: return launch_cfg<128, 2, 2>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
             default: break;
         }
     } else {
         switch (bn) {
-            case 224: return launch_cfg<224, 1, 1>(a, a_rows, b, b_rows, p, grid, stream);
-            case 192: return launch_cfg<192, 1, 1>(a, a_rows, b, b_rows, p, grid, stream);
-            case 160: return launch_cfg<160, 1, 1>(a, a_rows, b, b_rows, p, grid, stream);
-            case 128: return launch_cfg<128, 1, 1>(a, a_rows, b, b_rows, p, grid, stream);
+            case 224: return launch_cfg<224, 1, 1>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 192: return launch_cfg<192, 1, 1>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 160: return launch_cfg<160, 1, 1>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 128: return launch_cfg<128, 1, 1>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
             default: break;
         }
     }
@@ -198,7 +278,7 @@ struct Plan {
 };
 
 int plan_and_launch(dg::GemmParams p, const DeviceInfo &info, const Plan &plan, const void *a, long long a_rows,
-                    const void *b, long long b_rows, cudaStream_t stream) {
+                    const void *b, long long b_rows, const ScaleArgs &sc, cudaStream_t stream) {
     const int sms = effective_sms(info);
     bool pair = plan.pair_supported && sms >= 2;
     if (g_pair_policy == 0) pair = false;
@@ -211,10 +291,11 @@ int plan_and_launch(dg::GemmParams p, const DeviceInfo &info, const Plan &plan, 
     const int bn = dg_select_block_n(pair ? plan.sel2 : plan.sel1, p.N, units);
     p.num_n_blocks = (p.N + bn - 1) / bn;
     p.num_windows = static_cast<int>(p.mode == dg::MODE_MASKED ? 0 : (pair ? plan.windows2 : plan.windows1));
+    p.num_sf_groups = (p.K / dg::BLOCK_K + dg::SF_GROUP - 1) / dg::SF_GROUP;
     const long long tiles = (pair ? plan.bound2 : plan.bound1) * p.num_n_blocks;
     const int grid = static_cast<int>(tiles < units ? tiles : units);
     if (grid <= 0) return DG_OK;
-    return launch_bn(bn, pair ? 2 : 1, a, a_rows, b, b_rows, p, grid, stream);
+    return launch_bn(bn, pair ? 2 : 1, a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
 }
 
 unsigned *device_error_word() {
@@ -312,14 +393,13 @@ int dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const float *
     dg::GemmParams p{};
     p.mode = dg::MODE_DENSE;
     p.M = M; p.N = N; p.K = K; p.G = 1;
-    p.sfa_ld = dg_get_tma_aligned_size(M, 4);
-    p.sfa = sfa; p.sfb = sfb;
+    const ScaleArgs sc{sfa, dg_get_tma_aligned_size(M, 4), sfb};
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.err = device_error_word();
     if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
     const long long w1 = (M + dg::BLOCK_M - 1) / dg::BLOCK_M, w2 = (M + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M);
     const Plan plan{w1, w2, w1, w2, w1, w2, true};
-    return plan_and_launch(p, info, plan, a, M, b, N, reinterpret_cast<cudaStream_t>(stream));
+    return plan_and_launch(p, info, plan, a, M, b, N, sc, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
@@ -338,8 +418,7 @@ int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const v
     dg::GemmParams p{};
     p.mode = dg::MODE_CONTIGUOUS;
     p.M = M_total; p.N = N; p.K = K; p.G = G;
-    p.sfa_ld = dg_get_tma_aligned_size(M_total, 4);
-    p.sfa = sfa; p.sfb = sfb;
+    const ScaleArgs sc{sfa, dg_get_tma_aligned_size(M_total, 4), sfb};
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.m_indices = m_indices;
     p.err = device_error_word();
@@ -348,7 +427,7 @@ int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const v
     // a 256-row window holds at most two tiles (its halves may belong to two groups)
     const long long bound = w2 + (w2 < G ? w2 : G);
     const Plan plan{w1, w2, w1, bound, w1, w2, w2 <= dg::MAX_PAIR_WINDOWS};
-    return plan_and_launch(p, info, plan, a, M_total, b, static_cast<long long>(G) * N,
+    return plan_and_launch(p, info, plan, a, M_total, b, static_cast<long long>(G) * N, sc,
                            reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -368,8 +447,8 @@ int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const void 
     dg::GemmParams p{};
     p.mode = dg::MODE_MASKED;
     p.M = M_max; p.N = N; p.K = K; p.G = G;
-    p.sfa_ld = dg_get_tma_aligned_size(M_max, 4);
-    p.sfa = sfa; p.sfb = sfb;
+    const ScaleArgs sc{sfa, dg_get_tma_aligned_size(M_max, 4), sfb};
+    p.sfa_blocks = (M_max + dg::BLOCK_M - 1) / dg::BLOCK_M;
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.masked_m = masked_m;
     p.err = device_error_word();
@@ -381,7 +460,7 @@ int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const void 
     const long long max1 = static_cast<long long>(G) * ((M_max + dg::BLOCK_M - 1) / dg::BLOCK_M);
     const long long max2 = static_cast<long long>(G) * ((M_max + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M));
     const Plan plan{h1, h2, max1, max2, 0, 0, true};
-    return plan_and_launch(p, info, plan, a, static_cast<long long>(G) * M_max, b, static_cast<long long>(G) * N,
+    return plan_and_launch(p, info, plan, a, static_cast<long long>(G) * M_max, b, static_cast<long long>(G) * N, sc,
                            reinterpret_cast<cudaStream_t>(stream));
 }
 

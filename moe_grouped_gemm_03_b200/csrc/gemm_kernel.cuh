@@ -6,27 +6,26 @@
 // call shapes, "Optimizations" for persistent warp specialisation, the unified block scheduler, larger
 // blocks and unaligned block sizes.)
 //
+// The per-128-K scale promotion runs inside the tensor core: the MMA is tcgen05.mma kind::mxf8f6f4 with
+// block scaling (one UE8M0 scale per 32 K elements and row/column).  The fp32 power-of-two scales are packed
+// beforehand (scale_pack.cuh) into 32-bit words holding the UE8M0 bytes of four consecutive 128-K blocks,
+// already in the shared-memory layout tcgen05.cp reads; the MMAs of K block kb select byte kb % 4 through
+// the scale-factor ids of the instruction descriptor for all four 32-wide K sub-blocks, which applies the
+// 1x128 / 128x128 recipe exactly.
+//
 // CTAS = 1: one CTA computes a 128 x BN output tile.  CTAS = 2: a cluster of two CTAs (a CTA pair) computes
 // a 256 x BN tile with tcgen05.mma.cta_group::2: each CTA loads its own 128 rows of A and its own BN/2 rows
-// of B (no multicast), the leader CTA issues the MMAs, and each CTA's TMEM holds its 128 rows of D.  The
-// pair halves the B bytes each SM pulls from L2 per FLOP.
+// of B (no multicast), the leader CTA issues the MMAs, and each CTA's TMEM holds its 128 rows of D.  All
+// cross-CTA data arrives by TMA whose byte counts complete the leader's barrier.
 //
-// Per CTA, 256 threads:
-//   warp 0      TMA producer: A [128 x 128 B] and B [BN/CTAS x 128 B] per 128-K block, KPS K blocks per
-//               stage of a STAGES-deep ring (128-byte swizzle; one barrier wait and one commit per stage).
-//   warp 1      TMEM owner (both CTAs) and MMA issuer (one thread of the leader CTA): per group of four
-//               128-K blocks it copies the group's scale factors shared -> TMEM (tcgen05.cp); per 128-K
-//               block it issues four tcgen05.mma kind::mxf8f6f4 (K = 32 each) into one of two TMEM
-//               accumulators (BN fp32 columns).
-//   warp 2      scale-factor packer, one group of four 128-K blocks at a time: prefetches the groups' fp32
-//               SFA [4 x 128] by TMA into its own ring (RAW_SLOTS groups ahead), turns the power-of-two
-//               scales into UE8M0 bytes (the fp32 exponent field) and packs the four K blocks' bytes of a
-//               row into one 32-bit word in the layout tcgen05.cp / the block-scaled MMA read.  The MMAs of
-//               K block kb select byte kb % 4 through the scale-factor ids of the instruction descriptor,
-//               for all four 32-wide K sub-blocks, so the per-32 scaling of the MMA applies the 1x128 /
-//               128x128 recipe exactly and the per-K-block promotion happens inside the tensor core.  SFB
-//               rows of the tile are kept in registers, prefetched one tile ahead.
-//   warps 4..7  epilogue: TMEM -> registers -> bf16 (RNE) -> global, only for rows the GEMM owns, while the
+// Per CTA, 192 threads:
+//   warp 0      TMA producer: per pipeline stage KPS 128-K blocks of A [128 x 128 B] and B [BN/CTAS x 128 B]
+//               (128-byte swizzle) and, at the first stage of each group of four K blocks, the packed scale
+//               atoms of the group (SFA of this CTA's rows, SFB of the whole tile).
+//   warp 1      TMEM owner (both CTAs) and MMA issuer (one thread of the leader CTA): copies a group's scale
+//               atoms shared -> TMEM (tcgen05.cp), then issues four tcgen05.mma (K = 32 each) per 128-K
+//               block into one of two TMEM accumulators (BN fp32 columns).
+//   warps 2..5  epilogue: TMEM -> registers -> bf16 (RNE) -> global, only for rows the GEMM owns, while the
 //               MMA already fills the other accumulator with the next tile.
 //
 // Tile scheduler (every role walks the same sequence): windows of 128*CTAS rows x BN columns, N fastest,
@@ -54,13 +53,12 @@ enum : int { MODE_DENSE = 0, MODE_CONTIGUOUS = 1, MODE_MASKED = 2 };
 constexpr int BLOCK_M = 128;  // rows per CTA
 constexpr int BLOCK_K = 128;  // = the scale block along K
 constexpr int MMA_K = 32;     // K of one kind::mxf8f6f4 MMA
-constexpr int NUM_THREADS = 256;
+constexpr int SF_GROUP = 4;   // 128-K blocks whose scales share one 32-bit word (one byte each)
+constexpr int SF_ATOM_WORDS = 128;  // a packed scale atom: 128 rows x one 32-bit word (512 bytes)
+constexpr int NUM_THREADS = 192;
+constexpr int EPI_WARP0 = 2;        // epilogue warps 2..5 (TMEM lane quarter = warp % 4)
 constexpr int MAX_MASKED_GROUPS = 1024;
 constexpr int MAX_PAIR_WINDOWS = 4096;  // contiguous layout with CTA pairs: M_total <= 4096 * 256
-constexpr int SFB_KB_REGS = 4;          // K blocks of SFB held per lane: K <= 32 * 4 * 128 = 16384 fast path
-constexpr int SF_GROUP = 4;             // 128-K blocks whose scales share one 32-bit word (one byte each)
-constexpr int SF_SLOTS = 3;             // packed scale groups in flight (shared memory and TMEM slots)
-constexpr int RAW_SLOTS = 4;            // fp32 SFA groups the scale-factor warp prefetches ahead
 constexpr int TMEM_COLS = 512;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s for any single wait
 constexpr int SMEM_LIMIT = 232448;                  // 227 KB of dynamic shared memory per CTA
@@ -73,11 +71,10 @@ struct GemmParams {
     int mode;
     int M;             // dense: M; contiguous: M_total; masked: M_max
     int N, K, G;
-    int num_windows;   // dense / contiguous(single): total; masked: per group; contiguous(pair): windows
-    int num_n_blocks;
-    int sfa_ld;        // sfa floats per K block (the MN-major row extent)
-    const float *sfa;
-    const float *sfb;
+    int num_windows;   // dense / contiguous: windows (128- or 256-row); masked: unused
+    int num_n_blocks;  // ceil(N / BN)
+    int num_sf_groups; // ceil(K / (128 * SF_GROUP))
+    int sfa_blocks;    // 128-row blocks per group of the packed SFA (masked layout)
     __nv_bfloat16 *d;
     const int *m_indices;
     const int *masked_m;
@@ -96,22 +93,21 @@ struct Cfg {
     static constexpr int B_BYTES1 = B_ROWS * BLOCK_K;             // one K block of this CTA's B rows
     static constexpr int A_BYTES = KPS * A_BYTES1;                // per stage
     static constexpr int B_BYTES = KPS * B_BYTES1;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int SF_WORDS = 128 + 128 * SFB_ATOMS;        // packed 32-bit words per slot (SFA, then SFB)
-    static constexpr int SFA_RAW_BYTES = SF_GROUP * TILE_M * 4;   // fp32 SFA [4 K blocks][TILE_M rows], by TMA
-    static constexpr int SF_COLS = 4 + 4 * SFB_ATOMS;             // TMEM columns per slot
+    static constexpr int SF_BYTES = (1 + SFB_ATOMS) * SF_ATOM_WORDS * 4;  // SFA atom + SFB atoms
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SF_BYTES;
+    static constexpr int SF_COLS = 4 + 4 * SFB_ATOMS;             // TMEM columns of one stage's scales
     static constexpr int SF_TMEM_BASE = 2 * BN;                   // after the two accumulators
     static constexpr int TABLE_INTS = (CTAS == 2 ? MAX_PAIR_WINDOWS : MAX_MASKED_GROUPS) + 1;
-    static constexpr int FIXED_BYTES = SF_SLOTS * SF_WORDS * 4 + RAW_SLOTS * SFA_RAW_BYTES + 8 * (2 * SF_SLOTS + RAW_SLOTS + 5) + 16 +
-                                       4 * TABLE_INTS + 4 * MAX_MASKED_GROUPS + 1024 + 8 * 2 * 8;
-    static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
-    static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-    static constexpr int NUM_BARRIERS = 2 * STAGES + 2 * SF_SLOTS + RAW_SLOTS + 5;
+    static constexpr int FIXED_BYTES = 4 * TABLE_INTS + 4 * MAX_MASKED_GROUPS + 16 + 8 * 16 + 1024;
+    static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES - 8 * 2 * 8) / STAGE_BYTES;
+    static constexpr int STAGES_TMEM = (TMEM_COLS - SF_TMEM_BASE) / SF_COLS;
+    static constexpr int STAGES_MAX = STAGES_FIT < STAGES_TMEM ? STAGES_FIT : STAGES_TMEM;
+    static constexpr int STAGES = STAGES_MAX > 8 ? 8 : STAGES_MAX;
+    static constexpr int NUM_BARRIERS = 2 * STAGES + 5;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;
-    static constexpr int OFF_SFA_RAW = OFF_SF + SF_SLOTS * SF_WORDS * 4;
-    static constexpr int OFF_BAR = OFF_SFA_RAW + RAW_SLOTS * SFA_RAW_BYTES;
+    static constexpr int OFF_BAR = OFF_SF + STAGES * SF_BYTES;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARRIERS * 8;   // tmem base, abort flag
     static constexpr int OFF_PREFIX = OFF_MISC + 16;               // int[TABLE_INTS]
     static constexpr int OFF_MM = OFF_PREFIX + 4 * TABLE_INTS;     // masked: clamped masked_m
@@ -120,7 +116,7 @@ struct Cfg {
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32, 256]");
     static_assert(B_ROWS % 8 == 0, "B tile rows must fill whole 8-row swizzle atoms");
     static_assert(STAGES >= 3, "pipeline too shallow");
-    static_assert(SF_TMEM_BASE + SF_SLOTS * SF_COLS <= TMEM_COLS, "TMEM budget");
+    static_assert(SF_TMEM_BASE + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
     static_assert(A_BYTES1 % 1024 == 0 && B_BYTES1 % 1024 == 0, "swizzle atoms need 1024-byte alignment");
     static_assert(SF_GROUP % KPS == 0, "a stage must not straddle a scale group");
@@ -130,6 +126,7 @@ struct Tile {
     int row0;        // first row of the window in A / D (flattened [rows, K] / [rows, N])
     int local_row0;  // first row of the window inside its group (masked) or = row0
     int n0;
+    int nb;
     int g;
 };
 
@@ -163,7 +160,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
 }
 
 // Whole-warp wait: lane 0 waits, the verdict is broadcast, and the warp leaves converged (the callers
-// follow with .sync.aligned tcgen05 instructions or shared-memory accesses guarded by the barrier).
+// follow with .sync.aligned tcgen05 instructions).
 __device__ __forceinline__ bool warp_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort,
                                                   unsigned *err, int lane) {
     int ok = 1;
@@ -197,8 +194,8 @@ __device__ __forceinline__ int upper_index(const int *table, int n, int v) {
 template <class C>
 __device__ __forceinline__ bool decode_tile(const GemmParams &p, const SharedCtl &ctl, int t, Tile &ti) {
     const int w = t / p.num_n_blocks;  // window-tile index
-    const int nb = t - w * p.num_n_blocks;
-    ti.n0 = nb * C::BN;
+    ti.nb = t - w * p.num_n_blocks;
+    ti.n0 = ti.nb * C::BN;
     if (p.mode == MODE_DENSE) {
         ti.g = 0;
         ti.row0 = ti.local_row0 = w * C::TILE_M;
@@ -223,11 +220,6 @@ __device__ __forceinline__ bool decode_tile(const GemmParams &p, const SharedCtl
     ti.local_row0 = (w - ctl.prefix[g]) * C::TILE_M;
     ti.row0 = g * p.M + ti.local_row0;
     return true;
-}
-
-__device__ __forceinline__ uint32_t ue8m0(float s) {
-    // the biased exponent of a power-of-two fp32 is its UE8M0 code
-    return (__float_as_uint(s) >> 23) & 0xFFu;
 }
 
 // Builds the scheduler table in shared memory (one warp).
@@ -276,7 +268,8 @@ __device__ void build_schedule_table(const GemmParams &p, int *prefix, int *mm, 
 template <class C>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                    const __grid_constant__ CUtensorMap tmap_sfa, const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
+                    const GemmParams p) {
     constexpr int BN = C::BN;
     constexpr int STAGES = C::STAGES;
     constexpr int CTAS = C::CTAS;
@@ -285,17 +278,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem + C::OFF_A;
     uint8_t *sB = smem + C::OFF_B;
-    uint32_t *sSF = reinterpret_cast<uint32_t *>(smem + C::OFF_SF);
-    float *sSFA_raw = reinterpret_cast<float *>(smem + C::OFF_SFA_RAW);
+    uint8_t *sSF = smem + C::OFF_SF;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *full = bars;                       // [STAGES] A + B landed (the leader's counts both CTAs' bytes)
-    uint64_t *empty = bars + STAGES;             // [STAGES] MMAs done with the stage (both CTAs, by commit)
-    uint64_t *raw_full = bars + 2 * STAGES;      // [RAW_SLOTS] this CTA's fp32 SFA group landed
-    uint64_t *sf_full = raw_full + RAW_SLOTS;    // [SF_SLOTS] packed scales of the whole tile ready
-    uint64_t *sf_empty = sf_full + SF_SLOTS;     // [SF_SLOTS] MMAs done with the slot (both CTAs, by commit)
-    uint64_t *tmem_full = sf_empty + SF_SLOTS;   // [2]
-    uint64_t *tmem_empty = tmem_full + 2;        // [2] (the leader's counts the epilogue warps of both CTAs)
-    uint64_t *drain = tmem_empty + 2;            // [1]
+    uint64_t *full = bars;                  // [STAGES] stage landed (the leader's counts both CTAs' bytes)
+    uint64_t *empty = bars + STAGES;        // [STAGES] MMAs done with the stage (both CTAs, by commit)
+    uint64_t *tmem_full = bars + 2 * STAGES;  // [2]
+    uint64_t *tmem_empty = tmem_full + 2;   // [2] (the leader's counts the epilogue warps of both CTAs)
+    uint64_t *drain = tmem_empty + 2;       // [1]
     uint32_t *s_tmem_base = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     int *s_prefix = reinterpret_cast<int *>(smem + C::OFF_PREFIX);
@@ -309,14 +298,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);  // the leader's producer arms it with both CTAs' bytes
+            mbar_init(&full[s], 1);  // armed by the leader's producer with every byte of the stage
             mbar_init(&empty[s], 1);
         }
-        for (int j = 0; j < SF_SLOTS; ++j) {
-            mbar_init(&sf_full[j], 1);
-            mbar_init(&sf_empty[j], 1);
-        }
-        for (int j = 0; j < RAW_SLOTS; ++j) mbar_init(&raw_full[j], 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tmem_full[i], 1);
             mbar_init(&tmem_empty[i], 4 * CTAS);  // one arrival per epilogue warp of each CTA
@@ -328,12 +312,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tma_prefetch_desc(&tmap_a);
         tma_prefetch_desc(&tmap_b);
         tma_prefetch_desc(&tmap_sfa);
+        tma_prefetch_desc(&tmap_sfb);
     }
     if (warp == 1) {
         tmem_alloc<CTAS>(s_tmem_base, TMEM_COLS);
         tmem_relinquish<CTAS>();
     }
-    if (warp == 2 && (p.mode == MODE_MASKED || (PAIR && p.mode == MODE_CONTIGUOUS)))
+    if (warp == EPI_WARP0 && (p.mode == MODE_MASKED || (PAIR && p.mode == MODE_CONTIGUOUS)))
         build_schedule_table<C>(p, s_prefix, s_mm, lane);
     tc_fence_before_sync();
     __syncthreads();
@@ -356,32 +341,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
+            grid_dependency_wait();  // the packed scales come from the kernel launched just before
             int s = 0;
             uint32_t ph = 0;
             uint32_t armed = 0, armed_ph = 0;  // stages armed at least once / parity of their last arming
             bool ok = true;
+            const uint32_t full_leader0 = PAIR ? map_shared_rank(smem_u32(&full[0]), 0) : 0u;
             for (int t = cluster_id; t < total_tiles && ok; t += num_clusters) {
                 Tile ti;
                 if (!decode_tile<C>(p, ctl, t, ti)) continue;
                 const int arow = ti.row0 + my_rows;
                 const int brow = ti.g * p.N + ti.n0 + static_cast<int>(rank) * C::B_ROWS;
+                // packed scale atoms: SFA [block][group], SFB [g][n block][group][atom]
+                const int sfa_block = p.mode == MODE_MASKED ? ti.g * p.sfa_blocks + (ti.local_row0 + my_rows) / BLOCK_M
+                                                            : (ti.row0 + my_rows) / BLOCK_M;
+                const int sfa_y0 = sfa_block * p.num_sf_groups;
+                const int sfb_y0 = (ti.g * p.num_n_blocks + ti.nb) * p.num_sf_groups * C::SFB_ATOMS;
                 for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
                     const int nk = min(C::KPS, nkb - kb0);  // K blocks in this stage
+                    const bool group_start = kb0 % SF_GROUP == 0;
                     if (!wait_bounded(&empty[s], ph ^ 1u, s_abort, p.err)) { ok = false; break; }
                     uint8_t *a_dst = sA + s * C::A_BYTES;
                     uint8_t *b_dst = sB + s * C::B_BYTES;
-                    const uint32_t bytes = static_cast<uint32_t>(nk * (C::A_BYTES1 + C::B_BYTES1));
+                    uint8_t *sf_dst = sSF + s * C::SF_BYTES;
+                    const int q = kb0 / SF_GROUP;
+                    const uint32_t bytes =
+                        static_cast<uint32_t>(nk * (C::A_BYTES1 + C::B_BYTES1) + (group_start ? C::SF_BYTES : 0));
                     if constexpr (PAIR) {
-                        // Only the leader arrives (with both CTAs' bytes); the peer's loads just count their
-                        // bytes on the leader's barrier.  A peer load may land before the leader arms the
-                        // phase: the transaction count dips below zero but the phase cannot complete before
-                        // the leader's arrival.  (No cross-CTA release in this loop: it would wait for this
-                        // thread's loads in flight.)
-                        const uint32_t leader_full = map_shared_rank(smem_u32(&full[s]), 0);
+                        // Only the leader arms the barrier (with both CTAs' bytes); the peer's loads just count
+                        // their bytes on it.  A peer load may land before the leader arms the phase: the
+                        // transaction count dips below zero but the phase cannot complete before the arrival.
+                        const uint32_t leader_full = full_leader0 + 8u * static_cast<uint32_t>(s);
                         if (rank == 0) mbar_arrive_expect_tx(&full[s], CTAS * bytes);
                         for (int i = 0; i < nk; ++i) {
                             tma_load_2d_pair(a_dst + i * C::A_BYTES1, &tmap_a, leader_full, (kb0 + i) * BLOCK_K, arow);
                             tma_load_2d_pair(b_dst + i * C::B_BYTES1, &tmap_b, leader_full, (kb0 + i) * BLOCK_K, brow);
+                        }
+                        if (group_start) {
+                            tma_load_2d_pair(sf_dst, &tmap_sfa, leader_full, 0, sfa_y0 + q);
+                            tma_load_2d_pair(sf_dst + SF_ATOM_WORDS * 4, &tmap_sfb, leader_full, 0,
+                                             sfb_y0 + q * C::SFB_ATOMS);
                         }
                     } else {
                         mbar_arrive_expect_tx(&full[s], bytes);
@@ -389,22 +388,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             tma_load_2d(a_dst + i * C::A_BYTES1, &tmap_a, &full[s], (kb0 + i) * BLOCK_K, arow);
                             tma_load_2d(b_dst + i * C::B_BYTES1, &tmap_b, &full[s], (kb0 + i) * BLOCK_K, brow);
                         }
+                        if (group_start) {
+                            tma_load_2d(sf_dst, &tmap_sfa, &full[s], 0, sfa_y0 + q);
+                            tma_load_2d(sf_dst + SF_ATOM_WORDS * 4, &tmap_sfb, &full[s], 0, sfb_y0 + q * C::SFB_ATOMS);
+                        }
                     }
                     armed |= 1u << s;
                     armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
             }
-            if (!ok) {
-                // let the loads still in flight land before shared memory goes away (in a pair the A/B
-                // bytes of both CTAs are counted on the leader's barrier)
+            if (!ok && (!PAIR || rank == 0)) {
+                // let the loads still in flight land before shared memory goes away (in a pair the bytes of
+                // both CTAs are counted on the leader's barrier; the final cluster barrier holds the peer)
                 for (int i = 0; i < STAGES; ++i) {
                     if (!(armed >> i & 1u)) continue;
-                    if (!PAIR || rank == 0) {
-                        const uint64_t t1 = global_timer_ns();
-                        while (!mbar_try_wait(&full[i], (armed_ph >> i) & 1u) &&
-                               global_timer_ns() - t1 < WAIT_LIMIT_NS) {
-                        }
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(&full[i], (armed_ph >> i) & 1u) && global_timer_ns() - t0 < WAIT_LIMIT_NS) {
                     }
                 }
             }
@@ -415,8 +415,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             constexpr uint32_t IDESC = idesc_mxf8_e4m3(C::TILE_M, BN);
             int s = 0;
             uint32_t ph = 0;
-            int slot = 0;
-            uint32_t slot_ph = 0;
             int acc = 0;
             uint32_t acc_ph = 0;
             bool ok = true;
@@ -429,19 +427,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 uint32_t sf_tmem = 0;
                 for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
                     const int nk = min(C::KPS, nkb - kb0);
+                    if (!wait_bounded(&full[s], ph, s_abort, p.err)) { ok = false; break; }
+                    tc_fence_after_sync();
                     if (kb0 % SF_GROUP == 0) {
-                        if (!wait_bounded(&sf_full[slot], slot_ph, s_abort, p.err)) { ok = false; break; }
-                        tc_fence_after_sync();
-                        sf_tmem = tmem_base + static_cast<uint32_t>(C::SF_TMEM_BASE + slot * C::SF_COLS);
-                        const uint32_t sf_smem = smem_u32(sSF + slot * C::SF_WORDS);
+                        // the group's scales into this stage's TMEM slot (the slot's previous readers were
+                        // issued at least STAGES stages ago and the tensor pipe runs them in order)
+                        sf_tmem = tmem_base + static_cast<uint32_t>(C::SF_TMEM_BASE + s * C::SF_COLS);
+                        const uint32_t sf_smem = smem_u32(sSF + s * C::SF_BYTES);
                         tc_cp_32x128b_warpx4<CTAS>(sf_tmem, sdesc_rows16_noswizzle(sf_smem));
 #pragma unroll
                         for (int a = 0; a < C::SFB_ATOMS; ++a)
                             tc_cp_32x128b_warpx4<CTAS>(sf_tmem + 4 + 4 * a,
                                                        sdesc_rows16_noswizzle(sf_smem + 512 + 512 * a));
                     }
-                    if (!wait_bounded(&full[s], ph, s_abort, p.err)) { ok = false; break; }
-                    tc_fence_after_sync();
                     const uint32_t a_stage = smem_u32(sA + s * C::A_BYTES);
                     const uint32_t b_stage = smem_u32(sB + s * C::B_BYTES);
                     for (int i = 0; i < nk; ++i) {
@@ -459,11 +457,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                     tc_commit<CTAS>(&empty[s]);
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
-                    const int last = kb0 + nk - 1;
-                    if (last % SF_GROUP == SF_GROUP - 1 || last == nkb - 1) {
-                        tc_commit<CTAS>(&sf_empty[slot]);
-                        if (++slot == SF_SLOTS) { slot = 0; slot_ph ^= 1u; }
-                    }
                 }
                 if (!ok) break;
                 tc_commit<CTAS>(&tmem_full[acc]);
@@ -476,183 +469,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < WAIT_LIMIT_NS) {
             }
         }
-    } else if (warp == 2 && rank == 0) {
-        // ---------------------------------------------------------------- scale-factor packer (leader CTA)
-        // In a pair the leader packs the scales of both CTAs' rows and stores the peer's words straight into
-        // the peer's shared memory (same offsets), so the MMA thread waits on one local barrier.
-        // Two cursors walk this CTA's (tile, group-of-4-K-blocks) sequence: the prefetch cursor keeps up to
-        // RAW_SLOTS groups of fp32 SFA in flight (TMA into this warp's own ring, which depends on nothing but
-        // this warp's progress), the consume cursor packs one group at a time into a slot the MMAs released.
-        const int nnb128 = (p.N + 127) / 128;
-        const bool sfb_in_regs = nkb <= 32 * SFB_KB_REGS;
-        const uint32_t sf_peer0 = PAIR ? map_shared_rank(smem_u32(sSF), 1) : 0u;  // the peer's packed words
-        auto next_valid = [&](int &t, Tile &ti) {
-            for (; t < total_tiles; t += num_clusters)
-                if (decode_tile<C>(p, ctl, t, ti)) return true;
-            return false;
-        };
-        struct Cursor {
-            int t;
-            Tile ti;
-            int kb0;
-            bool have;
-        };
-        auto advance = [&](Cursor &c) {
-            c.kb0 += SF_GROUP;
-            if (c.kb0 >= nkb) {
-                c.kb0 = 0;
-                c.t += num_clusters;
-                c.have = next_valid(c.t, c.ti);
-            }
-        };
-        Cursor pf{cluster_id, Tile{}, 0, false};
-        pf.have = next_valid(pf.t, pf.ti);
-        Cursor cs = pf;
-        uint32_t issued = 0, consumed = 0;
-        auto prefetch = [&]() {
-            while (pf.have && issued - consumed < static_cast<uint32_t>(RAW_SLOTS)) {
-                if (lane == 0) {
-                    const int rs = static_cast<int>(issued % RAW_SLOTS);
-                    const int x = pf.ti.local_row0;
-                    const int y = (p.mode == MODE_MASKED ? pf.ti.g * nkb : 0) + pf.kb0;
-                    mbar_arrive_expect_tx(&raw_full[rs], C::SFA_RAW_BYTES);
-                    tma_load_2d(sSFA_raw + rs * SF_GROUP * C::TILE_M, &tmap_sfa, &raw_full[rs], x, y);
-                }
-                ++issued;
-                advance(pf);
-            }
-        };
-        // SFB of the consume cursor's tile (cur) and of the next tile (nxt), in registers
-        float cur[3][SFB_KB_REGS], nxt[3][SFB_KB_REGS];
-        auto load_sfb = [&](const Tile &ti, float (&v)[3][SFB_KB_REGS]) {
-            const float *sfb_g = p.sfb + static_cast<size_t>(ti.g) * nnb128 * nkb;
-            const int nb0 = ti.n0 >> 7;
-#pragma unroll
-            for (int j = 0; j < 3; ++j)
-#pragma unroll
-                for (int i = 0; i < SFB_KB_REGS; ++i) {
-                    const int kb = lane + 32 * i;
-                    v[j][i] = (nb0 + j < nnb128 && kb < nkb) ? __ldg(sfb_g + (nb0 + j) * nkb + kb) : 1.f;
-                }
-        };
-        int t_next = cs.t + num_clusters;
-        Tile ti_next;
-        bool have_next = cs.have && next_valid(t_next, ti_next);
-        if (cs.have && sfb_in_regs) load_sfb(cs.ti, cur);
-        if (have_next && sfb_in_regs) load_sfb(ti_next, nxt);
-        int slot = 0;
-        uint32_t slot_ph = 0;
-        bool ok = true;
-        while (cs.have) {
-            prefetch();
-            const Tile &ti = cs.ti;
-            const int kb0 = cs.kb0;
-            const int nb0 = ti.n0 >> 7;
-            // packed SFB word of each of the tile's (up to) three 128-row scale blocks
-            const float *sfb_g = p.sfb + static_cast<size_t>(ti.g) * nnb128 * nkb;
-            uint32_t wb[3];
-#pragma unroll
-            for (int j = 0; j < 3; ++j) {
-                uint32_t word = 0;
-#pragma unroll
-                for (int i = 0; i < SF_GROUP; ++i) {
-                    const int kb = kb0 + i;
-                    float v;
-                    if (sfb_in_regs) {
-                        const int reg = kb >> 5;
-                        float x = cur[j][0];
-#pragma unroll
-                        for (int r = 1; r < SFB_KB_REGS; ++r) x = reg == r ? cur[j][r] : x;
-                        v = __shfl_sync(0xffffffffu, x, kb & 31);
-                    } else {
-                        v = (nb0 + j < nnb128 && kb < nkb) ? __ldg(sfb_g + (nb0 + j) * nkb + kb) : 1.f;
-                    }
-                    word |= ue8m0(v) << (8 * i);
-                }
-                wb[j] = word;
-            }
-            // the group's fp32 SFA -> one packed word per row (byte i = K block kb0 + i)
-            const int rs = static_cast<int>(consumed % RAW_SLOTS);
-            if (!warp_wait_bounded(&raw_full[rs], (consumed / RAW_SLOTS) & 1u, s_abort, p.err, lane)) {
-                ok = false;
-                break;
-            }
-            const float *raw = sSFA_raw + rs * SF_GROUP * C::TILE_M;
-            uint32_t wa[CTAS][4];
-#pragma unroll
-            for (int c = 0; c < CTAS; ++c) {
-                wa[c][0] = wa[c][1] = wa[c][2] = wa[c][3] = 0u;
-#pragma unroll
-                for (int i = 0; i < SF_GROUP; ++i) {
-                    const float4 v = reinterpret_cast<const float4 *>(raw + i * C::TILE_M + c * BLOCK_M)[lane];
-                    wa[c][0] |= ue8m0(v.x) << (8 * i);
-                    wa[c][1] |= ue8m0(v.y) << (8 * i);
-                    wa[c][2] |= ue8m0(v.z) << (8 * i);
-                    wa[c][3] |= ue8m0(v.w) << (8 * i);
-                }
-            }
-            fence_proxy_async_smem();  // the raw slot's next TMA write comes after these reads
-            __syncwarp();
-            ++consumed;
-            prefetch();
-            if (!warp_wait_bounded(&sf_empty[slot], slot_ph ^ 1u, s_abort, p.err, lane)) { ok = false; break; }
-            uint32_t *w = sSF + slot * C::SF_WORDS;
-            const uint32_t w_peer = sf_peer0 + 4u * static_cast<uint32_t>(slot * C::SF_WORDS);
-            // tcgen05.cp 32x128b source: word (r % 32) * 4 + r / 32 holds row r of a 128-row atom
-            const int r0 = 4 * lane;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int idx = ((r0 + i) & 31) * 4 + ((r0 + i) >> 5);
-                w[idx] = wa[0][i];
-                if constexpr (PAIR) st_shared_cluster(w_peer + 4u * idx, wa[CTAS - 1][i]);
-            }
-#pragma unroll
-            for (int j = 0; j < C::SFB_ATOMS * 4; ++j) {
-                const int r = lane + 32 * j;                        // row inside the BN tile
-                const int which = ((ti.n0 + r) >> 7) - nb0;         // 0, 1 or 2
-                const int idx = 128 + (r >> 7) * 128 + (r & 31) * 4 + ((r >> 5) & 3);
-                const uint32_t v = which == 0 ? wb[0] : (which == 1 ? wb[1] : wb[2]);
-                w[idx] = v;
-                if constexpr (PAIR) st_shared_cluster(w_peer + 4u * idx, v);
-            }
-            if constexpr (PAIR) fence_proxy_async_all(); else fence_proxy_async_smem();
-            __syncwarp();
-            // lane 1 signals: lane 0 issues this warp's TMA loads, and a release by the thread that issued
-            // them could wait for them to land
-            if (lane == 1) {
-                if constexpr (PAIR)
-                    mbar_arrive_cluster(map_shared_rank(smem_u32(&sf_full[slot]), 0));
-                else
-                    mbar_arrive(&sf_full[slot]);
-            }
-            if (++slot == SF_SLOTS) { slot = 0; slot_ph ^= 1u; }
-            const int t_before = cs.t;
-            advance(cs);
-            if (cs.have && cs.t != t_before) {
-                // moved to the next tile: its SFB is in nxt; fetch the one after
-                if (sfb_in_regs) {
-#pragma unroll
-                    for (int j = 0; j < 3; ++j)
-#pragma unroll
-                        for (int i = 0; i < SFB_KB_REGS; ++i) cur[j][i] = nxt[j][i];
-                }
-                t_next = cs.t + num_clusters;
-                have_next = next_valid(t_next, ti_next);
-                if (have_next && sfb_in_regs) load_sfb(ti_next, nxt);
-            }
-        }
-        if (!ok && lane == 0) {
-            // let this warp's loads still in flight land before shared memory goes away
-            for (uint32_t q = consumed; q != issued; ++q) {
-                const uint64_t t0 = global_timer_ns();
-                while (!mbar_try_wait(&raw_full[q % RAW_SLOTS], (q / RAW_SLOTS) & 1u) &&
-                       global_timer_ns() - t0 < WAIT_LIMIT_NS) {
-                }
-            }
-        }
-        __syncwarp();
-    } else if (warp >= 4) {
-        // ---------------------------------------------------------------- epilogue
+    } else {
+        // ---------------------------------------------------------------- epilogue (warps 2..5)
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const uint32_t tmem_empty_leader0 = PAIR ? map_shared_rank(smem_u32(&tmem_empty[0]), 0) : 0u;
         int acc = 0;

@@ -78,6 +78,17 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ------------------------------------------------------------------------------------------------
+// Programmatic dependent launch
+// ------------------------------------------------------------------------------------------------
+// Blocks until the grid this one depends on has completed and its memory operations are visible (a no-op
+// when the kernel was not launched as a programmatic dependent).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the dependent grid start launching (its prologue overlaps the rest of this grid).
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------------------------------
 // Clusters
 // ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_cta_rank() {
