@@ -103,6 +103,23 @@ DG_EXPORT int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, c
                                     void *d, const int *masked_m, int G, int M_max, int N, int K,
                                     int expected_m, dg_stream_t stream);
 
+/* Dense NT GEMM that allocates no device memory (the pages have no counterpart: it exists for callers of this
+ * library).  Same arguments, layouts, validation and results as dg_fp8_gemm_nt.  dg_fp8_gemm_nt takes a small
+ * stream-ordered scratch buffer per call for its packed scale factors; callers that may not allocate during the
+ * call -- code running under a global-mode stream capture, where allocation calls are refused, or engines whose
+ * own memory manager owns all of device memory -- use this entry point instead, which puts the packed scales in a
+ * fixed 16 MiB buffer that lives as long as the library is loaded (every device that loads the library holds
+ * one).  It never calls cudaMalloc, cudaFree or any allocating routine.
+ *   - Limit: the packed scales take at most (ceil(M/128) + 2*ceil(N/BN)) * ceil(K/512) * 512 bytes (BN is the
+ *     chosen tile width, 128..224); a shape needing more than 16 MiB returns DG_ERR_UNSUPPORTED and launches
+ *     nothing (M = N = K = 16384 needs about 4.5 MB).
+ *   - The first call on each device looks up the buffer's device address with that device current; make that
+ *     first call before any stream capture.
+ *   - All calls share the buffer and each call rewrites every word it uses: calls whose work overlaps on the GPU
+ *     (unordered streams) race; calls ordered on one stream are safe. */
+DG_EXPORT int dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
+                                     int M, int N, int K, dg_stream_t stream);
+
 /* Tile-shape policy for the next calls on any thread: -1 (default) lets the library choose between one
  * CTA per 128-row tile and CTA pairs (2-CTA clusters, tcgen05 cta_group::2) computing 256-row tiles;
  * 0 forces single CTAs; 1 uses pairs wherever the layout allows.  Results agree within the tolerance of

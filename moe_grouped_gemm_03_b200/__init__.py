@@ -53,6 +53,7 @@ _SIGNATURES = {
     "dg_fp8_gemm_nt": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_gemm_nt_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_gemm_nt_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "dg_fp8_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_set_cta_pair_policy": (_I, [_I]),
     "dg_last_error": (ctypes.c_char_p, []),
     "dg_check_device_error": (_I, [_P]),
@@ -162,6 +163,26 @@ def fp8_gemm_nt(lhs: Tuple[torch.Tensor, torch.Tensor], rhs: Tuple[torch.Tensor,
     _check(_lib.dg_fp8_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(out), M, N, K, _stream()))
 
 
+def fp8_gemm_nt_noalloc(lhs: Tuple[torch.Tensor, torch.Tensor], rhs: Tuple[torch.Tensor, torch.Tensor],
+                        out: torch.Tensor) -> None:
+    """Same as fp8_gemm_nt but allocates no device memory: the packed scales go to the library's fixed 16 MiB
+    buffer (for callers that may not allocate during the call, e.g. under a global-mode stream capture).
+    Calls overlapping on the GPU share that buffer and race; calls on one stream are safe."""
+    a, sfa = lhs
+    b, sfb = rhs
+    _check_operand("a", a, 2, _FP8_TYPES)
+    _check_operand("b", b, 2, _FP8_TYPES)
+    _check_operand("sfa", sfa, 2, (torch.float32,))
+    _check_operand("sfb", sfb, 2, (torch.float32,))
+    _check_operand("out", out, 2, (torch.bfloat16,))
+    M, K = a.shape
+    N = b.shape[0]
+    _need(b.shape[1] == K and tuple(out.shape) == (M, N), "shape mismatch between a, b and out")
+    _need(sfa.shape == (K // 128, get_tma_aligned_size(M, 4)), f"sfa must be [{K // 128}, {get_tma_aligned_size(M, 4)}]")
+    _need(sfb.shape == ((N + 127) // 128, K // 128), "sfb must be [ceil(N/128), K/128]")
+    _check(_lib.dg_fp8_gemm_nt_noalloc(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(out), M, N, K, _stream()))
+
+
 def m_grouped_fp8_gemm_nt_contiguous(lhs, rhs, out: torch.Tensor, m_indices: torch.Tensor) -> None:
     """Contiguous layout: out[m] = lhs[m] @ rhs[m_indices[m]]^T; rows with m_indices == -1 are untouched."""
     a, sfa = lhs
@@ -202,7 +223,7 @@ def m_grouped_fp8_gemm_nt_masked(lhs, rhs, out: torch.Tensor, masked_m: torch.Te
 
 
 __all__ = [
-    "DGError", "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
+    "DGError", "fp8_gemm_nt", "fp8_gemm_nt_noalloc", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
     "get_m_alignment_for_contiguous_layout", "get_tma_aligned_size", "set_num_sms", "get_num_sms", "num_tiles",
     "select_block_n", "set_cta_pair_policy", "check_device_error", "lib", "header_symbols", "last_error",
 ]
