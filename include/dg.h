@@ -88,7 +88,7 @@ DG_EXPORT int dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, con
  *   sfa [K/128][ld(M_total)], b [G][N][K] e4m3, sfb [G][ceil(N/128)][K/128],
  *   m_indices int32 [M_total] on the device: the group of each row, -1 for a padding row.  Every
  *   128-row block must hold one group (its first row decides; a block whose first row is -1 is skipped),
- *   d [M_total][N] bf16: rows with m_indices == -1 are left untouched.  M_total % 128 == 0. */
+ *   d [M_total][N] bf16: rows with m_indices == -1 are left untouched.  M_total % 128 == 0, 1 <= G <= 65534. */
 DG_EXPORT int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
                                         void *d, const int *m_indices, int M_total, int N, int K, int G,
                                         dg_stream_t stream);

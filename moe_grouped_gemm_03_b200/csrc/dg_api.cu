@@ -536,7 +536,7 @@ int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const v
     if (int rc = check_common(a, sfa, b, sfb, d, N, K)) return rc;
     if (!m_indices) return fail(DG_ERR_INVALID_ARG, "m_indices is null");
     if (!aligned(m_indices, 4)) return fail(DG_ERR_ALIGNMENT, "m_indices must be 4-byte aligned");
-    if (G < 1) return fail(DG_ERR_INVALID_ARG, "G=%d must be at least 1", G);
+    if (G < 1 || G > 65534) return fail(DG_ERR_INVALID_ARG, "G=%d must be in [1, 65534]", G);
     if (M_total < 0) return fail(DG_ERR_INVALID_ARG, "M_total=%d must be non-negative", M_total);
     if (M_total % dg::BLOCK_M)
         return fail(DG_ERR_ALIGNMENT, "M_total=%d must be a multiple of %d", M_total, dg::BLOCK_M);

@@ -37,6 +37,8 @@
 //               window table (tiles per window, prefix) is built on the device at kernel start.
 //   masked      per group ceil(masked_m[g] / 128*CTAS) windows, counted on the device, so the host never
 //               needs masked_m.
+// Each CTA decodes its tile sequence once at kernel start (all threads, into a shared-memory list), so no
+// role pays a decode -- a binary search and global loads of m_indices -- per tile.
 //
 // Every mbarrier wait is bounded: after WAIT_LIMIT_NS the waiting thread raises a CTA-wide abort flag and
 // records ERR_TIMEOUT in the device error word; every role then leaves its loop, the producer waits (bounded)
@@ -59,6 +61,7 @@ constexpr int NUM_THREADS = 192;
 constexpr int EPI_WARP0 = 2;        // epilogue warps 2..5 (TMEM lane quarter = warp % 4)
 constexpr int MAX_MASKED_GROUPS = 1024;
 constexpr int MAX_PAIR_WINDOWS = 4096;  // contiguous layout with CTA pairs: M_total <= 4096 * 256
+constexpr int TILE_LIST_CAP = 1024;     // tiles per CTA decoded up front (further tiles are decoded on the fly)
 constexpr int TMEM_COLS = 512;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s for any single wait
 constexpr int SMEM_LIMIT = 232448;                  // 227 KB of dynamic shared memory per CTA
@@ -98,7 +101,7 @@ struct Cfg {
     static constexpr int SF_COLS = 4 + 4 * SFB_ATOMS;             // TMEM columns of one stage's scales
     static constexpr int SF_TMEM_BASE = 2 * BN;                   // after the two accumulators
     static constexpr int TABLE_INTS = (CTAS == 2 ? MAX_PAIR_WINDOWS : MAX_MASKED_GROUPS) + 1;
-    static constexpr int FIXED_BYTES = 4 * TABLE_INTS + 4 * MAX_MASKED_GROUPS + 16 + 8 * 16 + 1024;
+    static constexpr int FIXED_BYTES = 4 * TABLE_INTS + 4 * MAX_MASKED_GROUPS + 16 + 8 * TILE_LIST_CAP + 16 + 8 * 16 + 1024;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES - 8 * 2 * 8) / STAGE_BYTES;
     static constexpr int STAGES_TMEM = (TMEM_COLS - SF_TMEM_BASE) / SF_COLS;
     static constexpr int STAGES_MAX = STAGES_FIT < STAGES_TMEM ? STAGES_FIT : STAGES_TMEM;
@@ -111,7 +114,8 @@ struct Cfg {
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARRIERS * 8;   // tmem base, abort flag
     static constexpr int OFF_PREFIX = OFF_MISC + 16;               // int[TABLE_INTS]
     static constexpr int OFF_MM = OFF_PREFIX + 4 * TABLE_INTS;     // masked: clamped masked_m
-    static constexpr int SMEM_BYTES = OFF_MM + 4 * MAX_MASKED_GROUPS + 1024;  // + alignment slack
+    static constexpr int OFF_TILES = (OFF_MM + 4 * MAX_MASKED_GROUPS + 15) / 16 * 16;  // uint2[TILE_LIST_CAP]
+    static constexpr int SMEM_BYTES = OFF_TILES + 8 * TILE_LIST_CAP + 1024;     // + alignment slack
     static_assert(CTAS == 1 || CTAS == 2, "single CTA or CTA pair");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32, 256]");
     static_assert(B_ROWS % 8 == 0, "B tile rows must fill whole 8-row swizzle atoms");
@@ -120,6 +124,9 @@ struct Cfg {
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
     static_assert(A_BYTES1 % 1024 == 0 && B_BYTES1 % 1024 == 0, "swizzle atoms need 1024-byte alignment");
     static_assert(SF_GROUP % KPS == 0, "a stage must not straddle a scale group");
+    static_assert(OFF_A % 1024 == 0 && OFF_B % 1024 == 0 && OFF_SF % 512 == 0, "TMA destinations");
+    static_assert(OFF_BAR % 8 == 0 && OFF_MISC % 8 == 0, "mbarriers need 8-byte alignment");
+    static_assert(OFF_PREFIX % 4 == 0 && OFF_MM % 4 == 0 && OFF_TILES % 16 == 0, "tables");
 };
 
 struct Tile {
@@ -222,6 +229,25 @@ __device__ __forceinline__ bool decode_tile(const GemmParams &p, const SharedCtl
     return true;
 }
 
+// A decoded tile packed into 8 bytes: row0, then (g + 1) in the low 16 bits and nb in the high 16 bits
+// (g + 1 = 0 marks a tile that computes nothing).  local_row0 = row0 - g * M for the masked layout, else row0.
+__device__ __forceinline__ uint2 pack_tile(bool valid, const Tile &ti) {
+    return make_uint2(static_cast<uint32_t>(ti.row0),
+                      (valid ? static_cast<uint32_t>(ti.g + 1) : 0u) | (static_cast<uint32_t>(ti.nb) << 16));
+}
+
+template <class C>
+__device__ __forceinline__ bool unpack_tile(const GemmParams &p, uint2 e, Tile &ti) {
+    const int g1 = static_cast<int>(e.y & 0xFFFFu);
+    if (g1 == 0) return false;
+    ti.g = g1 - 1;
+    ti.nb = static_cast<int>(e.y >> 16);
+    ti.n0 = ti.nb * C::BN;
+    ti.row0 = static_cast<int>(e.x);
+    ti.local_row0 = p.mode == MODE_MASKED ? ti.row0 - ti.g * p.M : ti.row0;
+    return true;
+}
+
 // Builds the scheduler table in shared memory (one warp).
 //   masked: mm[g] = clamp(masked_m[g]); prefix[g] = sum_{h<g} ceil(mm[h] / TILE_M); prefix[G] = total.
 //   contiguous, CTA pair: prefix[j] = tiles in windows before j (a window holds 0, 1 or 2 tiles).
@@ -289,6 +315,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     int *s_prefix = reinterpret_cast<int *>(smem + C::OFF_PREFIX);
     int *s_mm = reinterpret_cast<int *>(smem + C::OFF_MM);
+    uint2 *s_tiles = reinterpret_cast<uint2 *>(smem + C::OFF_TILES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -338,6 +365,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int total_tiles = total_windows * p.num_n_blocks;
     const int my_rows = BLOCK_M * static_cast<int>(rank);  // offset of this CTA's rows inside the window
 
+    // This CTA's (pair's) tile sequence t = cluster_id + k * num_clusters, decoded once by all threads; every
+    // role then reads tile k with one shared-memory load instead of decoding it (which can take global loads).
+    const int my_tiles = total_tiles > cluster_id ? (total_tiles - cluster_id + num_clusters - 1) / num_clusters : 0;
+    for (int k = threadIdx.x; k < min(my_tiles, TILE_LIST_CAP); k += NUM_THREADS) {
+        Tile ti;
+        const bool valid = decode_tile<C>(p, ctl, cluster_id + k * num_clusters, ti);
+        s_tiles[k] = pack_tile(valid, ti);
+    }
+    __syncthreads();
+    auto tile_at = [&](int k, Tile &ti) -> bool {
+        if (k < TILE_LIST_CAP) return unpack_tile<C>(p, s_tiles[k], ti);
+        return decode_tile<C>(p, ctl, cluster_id + k * num_clusters, ti);
+    };
+
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
@@ -347,9 +388,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t armed = 0, armed_ph = 0;  // stages armed at least once / parity of their last arming
             bool ok = true;
             const uint32_t full_leader0 = PAIR ? map_shared_rank(smem_u32(&full[0]), 0) : 0u;
-            for (int t = cluster_id; t < total_tiles && ok; t += num_clusters) {
+            for (int k = 0; k < my_tiles && ok; ++k) {
                 Tile ti;
-                if (!decode_tile<C>(p, ctl, t, ti)) continue;
+                if (!tile_at(k, ti)) continue;
                 const int arow = ti.row0 + my_rows;
                 const int brow = ti.g * p.N + ti.n0 + static_cast<int>(rank) * C::B_ROWS;
                 // packed scale atoms: SFA [block][group], SFB [g][n block][group][atom]
@@ -418,9 +459,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int acc = 0;
             uint32_t acc_ph = 0;
             bool ok = true;
-            for (int t = cluster_id; t < total_tiles && ok; t += num_clusters) {
+            for (int k = 0; k < my_tiles && ok; ++k) {
                 Tile ti;
-                if (!decode_tile<C>(p, ctl, t, ti)) continue;
+                if (!tile_at(k, ti)) continue;
                 if (!wait_bounded(&tmem_empty[acc], acc_ph ^ 1u, s_abort, p.err)) break;
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -475,9 +516,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t tmem_empty_leader0 = PAIR ? map_shared_rank(smem_u32(&tmem_empty[0]), 0) : 0u;
         int acc = 0;
         uint32_t acc_ph = 0;
-        for (int t = cluster_id; t < total_tiles; t += num_clusters) {
+        for (int k = 0; k < my_tiles; ++k) {
             Tile ti;
-            if (!decode_tile<C>(p, ctl, t, ti)) continue;
+            if (!tile_at(k, ti)) continue;
             if (!warp_wait_bounded(&tmem_full[acc], acc_ph, s_abort, p.err, lane)) break;
             tc_fence_after_sync();
             const int r_local = my_rows + 32 * q + lane;
