@@ -555,7 +555,9 @@ int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const v
     const long long w1 = M_total / dg::BLOCK_M, w2 = (w1 + 1) / 2;
     // a 256-row window holds at most two tiles (its halves may belong to two groups)
     const long long bound = w2 + (w2 < G ? w2 : G);
-    const Plan plan{w1, w2, w1, bound, w1, w2, w2 <= dg::MAX_PAIR_WINDOWS};
+    // pairs need the device-built window list to fit (at most NB/2 + G/2 windows) and group ids below 2^15
+    const bool pair_ok = (w1 + G) / 2 + 1 <= dg::MAX_PAIR_WINDOWS && G <= 32767;
+    const Plan plan{w1, w2, w1, bound, w1, w2, pair_ok};
     return plan_and_launch(p, info, plan, a, M_total, b, static_cast<long long>(G) * N, sc,
                            reinterpret_cast<cudaStream_t>(stream));
 }

@@ -32,9 +32,9 @@
 // handed round-robin to the persistent CTAs (pairs).
 //   dense       ceil(M / 128*CTAS) windows.
 //   contiguous  CTAS = 1: M_total/128 blocks, group = m_indices[first row], -1 skips the block.
-//               CTAS = 2: 256-row windows over the 128-aligned segments; a window whose two halves belong to
-//               different groups becomes two tiles (one per group, each storing only its own rows).  The
-//               window table (tiles per window, prefix) is built on the device at kernel start.
+//               CTAS = 2: 256-row windows starting at each group's first block (two blocks of one group; the
+//               last window of a group with an odd block count computes, and does not store, one block of
+//               the next rows).  The window list is built on the device at kernel start.
 //   masked      per group ceil(masked_m[g] / 128*CTAS) windows, counted on the device, so the host never
 //               needs masked_m.
 // Each CTA decodes its tile sequence once at kernel start (all threads, into a shared-memory list), so no
@@ -139,8 +139,9 @@ struct Tile {
 
 struct SharedCtl {
     volatile int *abort;
-    const int *prefix;
-    const int *mm;
+    const int *prefix;   // masked: window prefix per group; contiguous pairs: first block of each window
+    const int *mm;       // masked: clamped masked_m
+    const short *gblk;   // contiguous pairs, kernel prologue only: group of each 128-row block
 };
 
 __device__ __forceinline__ void raise_error(unsigned *err, unsigned code) { atomicCAS(err, 0u, code); }
@@ -214,11 +215,9 @@ __device__ __forceinline__ bool decode_tile(const GemmParams &p, const SharedCtl
             ti.g = group_of_block(p, w);
             return ti.g >= 0;
         } else {
-            const int j = upper_index(ctl.prefix, p.num_windows, w);
-            const int k = w - ctl.prefix[j];
-            const int ga = group_of_block(p, 2 * j), gb = group_of_block(p, 2 * j + 1);
-            ti.row0 = ti.local_row0 = j * C::TILE_M;
-            ti.g = (k == 0 && ga >= 0) ? ga : gb;
+            const int b0 = ctl.prefix[w];  // first block of the window
+            ti.row0 = ti.local_row0 = b0 * BLOCK_M;
+            ti.g = ctl.gblk ? ctl.gblk[b0] : group_of_block(p, b0);  // the staged table exists only in the prologue
             return ti.g >= 0;
         }
     }
@@ -248,47 +247,67 @@ __device__ __forceinline__ bool unpack_tile(const GemmParams &p, uint2 e, Tile &
     return true;
 }
 
-// Builds the scheduler table in shared memory (one warp).
-//   masked: mm[g] = clamp(masked_m[g]); prefix[g] = sum_{h<g} ceil(mm[h] / TILE_M); prefix[G] = total.
-//   contiguous, CTA pair: prefix[j] = tiles in windows before j (a window holds 0, 1 or 2 tiles).
-template <class C>
-__device__ void build_schedule_table(const GemmParams &p, int *prefix, int *mm, int lane) {
-    const bool masked = p.mode == MODE_MASKED;
-    const int n = masked ? p.G : p.num_windows;
-    const int chunk = (n + 31) / 32;
-    const int begin = min(lane * chunk, n), end = min(begin + chunk, n);
-    auto count = [&](int i) {
-        if (masked) {
-            int m = __ldg(p.masked_m + i);
-            if (m < 0 || m > p.M) {
-                raise_error(p.err, ERR_BAD_GROUP);
-                m = m < 0 ? 0 : p.M;
-            }
-            mm[i] = m;
-            return (m + C::TILE_M - 1) / C::TILE_M;
-        }
-        const int ga = group_of_block(p, 2 * i), gb = group_of_block(p, 2 * i + 1);
-        return (ga >= 0 ? 1 : 0) + (gb >= 0 && gb != ga ? 1 : 0);
-    };
-    int local = 0;
-    for (int i = begin; i < end; ++i) {
-        const int c = count(i);
-        prefix[i] = c;  // per-entry count for now
-        local += c;
-    }
-    int incl = local;
+// Warp-wide exclusive prefix sum of one int per lane; *total receives the sum over the warp.
+__device__ __forceinline__ int warp_exclusive_sum(int v, int lane, int *total) {
+    int incl = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
+        const int u = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += u;
     }
-    int run = incl - local;
-    for (int i = begin; i < end; ++i) {
-        const int c = prefix[i];
-        prefix[i] = run;
-        run += c;
+    *total = __shfl_sync(0xffffffffu, incl, 31);
+    return incl - v;
+}
+
+// Masked layout (one warp, after mm[] holds the clamped masked_m): prefix[g] = windows of groups before g,
+// prefix[G] = all windows.
+template <class C>
+__device__ void build_masked_prefix(const GemmParams &p, int *prefix, const int *mm, int lane) {
+    const int chunk = (p.G + 31) / 32;
+    const int begin = min(lane * chunk, p.G), end = min(begin + chunk, p.G);
+    int local = 0;
+    for (int g = begin; g < end; ++g) local += (mm[g] + C::TILE_M - 1) / C::TILE_M;
+    int total;
+    int run = warp_exclusive_sum(local, lane, &total);
+    for (int g = begin; g < end; ++g) {
+        prefix[g] = run;
+        run += (mm[g] + C::TILE_M - 1) / C::TILE_M;
     }
-    if (lane == 31) prefix[n] = incl;
+    if (lane == 0) prefix[p.G] = total;
+}
+
+// Contiguous layout with CTA pairs (one warp, after gblk[] holds each 128-row block's group or -1): the
+// 256-row windows start at each group's first block and advance by two blocks inside the group's run, so a
+// window never spans two groups except the last window of a run with an odd number of blocks, whose second
+// half computes rows it does not store.  list[0..n) = first block of each window, list[MAX_PAIR_WINDOWS] = n.
+__device__ void build_pair_windows(int num_blocks, const short *gblk, int *list, int lane) {
+    const int chunk = (num_blocks + 31) / 32;
+    const int begin = min(lane * chunk, num_blocks), end = min(begin + chunk, num_blocks);
+    auto run_head = [&](int b) { return gblk[b] >= 0 && (b == 0 || gblk[b - 1] != gblk[b]); };
+    // the last run head at or before each chunk's start (inclusive max-scan of run heads)
+    int last = -1;
+    for (int b = begin; b < end; ++b)
+        if (run_head(b)) last = b;
+    int carried = last;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, carried, off);
+        if (lane >= off) carried = max(carried, u);
+    }
+    int head = __shfl_up_sync(0xffffffffu, carried, 1);
+    if (lane == 0) head = -1;
+    int count = 0;
+    for (int b = begin, h = head; b < end; ++b) {
+        if (run_head(b)) h = b;
+        if (gblk[b] >= 0 && ((b - h) & 1) == 0) ++count;
+    }
+    int total;
+    int pos = warp_exclusive_sum(count, lane, &total);
+    for (int b = begin, h = head; b < end; ++b) {
+        if (run_head(b)) h = b;
+        if (gblk[b] >= 0 && ((b - h) & 1) == 0 && pos < MAX_PAIR_WINDOWS) list[pos++] = b;
+    }
+    if (lane == 0) list[MAX_PAIR_WINDOWS] = min(total, MAX_PAIR_WINDOWS);
 }
 
 template <class C>
@@ -345,21 +364,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_alloc<CTAS>(s_tmem_base, TMEM_COLS);
         tmem_relinquish<CTAS>();
     }
-    if (warp == EPI_WARP0 && (p.mode == MODE_MASKED || (PAIR && p.mode == MODE_CONTIGUOUS)))
-        build_schedule_table<C>(p, s_prefix, s_mm, lane);
+    // Scheduler tables.  Loads first, by all threads (independent loads in flight together), into shared
+    // memory: masked_m, or the group of every 128-row block (staged in the A ring, unused until the producer
+    // starts); then one warp scans them.
+    const bool pair_contig = PAIR && p.mode == MODE_CONTIGUOUS;
+    short *s_gblk = reinterpret_cast<short *>(sA);
+    const int num_blocks = p.M / BLOCK_M;
+    if (p.mode == MODE_MASKED) {
+        for (int g = threadIdx.x; g < p.G; g += NUM_THREADS) {
+            int m = __ldg(p.masked_m + g);
+            if (m < 0 || m > p.M) {
+                raise_error(p.err, ERR_BAD_GROUP);
+                m = m < 0 ? 0 : p.M;
+            }
+            s_mm[g] = m;
+        }
+    } else if (pair_contig) {
+        for (int b = threadIdx.x; b < num_blocks; b += NUM_THREADS) s_gblk[b] = static_cast<short>(group_of_block(p, b));
+    }
+    __syncthreads();
+    if (warp == EPI_WARP0) {
+        if (p.mode == MODE_MASKED) build_masked_prefix<C>(p, s_prefix, s_mm, lane);
+        else if (pair_contig) build_pair_windows(num_blocks, s_gblk, s_prefix, lane);
+    }
     tc_fence_before_sync();
     __syncthreads();
     if constexpr (PAIR) cluster_sync();  // the peer's barriers exist before any cross-CTA signal
     tc_fence_after_sync();
     const uint32_t tmem_base = *s_tmem_base;
 
-    const SharedCtl ctl{s_abort, s_prefix, s_mm};
+    const SharedCtl ctl{s_abort, s_prefix, s_mm, s_gblk};
     const int nkb = p.K / BLOCK_K;
     int total_windows;
     if (p.mode == MODE_MASKED)
         total_windows = s_prefix[p.G];
-    else if (PAIR && p.mode == MODE_CONTIGUOUS)
-        total_windows = s_prefix[p.num_windows];
+    else if (pair_contig)
+        total_windows = s_prefix[MAX_PAIR_WINDOWS];
     else
         total_windows = p.num_windows;
     const int total_tiles = total_windows * p.num_n_blocks;
@@ -374,9 +414,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         s_tiles[k] = pack_tile(valid, ti);
     }
     __syncthreads();
+    const SharedCtl ctl_main{s_abort, s_prefix, s_mm, nullptr};  // the A ring is operand data from here on
     auto tile_at = [&](int k, Tile &ti) -> bool {
         if (k < TILE_LIST_CAP) return unpack_tile<C>(p, s_tiles[k], ti);
-        return decode_tile<C>(p, ctl, cluster_id + k * num_clusters, ti);
+        return decode_tile<C>(p, ctl_main, cluster_id + k * num_clusters, ti);
     };
 
     if (warp == 0) {
