@@ -96,6 +96,22 @@ int make_operand_map(CUtensorMap &map, const void *base, long long rows, int K, 
     return DG_OK;
 }
 
+// D, bf16 row-major [rows][N]: boxes of 32 rows x 32 columns (64-byte rows) with the 64-byte swizzle, the
+// layout the epilogue stages each chunk in.
+int make_output_map(CUtensorMap &map, void *base, long long rows, int N) {
+    EncodeTiledFn encode;
+    if (int rc = get_encode_fn(encode)) return rc;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", static_cast<int>(r));
+    return DG_OK;
+}
+
 // Packed scale atoms: rows of 128 32-bit words (512 bytes), boxes of `box_rows` atoms, no swizzle.
 int make_atom_map(CUtensorMap &map, const uint32_t *base, long long atoms, int box_rows) {
     EncodeTiledFn encode;
@@ -186,7 +202,8 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
         dg::pack_scales_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(pk);
         if ((e = cudaGetLastError()) != cudaSuccess) { rc = cuda_fail(e, "scale pack launch"); break; }
         // ---- tensor maps
-        CUtensorMap ta, tb, tsfa, tsfb;
+        CUtensorMap ta, tb, tsfa, tsfb, td;
+        if ((rc = make_output_map(td, p.d, a_rows, p.N))) break;
         if ((rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M))) break;
         if ((rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS))) break;
         if ((rc = make_atom_map(tsfa, pk.sfa_out, sfa_atoms, 1))) break;
@@ -232,7 +249,7 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
                             " scratch=%lld B\n",
                     p.mode, p.M, p.N, p.K, p.G, BN, C::STAGES, KPS, CTAS, cfg.gridDim.x, C::SMEM_BYTES, p.num_windows,
                     (pk.sfa_words + pk.sfb_words) * 4);
-        if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, tsfb, p)) != cudaSuccess) {
+        if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, tsfb, td, p)) != cudaSuccess) {
             rc = cuda_fail(e, "kernel launch");
             break;
         }
@@ -387,7 +404,8 @@ int launch_cfg_noalloc(const void *a, long long a_rows, const void *b, long long
     dg::pack_scales_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(pk);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "scale pack launch");
-    CUtensorMap ta, tb, tsfa, tsfb;
+    CUtensorMap ta, tb, tsfa, tsfb, td;
+    if (int rc = make_output_map(td, p.d, a_rows, p.N)) return rc;
     if (int rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M)) return rc;
     if (int rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS)) return rc;
     if (int rc = make_atom_map(tsfa, pk.sfa_out, sfa_atoms, 1)) return rc;
@@ -417,7 +435,7 @@ int launch_cfg_noalloc(const void *a, long long a_rows, const void *b, long long
         }
         if (grid > n) cfg.gridDim.x = static_cast<unsigned>(n * CTAS);
     }
-    if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, tsfb, p)) != cudaSuccess)
+    if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, tsfb, td, p)) != cudaSuccess)
         return cuda_fail(e, "kernel launch");
     return DG_OK;
 }

@@ -60,8 +60,9 @@ constexpr int SF_ATOM_WORDS = 128;  // a packed scale atom: 128 rows x one 32-bi
 constexpr int NUM_THREADS = 192;
 constexpr int EPI_WARP0 = 2;        // epilogue warps 2..5 (TMEM lane quarter = warp % 4)
 constexpr int MAX_MASKED_GROUPS = 1024;
-constexpr int MAX_PAIR_WINDOWS = 4096;  // contiguous layout with CTA pairs: M_total <= 4096 * 256
+constexpr int MAX_PAIR_WINDOWS = 2048;  // contiguous layout with CTA pairs: at most 2048 256-row windows
 constexpr int TILE_LIST_CAP = 1024;     // tiles per CTA decoded up front (further tiles are decoded on the fly)
+constexpr int EPI_CHUNK_BYTES = 32 * 32 * 2;  // one epilogue staging chunk: 32 rows x 32 bf16 columns
 constexpr int TMEM_COLS = 512;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s for any single wait
 constexpr int SMEM_LIMIT = 232448;                  // 227 KB of dynamic shared memory per CTA
@@ -101,7 +102,9 @@ struct Cfg {
     static constexpr int SF_COLS = 4 + 4 * SFB_ATOMS;             // TMEM columns of one stage's scales
     static constexpr int SF_TMEM_BASE = 2 * BN;                   // after the two accumulators
     static constexpr int TABLE_INTS = (CTAS == 2 ? MAX_PAIR_WINDOWS : MAX_MASKED_GROUPS) + 1;
-    static constexpr int FIXED_BYTES = 4 * TABLE_INTS + 4 * MAX_MASKED_GROUPS + 16 + 8 * TILE_LIST_CAP + 16 + 8 * 16 + 1024;
+    static constexpr int EPI_BYTES = 4 * 2 * EPI_CHUNK_BYTES;    // per epilogue warp: two staging chunks
+    static constexpr int FIXED_BYTES =
+        EPI_BYTES + 4 * TABLE_INTS + 4 * MAX_MASKED_GROUPS + 16 + 8 * TILE_LIST_CAP + 16 + 8 * 16 + 1024;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES - 8 * 2 * 8) / STAGE_BYTES;
     static constexpr int STAGES_TMEM = (TMEM_COLS - SF_TMEM_BASE) / SF_COLS;
     static constexpr int STAGES_MAX = STAGES_FIT < STAGES_TMEM ? STAGES_FIT : STAGES_TMEM;
@@ -110,7 +113,8 @@ struct Cfg {
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;
-    static constexpr int OFF_BAR = OFF_SF + STAGES * SF_BYTES;
+    static constexpr int OFF_EPI = OFF_SF + STAGES * SF_BYTES;    // 1024-aligned (64-byte swizzle atoms)
+    static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARRIERS * 8;   // tmem base, abort flag
     static constexpr int OFF_PREFIX = OFF_MISC + 16;               // int[TABLE_INTS]
     static constexpr int OFF_MM = OFF_PREFIX + 4 * TABLE_INTS;     // masked: clamped masked_m
@@ -124,7 +128,7 @@ struct Cfg {
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
     static_assert(A_BYTES1 % 1024 == 0 && B_BYTES1 % 1024 == 0, "swizzle atoms need 1024-byte alignment");
     static_assert(SF_GROUP % KPS == 0, "a stage must not straddle a scale group");
-    static_assert(OFF_A % 1024 == 0 && OFF_B % 1024 == 0 && OFF_SF % 512 == 0, "TMA destinations");
+    static_assert(OFF_A % 1024 == 0 && OFF_B % 1024 == 0 && OFF_SF % 512 == 0 && OFF_EPI % 512 == 0, "TMA buffers");
     static_assert(OFF_BAR % 8 == 0 && OFF_MISC % 8 == 0, "mbarriers need 8-byte alignment");
     static_assert(OFF_PREFIX % 4 == 0 && OFF_MM % 4 == 0 && OFF_TILES % 16 == 0, "tables");
 };
@@ -314,7 +318,7 @@ template <class C>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
-                    const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmap_d, const GemmParams p) {
     constexpr int BN = C::BN;
     constexpr int STAGES = C::STAGES;
     constexpr int CTAS = C::CTAS;
@@ -324,6 +328,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint8_t *sA = smem + C::OFF_A;
     uint8_t *sB = smem + C::OFF_B;
     uint8_t *sSF = smem + C::OFF_SF;
+    uint8_t *sEpi = smem + C::OFF_EPI;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *full = bars;                  // [STAGES] stage landed (the leader's counts both CTAs' bytes)
     uint64_t *empty = bars + STAGES;        // [STAGES] MMAs done with the stage (both CTAs, by commit)
@@ -359,6 +364,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tma_prefetch_desc(&tmap_b);
         tma_prefetch_desc(&tmap_sfa);
         tma_prefetch_desc(&tmap_sfb);
+        tma_prefetch_desc(&tmap_d);
     }
     if (warp == 1) {
         tmem_alloc<CTAS>(s_tmem_base, TMEM_COLS);
@@ -553,10 +559,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else {
         // ---------------------------------------------------------------- epilogue (warps 2..5)
+        // Each warp owns 32 rows (its TMEM lane quarter).  A 32-column chunk is converted to bf16 and, when all
+        // 32 rows belong to the call, staged in shared memory (64-byte rows, 16-byte chunks XOR-swizzled by
+        // (row / 2) % 4, the layout of a 64-byte-swizzle TMA box) and written by one TMA tensor store; rows and
+        // columns outside D are clipped by the store.  Warps with rows the call must not write store their
+        // owned rows directly.
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const uint32_t tmem_empty_leader0 = PAIR ? map_shared_rank(smem_u32(&tmem_empty[0]), 0) : 0u;
+        uint8_t *stage_buf = sEpi + (warp - EPI_WARP0) * 2 * EPI_CHUNK_BYTES;
         int acc = 0;
         uint32_t acc_ph = 0;
+        int chunk_count = 0;  // chunks this warp has staged (selects the staging buffer)
         for (int k = 0; k < my_tiles; ++k) {
             Tile ti;
             if (!tile_at(k, ti)) continue;
@@ -571,6 +584,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 valid = row < p.M && __ldg(p.m_indices + row) == ti.g;
             else
                 valid = ti.local_row0 + r_local < ctl.mm[ti.g];
+            // dense rows past M lie outside D and are clipped by the store
+            const bool tma_ok = p.mode == MODE_DENSE || __all_sync(0xffffffffu, valid);
             __nv_bfloat16 *out = p.d + static_cast<size_t>(row) * p.N + ti.n0;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
@@ -578,22 +593,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_row + 32 * c, r);
                 tmem_ld_wait_regs(r);
-                if (valid) {
+                uint32_t h[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                    h[j] = *reinterpret_cast<uint32_t *>(&v);
+                }
+                if (tma_ok) {
+                    uint8_t *buf = stage_buf + (chunk_count & 1) * EPI_CHUNK_BYTES;
+                    if (chunk_count >= 2) {
+                        if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
+                        __syncwarp();
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int sw = j ^ ((lane >> 1) & 3);
+                        *reinterpret_cast<uint4 *>(buf + lane * 64 + sw * 16) =
+                            make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmap_d, buf, ti.n0 + 32 * c, ti.row0 + my_rows + 32 * q);
+                        bulk_commit_group();
+                    }
+                    ++chunk_count;
+                } else if (valid) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int col = ti.n0 + 32 * c + 8 * j;
-                        if (col < p.N) {
-                            uint4 v;
-                            __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
-                            __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
-                            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
-                            __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
-                            v.x = *reinterpret_cast<uint32_t *>(&h0);
-                            v.y = *reinterpret_cast<uint32_t *>(&h1);
-                            v.z = *reinterpret_cast<uint32_t *>(&h2);
-                            v.w = *reinterpret_cast<uint32_t *>(&h3);
-                            *reinterpret_cast<uint4 *>(out + 32 * c + 8 * j) = v;
-                        }
+                        if (col < p.N)
+                            *reinterpret_cast<uint4 *>(out + 32 * c + 8 * j) =
+                                make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
                     }
                 }
             }
@@ -608,6 +639,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             acc ^= 1;
             if (acc == 0) acc_ph ^= 1u;
         }
+        if (lane == 0) bulk_wait_group_all();  // the tensor stores finish before the CTA's shared memory goes away
+        __syncwarp();
     }
 
     tc_fence_before_sync();
