@@ -73,8 +73,9 @@ DG_EXPORT int dg_get_num_sms(void);
  * README "Unaligned block sizes": M=256, N=7168 gives 112 tiles at 128x128 and 128 tiles at 128x112. */
 DG_EXPORT long long dg_num_tiles(long long M, long long N, int block_m, int block_n);
 
-/* The N tile the library picks for `num_m_blocks` 128-row blocks of an N-wide output on `num_sms` SMs:
- * the candidate with the fewest SM-waves weighted by tile width (README "Unaligned block sizes"). */
+/* The N tile the library picks for `num_m_blocks` 128-row single-CTA tiles of an N-wide output on `num_sms`
+ * SMs: the candidate (224, 192, 160, 128) minimising waves x (128 + BN), the operand rows a CTA loads per K
+ * block (README "Unaligned block sizes": wave quantisation on the SM count). */
 DG_EXPORT int dg_select_block_n(long long num_m_blocks, int N, int num_sms);
 
 /* Dense NT GEMM (README "Normal dense GEMMs", gemm_fp8_fp8_bf16_nt).

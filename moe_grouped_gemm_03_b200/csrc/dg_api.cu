@@ -285,6 +285,27 @@ int launch_bn(int bn, int ctas, const void *a, long long a_rows, const void *b, 
     return fail(DG_ERR_UNSUPPORTED, "no kernel instantiated for BN=%d with %d CTA(s) per tile", bn, ctas);
 }
 
+// Tile width for `windows` row windows (128 rows per CTA, `ctas` CTAs per tile) of an N-wide output on
+// `units` SMs or SM pairs.  The persistent kernel is bound by the operand bytes each CTA pulls per K block
+// (128 A rows + BN/ctas B rows), so a pass costs about waves x (128 + BN/ctas); wider tiles win unless they
+// add a wave (README "Unaligned block sizes": wave quantisation on the SM count).
+int select_block_n(long long windows, int N, int units, int ctas) {
+    if (units <= 0) units = 1;
+    if (windows <= 0) windows = 1;
+    int best = kCandidateBN[0];
+    long long best_cost = -1;
+    for (int bn : kCandidateBN) {
+        const long long tiles = windows * ((N + bn - 1) / bn);
+        const long long waves = (tiles + units - 1) / units;
+        const long long cost = waves * (dg::BLOCK_M + bn / ctas);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
+}
+
 // Shape and launch: picks single CTAs or CTA pairs, the tile width, and the persistent grid.
 //   sel1 / sel2:     128-row / 256-row windows the tile shape is chosen for (a hint for the masked layout)
 //   bound1 / bound2: the most 128-row / 256-row tiles the device may find (sizes the grid)
@@ -301,11 +322,13 @@ int plan_and_launch(dg::GemmParams p, const DeviceInfo &info, const Plan &plan, 
     if (g_pair_policy == 0) pair = false;
     if (g_pair_policy < 0 && pair) {
         // pairs pay once there is at least a wave of them
-        const int bn = dg_select_block_n(plan.sel2, p.N, sms / 2);
+        const int bn = select_block_n(plan.sel2, p.N, sms / 2, 2);
         pair = plan.sel2 * ((p.N + bn - 1) / bn) >= sms / 2;
     }
     const int units = pair ? sms / 2 : sms;
-    const int bn = dg_select_block_n(pair ? plan.sel2 : plan.sel1, p.N, units);
+    int bn = select_block_n(pair ? plan.sel2 : plan.sel1, p.N, units, pair ? 2 : 1);
+    static const int forced_bn = getenv("DG_BLOCK_N") ? atoi(getenv("DG_BLOCK_N")) : 0;  // tuning override
+    if (forced_bn > 0) bn = forced_bn;
     p.num_n_blocks = (p.N + bn - 1) / bn;
     p.num_windows = static_cast<int>(p.mode == dg::MODE_MASKED ? 0 : (pair ? plan.windows2 : plan.windows1));
     p.num_sf_groups = (p.K / dg::BLOCK_K + dg::SF_GROUP - 1) / dg::SF_GROUP;
@@ -494,24 +517,7 @@ long long dg_num_tiles(long long M, long long N, int block_m, int block_n) {
     return ((M + block_m - 1) / block_m) * ((N + block_n - 1) / block_n);
 }
 
-int dg_select_block_n(long long num_m_blocks, int N, int num_sms) {
-    if (num_sms <= 0) num_sms = 1;
-    if (num_m_blocks <= 0) num_m_blocks = 1;
-    // Time of a persistent pass ~ waves x per-tile time; a tile's time grows with its width plus a fixed
-    // cost (prologue, epilogue drain) worth about 32 columns.
-    int best = kCandidateBN[0];
-    long long best_cost = -1;
-    for (int bn : kCandidateBN) {
-        const long long tiles = num_m_blocks * ((N + bn - 1) / bn);
-        const long long waves = (tiles + num_sms - 1) / num_sms;
-        const long long cost = waves * (bn + 32);
-        if (best_cost < 0 || cost < best_cost) {
-            best_cost = cost;
-            best = bn;
-        }
-    }
-    return best;
-}
+int dg_select_block_n(long long num_m_blocks, int N, int num_sms) { return select_block_n(num_m_blocks, N, num_sms, 1); }
 
 const char *dg_last_error(void) { return g_last_error.c_str(); }
 
@@ -638,11 +644,11 @@ int dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void *b, const
     bool pair = sms >= 2;
     if (g_pair_policy == 0) pair = false;
     if (g_pair_policy < 0 && pair) {
-        const int bn2 = dg_select_block_n(w2, N, sms / 2);
+        const int bn2 = select_block_n(w2, N, sms / 2, 2);
         pair = w2 * ((N + bn2 - 1) / bn2) >= sms / 2;
     }
     const int units = pair ? sms / 2 : sms;
-    const int bn = dg_select_block_n(pair ? w2 : w1, N, units);
+    const int bn = select_block_n(pair ? w2 : w1, N, units, pair ? 2 : 1);
     p.num_n_blocks = (N + bn - 1) / bn;
     p.num_windows = static_cast<int>(pair ? w2 : w1);
     p.num_sf_groups = (K / dg::BLOCK_K + dg::SF_GROUP - 1) / dg::SF_GROUP;
