@@ -128,6 +128,18 @@ DG_EXPORT int dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void
  * sizes up to 256x256.) */
 DG_EXPORT int dg_set_cta_pair_policy(int policy);
 
+/* Testing aid for the bounded waits (no counterpart in the method; it exists so that the timeout path can be
+ * exercised without faulting or hanging a GPU).
+ *   limit_ns          limit of every mbarrier wait inside the GEMM kernel: 0 restores the default of 2 s,
+ *                     otherwise 1e6 .. 2e9 ns.  Stays in force for every later launch.
+ *   drop_first_stage  non-zero: the NEXT GEMM launch only (any entry point) leaves the first operand stage of its
+ *                     first CTA (or CTA pair) unloaded, so that CTA's tensor-core thread waits for data that never
+ *                     comes.  Its wait runs out after limit_ns, the CTA abandons its tiles (their rows of D are
+ *                     left unwritten), the other CTAs finish, and dg_check_device_error() returns
+ *                     DG_ERR_DEVICE_TIMEOUT.  The CUDA context stays usable.
+ * Process-wide, not thread-safe; call it between launches.  Returns DG_OK or DG_ERR_INVALID_ARG. */
+DG_EXPORT int dg_debug_bounded_wait(unsigned long long limit_ns, int drop_first_stage);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 DG_EXPORT const char *dg_last_error(void);
 

@@ -55,6 +55,7 @@ _SIGNATURES = {
     "dg_m_grouped_fp8_gemm_nt_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "dg_fp8_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_set_cta_pair_policy": (_I, [_I]),
+    "dg_debug_bounded_wait": (_I, [ctypes.c_ulonglong, _I]),
     "dg_last_error": (ctypes.c_char_p, []),
     "dg_check_device_error": (_I, [_P]),
 }
@@ -136,6 +137,12 @@ def select_block_n(num_m_blocks: int, N: int, num_sms: int) -> int:
 def set_cta_pair_policy(policy: int) -> int:
     """-1: library decides; 0: single-CTA 128-row tiles only; 1: 2-CTA 256-row tiles wherever possible."""
     return _lib.dg_set_cta_pair_policy(policy)
+
+
+def debug_bounded_wait(limit_ns: int = 0, drop_first_stage: bool = False) -> None:
+    """Testing aid: set the in-kernel wait limit (0 = default 2 s) and, optionally, make the next GEMM launch
+    leave one operand stage unloaded so a wait runs out and DG_ERR_DEVICE_TIMEOUT is recorded."""
+    _check(_lib.dg_debug_bounded_wait(int(limit_ns), 1 if drop_first_stage else 0))
 
 
 def check_device_error(stream=None) -> None:

@@ -150,6 +150,15 @@ int scratch_pool(int device, cudaMemPool_t &pool) {
 
 // ----------------------------------------------------------------------------------------------- launch
 int g_pair_policy = -1;  // -1: library decides; 0: single CTAs only; 1: CTA pairs whenever supported
+unsigned long long g_wait_limit_ns = dg::WAIT_LIMIT_NS;  // limit of every in-kernel wait
+bool g_drop_first_stage = false;  // testing aid: the next GEMM launch leaves one stage unloaded
+
+// Per-launch wait settings; the dropped stage applies to one launch only.
+void apply_wait_settings(dg::GemmParams &p) {
+    p.wait_limit_ns = g_wait_limit_ns;
+    p.skip_first_load = g_drop_first_stage ? 1 : 0;
+    g_drop_first_stage = false;
+}
 
 struct ScaleArgs {
     const float *sfa;
@@ -249,6 +258,7 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
                             " scratch=%lld B\n",
                     p.mode, p.M, p.N, p.K, p.G, BN, C::STAGES, KPS, CTAS, cfg.gridDim.x, C::SMEM_BYTES, p.num_windows,
                     (pk.sfa_words + pk.sfb_words) * 4);
+        apply_wait_settings(p);
         if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, tsfb, td, p)) != cudaSuccess) {
             rc = cuda_fail(e, "kernel launch");
             break;
@@ -458,6 +468,7 @@ int launch_cfg_noalloc(const void *a, long long a_rows, const void *b, long long
         }
         if (grid > n) cfg.gridDim.x = static_cast<unsigned>(n * CTAS);
     }
+    apply_wait_settings(p);
     if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, tsfb, td, p)) != cudaSuccess)
         return cuda_fail(e, "kernel launch");
     return DG_OK;
@@ -617,6 +628,14 @@ int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const void 
     const Plan plan{h1, h2, max1, max2, 0, 0, true};
     return plan_and_launch(p, info, plan, a, static_cast<long long>(G) * M_max, b, static_cast<long long>(G) * N, sc,
                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dg_debug_bounded_wait(unsigned long long limit_ns, int drop_first_stage) {
+    if (limit_ns != 0 && (limit_ns < 1000000ull || limit_ns > dg::WAIT_LIMIT_NS))
+        return fail(DG_ERR_INVALID_ARG, "limit_ns=%llu must be 0 or within [1 ms, 2 s]", limit_ns);
+    g_wait_limit_ns = limit_ns == 0 ? dg::WAIT_LIMIT_NS : limit_ns;
+    g_drop_first_stage = drop_first_stage != 0;
+    return DG_OK;
 }
 
 int dg_set_cta_pair_policy(int policy) {

@@ -64,7 +64,7 @@ constexpr int MAX_PAIR_WINDOWS = 2048;  // contiguous layout with CTA pairs: at 
 constexpr int TILE_LIST_CAP = 1024;     // tiles per CTA decoded up front (further tiles are decoded on the fly)
 constexpr int EPI_CHUNK_BYTES = 32 * 32 * 2;  // one epilogue staging chunk: 32 rows x 32 bf16 columns
 constexpr int TMEM_COLS = 512;
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s for any single wait
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // default limit of any single wait: 2 s
 constexpr int SMEM_LIMIT = 232448;                  // 227 KB of dynamic shared memory per CTA
 
 // device error word codes
@@ -83,6 +83,8 @@ struct GemmParams {
     const int *m_indices;
     const int *masked_m;
     unsigned *err;
+    unsigned long long wait_limit_ns;  // limit of any single wait
+    int skip_first_load;               // test hook: the first CTA (pair) never loads stage 0
 };
 
 template <int BN_, int CTAS_, int KPS_>
@@ -151,13 +153,14 @@ struct SharedCtl {
 __device__ __forceinline__ void raise_error(unsigned *err, unsigned code) { atomicCAS(err, 0u, code); }
 
 // Slow path of the bounded mbarrier wait.  false = gave up (this CTA is aborting).
-__device__ __noinline__ bool wait_bounded_slow(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err) {
+__device__ __noinline__ bool wait_bounded_slow(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err,
+                                               uint64_t limit) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
         if ((it & 3u) == 0) {
             if (*abort) return false;
-            if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+            if (global_timer_ns() - t0 > limit) {
                 *abort = 1;
                 raise_error(err, ERR_TIMEOUT);
                 return false;
@@ -166,17 +169,18 @@ __device__ __noinline__ bool wait_bounded_slow(uint64_t *bar, uint32_t parity, v
     }
 }
 
-__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err) {
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err,
+                                             uint64_t limit) {
     if (mbar_try_wait(bar, parity)) return true;
-    return wait_bounded_slow(bar, parity, abort, err);
+    return wait_bounded_slow(bar, parity, abort, err, limit);
 }
 
 // Whole-warp wait: lane 0 waits, the verdict is broadcast, and the warp leaves converged (the callers
 // follow with .sync.aligned tcgen05 instructions).
 __device__ __forceinline__ bool warp_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                                  unsigned *err, int lane) {
+                                                  unsigned *err, uint64_t limit, int lane) {
     int ok = 1;
-    if (lane == 0) ok = wait_bounded(bar, parity, abort, err) ? 1 : 0;
+    if (lane == 0) ok = wait_bounded(bar, parity, abort, err, limit) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;
@@ -435,6 +439,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t armed = 0, armed_ph = 0;  // stages armed at least once / parity of their last arming
             bool ok = true;
             const uint32_t full_leader0 = PAIR ? map_shared_rank(smem_u32(&full[0]), 0) : 0u;
+            // test hook: the first CTA (pair) starts its ring at stage 1, so stage 0 is never armed or loaded and
+            // the tensor-core thread's first wait runs out
+            if (p.skip_first_load && cluster_id == 0) s = 1;
             for (int k = 0; k < my_tiles && ok; ++k) {
                 Tile ti;
                 if (!tile_at(k, ti)) continue;
@@ -448,7 +455,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
                     const int nk = min(C::KPS, nkb - kb0);  // K blocks in this stage
                     const bool group_start = kb0 % SF_GROUP == 0;
-                    if (!wait_bounded(&empty[s], ph ^ 1u, s_abort, p.err)) { ok = false; break; }
+                    if (!wait_bounded(&empty[s], ph ^ 1u, s_abort, p.err, p.wait_limit_ns)) { ok = false; break; }
                     uint8_t *a_dst = sA + s * C::A_BYTES;
                     uint8_t *b_dst = sB + s * C::B_BYTES;
                     uint8_t *sf_dst = sSF + s * C::SF_BYTES;
@@ -486,13 +493,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
             }
-            if (!ok && (!PAIR || rank == 0)) {
-                // let the loads still in flight land before shared memory goes away (in a pair the bytes of
-                // both CTAs are counted on the leader's barrier; the final cluster barrier holds the peer)
+            if (!PAIR || rank == 0) {
+                // let the loads still in flight land before shared memory goes away, also when a consumer gave
+                // up on them (in a pair the bytes of both CTAs are counted on the leader's barrier; the final
+                // cluster barrier holds the peer).  On the normal path every armed phase has completed already.
                 for (int i = 0; i < STAGES; ++i) {
                     if (!(armed >> i & 1u)) continue;
                     const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(&full[i], (armed_ph >> i) & 1u) && global_timer_ns() - t0 < WAIT_LIMIT_NS) {
+                    while (!mbar_try_wait(&full[i], (armed_ph >> i) & 1u) && global_timer_ns() - t0 < p.wait_limit_ns) {
                     }
                 }
             }
@@ -509,13 +517,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int k = 0; k < my_tiles && ok; ++k) {
                 Tile ti;
                 if (!tile_at(k, ti)) continue;
-                if (!wait_bounded(&tmem_empty[acc], acc_ph ^ 1u, s_abort, p.err)) break;
+                if (!wait_bounded(&tmem_empty[acc], acc_ph ^ 1u, s_abort, p.err, p.wait_limit_ns)) break;
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
                 uint32_t sf_tmem = 0;
                 for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
                     const int nk = min(C::KPS, nkb - kb0);
-                    if (!wait_bounded(&full[s], ph, s_abort, p.err)) { ok = false; break; }
+                    if (!wait_bounded(&full[s], ph, s_abort, p.err, p.wait_limit_ns)) { ok = false; break; }
                     tc_fence_after_sync();
                     if (kb0 % SF_GROUP == 0) {
                         // the group's scales into this stage's TMEM slot (the slot's previous readers were
@@ -554,7 +562,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // all tensor-core work of the pair must be complete before TMEM is released
             tc_commit<CTAS>(drain);
             const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < WAIT_LIMIT_NS) {
+            while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < p.wait_limit_ns) {
             }
         }
     } else {
@@ -573,7 +581,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int k = 0; k < my_tiles; ++k) {
             Tile ti;
             if (!tile_at(k, ti)) continue;
-            if (!warp_wait_bounded(&tmem_full[acc], acc_ph, s_abort, p.err, lane)) break;
+            if (!warp_wait_bounded(&tmem_full[acc], acc_ph, s_abort, p.err, p.wait_limit_ns, lane)) break;
             tc_fence_after_sync();
             const int r_local = my_rows + 32 * q + lane;
             const int row = ti.row0 + r_local;

@@ -95,3 +95,11 @@ def test_grouped_validation():
     assert L.dg_m_grouped_fp8_gemm_nt_masked(*ok.values(), P(256), 4, 0, 256, 512, 128, None) == -1
     assert L.dg_m_grouped_fp8_gemm_nt_masked(*ok.values(), None, 4, 256, 256, 512, 128, None) == -1
     assert L.dg_m_grouped_fp8_gemm_nt_masked(*ok.values(), P(256), 4, 256, 250, 512, 128, None) == -2
+
+
+def test_debug_wait_limit_range():
+    """The wait-limit testing aid accepts 0 (default) or 1 ms .. 2 s, and needs no device."""
+    assert L.dg_debug_bounded_wait(ctypes.c_ulonglong(5), 0) == -1
+    assert L.dg_debug_bounded_wait(ctypes.c_ulonglong(3_000_000_000), 0) == -1
+    assert L.dg_debug_bounded_wait(ctypes.c_ulonglong(1_000_000), 0) == 0
+    assert L.dg_debug_bounded_wait(ctypes.c_ulonglong(0), 0) == 0
