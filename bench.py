@@ -139,7 +139,7 @@ def dist_setup(args):
         import torch.distributed as dist
 
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
@@ -159,9 +159,17 @@ def max_over_ranks(x, world):
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    device = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_throughput(flops_per_rank, local_ms, world):
+    """(slowest rank's ms per step, TFLOP/s of all ranks together): every rank runs its own replica of the
+    workload, so the job processes world x flops_per_rank per step in the slowest rank's time."""
+    ms = max_over_ranks(local_ms, world)
+    return ms, world * flops_per_rank / (ms * 1e-3) / 1e12
 
 
 def call_library(p, t, out):
@@ -285,8 +293,7 @@ def run_ours(args, world, rank, local):
     barrier(world)
     dg.check_device_error()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = max_over_ranks(statistics.mean(step_ms), world)
-    value = world * flops / (ms * 1e-3) / 1e12
+    ms, value = whole_job_throughput(flops, statistics.mean(step_ms), world)
 
     # end to end through the public API: pinned host inputs -> device, GEMM, result -> pinned host
     host = {k: v.cpu().pin_memory() for k, v in t.items()}
