@@ -166,6 +166,25 @@ struct ScaleArgs {
     const float *sfb;
 };
 
+// Launch of the scale pre-pass: one warp per atom, spread over every SM (one block each), so that every SM is
+// free for the GEMM (a programmatic dependent) at about the same time.  An SM running a pre-pass block takes no
+// GEMM CTA until that block is done (the pre-pass keeps the default shared-memory carveout).
+int launch_pack(const dg::PackParams &pk, int device, cudaStream_t stream) {
+    const long long atoms = (pk.sfa_words + pk.sfb_words) / dg::SF_ATOM_WORDS;
+    constexpr long long kMaxWarps = dg::PACK_THREADS / 32;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms <= 0) sms = 1;
+    long long blocks = atoms < sms ? atoms : sms;
+    if (blocks < 1) blocks = 1;
+    long long warps = (atoms + blocks - 1) / blocks;
+    if (warps > kMaxWarps) warps = kMaxWarps;
+    if (warps < 1) warps = 1;
+    dg::pack_scales_kernel<<<static_cast<unsigned>(blocks), static_cast<unsigned>(32 * warps), 0, stream>>>(pk);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "scale pack launch");
+    return DG_OK;
+}
+
 template <int BN, int CTAS, int KPS>
 int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows, const ScaleArgs &sc, dg::GemmParams p,
                int grid, int device, cudaStream_t stream) {
@@ -205,12 +224,7 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
     pk.sfb_out = pk.sfa_out + pk.sfa_words;
     int rc = DG_OK;
     do {
-        const long long total = pk.sfa_words + pk.sfb_words;
-        long long blocks = (total + 255) / 256;
-        if (blocks > 4096) blocks = 4096;
-        dg::pack_scales_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(pk);
-        if ((e = cudaGetLastError()) != cudaSuccess) { rc = cuda_fail(e, "scale pack launch"); break; }
-        // ---- tensor maps
+        // ---- tensor maps (all host work is done before the two launches, so they reach the GPU back to back)
         CUtensorMap ta, tb, tsfa, tsfb, td;
         if ((rc = make_output_map(td, p.d, a_rows, p.N))) break;
         if ((rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M))) break;
@@ -259,6 +273,7 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
                     p.mode, p.M, p.N, p.K, p.G, BN, C::STAGES, KPS, CTAS, cfg.gridDim.x, C::SMEM_BYTES, p.num_windows,
                     (pk.sfa_words + pk.sfb_words) * 4);
         apply_wait_settings(p);
+        if ((rc = launch_pack(pk, device, stream))) break;
         if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, tsfb, td, p)) != cudaSuccess) {
             rc = cuda_fail(e, "kernel launch");
             break;
@@ -431,12 +446,7 @@ int launch_cfg_noalloc(const void *a, long long a_rows, const void *b, long long
     if (int rc = noalloc_scratch(device, &scratch)) return rc;
     pk.sfa_out = scratch;
     pk.sfb_out = scratch + pk.sfa_words;  // every word of both regions is written by the pre-pass
-    const long long total = pk.sfa_words + pk.sfb_words;
-    long long blocks = (total + 255) / 256;
-    if (blocks > 4096) blocks = 4096;
-    dg::pack_scales_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(pk);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "scale pack launch");
+    cudaError_t e;
     CUtensorMap ta, tb, tsfa, tsfb, td;
     if (int rc = make_output_map(td, p.d, a_rows, p.N)) return rc;
     if (int rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M)) return rc;
@@ -469,6 +479,7 @@ int launch_cfg_noalloc(const void *a, long long a_rows, const void *b, long long
         if (grid > n) cfg.gridDim.x = static_cast<unsigned>(n * CTAS);
     }
     apply_wait_settings(p);
+    if (int rc = launch_pack(pk, device, stream)) return rc;
     if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, tsfb, td, p)) != cudaSuccess)
         return cuda_fail(e, "kernel launch");
     return DG_OK;

@@ -101,15 +101,17 @@ struct Cfg {
     static constexpr int B_BYTES = KPS * B_BYTES1;
     static constexpr int SF_BYTES = (1 + SFB_ATOMS) * SF_ATOM_WORDS * 4;  // SFA atom + SFB atoms
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SF_BYTES;
-    static constexpr int SF_COLS = 4 + 4 * SFB_ATOMS;             // TMEM columns of one stage's scales
+    static constexpr int SF_COLS = 4 + 4 * SFB_ATOMS;             // TMEM columns of one scale group's scales
     static constexpr int SF_TMEM_BASE = 2 * BN;                   // after the two accumulators
+    // scale slots in TMEM, used round-robin by successive scale groups (not by stages)
+    static constexpr int SF_SLOTS_FIT = (TMEM_COLS - SF_TMEM_BASE) / SF_COLS;
+    static constexpr int SF_SLOTS = SF_SLOTS_FIT > 4 ? 4 : SF_SLOTS_FIT;
     static constexpr int TABLE_INTS = (CTAS == 2 ? MAX_PAIR_WINDOWS : MAX_MASKED_GROUPS) + 1;
     static constexpr int EPI_BYTES = 4 * 2 * EPI_CHUNK_BYTES;    // per epilogue warp: two staging chunks
     static constexpr int FIXED_BYTES =
         EPI_BYTES + 4 * TABLE_INTS + 4 * MAX_MASKED_GROUPS + 16 + 8 * TILE_LIST_CAP + 16 + 8 * 16 + 1024;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES - 8 * 2 * 8) / STAGE_BYTES;
-    static constexpr int STAGES_TMEM = (TMEM_COLS - SF_TMEM_BASE) / SF_COLS;
-    static constexpr int STAGES_MAX = STAGES_FIT < STAGES_TMEM ? STAGES_FIT : STAGES_TMEM;
+    static constexpr int STAGES_MAX = STAGES_FIT;
     static constexpr int STAGES = STAGES_MAX > 8 ? 8 : STAGES_MAX;
     static constexpr int NUM_BARRIERS = 2 * STAGES + 5;
     static constexpr int OFF_A = 0;
@@ -126,7 +128,7 @@ struct Cfg {
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32, 256]");
     static_assert(B_ROWS % 8 == 0, "B tile rows must fill whole 8-row swizzle atoms");
     static_assert(STAGES >= 3, "pipeline too shallow");
-    static_assert(SF_TMEM_BASE + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
+    static_assert(SF_SLOTS >= 2 && SF_TMEM_BASE + SF_SLOTS * SF_COLS <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
     static_assert(A_BYTES1 % 1024 == 0 && B_BYTES1 % 1024 == 0, "swizzle atoms need 1024-byte alignment");
     static_assert(SF_GROUP % KPS == 0, "a stage must not straddle a scale group");
@@ -186,15 +188,19 @@ __device__ __forceinline__ bool warp_wait_bounded(uint64_t *bar, uint32_t parity
     return ok != 0;
 }
 
-__device__ __forceinline__ int group_of_block(const GemmParams &p, int block) {
-    const int row = block * BLOCK_M;
-    if (row >= p.M) return -1;
-    const int g = __ldg(p.m_indices + row);
+// A group id read from m_indices: -1 for padding; ids >= G are reported and treated as padding.
+__device__ __forceinline__ int checked_group(const GemmParams &p, int g) {
     if (g >= p.G) {
         raise_error(p.err, ERR_BAD_GROUP);
         return -1;
     }
     return g < 0 ? -1 : g;
+}
+
+__device__ __forceinline__ int group_of_block(const GemmParams &p, int block) {
+    const int row = block * BLOCK_M;
+    if (row >= p.M) return -1;
+    return checked_group(p, __ldg(p.m_indices + row));
 }
 
 // largest i in [0, n) with table[i] <= v, given table[0] <= v < table[n]
@@ -390,7 +396,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             s_mm[g] = m;
         }
     } else if (pair_contig) {
-        for (int b = threadIdx.x; b < num_blocks; b += NUM_THREADS) s_gblk[b] = static_cast<short>(group_of_block(p, b));
+        // several independent loads in flight per thread (m_indices is usually cold in L2 here)
+        constexpr int U = 8;
+        for (int b0 = threadIdx.x; b0 < num_blocks; b0 += NUM_THREADS * U) {
+            int g[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int b = b0 + u * NUM_THREADS;
+                g[u] = b < num_blocks ? __ldg(p.m_indices + static_cast<size_t>(b) * BLOCK_M) : -1;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int b = b0 + u * NUM_THREADS;
+                if (b < num_blocks) s_gblk[b] = static_cast<short>(checked_group(p, g[u]));
+            }
+        }
     }
     __syncthreads();
     if (warp == EPI_WARP0) {
@@ -433,12 +453,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
-            grid_dependency_wait();  // the packed scales come from the kernel launched just before
             int s = 0;
             uint32_t ph = 0;
             uint32_t armed = 0, armed_ph = 0;  // stages armed at least once / parity of their last arming
             bool ok = true;
             const uint32_t full_leader0 = PAIR ? map_shared_rank(smem_u32(&full[0]), 0) : 0u;
+            // The packed scale atoms come from the pre-pass launched just before this kernel.  The first STAGES
+            // stages' operand loads go out before waiting for it; their scale loads follow once it has finished
+            // (their barriers are armed with the scale bytes up front, so no stage completes without them).
+            auto load_scales = [&](int st, int ya, int yb) {
+                uint8_t *sf_dst = sSF + st * C::SF_BYTES;
+                if constexpr (PAIR) {
+                    const uint32_t leader_full = full_leader0 + 8u * static_cast<uint32_t>(st);
+                    tma_load_2d_pair(sf_dst, &tmap_sfa, leader_full, 0, ya);
+                    tma_load_2d_pair(sf_dst + SF_ATOM_WORDS * 4, &tmap_sfb, leader_full, 0, yb);
+                } else {
+                    tma_load_2d(sf_dst, &tmap_sfa, &full[st], 0, ya);
+                    tma_load_2d(sf_dst + SF_ATOM_WORDS * 4, &tmap_sfb, &full[st], 0, yb);
+                }
+            };
+            bool scales_ready = false;
+            int n_deferred = 0, issued = 0;
+            int def_stage[8], def_ya[8], def_yb[8];
+            static_assert(STAGES <= 8, "deferred scale loads are kept for at most 8 stages");
+            auto wait_for_scales = [&]() {
+                if (scales_ready) return;
+                grid_dependency_wait();
+                scales_ready = true;
+                for (int i = 0; i < n_deferred; ++i) load_scales(def_stage[i], def_ya[i], def_yb[i]);
+                n_deferred = 0;
+            };
             // test hook: the first CTA (pair) starts its ring at stage 1, so stage 0 is never armed or loaded and
             // the tensor-core thread's first wait runs out
             if (p.skip_first_load && cluster_id == 0) s = 1;
@@ -455,10 +499,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
                     const int nk = min(C::KPS, nkb - kb0);  // K blocks in this stage
                     const bool group_start = kb0 % SF_GROUP == 0;
+                    if (issued == STAGES) wait_for_scales();  // the ring is full: the MMAs need the scales now
                     if (!wait_bounded(&empty[s], ph ^ 1u, s_abort, p.err, p.wait_limit_ns)) { ok = false; break; }
                     uint8_t *a_dst = sA + s * C::A_BYTES;
                     uint8_t *b_dst = sB + s * C::B_BYTES;
-                    uint8_t *sf_dst = sSF + s * C::SF_BYTES;
                     const int q = kb0 / SF_GROUP;
                     const uint32_t bytes =
                         static_cast<uint32_t>(nk * (C::A_BYTES1 + C::B_BYTES1) + (group_start ? C::SF_BYTES : 0));
@@ -472,27 +516,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             tma_load_2d_pair(a_dst + i * C::A_BYTES1, &tmap_a, leader_full, (kb0 + i) * BLOCK_K, arow);
                             tma_load_2d_pair(b_dst + i * C::B_BYTES1, &tmap_b, leader_full, (kb0 + i) * BLOCK_K, brow);
                         }
-                        if (group_start) {
-                            tma_load_2d_pair(sf_dst, &tmap_sfa, leader_full, 0, sfa_y0 + q);
-                            tma_load_2d_pair(sf_dst + SF_ATOM_WORDS * 4, &tmap_sfb, leader_full, 0,
-                                             sfb_y0 + q * C::SFB_ATOMS);
-                        }
                     } else {
                         mbar_arrive_expect_tx(&full[s], bytes);
                         for (int i = 0; i < nk; ++i) {
                             tma_load_2d(a_dst + i * C::A_BYTES1, &tmap_a, &full[s], (kb0 + i) * BLOCK_K, arow);
                             tma_load_2d(b_dst + i * C::B_BYTES1, &tmap_b, &full[s], (kb0 + i) * BLOCK_K, brow);
                         }
-                        if (group_start) {
-                            tma_load_2d(sf_dst, &tmap_sfa, &full[s], 0, sfa_y0 + q);
-                            tma_load_2d(sf_dst + SF_ATOM_WORDS * 4, &tmap_sfb, &full[s], 0, sfb_y0 + q * C::SFB_ATOMS);
+                    }
+                    if (group_start) {
+                        if (scales_ready) {
+                            load_scales(s, sfa_y0 + q, sfb_y0 + q * C::SFB_ATOMS);
+                        } else {
+                            def_stage[n_deferred] = s;
+                            def_ya[n_deferred] = sfa_y0 + q;
+                            def_yb[n_deferred] = sfb_y0 + q * C::SFB_ATOMS;
+                            ++n_deferred;
                         }
                     }
+                    ++issued;
                     armed |= 1u << s;
                     armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
             }
+            wait_for_scales();  // (also after an abort: every armed stage gets all its bytes)
             if (!PAIR || rank == 0) {
                 // let the loads still in flight land before shared memory goes away, also when a consumer gave
                 // up on them (in a pair the bytes of both CTAs are counted on the leader's barrier; the final
@@ -513,6 +560,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t ph = 0;
             int acc = 0;
             uint32_t acc_ph = 0;
+            int sf_slot = 0;  // TMEM scale slot of the next scale group
             bool ok = true;
             for (int k = 0; k < my_tiles && ok; ++k) {
                 Tile ti;
@@ -526,9 +574,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     if (!wait_bounded(&full[s], ph, s_abort, p.err, p.wait_limit_ns)) { ok = false; break; }
                     tc_fence_after_sync();
                     if (kb0 % SF_GROUP == 0) {
-                        // the group's scales into this stage's TMEM slot (the slot's previous readers were
-                        // issued at least STAGES stages ago and the tensor pipe runs them in order)
-                        sf_tmem = tmem_base + static_cast<uint32_t>(C::SF_TMEM_BASE + s * C::SF_COLS);
+                        // the group's scales into the next TMEM slot (the slot's previous readers, the MMAs of
+                        // the group SF_SLOTS groups back, were issued earlier and the tensor pipe runs in order)
+                        sf_tmem = tmem_base + static_cast<uint32_t>(C::SF_TMEM_BASE + sf_slot * C::SF_COLS);
+                        if (++sf_slot == C::SF_SLOTS) sf_slot = 0;
                         const uint32_t sf_smem = smem_u32(sSF + s * C::SF_BYTES);
                         tc_cp_32x128b_warpx4<CTAS>(sf_tmem, sdesc_rows16_noswizzle(sf_smem));
 #pragma unroll

@@ -36,51 +36,64 @@ struct PackParams {
 
 __device__ __forceinline__ uint32_t ue8m0_code(float s) { return (__float_as_uint(s) >> 23) & 0xFFu; }
 
-__global__ void __launch_bounds__(256) pack_scales_kernel(const PackParams p) {
+// Most threads per block of the pre-pass (the host launches at most one block per SM).
+constexpr int PACK_THREADS = 1024;
+
+// One warp per atom: lane l builds the words of rows l, l+32, l+64, l+96 (words 4l .. 4l+3) and writes them
+// with one 16-byte store, so an atom is one coalesced 512-byte write.
+__global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackParams p) {
     grid_launch_dependents();  // the GEMM may start its prologue; it waits for this grid before reading
-    const long long total = p.sfa_words + p.sfb_words;
+    const long long sfa_atoms = p.sfa_words / SF_ATOM_WORDS;
+    const long long total = sfa_atoms + p.sfb_words / SF_ATOM_WORDS;
+    const int lane = threadIdx.x & 31;
+    const int warps_per_block = blockDim.x >> 5;
+    const long long num_warps = static_cast<long long>(gridDim.x) * warps_per_block;
     const int nnb128 = (p.N + 127) / 128;
-    for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
-         idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const int w = static_cast<int>(idx % SF_ATOM_WORDS);
-        const int r = (w >> 2) + 32 * (w & 3);  // atom row stored at word w
-        uint32_t word = 0;
-        if (idx < p.sfa_words) {
-            const long long atom = idx / SF_ATOM_WORDS;
+    for (long long atom = static_cast<long long>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5); atom < total;
+         atom += num_warps) {
+        uint32_t word[4] = {0u, 0u, 0u, 0u};
+        uint32_t *dst;
+        if (atom < sfa_atoms) {
             const int q = static_cast<int>(atom % p.num_sf_groups);
             const long long block = atom / p.num_sf_groups;
             const int g = static_cast<int>(block / p.blocks_per_group);
             const int lb = static_cast<int>(block % p.blocks_per_group);
-            const int row = lb * 128 + r;
             const float *base = p.sfa + static_cast<size_t>(g) * p.nkb * p.sfa_ld;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int kb = 4 * q + i;
-                const uint32_t code = (row < p.sfa_ld && row < p.rows_per_group && kb < p.nkb)
-                                          ? ue8m0_code(__ldg(base + static_cast<size_t>(kb) * p.sfa_ld + row))
-                                          : 0x7Fu;
-                word |= code << (8 * i);
-            }
-            p.sfa_out[idx] = word;
-        } else {
-            const long long j = idx - p.sfa_words;
-            long long atom = j / SF_ATOM_WORDS;
-            const int a = static_cast<int>(atom % p.sfb_atoms);
-            atom /= p.sfb_atoms;
-            const int q = static_cast<int>(atom % p.num_sf_groups);
-            atom /= p.num_sf_groups;
-            const int nt = static_cast<int>(atom % p.n_tiles);
-            const int g = static_cast<int>(atom / p.n_tiles);
-            const int n = nt * p.bn + a * 128 + r;
-            const float *base = p.sfb + (static_cast<size_t>(g) * nnb128 + n / 128) * p.nkb;
+            for (int j = 0; j < 4; ++j) {
+                const int row = lb * 128 + lane + 32 * j;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int kb = 4 * q + i;
-                const uint32_t code = (n < p.N && kb < p.nkb) ? ue8m0_code(__ldg(base + kb)) : 0x7Fu;
-                word |= code << (8 * i);
+                for (int i = 0; i < 4; ++i) {
+                    const int kb = 4 * q + i;
+                    const uint32_t code = (row < p.sfa_ld && row < p.rows_per_group && kb < p.nkb)
+                                              ? ue8m0_code(__ldg(base + static_cast<size_t>(kb) * p.sfa_ld + row))
+                                              : 0x7Fu;
+                    word[j] |= code << (8 * i);
+                }
             }
-            p.sfb_out[j] = word;
+            dst = p.sfa_out + atom * SF_ATOM_WORDS;
+        } else {
+            const long long b = atom - sfa_atoms;
+            const int a = static_cast<int>(b % p.sfb_atoms);
+            long long rest = b / p.sfb_atoms;
+            const int q = static_cast<int>(rest % p.num_sf_groups);
+            rest /= p.num_sf_groups;
+            const int nt = static_cast<int>(rest % p.n_tiles);
+            const int g = static_cast<int>(rest / p.n_tiles);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int n = nt * p.bn + a * 128 + lane + 32 * j;
+                const float *base = p.sfb + (static_cast<size_t>(g) * nnb128 + n / 128) * p.nkb;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int kb = 4 * q + i;
+                    const uint32_t code = (n < p.N && kb < p.nkb) ? ue8m0_code(__ldg(base + kb)) : 0x7Fu;
+                    word[j] |= code << (8 * i);
+                }
+            }
+            dst = p.sfb_out + b * SF_ATOM_WORDS;
         }
+        *reinterpret_cast<uint4 *>(dst + 4 * lane) = make_uint4(word[0], word[1], word[2], word[3]);
     }
 }
 
