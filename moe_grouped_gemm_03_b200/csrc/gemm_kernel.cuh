@@ -497,31 +497,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int sfa_y0 = sfa_block * p.num_sf_groups;
                 const int sfb_y0 = (ti.g * p.num_n_blocks + ti.nb) * p.num_sf_groups * C::SFB_ATOMS;
                 for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
-                    const int nk = min(C::KPS, nkb - kb0);  // K blocks in this stage
                     const bool group_start = kb0 % SF_GROUP == 0;
                     if (issued == STAGES) wait_for_scales();  // the ring is full: the MMAs need the scales now
                     if (!wait_bounded(&empty[s], ph ^ 1u, s_abort, p.err, p.wait_limit_ns)) { ok = false; break; }
                     uint8_t *a_dst = sA + s * C::A_BYTES;
                     uint8_t *b_dst = sB + s * C::B_BYTES;
                     const int q = kb0 / SF_GROUP;
+                    // one 3-D box per operand brings KPS K blocks (a block past K arrives zero-filled and unused)
                     const uint32_t bytes =
-                        static_cast<uint32_t>(nk * (C::A_BYTES1 + C::B_BYTES1) + (group_start ? C::SF_BYTES : 0));
+                        static_cast<uint32_t>(C::A_BYTES + C::B_BYTES + (group_start ? C::SF_BYTES : 0));
                     if constexpr (PAIR) {
                         // Only the leader arms the barrier (with both CTAs' bytes); the peer's loads just count
                         // their bytes on it.  A peer load may land before the leader arms the phase: the
                         // transaction count dips below zero but the phase cannot complete before the arrival.
                         const uint32_t leader_full = full_leader0 + 8u * static_cast<uint32_t>(s);
                         if (rank == 0) mbar_arrive_expect_tx(&full[s], CTAS * bytes);
-                        for (int i = 0; i < nk; ++i) {
-                            tma_load_2d_pair(a_dst + i * C::A_BYTES1, &tmap_a, leader_full, (kb0 + i) * BLOCK_K, arow);
-                            tma_load_2d_pair(b_dst + i * C::B_BYTES1, &tmap_b, leader_full, (kb0 + i) * BLOCK_K, brow);
-                        }
+                        tma_load_3d_pair(a_dst, &tmap_a, leader_full, 0, arow, kb0);
+                        tma_load_3d_pair(b_dst, &tmap_b, leader_full, 0, brow, kb0);
                     } else {
                         mbar_arrive_expect_tx(&full[s], bytes);
-                        for (int i = 0; i < nk; ++i) {
-                            tma_load_2d(a_dst + i * C::A_BYTES1, &tmap_a, &full[s], (kb0 + i) * BLOCK_K, arow);
-                            tma_load_2d(b_dst + i * C::B_BYTES1, &tmap_b, &full[s], (kb0 + i) * BLOCK_K, brow);
-                        }
+                        tma_load_3d(a_dst, &tmap_a, &full[s], 0, arow, kb0);
+                        tma_load_3d(b_dst, &tmap_b, &full[s], 0, brow, kb0);
                     }
                     if (group_start) {
                         if (scales_ready) {
