@@ -14,6 +14,9 @@ deep_gemm wrapper API list).  This module only selects rows and marshals pointer
 Grouped layouts (same README, "Grouped GEMMs (contiguous layout)" / "(masked layout)"):
 * contiguous: row m belongs to group m_indices[m]; rows with m_indices == -1 are padding and produce nothing.
 * masked: group g owns rows 0 .. masked_m[g]-1 of its [M_max, K] slab; the other rows produce nothing.
+* no padding (same README, "Grouped GEMMs (nopad layout)"): the groups' rows are concatenated in group order
+  with no alignment; group g owns rows off_g .. off_g + counts[g] - 1 with off_g = counts[0] + ... +
+  counts[g-1]; rows past the sum of the counts produce nothing.
 Rows that produce nothing are returned as NaN (the "left untouched" sentinel).
 """
 from __future__ import annotations
@@ -142,3 +145,18 @@ def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, masked_m):
     out = np.full((G * M_max, N), np.nan)
     out[rows] = gemm_rows(a.reshape(G * M_max, K), g * nkb * Ma + rows - g * M_max, Ma, sfa, b, sfb, rows, g, N, K)
     return out.reshape(G, M_max, N)
+
+
+def m_grouped_fp8_gemm_nt_nopad(a, sfa, b, sfb, counts):
+    """a [M_total,K], sfa [K/128, >=M_total], b [G,N,K], sfb [G, ceil(N/128), K/128], counts [G]
+    (sum(counts) <= M_total)."""
+    M, K = a.shape
+    G, N, _ = b.shape
+    counts = np.asarray(counts, np.int64)
+    off = np.concatenate([[0], np.cumsum(counts)[:-1]])
+    rows = np.concatenate([off[g] + np.arange(counts[g]) for g in range(G)]).astype(np.int64)
+    groups = np.concatenate([np.full(counts[g], g) for g in range(G)]).astype(np.int32)
+    out = np.full((M, N), np.nan)
+    if len(rows):
+        out[rows] = gemm_rows(a, rows, sfa.shape[1], sfa, b, sfb, rows, groups, N, K)
+    return out

@@ -2,7 +2,7 @@
 
 This module only *prepares inputs*: it draws fp32 N(0,1) data from ``numpy.random.default_rng(seed)``,
 quantises it to OCP e4m3 with power-of-two (UE8M0-representable) scales, and builds the grouping metadata
-(``m_indices`` / ``masked_m``).  It holds none of the GEMM arithmetic.  Both the CPU oracle and the CUDA
+(``m_indices`` / ``masked_m`` / per-group ``counts``).  It holds none of the GEMM arithmetic.  Both the CPU oracle and the CUDA
 path consume what it returns, and neither is imported here.
 
 Recipe (fine-grained scaling, "FP8 GEMM kernels with fine-grained scaling", DeepGEMM-for-PPU README,
@@ -14,8 +14,10 @@ Recipe (fine-grained scaling, "FP8 GEMM kernels with fine-grained scaling", Deep
 * q = e4m3_RNE(x / s) (torch's fp32 -> float8_e4m3fn cast, round-to-nearest-even; |x / s| <= 448).
 * sfa is stored MN-major ("LHS scale TMA-aligned and transposed"): [K/128][align4(rows)] fp32
   (masked: [G][K/128][align4(M_max)]).  sfb is [G][ceil(N/128)][K/128] fp32.
-* Rows that no group owns (contiguous padding, masked rows >= masked_m[g]) hold garbage: random bytes,
-  e4m3 NaN codes included, with random power-of-two scales.
+* Rows that no group owns (contiguous padding, masked rows >= masked_m[g], no-padding rows past the sum of
+  the counts) hold garbage: random bytes, e4m3 NaN codes included, with random power-of-two scales.
+* No-padding layout ("Grouped GEMMs (nopad layout)"): the groups' rows are concatenated in group order with
+  no alignment; group g owns rows off_g .. off_g + counts[g] - 1, off_g = counts[0] + ... + counts[g-1].
 
 Draw order per problem: group sizes (or masked_m) -> A fp32 -> B fp32 (group by group) -> garbage.
 """
@@ -44,17 +46,18 @@ def tma_aligned_rows(rows: int) -> int:
 class Problem:
     """One GEMM problem in the layouts the library takes.
 
-    kind       'dense' | 'contiguous' | 'masked'
+    kind       'dense' | 'contiguous' | 'masked' | 'nopad'
     a          uint8 e4m3 codes, [rows, K]; masked: [G * M_max, K] (= [G, M_max, K] flattened)
     sfa        fp32, dense/contiguous [K/128, align4(rows)]; masked [G, K/128, align4(M_max)]
     b          uint8 e4m3 codes, [G, N, K] (G = 1 for dense)
     sfb        fp32, [G, ceil(N/128), K/128]
     m_indices  int32 [rows] (contiguous only): group id of each row, -1 for padding rows
     masked_m   int32 [G] (masked only): number of valid rows of each group
+    counts     int32 [G]: contiguous -- valid rows per group (metadata); nopad -- the call's per-group row counts
     """
 
     kind: str
-    M: int  # dense: M; contiguous: M_total (padded); masked: M_max
+    M: int  # dense: M; contiguous: M_total (padded); masked: M_max; nopad: M_total (>= sum of counts)
     N: int
     K: int
     G: int
@@ -78,6 +81,8 @@ class Problem:
             return np.arange(self.M, dtype=np.int64)
         if self.kind == "contiguous":
             return np.nonzero(self.m_indices >= 0)[0].astype(np.int64)
+        if self.kind == "nopad":
+            return np.arange(int(np.sum(self.counts, dtype=np.int64)), dtype=np.int64)
         out = [g * self.M + np.arange(int(self.masked_m[g]), dtype=np.int64) for g in range(self.G)]
         return np.concatenate(out) if out else np.zeros(0, np.int64)
 
@@ -86,6 +91,9 @@ class Problem:
             return np.zeros(len(rows), np.int32)
         if self.kind == "contiguous":
             return self.m_indices[rows].astype(np.int32)
+        if self.kind == "nopad":
+            ends = np.cumsum(np.asarray(self.counts, np.int64))
+            return np.searchsorted(ends, rows, side="right").astype(np.int32)
         return (rows // self.M).astype(np.int32)
 
     def flops(self) -> int:
@@ -211,6 +219,26 @@ def make_contiguous(counts: Sequence[int], N: int, K: int, seed: int = 0, name: 
                    counts=counts.astype(np.int32), name=name or f"contiguous G={G} N={N} K={K}")
 
 
+def make_nopad(counts: Sequence[int], N: int, K: int, seed: int = 0, extra_rows: int = 0, name: str = "",
+               rng: Optional[np.random.Generator] = None) -> Problem:
+    """Groups' rows concatenated with no padding, then ``extra_rows`` rows that no group owns (garbage)."""
+    rng = rng if rng is not None else np.random.default_rng(seed)
+    counts = np.asarray(counts, np.int64)
+    assert (counts >= 0).all()
+    G = len(counts)
+    valid = int(counts.sum())
+    M_total = valid + int(extra_rows)
+    codes = np.zeros((M_total, K), np.uint8)
+    sfa = np.ones((K // SCALE_BLOCK, tma_aligned_rows(max(M_total, 1))), np.float32)
+    qa, s = quantize_rows(_draw_normal(rng, (valid, K)))
+    codes[:valid] = qa
+    sfa[:, :valid] = s.T
+    b, sfb = _quantize_b(rng, G, N, K)
+    _garbage_rows(rng, codes, sfa, np.arange(valid, M_total))
+    return Problem("nopad", M_total, N, K, G, codes, sfa, b, sfb, counts=counts.astype(np.int32),
+                   name=name or f"nopad G={G} N={N} K={K}")
+
+
 def make_masked(G: int, M_max: int, N: int, K: int, masked_m: Optional[Sequence[int]] = None,
                 seed: int = 0, expected_m: int = 0, name: str = "") -> Problem:
     """[G, M_max, K] activations; rows >= masked_m[g] of each group are garbage and must stay unwritten.
@@ -246,13 +274,14 @@ def zipf_counts(total: int, G: int, s: float) -> np.ndarray:
     return counts
 
 
-# The five workloads (all seed 0).
+# The five workloads (all seed 0), and as 6 the no-padding layout of workload 5's token split.
 CONFIGS = {
     1: "dense FP8 NT GEMM M=128 N=256 K=512",
     2: "dense FP8 NT GEMM M=4096 N=7168 K=7168",
     3: "M-grouped contiguous FP8 GEMM G=8 N=4096 K=7168, tokens U[1024,8192] per group",
     4: "M-grouped masked FP8 GEMM G=32 M_max=256 N=7168 K=2048, masked_m U[0,256], expected_m=128",
     5: "M-grouped contiguous FP8 GEMM G=64 N=7168 K=2048, Zipf(1.2) split of 65536 tokens",
+    6: "M-grouped no-padding FP8 GEMM G=64 N=7168 K=2048, Zipf(1.2) split of 65536 tokens",
 }
 
 
@@ -270,6 +299,9 @@ def make_config(i: int, seed: int = 0) -> Problem:
     if i == 5:
         rng = np.random.default_rng(seed)
         return make_contiguous(zipf_counts(65536, 64, 1.2), 7168, 2048, rng=rng, name=CONFIGS[5])
+    if i == 6:
+        rng = np.random.default_rng(seed)
+        return make_nopad(zipf_counts(65536, 64, 1.2), 7168, 2048, rng=rng, name=CONFIGS[6])
     raise ValueError(f"unknown config {i}")
 
 
@@ -289,4 +321,6 @@ def to_torch(p: Problem, device="cuda"):
         out["masked_m"] = t(p.masked_m)
     if p.kind == "contiguous":
         out["m_indices"] = t(p.m_indices)
+    if p.kind == "nopad":
+        out["counts"] = t(p.counts)
     return out

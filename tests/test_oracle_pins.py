@@ -181,6 +181,47 @@ def test_masked_equals_per_group_dense_and_leaves_rows_untouched():
         assert np.isnan(full[g, mm:]).all()
 
 
+def test_nopad_equals_per_group_dense_and_leaves_tail_untouched():
+    """No-padding layout: group g's rows off_g .. off_g + counts[g] - 1 equal a dense GEMM of exactly those rows
+    with B_g; a zero-count group owns no row; rows past the sum of the counts stay untouched."""
+    counts = [130, 1, 0, 256, 77]
+    p = synth.make_nopad(counts, N=256, K=256, seed=16, extra_rows=9)
+    full = oracle.problem_full(p)
+    off = np.concatenate([[0], np.cumsum(counts)])
+    for g, c in enumerate(counts):
+        if c == 0:
+            continue
+        s = off[g]
+        sfa = np.ascontiguousarray(p.sfa[:, s:s + synth.tma_aligned_rows(c)])
+        dense = oracle.fp8_gemm_nt(p.a[s:s + c], sfa, p.b[g], p.sfb[g])
+        np.testing.assert_array_equal(full[s:s + c], dense)
+    assert np.isnan(full[off[-1]:]).all() and not np.isnan(full[:off[-1]]).any()
+
+
+def test_nopad_equals_contiguous_layout_of_the_same_rows():
+    """The same tokens in the padded contiguous layout give the same products row for row."""
+    counts = [3, 129, 128, 0, 200]
+    q = synth.make_nopad(counts, N=128, K=256, seed=17)
+    padded = [synth.align_up(c, 128) for c in counts]
+    starts = np.concatenate([[0], np.cumsum(padded)])
+    M_total = int(starts[-1])
+    a = np.zeros((M_total, q.K), np.uint8)
+    sfa = np.ones((q.K // 128, synth.tma_aligned_rows(M_total)), np.float32)
+    m_indices = np.full(M_total, -1, np.int32)
+    src = 0
+    for g, c in enumerate(counts):
+        a[starts[g]:starts[g] + c] = q.a[src:src + c]
+        sfa[:, starts[g]:starts[g] + c] = q.sfa[:, src:src + c]
+        m_indices[starts[g]:starts[g] + c] = g
+        src += c
+    contig = oracle.m_grouped_fp8_gemm_nt_contiguous(a, sfa, q.b, q.sfb, m_indices)
+    nopad = oracle.problem_full(q)
+    src = 0
+    for g, c in enumerate(counts):
+        np.testing.assert_array_equal(nopad[src:src + c], contig[starts[g]:starts[g] + c])
+        src += c
+
+
 def test_library_call_shapes_agree_with_problem_driver():
     p = synth.make_masked(G=3, M_max=64, N=128, K=128, masked_m=[3, 64, 0], seed=8)
     a = p.a.reshape(p.G, p.M, p.K)
@@ -190,3 +231,7 @@ def test_library_call_shapes_agree_with_problem_driver():
     q = synth.make_contiguous([5, 200], N=128, K=128, seed=9)
     got = oracle.m_grouped_fp8_gemm_nt_contiguous(q.a, q.sfa, q.b, q.sfb, q.m_indices)
     np.testing.assert_array_equal(np.nan_to_num(got), np.nan_to_num(oracle.problem_full(q)))
+    r = synth.make_nopad([7, 0, 140], N=128, K=128, seed=10, extra_rows=3)
+    got = oracle.m_grouped_fp8_gemm_nt_nopad(r.a, r.sfa, r.b, r.sfb, r.counts)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(oracle.problem_full(r)))
+    np.testing.assert_array_equal(np.nan_to_num(got), np.nan_to_num(oracle.problem_full(r)))

@@ -59,6 +59,14 @@ def test_contiguous_layout():
     assert (p.a[3:128, 0] == 0x7F).all()
 
 
+def test_nopad_layout():
+    p = synth.make_nopad([3, 0, 130], N=128, K=256, seed=1, extra_rows=5)
+    assert p.rows == 138 and p.sfa.shape == (2, 140) and p.sfb.shape == (3, 1, 2)
+    np.testing.assert_array_equal(p.valid_rows(), np.arange(133))
+    np.testing.assert_array_equal(p.row_groups(np.array([0, 2, 3, 132])), [0, 0, 2, 2])
+    assert (p.a[133:, 0] == 0x7F).all() and p.flops() == 2 * 133 * 128 * 256
+
+
 def test_masked_layout():
     p = synth.make_masked(G=2, M_max=10, N=128, K=256, masked_m=[0, 10], seed=1)
     assert p.a.shape == (20, 256) and p.sfa.shape == (2, 2, 12) and p.sfb.shape == (2, 1, 2)
