@@ -53,7 +53,8 @@ typedef enum {
     DG_ERR_UNSUPPORTED = -3,   /* device is not sm_100, or a shape outside the supported set */
     DG_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed */
     DG_ERR_DEVICE_TIMEOUT = -5,/* (device error word) a bounded wait inside the kernel ran out */
-    DG_ERR_BAD_GROUP = -6      /* (device error word) a group id outside [-1, G) or masked_m outside [0, M_max] */
+    DG_ERR_BAD_GROUP = -6      /* (device error word) a group id outside [-1, G), masked_m outside [0, M_max],
+                                  or no-padding counts that are negative or sum past M_total */
 } dg_status;
 
 /* Per-segment M padding of the contiguous layout: each group's rows start on a multiple of this (128).
@@ -103,6 +104,19 @@ DG_EXPORT int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sf
 DG_EXPORT int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const void *b, const float *sfb,
                                     void *d, const int *masked_m, int G, int M_max, int N, int K,
                                     int expected_m, dg_stream_t stream);
+
+/* M-grouped GEMM, no-padding layout (README "Grouped GEMMs (nopad layout)": a per-group token count replaces
+ * the alignment of each group's rows to the M block).
+ *   a [M_total][K] e4m3: group g's rows are off_g .. off_g + counts[g] - 1, off_g = counts[0] + ... +
+ *     counts[g-1] (groups in order, no gaps, no alignment); rows from sum(counts) to M_total - 1 belong to no
+ *     group.  sfa [K/128][ld(M_total)] (as for the dense call), b [G][N][K] e4m3, sfb [G][ceil(N/128)][K/128].
+ *   counts int32 [G] on the device; the host never reads it.
+ *   d [M_total][N] bf16: rows no group owns are left untouched.
+ *   Negative counts count as 0; counts whose sum exceeds M_total are clipped at row M_total.  Both are
+ *   reported by dg_check_device_error() as DG_ERR_BAD_GROUP.  1 <= G <= 1024; M_total has no alignment
+ *   requirement (0 launches nothing). */
+DG_EXPORT int dg_m_grouped_fp8_gemm_nt_nopad(const void *a, const float *sfa, const void *b, const float *sfb,
+                                   void *d, const int *counts, int M_total, int N, int K, int G, dg_stream_t stream);
 
 /* Dense NT GEMM that allocates no device memory (the pages have no counterpart: it exists for callers of this
  * library).  Same arguments, layouts, validation and results as dg_fp8_gemm_nt.  dg_fp8_gemm_nt takes a small

@@ -53,6 +53,7 @@ _SIGNATURES = {
     "dg_fp8_gemm_nt": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_gemm_nt_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_gemm_nt_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "dg_m_grouped_fp8_gemm_nt_nopad": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_fp8_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_set_cta_pair_policy": (_I, [_I]),
     "dg_debug_bounded_wait": (_I, [ctypes.c_ulonglong, _I]),
@@ -229,8 +230,30 @@ def m_grouped_fp8_gemm_nt_masked(lhs, rhs, out: torch.Tensor, masked_m: torch.Te
                                                 G, M_max, N, K, int(expected_m), _stream()))
 
 
+def m_grouped_fp8_gemm_nt_nopad(lhs, rhs, out: torch.Tensor, counts: torch.Tensor) -> None:
+    """No-padding layout: group g's rows are off_g .. off_g + counts[g] - 1 (off_g = sum of the earlier counts);
+    out rows of group g = lhs rows of group g @ rhs[g]^T; rows past sum(counts) are untouched."""
+    a, sfa = lhs
+    b, sfb = rhs
+    _check_operand("a", a, 2, _FP8_TYPES)
+    _check_operand("b", b, 3, _FP8_TYPES)
+    _check_operand("sfa", sfa, 2, (torch.float32,))
+    _check_operand("sfb", sfb, 3, (torch.float32,))
+    _check_operand("out", out, 2, (torch.bfloat16,))
+    _check_operand("counts", counts, 1, (torch.int32,))
+    M, K = a.shape
+    G, N, _ = b.shape
+    _need(b.shape[2] == K and tuple(out.shape) == (M, N) and counts.shape[0] == G, "shape mismatch")
+    _need(sfa.shape[0] == K // 128 and sfa.shape[1] == get_tma_aligned_size(M, 4),
+          "sfa must be [K/128, tma_aligned(M_total)]")
+    _need(sfb.shape == (G, (N + 127) // 128, K // 128), "sfb must be [G, ceil(N/128), K/128]")
+    _check(_lib.dg_m_grouped_fp8_gemm_nt_nopad(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(out), _ptr(counts),
+                                               M, N, K, G, _stream()))
+
+
 __all__ = [
     "DGError", "fp8_gemm_nt", "fp8_gemm_nt_noalloc", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
+    "m_grouped_fp8_gemm_nt_nopad",
     "get_m_alignment_for_contiguous_layout", "get_tma_aligned_size", "set_num_sms", "get_num_sms", "num_tiles",
     "select_block_n", "set_cta_pair_policy", "check_device_error", "lib", "header_symbols", "last_error",
 ]

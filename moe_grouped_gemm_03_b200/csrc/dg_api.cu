@@ -207,10 +207,18 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
     pk.sfb_atoms = C::SFB_ATOMS;
     pk.nkb = nkb;
     pk.num_sf_groups = p.num_sf_groups;
+    pk.mode = p.mode;
+    pk.counts = p.masked_m;
+    pk.tile_m = C::TILE_M;
     if (p.mode == dg::MODE_MASKED) {
         pk.rows_per_group = p.M;
         pk.blocks_per_group = p.sfa_blocks;
         pk.sfa_groups = p.G;
+    } else if (p.mode == dg::MODE_NOPAD) {
+        // every group's windows, at most ceil(M_total / TILE_M) + G of them, CTAS blocks each
+        pk.rows_per_group = p.M;
+        pk.blocks_per_group = CTAS * ((p.M + C::TILE_M - 1) / C::TILE_M + p.G);
+        pk.sfa_groups = 1;
     } else {
         pk.rows_per_group = p.M;
         pk.blocks_per_group = (p.M + dg::BLOCK_M - 1) / dg::BLOCK_M;
@@ -360,7 +368,8 @@ int plan_and_launch(dg::GemmParams p, const DeviceInfo &info, const Plan &plan, 
     static const int forced_bn = getenv("DG_BLOCK_N") ? atoi(getenv("DG_BLOCK_N")) : 0;  // tuning override
     if (forced_bn > 0) bn = forced_bn;
     p.num_n_blocks = (p.N + bn - 1) / bn;
-    p.num_windows = static_cast<int>(p.mode == dg::MODE_MASKED ? 0 : (pair ? plan.windows2 : plan.windows1));
+    const bool device_windows = p.mode == dg::MODE_MASKED || p.mode == dg::MODE_NOPAD;  // counted by the kernel
+    p.num_windows = static_cast<int>(device_windows ? 0 : (pair ? plan.windows2 : plan.windows1));
     p.num_sf_groups = (p.K / dg::BLOCK_K + dg::SF_GROUP - 1) / dg::SF_GROUP;
     const long long tiles = (pair ? plan.bound2 : plan.bound1) * p.num_n_blocks;
     const int grid = static_cast<int>(tiles < units ? tiles : units);
@@ -652,6 +661,34 @@ int dg_debug_bounded_wait(unsigned long long limit_ns, int drop_first_stage) {
     g_wait_limit_ns = limit_ns == 0 ? dg::WAIT_LIMIT_NS : limit_ns;
     g_drop_first_stage = drop_first_stage != 0;
     return DG_OK;
+}
+
+int dg_m_grouped_fp8_gemm_nt_nopad(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
+                                   const int *counts, int M_total, int N, int K, int G, dg_stream_t stream) {
+    if (int rc = check_common(a, sfa, b, sfb, d, N, K)) return rc;
+    if (!counts) return fail(DG_ERR_INVALID_ARG, "counts is null");
+    if (!aligned(counts, 4)) return fail(DG_ERR_ALIGNMENT, "counts must be 4-byte aligned");
+    if (G < 1 || G > dg::MAX_MASKED_GROUPS)
+        return fail(DG_ERR_INVALID_ARG, "G=%d must be in [1, %d]", G, dg::MAX_MASKED_GROUPS);
+    if (M_total < 0) return fail(DG_ERR_INVALID_ARG, "M_total=%d must be non-negative", M_total);
+    if (static_cast<long long>(G) * N > 0x7fffffffLL) return fail(DG_ERR_INVALID_ARG, "G*N exceeds 2^31");
+    if (M_total == 0) return DG_OK;
+    DeviceInfo info;
+    if (int rc = device_info(info)) return rc;
+    dg::GemmParams p{};
+    p.mode = dg::MODE_NOPAD;
+    p.M = M_total; p.N = N; p.K = K; p.G = G;
+    const ScaleArgs sc{sfa, dg_get_tma_aligned_size(M_total, 4), sfb};
+    p.d = static_cast<__nv_bfloat16 *>(d);
+    p.masked_m = counts;
+    p.err = device_error_word();
+    if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
+    // Windows: each group adds at most one partial window to ceil(M_total / rows per window); the tile shape
+    // is chosen for half a partial window per group.
+    const long long w1 = (M_total + dg::BLOCK_M - 1) / dg::BLOCK_M, w2 = (M_total + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M);
+    const Plan plan{w1 + G / 2, w2 + G / 2, w1 + G, w2 + G, 0, 0, true};
+    return plan_and_launch(p, info, plan, a, M_total, b, static_cast<long long>(G) * N, sc,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dg_set_cta_pair_policy(int policy) {

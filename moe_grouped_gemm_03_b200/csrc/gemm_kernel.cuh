@@ -37,6 +37,8 @@
 //               the next rows).  The window list is built on the device at kernel start.
 //   masked      per group ceil(masked_m[g] / 128*CTAS) windows, counted on the device, so the host never
 //               needs masked_m.
+//   no padding  the same per-group windows over the groups' row counts, each group starting at the sum of
+//               the earlier counts (no alignment); rows past a group's count are computed and not stored.
 // Each CTA decodes its tile sequence once at kernel start (all threads, into a shared-memory list), so no
 // role pays a decode -- a binary search and global loads of m_indices -- per tile.
 //
@@ -50,7 +52,7 @@
 
 namespace dg {
 
-enum : int { MODE_DENSE = 0, MODE_CONTIGUOUS = 1, MODE_MASKED = 2 };
+enum : int { MODE_DENSE = 0, MODE_CONTIGUOUS = 1, MODE_MASKED = 2, MODE_NOPAD = 3 };
 
 constexpr int BLOCK_M = 128;  // rows per CTA
 constexpr int BLOCK_K = 128;  // = the scale block along K
@@ -73,15 +75,15 @@ constexpr unsigned ERR_BAD_GROUP = 2u;
 
 struct GemmParams {
     int mode;
-    int M;             // dense: M; contiguous: M_total; masked: M_max
+    int M;             // dense: M; contiguous / no padding: M_total; masked: M_max
     int N, K, G;
-    int num_windows;   // dense / contiguous: windows (128- or 256-row); masked: unused
+    int num_windows;   // dense / contiguous: windows (128- or 256-row); masked / no padding: unused
     int num_n_blocks;  // ceil(N / BN)
     int num_sf_groups; // ceil(K / (128 * SF_GROUP))
     int sfa_blocks;    // 128-row blocks per group of the packed SFA (masked layout)
     __nv_bfloat16 *d;
     const int *m_indices;
-    const int *masked_m;
+    const int *masked_m;  // masked: masked_m; no padding: the groups' row counts
     unsigned *err;
     unsigned long long wait_limit_ns;  // limit of any single wait
     int skip_first_load;               // test hook: the first CTA (pair) never loads stage 0
@@ -106,7 +108,9 @@ struct Cfg {
     // scale slots in TMEM, used round-robin by successive scale groups (not by stages)
     static constexpr int SF_SLOTS_FIT = (TMEM_COLS - SF_TMEM_BASE) / SF_COLS;
     static constexpr int SF_SLOTS = SF_SLOTS_FIT > 4 ? 4 : SF_SLOTS_FIT;
-    static constexpr int TABLE_INTS = (CTAS == 2 ? MAX_PAIR_WINDOWS : MAX_MASKED_GROUPS) + 1;
+    // window prefix (masked / no padding: G + 1 entries, then the groups' first rows) or pair windows
+    static constexpr int TABLE_INTS =
+        MAX_PAIR_WINDOWS + 1 > 2 * (MAX_MASKED_GROUPS + 1) ? MAX_PAIR_WINDOWS + 1 : 2 * (MAX_MASKED_GROUPS + 1);
     static constexpr int EPI_BYTES = 4 * 2 * EPI_CHUNK_BYTES;    // per epilogue warp: two staging chunks
     static constexpr int FIXED_BYTES =
         EPI_BYTES + 4 * TABLE_INTS + 4 * MAX_MASKED_GROUPS + 16 + 8 * TILE_LIST_CAP + 16 + 8 * 16 + 1024;
@@ -147,8 +151,9 @@ struct Tile {
 
 struct SharedCtl {
     volatile int *abort;
-    const int *prefix;   // masked: window prefix per group; contiguous pairs: first block of each window
-    const int *mm;       // masked: clamped masked_m
+    const int *prefix;   // masked / no padding: window prefix per group; contiguous pairs: first block of each window
+    const int *mm;       // masked / no padding: the groups' clamped row counts
+    const int *off;      // no padding: first row of each group
     const short *gblk;   // contiguous pairs, kernel prologue only: group of each 128-row block
 };
 
@@ -238,26 +243,32 @@ __device__ __forceinline__ bool decode_tile(const GemmParams &p, const SharedCtl
     const int g = upper_index(ctl.prefix, p.G, w);
     ti.g = g;
     ti.local_row0 = (w - ctl.prefix[g]) * C::TILE_M;
-    ti.row0 = g * p.M + ti.local_row0;
+    ti.row0 = (p.mode == MODE_MASKED ? g * p.M : ctl.off[g]) + ti.local_row0;
     return true;
 }
 
 // A decoded tile packed into 8 bytes: row0, then (g + 1) in the low 16 bits and nb in the high 16 bits
-// (g + 1 = 0 marks a tile that computes nothing).  local_row0 = row0 - g * M for the masked layout, else row0.
+// (g + 1 = 0 marks a tile that computes nothing).  local_row0 = row0 - (the group's first row) for the masked
+// and no-padding layouts, else row0.
 __device__ __forceinline__ uint2 pack_tile(bool valid, const Tile &ti) {
     return make_uint2(static_cast<uint32_t>(ti.row0),
                       (valid ? static_cast<uint32_t>(ti.g + 1) : 0u) | (static_cast<uint32_t>(ti.nb) << 16));
 }
 
 template <class C>
-__device__ __forceinline__ bool unpack_tile(const GemmParams &p, uint2 e, Tile &ti) {
+__device__ __forceinline__ bool unpack_tile(const GemmParams &p, const SharedCtl &ctl, uint2 e, Tile &ti) {
     const int g1 = static_cast<int>(e.y & 0xFFFFu);
     if (g1 == 0) return false;
     ti.g = g1 - 1;
     ti.nb = static_cast<int>(e.y >> 16);
     ti.n0 = ti.nb * C::BN;
     ti.row0 = static_cast<int>(e.x);
-    ti.local_row0 = p.mode == MODE_MASKED ? ti.row0 - ti.g * p.M : ti.row0;
+    if (p.mode == MODE_MASKED)
+        ti.local_row0 = ti.row0 - ti.g * p.M;
+    else if (p.mode == MODE_NOPAD)
+        ti.local_row0 = ti.row0 - ctl.off[ti.g];
+    else
+        ti.local_row0 = ti.row0;
     return true;
 }
 
@@ -275,19 +286,49 @@ __device__ __forceinline__ int warp_exclusive_sum(int v, int lane, int *total) {
 
 // Masked layout (one warp, after mm[] holds the clamped masked_m): prefix[g] = windows of groups before g,
 // prefix[G] = all windows.
-template <class C>
-__device__ void build_masked_prefix(const GemmParams &p, int *prefix, const int *mm, int lane) {
-    const int chunk = (p.G + 31) / 32;
-    const int begin = min(lane * chunk, p.G), end = min(begin + chunk, p.G);
+// Window prefix of the groups' row counts: prefix[g] = ceil(mm[0] / tile_m) + ... + ceil(mm[g-1] / tile_m),
+// prefix[G] = the total (one warp; lane l scans a contiguous chunk of groups).
+__device__ void build_window_prefix(int G, int tile_m, const int *mm, int *prefix, int lane) {
+    const int chunk = (G + 31) / 32;
+    const int begin = min(lane * chunk, G), end = min(begin + chunk, G);
     int local = 0;
-    for (int g = begin; g < end; ++g) local += (mm[g] + C::TILE_M - 1) / C::TILE_M;
+    for (int g = begin; g < end; ++g) local += (mm[g] + tile_m - 1) / tile_m;
     int total;
     int run = warp_exclusive_sum(local, lane, &total);
     for (int g = begin; g < end; ++g) {
         prefix[g] = run;
-        run += (mm[g] + C::TILE_M - 1) / C::TILE_M;
+        run += (mm[g] + tile_m - 1) / tile_m;
     }
-    if (lane == 0) prefix[p.G] = total;
+    if (lane == 0) prefix[G] = total;
+}
+
+// No-padding layout: the groups' first rows off[g] = counts[0] + ... + counts[g-1] (a 64-bit running sum), and
+// the counts (already >= 0) clamped so that every group ends by row M; rows past M are reported and dropped.
+// One warp, the same chunking as build_window_prefix.
+__device__ void build_group_rows(int G, int M, int *mm, int *off, unsigned *err, int lane) {
+    const int chunk = (G + 31) / 32;
+    const int begin = min(lane * chunk, G), end = min(begin + chunk, G);
+    long long local = 0;
+    for (int g = begin; g < end; ++g) local += mm[g];
+    long long incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    long long run = incl - local;
+    for (int g = begin; g < end; ++g) {
+        const long long c = mm[g];
+        const int start = static_cast<int>(run < M ? run : M);
+        int kept = static_cast<int>(c);
+        if (run + c > M) {
+            kept = M - start;
+            if (err) raise_error(err, ERR_BAD_GROUP);
+        }
+        off[g] = start;
+        mm[g] = kept;
+        run += c;
+    }
 }
 
 // Contiguous layout with CTA pairs (one warp, after gblk[] holds each 128-row block's group or -1): the
@@ -349,6 +390,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     int *s_prefix = reinterpret_cast<int *>(smem + C::OFF_PREFIX);
     int *s_mm = reinterpret_cast<int *>(smem + C::OFF_MM);
+    int *s_off = s_prefix + (MAX_MASKED_GROUPS + 1);  // no padding: the groups' first rows
     uint2 *s_tiles = reinterpret_cast<uint2 *>(smem + C::OFF_TILES);
 
     const int warp = threadIdx.x >> 5;
@@ -386,10 +428,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const bool pair_contig = PAIR && p.mode == MODE_CONTIGUOUS;
     short *s_gblk = reinterpret_cast<short *>(sA);
     const int num_blocks = p.M / BLOCK_M;
-    if (p.mode == MODE_MASKED) {
+    if (p.mode == MODE_MASKED || p.mode == MODE_NOPAD) {
         for (int g = threadIdx.x; g < p.G; g += NUM_THREADS) {
             int m = __ldg(p.masked_m + g);
-            if (m < 0 || m > p.M) {
+            if (m < 0 || (p.mode == MODE_MASKED && m > p.M)) {
                 raise_error(p.err, ERR_BAD_GROUP);
                 m = m < 0 ? 0 : p.M;
             }
@@ -414,7 +456,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     __syncthreads();
     if (warp == EPI_WARP0) {
-        if (p.mode == MODE_MASKED) build_masked_prefix<C>(p, s_prefix, s_mm, lane);
+        if (p.mode == MODE_NOPAD) {
+            build_group_rows(p.G, p.M, s_mm, s_off, p.err, lane);
+            __syncwarp();
+        }
+        if (p.mode == MODE_MASKED || p.mode == MODE_NOPAD) build_window_prefix(p.G, C::TILE_M, s_mm, s_prefix, lane);
         else if (pair_contig) build_pair_windows(num_blocks, s_gblk, s_prefix, lane);
     }
     tc_fence_before_sync();
@@ -423,10 +469,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after_sync();
     const uint32_t tmem_base = *s_tmem_base;
 
-    const SharedCtl ctl{s_abort, s_prefix, s_mm, s_gblk};
+    const SharedCtl ctl{s_abort, s_prefix, s_mm, s_off, s_gblk};
     const int nkb = p.K / BLOCK_K;
     int total_windows;
-    if (p.mode == MODE_MASKED)
+    if (p.mode == MODE_MASKED || p.mode == MODE_NOPAD)
         total_windows = s_prefix[p.G];
     else if (pair_contig)
         total_windows = s_prefix[MAX_PAIR_WINDOWS];
@@ -444,9 +490,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         s_tiles[k] = pack_tile(valid, ti);
     }
     __syncthreads();
-    const SharedCtl ctl_main{s_abort, s_prefix, s_mm, nullptr};  // the A ring is operand data from here on
+    const SharedCtl ctl_main{s_abort, s_prefix, s_mm, s_off, nullptr};  // the A ring is operand data from here on
     auto tile_at = [&](int k, Tile &ti) -> bool {
-        if (k < TILE_LIST_CAP) return unpack_tile<C>(p, s_tiles[k], ti);
+        if (k < TILE_LIST_CAP) return unpack_tile<C>(p, ctl_main, s_tiles[k], ti);
         return decode_tile<C>(p, ctl_main, cluster_id + k * num_clusters, ti);
     };
 
@@ -492,8 +538,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int arow = ti.row0 + my_rows;
                 const int brow = ti.g * p.N + ti.n0 + static_cast<int>(rank) * C::B_ROWS;
                 // packed scale atoms: SFA [block][group], SFB [g][n block][group][atom]
-                const int sfa_block = p.mode == MODE_MASKED ? ti.g * p.sfa_blocks + (ti.local_row0 + my_rows) / BLOCK_M
-                                                            : (ti.row0 + my_rows) / BLOCK_M;
+                // (no padding: atoms of each group's windows, CTAS blocks per window, after the earlier groups')
+                int sfa_block = (ti.local_row0 + my_rows) / BLOCK_M;
+                if (p.mode == MODE_MASKED)
+                    sfa_block += ti.g * p.sfa_blocks;
+                else if (p.mode == MODE_NOPAD)
+                    sfa_block += CTAS * ctl_main.prefix[ti.g];
+                else
+                    sfa_block = (ti.row0 + my_rows) / BLOCK_M;
                 const int sfa_y0 = sfa_block * p.num_sf_groups;
                 const int sfb_y0 = (ti.g * p.num_n_blocks + ti.nb) * p.num_sf_groups * C::SFB_ATOMS;
                 for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {

@@ -6,7 +6,9 @@
 // i.e. TMEM column c of the scale slot holds rows 32c .. 32c+31, which is where the block-scaled MMA reads
 // the scale of row (or column) 32c + lane.
 //
-//   SFA atoms: [128-row block][group]       block over A's rows (masked: G x blocks-per-group)
+//   SFA atoms: [128-row block][group]       block over A's rows (masked: G x blocks-per-group; no padding:
+//                                           the blocks of each group's windows, 128*CTAS rows per window,
+//                                           after the earlier groups', starting at the group's first row)
 //   SFB atoms: [g][N tile][group][atom a]   rows a*128 .. a*128+127 of the BN-wide N tile (tile-aligned,
 //                                           so a tile whose start is not a multiple of 128 still gets one
 //                                           word per output column in the right TMEM lane)
@@ -19,11 +21,14 @@
 namespace dg {
 
 struct PackParams {
+    int mode;             // the GEMM's layout (MODE_*)
+    const int *counts;    // no padding: the groups' row counts (device)
+    int tile_m;           // no padding: rows per window (128 * CTAS)
     // SFA: fp32 MN-major [K/128][ld] (masked: [G][K/128][ld])
     const float *sfa;
     int sfa_ld;
     int rows_per_group;   // masked: M_max; otherwise the row extent (M or M_total)
-    int blocks_per_group; // 128-row blocks per group (masked) or in total
+    int blocks_per_group; // 128-row blocks per group (masked) or in total (no padding: an upper bound)
     int sfa_groups;       // G for masked, 1 otherwise
     // SFB: fp32 [G][ceil(N/128)][K/128]
     const float *sfb;
@@ -43,6 +48,22 @@ constexpr int PACK_THREADS = 1024;
 // with one 16-byte store, so an atom is one coalesced 512-byte write.
 __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackParams p) {
     grid_launch_dependents();  // the GEMM may start its prologue; it waits for this grid before reading
+    // no padding: the groups' clamped counts, first rows and window prefix, as the GEMM derives them
+    __shared__ int s_cnt[MAX_MASKED_GROUPS], s_off[MAX_MASKED_GROUPS], s_wpre[MAX_MASKED_GROUPS + 1];
+    const bool nopad = p.mode == MODE_NOPAD;
+    if (nopad) {
+        for (int g = threadIdx.x; g < p.G; g += blockDim.x) {
+            const int c = __ldg(p.counts + g);
+            s_cnt[g] = c < 0 ? 0 : c;
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            build_group_rows(p.G, p.rows_per_group, s_cnt, s_off, nullptr, threadIdx.x);
+            __syncwarp();
+            build_window_prefix(p.G, p.tile_m, s_cnt, s_wpre, threadIdx.x);
+        }
+        __syncthreads();
+    }
     const long long sfa_atoms = p.sfa_words / SF_ATOM_WORDS;
     const long long total = sfa_atoms + p.sfb_words / SF_ATOM_WORDS;
     const int lane = threadIdx.x & 31;
@@ -56,16 +77,32 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
         if (atom < sfa_atoms) {
             const int q = static_cast<int>(atom % p.num_sf_groups);
             const long long block = atom / p.num_sf_groups;
-            const int g = static_cast<int>(block / p.blocks_per_group);
-            const int lb = static_cast<int>(block % p.blocks_per_group);
-            const float *base = p.sfa + static_cast<size_t>(g) * p.nkb * p.sfa_ld;
+            long long group_base = 0;  // masked: the group's scale array
+            int first = 0, rows = 0;   // the block's first row in the scale array, rows of it that exist
+            if (nopad) {
+                const int per_window = p.tile_m / 128;
+                const long long window = block / per_window;
+                if (window < s_wpre[p.G]) {  // (blocks past the last window are never read)
+                    const int g = upper_index(s_wpre, p.G, static_cast<int>(window));
+                    const int local = static_cast<int>(block - static_cast<long long>(per_window) * s_wpre[g]) * 128;
+                    first = s_off[g] + local;
+                    rows = s_cnt[g] - local;
+                }
+            } else {
+                const int g = static_cast<int>(block / p.blocks_per_group);
+                group_base = static_cast<long long>(g) * p.nkb * p.sfa_ld;
+                first = static_cast<int>(block % p.blocks_per_group) * 128;
+                rows = p.rows_per_group - first;
+            }
+            const float *base = p.sfa + group_base;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int row = lb * 128 + lane + 32 * j;
+                const int r = lane + 32 * j;
+                const int row = first + r;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int kb = 4 * q + i;
-                    const uint32_t code = (row < p.sfa_ld && row < p.rows_per_group && kb < p.nkb)
+                    const uint32_t code = (r < rows && row < p.sfa_ld && kb < p.nkb)
                                               ? ue8m0_code(__ldg(base + static_cast<size_t>(kb) * p.sfa_ld + row))
                                               : 0x7Fu;
                     word[j] |= code << (8 * i);

@@ -90,6 +90,70 @@ def test_masked_shapes(G, M_max, N, K, mm, policy):
     _full_check(synth.make_masked(G, M_max, N, K, masked_m=mm, seed=G + M_max, expected_m=M_max // 2))
 
 
+@pytest.mark.parametrize("counts,N,K,extra", [
+    ([0, 1, 127, 128, 129, 300], 512, 256, 0),
+    ([513, 7, 260], 4096, 384, 5),
+    ([1], 16, 128, 0),
+    ([129, 1, 130, 255, 256, 257, 3], 640, 256, 131),  # groups start at any row; a tail no group owns
+    ([37] * 40, 384, 256, 0),                          # forty small groups: every window is partial
+    ([0, 0, 0], 256, 128, 40),                         # no group owns a row: nothing is written
+])
+def test_nopad_shapes(counts, N, K, extra, policy):
+    _full_check(synth.make_nopad(counts, N, K, seed=sum(counts) + N + extra, extra_rows=extra))
+
+
+def test_nopad_counts_past_m_total_are_clipped_and_reported(policy):
+    """Counts summing past M_total: the rows up to M_total are computed as the clipped layout says, and the
+    device error word reports it; a negative count owns no row."""
+    import moe_grouped_gemm_03_b200 as dg
+
+    p = synth.make_nopad([100, 50], 256, 256, seed=15)
+    t = synth.to_torch(p)
+    t["counts"].copy_(torch.tensor([100, 80], dtype=torch.int32))
+    out = run_problem(p, tensors=t)
+    with pytest.raises(dg.DGError) as e:
+        dg.check_device_error()
+    assert e.value.status == -6
+    assert_close(bf16_to_f64(out), oracle.problem_full(p), "clipped counts")
+    q = synth.make_nopad([0, 64], 256, 256, seed=16)
+    tq = synth.to_torch(q)
+    tq["counts"].copy_(torch.tensor([-5, 64], dtype=torch.int32))
+    out = run_problem(q, tensors=tq)
+    with pytest.raises(dg.DGError):
+        dg.check_device_error()
+    assert_close(bf16_to_f64(out), oracle.problem_full(q), "negative count")
+
+
+def test_nopad_equals_contiguous_call_on_the_padded_layout(policy):
+    """The same tokens through the no-padding and the contiguous entry points give bit-identical rows."""
+    import moe_grouped_gemm_03_b200 as dg
+
+    counts = [200, 77, 384, 1]
+    q = synth.make_nopad(counts, 1024, 512, seed=18)
+    out_np = run_problem(q)
+    padded = [synth.align_up(c, 128) for c in counts]
+    starts = np.concatenate([[0], np.cumsum(padded)])
+    M_total = int(starts[-1])
+    a = np.zeros((M_total, q.K), np.uint8)
+    sfa = np.ones((q.K // 128, synth.tma_aligned_rows(M_total)), np.float32)
+    m_indices = np.full(M_total, -1, np.int32)
+    src = 0
+    for g, c in enumerate(counts):
+        a[starts[g]:starts[g] + c] = q.a[src:src + c]
+        sfa[:, starts[g]:starts[g] + c] = q.sfa[:, src:src + c]
+        m_indices[starts[g]:starts[g] + c] = g
+        src += c
+    t = synth.to_torch(q)
+    out_c = torch.empty(M_total, q.N, dtype=torch.bfloat16, device="cuda")
+    dg.m_grouped_fp8_gemm_nt_contiguous((torch.from_numpy(a).cuda(), torch.from_numpy(sfa).cuda()),
+                                        (t["b"], t["sfb"]), out_c, torch.from_numpy(m_indices).cuda())
+    dg.check_device_error()
+    src = 0
+    for g, c in enumerate(counts):
+        assert torch.equal(out_np[src:src + c], out_c[starts[g]:starts[g] + c]), f"group {g}"
+        src += c
+
+
 def test_masked_all_groups_empty_writes_nothing(policy):
     p = synth.make_masked(3, 128, 256, 256, masked_m=[0, 0, 0], seed=1)
     out = run_problem(p)
