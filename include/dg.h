@@ -57,9 +57,16 @@ typedef enum {
                                   or no-padding counts that are negative or sum past M_total */
 } dg_status;
 
-/* Per-segment M padding of the contiguous layout: each group's rows start on a multiple of this (128).
- * README "Grouped GEMMs (contiguous layout)": segments are aligned to the GEMM M block size. */
+/* Per-segment M padding of the contiguous layout: each group's rows start on a multiple of this (128 unless
+ * set to 256).  README "Grouped GEMMs (contiguous layout)": segments are aligned to the GEMM M block size;
+ * MATE docs "Contiguous Grouped GEMM Alignment": the alignment is 128 by default, 256 on request, nothing else. */
 DG_EXPORT int dg_get_m_alignment_for_contiguous_layout(void);
+
+/* Sets that alignment for the contiguous calls that follow (process-wide; not thread-safe against concurrent
+ * calls).  128 or 256; returns the value set, or DG_ERR_INVALID_ARG (nothing changes) for any other value.
+ * With 256 every group owns whole 256-row windows, so the 2-CTA tiles never straddle two groups; results do
+ * not depend on the alignment, only M_total's validation does (M_total % alignment == 0). */
+DG_EXPORT int dg_set_m_alignment_for_contiguous_layout(int alignment);
 
 /* Rows rounded up so that `mn` elements of `elem_bytes` bytes fill whole 16-byte units (README
  * "Utilities": get_tma_aligned_size).  Returns -1 for a non-positive elem_bytes. */
@@ -90,7 +97,8 @@ DG_EXPORT int dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, con
  *   sfa [K/128][ld(M_total)], b [G][N][K] e4m3, sfb [G][ceil(N/128)][K/128],
  *   m_indices int32 [M_total] on the device: the group of each row, -1 for a padding row.  Every
  *   128-row block must hold one group (its first row decides; a block whose first row is -1 is skipped),
- *   d [M_total][N] bf16: rows with m_indices == -1 are left untouched.  M_total % 128 == 0, 1 <= G <= 65534. */
+ *   d [M_total][N] bf16: rows with m_indices == -1 are left untouched.
+ *   M_total % dg_get_m_alignment_for_contiguous_layout() == 0, 1 <= G <= 65534. */
 DG_EXPORT int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
                                         void *d, const int *m_indices, int M_total, int N, int K, int G,
                                         dg_stream_t stream);

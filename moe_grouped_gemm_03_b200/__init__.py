@@ -45,6 +45,7 @@ _LL = ctypes.c_longlong
 
 _SIGNATURES = {
     "dg_get_m_alignment_for_contiguous_layout": (_I, []),
+    "dg_set_m_alignment_for_contiguous_layout": (_I, [_I]),
     "dg_get_tma_aligned_size": (_I, [_I, _I]),
     "dg_set_num_sms": (_I, [_I]),
     "dg_get_num_sms": (_I, []),
@@ -113,6 +114,13 @@ def _check_operand(name, t, dims, dtypes):
 # ------------------------------------------------------------------------------------------------ utilities
 def get_m_alignment_for_contiguous_layout() -> int:
     return _lib.dg_get_m_alignment_for_contiguous_layout()
+
+
+def set_m_alignment_for_contiguous_layout(alignment: int) -> int:
+    """128 (default) or 256: the per-segment M padding the contiguous calls expect from here on."""
+    rc = _lib.dg_set_m_alignment_for_contiguous_layout(int(alignment))
+    _check(rc if rc < 0 else DG_OK)
+    return rc
 
 
 def get_tma_aligned_size(mn: int, element_size: int) -> int:
@@ -254,6 +262,6 @@ def m_grouped_fp8_gemm_nt_nopad(lhs, rhs, out: torch.Tensor, counts: torch.Tenso
 __all__ = [
     "DGError", "fp8_gemm_nt", "fp8_gemm_nt_noalloc", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
     "m_grouped_fp8_gemm_nt_nopad",
-    "get_m_alignment_for_contiguous_layout", "get_tma_aligned_size", "set_num_sms", "get_num_sms", "num_tiles",
+    "get_m_alignment_for_contiguous_layout", "set_m_alignment_for_contiguous_layout", "get_tma_aligned_size", "set_num_sms", "get_num_sms", "num_tiles",
     "select_block_n", "set_cta_pair_policy", "check_device_error", "lib", "header_symbols", "last_error",
 ]

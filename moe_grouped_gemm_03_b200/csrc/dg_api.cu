@@ -154,6 +154,7 @@ int scratch_pool(int device, cudaMemPool_t &pool) {
 }
 
 // ----------------------------------------------------------------------------------------------- launch
+int g_m_alignment = dg::BLOCK_M;  // contiguous layout: per-segment M padding (128 or 256)
 int g_pair_policy = -1;  // -1: library decides; 0: single CTAs only; 1: CTA pairs whenever supported
 unsigned long long g_wait_limit_ns = dg::WAIT_LIMIT_NS;  // limit of every in-kernel wait
 bool g_drop_first_stage = false;  // testing aid: the next GEMM launch leaves one stage unloaded
@@ -525,7 +526,14 @@ int launch_bn_noalloc(int bn, int ctas, const void *a, long long a_rows, const v
 
 extern "C" {
 
-int dg_get_m_alignment_for_contiguous_layout(void) { return dg::BLOCK_M; }
+int dg_get_m_alignment_for_contiguous_layout(void) { return g_m_alignment; }
+
+int dg_set_m_alignment_for_contiguous_layout(int alignment) {
+    if (alignment != 128 && alignment != 256)
+        return fail(DG_ERR_INVALID_ARG, "alignment=%d must be 128 or 256", alignment);
+    g_m_alignment = alignment;
+    return alignment;
+}
 
 int dg_get_tma_aligned_size(int mn, int elem_bytes) {
     if (elem_bytes <= 0) return -1;
@@ -598,8 +606,8 @@ int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const v
     if (!aligned(m_indices, 4)) return fail(DG_ERR_ALIGNMENT, "m_indices must be 4-byte aligned");
     if (G < 1 || G > 65534) return fail(DG_ERR_INVALID_ARG, "G=%d must be in [1, 65534]", G);
     if (M_total < 0) return fail(DG_ERR_INVALID_ARG, "M_total=%d must be non-negative", M_total);
-    if (M_total % dg::BLOCK_M)
-        return fail(DG_ERR_ALIGNMENT, "M_total=%d must be a multiple of %d", M_total, dg::BLOCK_M);
+    if (M_total % g_m_alignment)
+        return fail(DG_ERR_ALIGNMENT, "M_total=%d must be a multiple of %d", M_total, g_m_alignment);
     if (static_cast<long long>(G) * N > 0x7fffffffLL) return fail(DG_ERR_INVALID_ARG, "G*N exceeds 2^31");
     if (M_total == 0) return DG_OK;
     DeviceInfo info;

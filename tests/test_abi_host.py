@@ -103,3 +103,24 @@ def test_debug_wait_limit_range():
     assert L.dg_debug_bounded_wait(ctypes.c_ulonglong(3_000_000_000), 0) == -1
     assert L.dg_debug_bounded_wait(ctypes.c_ulonglong(1_000_000), 0) == 0
     assert L.dg_debug_bounded_wait(ctypes.c_ulonglong(0), 0) == 0
+
+
+def test_contiguous_alignment_setting():
+    """128 (default) or 256 per the pages; other values are refused; M_total is validated against it."""
+    import moe_grouped_gemm_03_b200 as dg
+
+    P = ctypes.c_void_p
+    ok = dict(a=P(256), sfa=P(256), b=P(256), sfb=P(256), d=P(256))
+    assert L.dg_get_m_alignment_for_contiguous_layout() == 128
+    assert L.dg_set_m_alignment_for_contiguous_layout(64) == -1
+    assert L.dg_set_m_alignment_for_contiguous_layout(384) == -1
+    assert L.dg_get_m_alignment_for_contiguous_layout() == 128
+    try:
+        assert dg.set_m_alignment_for_contiguous_layout(256) == 256
+        assert dg.get_m_alignment_for_contiguous_layout() == 256
+        # 384 rows are 128-aligned but not 256-aligned
+        assert L.dg_m_grouped_fp8_gemm_nt_contiguous(*ok.values(), P(256), 384, 256, 512, 2, None) == -2
+        assert L.dg_m_grouped_fp8_gemm_nt_contiguous(*ok.values(), P(256), 0, 256, 512, 2, None) == 0
+    finally:
+        assert dg.set_m_alignment_for_contiguous_layout(128) == 128
+    assert L.dg_m_grouped_fp8_gemm_nt_contiguous(*ok.values(), P(256), 200, 256, 512, 2, None) == -2

@@ -90,6 +90,25 @@ def test_masked_shapes(G, M_max, N, K, mm, policy):
     _full_check(synth.make_masked(G, M_max, N, K, masked_m=mm, seed=G + M_max, expected_m=M_max // 2))
 
 
+@pytest.fixture
+def alignment_256():
+    import moe_grouped_gemm_03_b200 as dg
+
+    dg.set_m_alignment_for_contiguous_layout(256)
+    yield 256
+    dg.set_m_alignment_for_contiguous_layout(128)
+
+
+@pytest.mark.parametrize("counts,N,K", [
+    ([0, 1, 127, 128, 129, 300], 512, 256),
+    ([129, 1, 130, 255, 256, 257, 3], 640, 384),
+    ([256] * 5, 256, 128),
+])
+def test_contiguous_alignment_256(counts, N, K, policy, alignment_256):
+    """Segments padded to 256 rows (the optional alignment): every 256-row window holds one group."""
+    _full_check(synth.make_contiguous(counts, N, K, seed=sum(counts) + 256, alignment=256))
+
+
 @pytest.mark.parametrize("counts,N,K,extra", [
     ([0, 1, 127, 128, 129, 300], 512, 256, 0),
     ([513, 7, 260], 4096, 384, 5),
