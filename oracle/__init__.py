@@ -14,6 +14,9 @@ deep_gemm wrapper API list).  This module only selects rows and marshals pointer
 Grouped layouts (same README, "Grouped GEMMs (contiguous layout)" / "(masked layout)"):
 * contiguous: row m belongs to group m_indices[m]; rows with m_indices == -1 are padding and produce nothing.
 * masked: group g owns rows 0 .. masked_m[g]-1 of its [M_max, K] slab; the other rows produce nothing.
+* NN (MATE docs, 0.2.7 additions, `m_grouped_fp8_gemm_nn_contiguous`): the contiguous layout with each group's
+  B stored [K, N]; the product is the same contraction, D[m, n] = sum_k A[m, k] B_g[k, n], with B's 128x128
+  block scales stored [K/128, ceil(N/128)].  The oracle reads B_g[k, n] as the NT definition's b_g[n, k].
 * no padding (same README, "Grouped GEMMs (nopad layout)"): the groups' rows are concatenated in group order
   with no alignment; group g owns rows off_g .. off_g + counts[g] - 1 with off_g = counts[0] + ... +
   counts[g-1]; rows past the sum of the counts produce nothing.
@@ -94,6 +97,11 @@ def problem_rows(p, rows) -> np.ndarray:
     """Selected global rows of a ``synth.Problem`` (rows must be rows the GEMM produces)."""
     rows = np.asarray(rows, np.int64)
     groups = p.row_groups(rows)
+    if p.kind == "contiguous_nn":
+        # B_g[k, n] is the definition's b_g[n, k]; sfb_g[kb, nb] its s_b(g, nb, kb)
+        b = np.ascontiguousarray(p.b.transpose(0, 2, 1))
+        sfb = np.ascontiguousarray(p.sfb.transpose(0, 2, 1))
+        return gemm_rows(p.a, rows, p.sfa.shape[1], p.sfa, b, sfb, rows, groups, p.N, p.K)
     if p.kind == "masked":
         Ma = p.sfa.shape[2]
         nkb = p.sfa.shape[1]
@@ -160,3 +168,9 @@ def m_grouped_fp8_gemm_nt_nopad(a, sfa, b, sfb, counts):
     if len(rows):
         out[rows] = gemm_rows(a, rows, sfa.shape[1], sfa, b, sfb, rows, groups, N, K)
     return out
+
+
+def m_grouped_fp8_gemm_nn_contiguous(a, sfa, b, sfb, m_indices):
+    """a [M_total,K], sfa [K/128, >=M_total], b [G,K,N], sfb [G, K/128, ceil(N/128)], m_indices [M_total]."""
+    return m_grouped_fp8_gemm_nt_contiguous(a, sfa, np.ascontiguousarray(np.transpose(b, (0, 2, 1))),
+                                            np.ascontiguousarray(np.transpose(sfb, (0, 2, 1))), m_indices)

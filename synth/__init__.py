@@ -46,11 +46,11 @@ def tma_aligned_rows(rows: int) -> int:
 class Problem:
     """One GEMM problem in the layouts the library takes.
 
-    kind       'dense' | 'contiguous' | 'masked' | 'nopad'
+    kind       'dense' | 'contiguous' | 'masked' | 'nopad' | 'contiguous_nn'
     a          uint8 e4m3 codes, [rows, K]; masked: [G * M_max, K] (= [G, M_max, K] flattened)
     sfa        fp32, dense/contiguous [K/128, align4(rows)]; masked [G, K/128, align4(M_max)]
-    b          uint8 e4m3 codes, [G, N, K] (G = 1 for dense)
-    sfb        fp32, [G, ceil(N/128), K/128]
+    b          uint8 e4m3 codes, [G, N, K] (G = 1 for dense); contiguous_nn: [G, K, N]
+    sfb        fp32, [G, ceil(N/128), K/128]; contiguous_nn: [G, K/128, ceil(N/128)]
     m_indices  int32 [rows] (contiguous only): group id of each row, -1 for padding rows
     masked_m   int32 [G] (masked only): number of valid rows of each group
     counts     int32 [G]: contiguous -- valid rows per group (metadata); nopad -- the call's per-group row counts
@@ -79,7 +79,7 @@ class Problem:
         """Global row indices (into ``a`` / the flattened output) that the GEMM must produce."""
         if self.kind == "dense":
             return np.arange(self.M, dtype=np.int64)
-        if self.kind == "contiguous":
+        if self.kind in ("contiguous", "contiguous_nn"):
             return np.nonzero(self.m_indices >= 0)[0].astype(np.int64)
         if self.kind == "nopad":
             return np.arange(int(np.sum(self.counts, dtype=np.int64)), dtype=np.int64)
@@ -89,7 +89,7 @@ class Problem:
     def row_groups(self, rows: np.ndarray) -> np.ndarray:
         if self.kind == "dense":
             return np.zeros(len(rows), np.int32)
-        if self.kind == "contiguous":
+        if self.kind in ("contiguous", "contiguous_nn"):
             return self.m_indices[rows].astype(np.int32)
         if self.kind == "nopad":
             ends = np.cumsum(np.asarray(self.counts, np.int64))
@@ -219,6 +219,18 @@ def make_contiguous(counts: Sequence[int], N: int, K: int, seed: int = 0, name: 
                    counts=counts.astype(np.int32), name=name or f"contiguous G={G} N={N} K={K}")
 
 
+def make_contiguous_nn(counts: Sequence[int], N: int, K: int, seed: int = 0, name: str = "",
+                       rng: Optional[np.random.Generator] = None) -> Problem:
+    """The contiguous layout with B in the NN orientation: the same draws as ``make_contiguous``, with each
+    group's B stored [K, N] (N contiguous) and its 128x128 block scales [K/128, ceil(N/128)]."""
+    p = make_contiguous(counts, N, K, seed=seed, rng=rng)
+    p.kind = "contiguous_nn"
+    p.b = np.ascontiguousarray(p.b.transpose(0, 2, 1))
+    p.sfb = np.ascontiguousarray(p.sfb.transpose(0, 2, 1))
+    p.name = name or f"contiguous NN G={p.G} N={N} K={K}"
+    return p
+
+
 def make_nopad(counts: Sequence[int], N: int, K: int, seed: int = 0, extra_rows: int = 0, name: str = "",
                rng: Optional[np.random.Generator] = None) -> Problem:
     """Groups' rows concatenated with no padding, then ``extra_rows`` rows that no group owns (garbage)."""
@@ -274,7 +286,8 @@ def zipf_counts(total: int, G: int, s: float) -> np.ndarray:
     return counts
 
 
-# The five workloads (all seed 0), and as 6 the no-padding layout of workload 5's token split.
+# The five workloads (all seed 0); 6: workload 5's token split in the no-padding layout; 7: workload 3 with B
+# in the NN orientation.
 CONFIGS = {
     1: "dense FP8 NT GEMM M=128 N=256 K=512",
     2: "dense FP8 NT GEMM M=4096 N=7168 K=7168",
@@ -282,6 +295,7 @@ CONFIGS = {
     4: "M-grouped masked FP8 GEMM G=32 M_max=256 N=7168 K=2048, masked_m U[0,256], expected_m=128",
     5: "M-grouped contiguous FP8 GEMM G=64 N=7168 K=2048, Zipf(1.2) split of 65536 tokens",
     6: "M-grouped no-padding FP8 GEMM G=64 N=7168 K=2048, Zipf(1.2) split of 65536 tokens",
+    7: "M-grouped contiguous FP8 NN GEMM (B [G, K, N]) G=8 N=4096 K=7168, tokens U[1024,8192] per group",
 }
 
 
@@ -299,6 +313,10 @@ def make_config(i: int, seed: int = 0) -> Problem:
     if i == 5:
         rng = np.random.default_rng(seed)
         return make_contiguous(zipf_counts(65536, 64, 1.2), 7168, 2048, rng=rng, name=CONFIGS[5])
+    if i == 7:
+        rng = np.random.default_rng(seed)
+        counts = rng.integers(1024, 8192, endpoint=True, size=8)
+        return make_contiguous_nn(counts, 4096, 7168, rng=rng, name=CONFIGS[7])
     if i == 6:
         rng = np.random.default_rng(seed)
         return make_nopad(zipf_counts(65536, 64, 1.2), 7168, 2048, rng=rng, name=CONFIGS[6])
@@ -319,7 +337,7 @@ def to_torch(p: Problem, device="cuda"):
     if p.kind == "masked":
         out["a"] = out["a"].view(p.G, p.M, p.K)
         out["masked_m"] = t(p.masked_m)
-    if p.kind == "contiguous":
+    if p.kind in ("contiguous", "contiguous_nn"):
         out["m_indices"] = t(p.m_indices)
     if p.kind == "nopad":
         out["counts"] = t(p.counts)

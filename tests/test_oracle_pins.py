@@ -222,6 +222,35 @@ def test_nopad_equals_contiguous_layout_of_the_same_rows():
         src += c
 
 
+def test_nn_unit_scales_equal_matmul_of_k_by_n_b():
+    """NN orientation: with unit scales the product is decode(A) @ decode(B_g) with B_g read as [K, N] (a
+    transposed reading fails this for N != K)."""
+    p = synth.make_contiguous_nn([3, 130], N=256, K=384, seed=19)
+    p.sfa[:] = 1.0
+    p.sfb[:] = 1.0
+    full = oracle.problem_full(p)
+    starts = [0, 128]
+    for g, c in enumerate(p.counts):
+        s, c = starts[g], int(c)
+        want = oracle.decode_e4m3(p.a[s:s + c]) @ oracle.decode_e4m3(p.b[g])
+        np.testing.assert_allclose(full[s:s + c], want, rtol=0, atol=0)
+
+
+def test_nn_block_scale_orientation():
+    """Doubling B's scale block (kb=1, nb=0) of the NN layout changes exactly output columns 0..127 of that
+    group, by exactly that K block's contribution."""
+    p = synth.make_contiguous_nn([130], N=256, K=384, seed=20)
+    base = oracle.problem_full(p)
+    p.sfb[0, 1, 0] *= 2.0
+    moved = oracle.problem_full(p)
+    rows = np.arange(130)
+    assert np.array_equal(moved[rows, 128:], base[rows, 128:])
+    a = oracle.decode_e4m3(p.a[:130, 128:256]) * p.sfa[1, :130, None]
+    b = oracle.decode_e4m3(p.b[0, 128:256, :128])  # K block 1, columns 0..127
+    contribution = (a @ b) * (p.sfb[0, 1, 0] / 2.0)
+    np.testing.assert_allclose(moved[rows, :128] - base[rows, :128], contribution, rtol=1e-12, atol=1e-9)
+
+
 def test_library_call_shapes_agree_with_problem_driver():
     p = synth.make_masked(G=3, M_max=64, N=128, K=128, masked_m=[3, 64, 0], seed=8)
     a = p.a.reshape(p.G, p.M, p.K)
@@ -235,3 +264,6 @@ def test_library_call_shapes_agree_with_problem_driver():
     got = oracle.m_grouped_fp8_gemm_nt_nopad(r.a, r.sfa, r.b, r.sfb, r.counts)
     np.testing.assert_array_equal(np.isnan(got), np.isnan(oracle.problem_full(r)))
     np.testing.assert_array_equal(np.nan_to_num(got), np.nan_to_num(oracle.problem_full(r)))
+    n = synth.make_contiguous_nn([9, 130], N=128, K=256, seed=11)
+    got = oracle.m_grouped_fp8_gemm_nn_contiguous(n.a, n.sfa, n.b, n.sfb, n.m_indices)
+    np.testing.assert_array_equal(np.nan_to_num(got), np.nan_to_num(oracle.problem_full(n)))

@@ -67,6 +67,14 @@ def test_nopad_layout():
     assert (p.a[133:, 0] == 0x7F).all() and p.flops() == 2 * 133 * 128 * 256
 
 
+def test_contiguous_nn_layout():
+    p = synth.make_contiguous_nn([3, 129], N=256, K=384, seed=1)
+    q = synth.make_contiguous([3, 129], N=256, K=384, seed=1)
+    assert p.b.shape == (2, 384, 256) and p.sfb.shape == (2, 3, 2)
+    assert np.array_equal(p.b, q.b.transpose(0, 2, 1)) and np.array_equal(p.sfb, q.sfb.transpose(0, 2, 1))
+    assert np.array_equal(p.a, q.a) and np.array_equal(p.m_indices, q.m_indices)
+
+
 def test_masked_layout():
     p = synth.make_masked(G=2, M_max=10, N=128, K=256, masked_m=[0, 10], seed=1)
     assert p.a.shape == (20, 256) and p.sfa.shape == (2, 2, 12) and p.sfb.shape == (2, 1, 2)
