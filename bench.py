@@ -38,7 +38,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5, 6])
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
@@ -179,6 +179,8 @@ def call_library(p, t, out):
         dg.fp8_gemm_nt((t["a"], t["sfa"]), (t["b"], t["sfb"]), out)
     elif p.kind == "contiguous":
         dg.m_grouped_fp8_gemm_nt_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["m_indices"])
+    elif p.kind == "contiguous_nn":
+        dg.m_grouped_fp8_gemm_nn_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["m_indices"])
     elif p.kind == "nopad":
         dg.m_grouped_fp8_gemm_nt_nopad((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["counts"])
     else:

@@ -113,6 +113,17 @@ DG_EXPORT int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, c
                                     void *d, const int *masked_m, int G, int M_max, int N, int K,
                                     int expected_m, dg_stream_t stream);
 
+/* M-grouped GEMM, contiguous layout with B in the NN orientation (MATE docs, 0.2.7 additions,
+ * `m_grouped_fp8_gemm_nn_contiguous`: B is [num_groups, K, N]; recipe (1, 128, 128) only).
+ *   Same as dg_m_grouped_fp8_gemm_nt_contiguous except
+ *   b [G][K][N] e4m3 (N contiguous) and sfb [G][K/128][ceil(N/128)] (B's 128x128 block scales in B's
+ *   orientation): D[m][n] = sum_k A[m][k] * B_g[k][n] with the block scales as in the NT call.
+ *   The library transposes B into stream-ordered scratch of G*N*K bytes (one HBM read and write of B) and runs
+ *   the NT kernel on it; the scratch is released in stream order when the call's work is done. */
+DG_EXPORT int dg_m_grouped_fp8_gemm_nn_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
+                                        void *d, const int *m_indices, int M_total, int N, int K, int G,
+                                        dg_stream_t stream);
+
 /* M-grouped GEMM, no-padding layout (README "Grouped GEMMs (nopad layout)": a per-group token count replaces
  * the alignment of each group's rows to the M block).
  *   a [M_total][K] e4m3: group g's rows are off_g .. off_g + counts[g] - 1, off_g = counts[0] + ... +

@@ -55,6 +55,7 @@ _SIGNATURES = {
     "dg_m_grouped_fp8_gemm_nt_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_gemm_nt_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_gemm_nt_nopad": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "dg_m_grouped_fp8_gemm_nn_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_fp8_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_set_cta_pair_policy": (_I, [_I]),
     "dg_debug_bounded_wait": (_I, [ctypes.c_ulonglong, _I]),
@@ -238,6 +239,25 @@ def m_grouped_fp8_gemm_nt_masked(lhs, rhs, out: torch.Tensor, masked_m: torch.Te
                                                 G, M_max, N, K, int(expected_m), _stream()))
 
 
+def m_grouped_fp8_gemm_nn_contiguous(lhs, rhs, out: torch.Tensor, m_indices: torch.Tensor) -> None:
+    """Contiguous layout with rhs = (b [G, K, N], sfb [G, K/128, ceil(N/128)]): out = lhs @ rhs[g] per group."""
+    a, sfa = lhs
+    b, sfb = rhs
+    _check_operand("a", a, 2, _FP8_TYPES)
+    _check_operand("b", b, 3, _FP8_TYPES)
+    _check_operand("sfa", sfa, 2, (torch.float32,))
+    _check_operand("sfb", sfb, 3, (torch.float32,))
+    _check_operand("out", out, 2, (torch.bfloat16,))
+    _check_operand("m_indices", m_indices, 1, (torch.int32,))
+    M, K = a.shape
+    G, _, N = b.shape
+    _need(b.shape[1] == K and tuple(out.shape) == (M, N) and m_indices.shape[0] == M, "shape mismatch")
+    _need(sfa.shape == (K // 128, get_tma_aligned_size(M, 4)), "sfa must be [K/128, tma_aligned(M)]")
+    _need(sfb.shape == (G, K // 128, (N + 127) // 128), "sfb must be [G, K/128, ceil(N/128)]")
+    _check(_lib.dg_m_grouped_fp8_gemm_nn_contiguous(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(out),
+                                                    _ptr(m_indices), M, N, K, G, _stream()))
+
+
 def m_grouped_fp8_gemm_nt_nopad(lhs, rhs, out: torch.Tensor, counts: torch.Tensor) -> None:
     """No-padding layout: group g's rows are off_g .. off_g + counts[g] - 1 (off_g = sum of the earlier counts);
     out rows of group g = lhs rows of group g @ rhs[g]^T; rows past sum(counts) are untouched."""
@@ -261,7 +281,7 @@ def m_grouped_fp8_gemm_nt_nopad(lhs, rhs, out: torch.Tensor, counts: torch.Tenso
 
 __all__ = [
     "DGError", "fp8_gemm_nt", "fp8_gemm_nt_noalloc", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
-    "m_grouped_fp8_gemm_nt_nopad",
+    "m_grouped_fp8_gemm_nt_nopad", "m_grouped_fp8_gemm_nn_contiguous",
     "get_m_alignment_for_contiguous_layout", "set_m_alignment_for_contiguous_layout", "get_tma_aligned_size", "set_num_sms", "get_num_sms", "num_tiles",
     "select_block_n", "set_cta_pair_policy", "check_device_error", "lib", "header_symbols", "last_error",
 ]

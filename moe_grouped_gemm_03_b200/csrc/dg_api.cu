@@ -13,6 +13,7 @@
 #include "dg.h"
 #include "gemm_kernel.cuh"
 #include "scale_pack.cuh"
+#include "transpose.cuh"
 
 namespace {
 
@@ -170,6 +171,7 @@ struct ScaleArgs {
     const float *sfa;
     int sfa_ld;
     const float *sfb;
+    bool sfb_kn = false;  // SFB stored [G][K/128][ceil(N/128)] (B in the NN orientation)
 };
 
 // Launch of the scale pre-pass: one warp per atom, spread over every SM (one block each), so that every SM is
@@ -201,6 +203,7 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
     pk.sfa = sc.sfa;
     pk.sfa_ld = sc.sfa_ld;
     pk.sfb = sc.sfb;
+    pk.sfb_kn = sc.sfb_kn ? 1 : 0;
     pk.N = p.N;
     pk.G = p.G;
     pk.bn = BN;
@@ -437,6 +440,7 @@ int launch_cfg_noalloc(const void *a, long long a_rows, const void *b, long long
     pk.sfa = sc.sfa;
     pk.sfa_ld = sc.sfa_ld;
     pk.sfb = sc.sfb;
+    pk.sfb_kn = sc.sfb_kn ? 1 : 0;
     pk.N = p.N;
     pk.G = p.G;
     pk.bn = BN;
@@ -524,6 +528,45 @@ int launch_bn_noalloc(int bn, int ctas, const void *a, long long a_rows, const v
 
 }  // namespace
 
+namespace {
+
+int check_contiguous(const void *a, const float *sfa, const void *b, const float *sfb, const void *d,
+                     const int *m_indices, int M_total, int N, int K, int G) {
+    if (int rc = check_common(a, sfa, b, sfb, d, N, K)) return rc;
+    if (!m_indices) return fail(DG_ERR_INVALID_ARG, "m_indices is null");
+    if (!aligned(m_indices, 4)) return fail(DG_ERR_ALIGNMENT, "m_indices must be 4-byte aligned");
+    if (G < 1 || G > 65534) return fail(DG_ERR_INVALID_ARG, "G=%d must be in [1, 65534]", G);
+    if (M_total < 0) return fail(DG_ERR_INVALID_ARG, "M_total=%d must be non-negative", M_total);
+    if (M_total % g_m_alignment)
+        return fail(DG_ERR_ALIGNMENT, "M_total=%d must be a multiple of %d", M_total, g_m_alignment);
+    if (static_cast<long long>(G) * N > 0x7fffffffLL) return fail(DG_ERR_INVALID_ARG, "G*N exceeds 2^31");
+    return DG_OK;
+}
+
+// The contiguous GEMM on checked arguments (M_total > 0); `sfb_kn` selects the NN orientation of SFB.
+int launch_contiguous(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
+                      const int *m_indices, int M_total, int N, int K, int G, bool sfb_kn, const DeviceInfo &info,
+                      cudaStream_t stream) {
+    dg::GemmParams p{};
+    p.mode = dg::MODE_CONTIGUOUS;
+    p.M = M_total; p.N = N; p.K = K; p.G = G;
+    ScaleArgs sc{sfa, dg_get_tma_aligned_size(M_total, 4), sfb};
+    sc.sfb_kn = sfb_kn;
+    p.d = static_cast<__nv_bfloat16 *>(d);
+    p.m_indices = m_indices;
+    p.err = device_error_word();
+    if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
+    const long long w1 = M_total / dg::BLOCK_M, w2 = (w1 + 1) / 2;
+    // a 256-row window holds at most two tiles (its halves may belong to two groups)
+    const long long bound = w2 + (w2 < G ? w2 : G);
+    // pairs need the device-built window list to fit (at most NB/2 + G/2 windows) and group ids below 2^15
+    const bool pair_ok = (w1 + G) / 2 + 1 <= dg::MAX_PAIR_WINDOWS && G <= 32767;
+    const Plan plan{w1, w2, w1, bound, w1, w2, pair_ok};
+    return plan_and_launch(p, info, plan, a, M_total, b, static_cast<long long>(G) * N, sc, stream);
+}
+
+}  // namespace
+
 extern "C" {
 
 int dg_get_m_alignment_for_contiguous_layout(void) { return g_m_alignment; }
@@ -599,35 +642,42 @@ int dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const float *
     return plan_and_launch(p, info, plan, a, M, b, N, sc, reinterpret_cast<cudaStream_t>(stream));
 }
 
+
 int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
                                         const int *m_indices, int M_total, int N, int K, int G, dg_stream_t stream) {
-    if (int rc = check_common(a, sfa, b, sfb, d, N, K)) return rc;
-    if (!m_indices) return fail(DG_ERR_INVALID_ARG, "m_indices is null");
-    if (!aligned(m_indices, 4)) return fail(DG_ERR_ALIGNMENT, "m_indices must be 4-byte aligned");
-    if (G < 1 || G > 65534) return fail(DG_ERR_INVALID_ARG, "G=%d must be in [1, 65534]", G);
-    if (M_total < 0) return fail(DG_ERR_INVALID_ARG, "M_total=%d must be non-negative", M_total);
-    if (M_total % g_m_alignment)
-        return fail(DG_ERR_ALIGNMENT, "M_total=%d must be a multiple of %d", M_total, g_m_alignment);
-    if (static_cast<long long>(G) * N > 0x7fffffffLL) return fail(DG_ERR_INVALID_ARG, "G*N exceeds 2^31");
+    if (int rc = check_contiguous(a, sfa, b, sfb, d, m_indices, M_total, N, K, G)) return rc;
     if (M_total == 0) return DG_OK;
     DeviceInfo info;
     if (int rc = device_info(info)) return rc;
-    dg::GemmParams p{};
-    p.mode = dg::MODE_CONTIGUOUS;
-    p.M = M_total; p.N = N; p.K = K; p.G = G;
-    const ScaleArgs sc{sfa, dg_get_tma_aligned_size(M_total, 4), sfb};
-    p.d = static_cast<__nv_bfloat16 *>(d);
-    p.m_indices = m_indices;
-    p.err = device_error_word();
-    if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
-    const long long w1 = M_total / dg::BLOCK_M, w2 = (w1 + 1) / 2;
-    // a 256-row window holds at most two tiles (its halves may belong to two groups)
-    const long long bound = w2 + (w2 < G ? w2 : G);
-    // pairs need the device-built window list to fit (at most NB/2 + G/2 windows) and group ids below 2^15
-    const bool pair_ok = (w1 + G) / 2 + 1 <= dg::MAX_PAIR_WINDOWS && G <= 32767;
-    const Plan plan{w1, w2, w1, bound, w1, w2, pair_ok};
-    return plan_and_launch(p, info, plan, a, M_total, b, static_cast<long long>(G) * N, sc,
-                           reinterpret_cast<cudaStream_t>(stream));
+    return launch_contiguous(a, sfa, b, sfb, d, m_indices, M_total, N, K, G, false, info,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dg_m_grouped_fp8_gemm_nn_contiguous(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
+                                        const int *m_indices, int M_total, int N, int K, int G, dg_stream_t stream) {
+    if (int rc = check_contiguous(a, sfa, b, sfb, d, m_indices, M_total, N, K, G)) return rc;
+    if (M_total == 0) return DG_OK;
+    DeviceInfo info;
+    if (int rc = device_info(info)) return rc;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // B [G][K][N] -> K-major [G][N][K] in stream-ordered scratch, then the NT path
+    cudaMemPool_t pool;
+    if (int rc = scratch_pool(info.device, pool)) return rc;
+    const size_t bytes = static_cast<size_t>(G) * N * K;
+    void *bt = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(&bt, bytes, pool, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync (B transposed)");
+    const long long tiles = static_cast<long long>(G) * (K / dg::TRANSPOSE_TILE) *
+                            ((N + dg::TRANSPOSE_TILE - 1) / dg::TRANSPOSE_TILE);
+    const long long cap = 8LL * info.num_sms;
+    dg::transpose_kn_to_nk_kernel<<<static_cast<unsigned>(tiles < cap ? tiles : cap), dg::TRANSPOSE_THREADS, 0, s>>>(
+        static_cast<const uint8_t *>(b), static_cast<uint8_t *>(bt), G, K, N);
+    int rc = DG_OK;
+    if ((e = cudaGetLastError()) != cudaSuccess) rc = cuda_fail(e, "transpose launch");
+    if (rc == DG_OK) rc = launch_contiguous(a, sfa, bt, sfb, d, m_indices, M_total, N, K, G, true, info, s);
+    const cudaError_t ef = cudaFreeAsync(bt, s);
+    if (rc == DG_OK && ef != cudaSuccess) rc = cuda_fail(ef, "cudaFreeAsync (B transposed)");
+    return rc;
 }
 
 int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const void *b, const float *sfb, void *d,

@@ -30,8 +30,9 @@ struct PackParams {
     int rows_per_group;   // masked: M_max; otherwise the row extent (M or M_total)
     int blocks_per_group; // 128-row blocks per group (masked) or in total (no padding: an upper bound)
     int sfa_groups;       // G for masked, 1 otherwise
-    // SFB: fp32 [G][ceil(N/128)][K/128]
+    // SFB: fp32 [G][ceil(N/128)][K/128], or [G][K/128][ceil(N/128)] when sfb_kn (B in the NN orientation)
     const float *sfb;
+    int sfb_kn;
     int N, G, bn, n_tiles, sfb_atoms;
     int nkb, num_sf_groups;
     uint32_t *sfa_out;    // [sfa_groups * blocks_per_group][num_sf_groups][128]
@@ -120,11 +121,14 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int n = nt * p.bn + a * 128 + lane + 32 * j;
-                const float *base = p.sfb + (static_cast<size_t>(g) * nnb128 + n / 128) * p.nkb;
+                // SFB element (g, n/128, kb) sits at base + kb * stride_kb
+                const size_t stride_kb = p.sfb_kn ? static_cast<size_t>(nnb128) : 1;
+                const float *base = p.sfb_kn ? p.sfb + static_cast<size_t>(g) * p.nkb * nnb128 + n / 128
+                                             : p.sfb + (static_cast<size_t>(g) * nnb128 + n / 128) * p.nkb;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int kb = 4 * q + i;
-                    const uint32_t code = (n < p.N && kb < p.nkb) ? ue8m0_code(__ldg(base + kb)) : 0x7Fu;
+                    const uint32_t code = (n < p.N && kb < p.nkb) ? ue8m0_code(__ldg(base + kb * stride_kb)) : 0x7Fu;
                     word[j] |= code << (8 * i);
                 }
             }

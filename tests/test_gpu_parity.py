@@ -90,6 +90,29 @@ def test_masked_shapes(G, M_max, N, K, mm, policy):
     _full_check(synth.make_masked(G, M_max, N, K, masked_m=mm, seed=G + M_max, expected_m=M_max // 2))
 
 
+@pytest.mark.parametrize("counts,N,K", [
+    ([0, 1, 127, 128, 129, 300], 512, 256),
+    ([513, 7, 260], 4096, 384),
+    ([1], 16, 128),
+    ([129, 1, 130, 255, 256, 257, 3], 640, 256),
+])
+def test_contiguous_nn_shapes(counts, N, K, policy):
+    _full_check(synth.make_contiguous_nn(counts, N, K, seed=sum(counts) + N))
+
+
+def test_nn_equals_nt_on_the_transposed_b(policy):
+    """The NN call on B [G, K, N] and the NT call on the same B stored [G, N, K] give bit-identical outputs."""
+    nn = synth.make_contiguous_nn([200, 77, 384], 1040, 512, seed=22)
+    nt = synth.make_contiguous([200, 77, 384], 1040, 512, seed=22)
+    a = run_problem(nn).clone()
+    b = run_problem(nt)
+    import moe_grouped_gemm_03_b200 as dg
+
+    dg.check_device_error()
+    valid = torch.from_numpy(nt.m_indices >= 0).cuda()
+    assert torch.equal(a[valid], b[valid])
+
+
 @pytest.fixture
 def alignment_256():
     import moe_grouped_gemm_03_b200 as dg
