@@ -17,6 +17,11 @@ Grouped layouts (same README, "Grouped GEMMs (contiguous layout)" / "(masked lay
 * NN (MATE docs, 0.2.7 additions, `m_grouped_fp8_gemm_nn_contiguous`): the contiguous layout with each group's
   B stored [K, N]; the product is the same contraction, D[m, n] = sum_k A[m, k] B_g[k, n], with B's 128x128
   block scales stored [K/128, ceil(N/128)].  The oracle reads B_g[k, n] as the NT definition's b_g[n, k].
+* K-grouped (MATE docs, 0.2.7 additions, `k_grouped_fp8_gemm_nt_contiguous`, recipe (1, 1, 128)): A [M, sum K]
+  and B [N, sum K], both K-major, with the groups' K segments concatenated; one scale per (row, 128-K block) on
+  both sides; D_g[m, n] = C_g[m, n] + sum over the 128-K blocks kb of group g of
+  sfa(m, kb) * sfb(n, kb) * sum_{k in kb} dec(a[m, k]) * dec(b[n, k]).  Computed here with numpy in float64,
+  one 128-K block at a time (each block's sum of 128 products of e4m3 values is exact in float64).
 * no padding (same README, "Grouped GEMMs (nopad layout)"): the groups' rows are concatenated in group order
   with no alignment; group g owns rows off_g .. off_g + counts[g] - 1 with off_g = counts[0] + ... +
   counts[g-1]; rows past the sum of the counts produce nothing.
@@ -96,6 +101,12 @@ def gemm_rows(a, sfa_row_off, sfa_kb_stride, sfa, b, sfb, rows, groups, N, K) ->
 def problem_rows(p, rows) -> np.ndarray:
     """Selected global rows of a ``synth.Problem`` (rows must be rows the GEMM produces)."""
     rows = np.asarray(rows, np.int64)
+    if p.kind == "k_grouped":  # rows of the flattened [G * M, N] output
+        out = np.zeros((len(rows), p.N))
+        for g in np.unique(rows // p.M):
+            sel = rows // p.M == g
+            out[sel] = k_grouped_rows(p, int(g), rows[sel] - g * p.M)
+        return out
     groups = p.row_groups(rows)
     if p.kind == "contiguous_nn":
         # B_g[k, n] is the definition's b_g[n, k]; sfb_g[kb, nb] its s_b(g, nb, kb)
@@ -114,8 +125,24 @@ def problem_rows(p, rows) -> np.ndarray:
     return gemm_rows(p.a, off, kb_stride, p.sfa, p.b, p.sfb, rows, groups, p.N, p.K)
 
 
+def k_grouped_rows(p, g, rows) -> np.ndarray:
+    """Rows ``rows`` (of M) of group g's output of a K-grouped ``synth.Problem`` (C added when present)."""
+    rows = np.asarray(rows, np.int64)
+    ks = np.asarray(p.counts, np.int64)
+    kb0 = int(ks[:g].sum()) // 128
+    out = np.zeros((len(rows), p.N)) if p.c is None else p.c[g][rows].astype(np.float64)
+    for kb in range(kb0, kb0 + int(ks[g]) // 128):
+        blk = slice(128 * kb, 128 * kb + 128)
+        a = decode_e4m3(p.a[rows, blk]) * p.sfa[kb, rows][:, None]
+        b = decode_e4m3(p.b[:, blk]) * p.sfb[kb, :p.N][:, None]
+        out += a @ b.T
+    return out
+
+
 def problem_full(p) -> np.ndarray:
     """The whole output of a ``synth.Problem`` in its output shape; rows that produce nothing are NaN."""
+    if p.kind == "k_grouped":
+        return np.stack([k_grouped_rows(p, g, np.arange(p.M)) for g in range(p.G)])
     rows = p.valid_rows()
     out = np.full((p.rows, p.N), np.nan, np.float64)
     out[rows] = problem_rows(p, rows)

@@ -46,14 +46,18 @@ def tma_aligned_rows(rows: int) -> int:
 class Problem:
     """One GEMM problem in the layouts the library takes.
 
-    kind       'dense' | 'contiguous' | 'masked' | 'nopad' | 'contiguous_nn'
+    kind       'dense' | 'contiguous' | 'masked' | 'nopad' | 'contiguous_nn' | 'k_grouped'
     a          uint8 e4m3 codes, [rows, K]; masked: [G * M_max, K] (= [G, M_max, K] flattened)
     sfa        fp32, dense/contiguous [K/128, align4(rows)]; masked [G, K/128, align4(M_max)]
     b          uint8 e4m3 codes, [G, N, K] (G = 1 for dense); contiguous_nn: [G, K, N]
     sfb        fp32, [G, ceil(N/128), K/128]; contiguous_nn: [G, K/128, ceil(N/128)]
     m_indices  int32 [rows] (contiguous only): group id of each row, -1 for padding rows
     masked_m   int32 [G] (masked only): number of valid rows of each group
-    counts     int32 [G]: contiguous -- valid rows per group (metadata); nopad -- the call's per-group row counts
+    counts     int32 [G]: contiguous -- valid rows per group (metadata); nopad -- the call's per-group row counts;
+               k_grouped -- the groups' K extents (multiples of 128)
+    k_grouped  a [M, sum K] and b [N, sum K] (both K-major, the groups' K segments concatenated); sfa
+               [sum K / 128, align4(M)] and sfb [sum K / 128, align4(N)] (one scale per row and 128-K block,
+               recipe (1, 1, 128)); c fp32 [G, M, N] or None; output fp32 [G, M, N]
     """
 
     kind: str
@@ -70,6 +74,7 @@ class Problem:
     expected_m: int = 0
     counts: Optional[np.ndarray] = None  # contiguous: valid rows per group
     name: str = ""
+    c: Optional[np.ndarray] = None  # k_grouped: the accumulator input
 
     @property
     def rows(self) -> int:
@@ -77,6 +82,8 @@ class Problem:
 
     def valid_rows(self) -> np.ndarray:
         """Global row indices (into ``a`` / the flattened output) that the GEMM must produce."""
+        if self.kind == "k_grouped":
+            return np.arange(self.G * self.M, dtype=np.int64)  # rows of the flattened [G * M, N] output
         if self.kind == "dense":
             return np.arange(self.M, dtype=np.int64)
         if self.kind in ("contiguous", "contiguous_nn"):
@@ -87,6 +94,8 @@ class Problem:
         return np.concatenate(out) if out else np.zeros(0, np.int64)
 
     def row_groups(self, rows: np.ndarray) -> np.ndarray:
+        if self.kind == "k_grouped":
+            return (rows // self.M).astype(np.int32)
         if self.kind == "dense":
             return np.zeros(len(rows), np.int32)
         if self.kind in ("contiguous", "contiguous_nn"):
@@ -97,9 +106,13 @@ class Problem:
         return (rows // self.M).astype(np.int32)
 
     def flops(self) -> int:
+        if self.kind == "k_grouped":  # each group contracts its own K segment
+            return 2 * self.M * self.N * self.K
         return 2 * int(len(self.valid_rows())) * self.N * self.K
 
     def out_shape(self):
+        if self.kind == "k_grouped":
+            return (self.G, self.M, self.N)
         if self.kind == "masked":
             return (self.G, self.M, self.N)
         return (self.rows, self.N)
@@ -231,6 +244,25 @@ def make_contiguous_nn(counts: Sequence[int], N: int, K: int, seed: int = 0, nam
     return p
 
 
+def make_k_grouped(ks: Sequence[int], M: int, N: int, seed: int = 0, with_c: bool = True, name: str = "",
+                   rng: Optional[np.random.Generator] = None) -> Problem:
+    """K-grouped operands: A [M, sum K] and B [N, sum K] with one scale per (row, 128-K block) (recipe
+    (1, 1, 128)); group g contracts its own K segment.  c ~ N(0, 1) fp32 [G, M, N] when ``with_c``."""
+    rng = rng if rng is not None else np.random.default_rng(seed)
+    ks = np.asarray(ks, np.int64)
+    assert (ks >= 0).all() and (ks % SCALE_BLOCK == 0).all()
+    G, Kt = len(ks), int(ks.sum())
+    a, sa = quantize_rows(_draw_normal(rng, (M, Kt)))
+    b, sb = quantize_rows(_draw_normal(rng, (N, Kt)))
+    sfa = np.ones((Kt // SCALE_BLOCK, tma_aligned_rows(M)), np.float32)
+    sfa[:, :M] = sa.T
+    sfb = np.ones((Kt // SCALE_BLOCK, tma_aligned_rows(N)), np.float32)
+    sfb[:, :N] = sb.T
+    c = _draw_normal(rng, (G, M, N)) if with_c else None
+    return Problem("k_grouped", M, N, Kt, G, a, sfa, b, sfb, counts=ks.astype(np.int32), c=c,
+                   name=name or f"k-grouped G={G} M={M} N={N}")
+
+
 def make_nopad(counts: Sequence[int], N: int, K: int, seed: int = 0, extra_rows: int = 0, name: str = "",
                rng: Optional[np.random.Generator] = None) -> Problem:
     """Groups' rows concatenated with no padding, then ``extra_rows`` rows that no group owns (garbage)."""
@@ -287,7 +319,7 @@ def zipf_counts(total: int, G: int, s: float) -> np.ndarray:
 
 
 # The five workloads (all seed 0); 6: workload 5's token split in the no-padding layout; 7: workload 3 with B
-# in the NN orientation.
+# in the NN orientation; 8: workload 3's token counts as the K extents of a K-grouped (weight-gradient) GEMM.
 CONFIGS = {
     1: "dense FP8 NT GEMM M=128 N=256 K=512",
     2: "dense FP8 NT GEMM M=4096 N=7168 K=7168",
@@ -296,6 +328,7 @@ CONFIGS = {
     5: "M-grouped contiguous FP8 GEMM G=64 N=7168 K=2048, Zipf(1.2) split of 65536 tokens",
     6: "M-grouped no-padding FP8 GEMM G=64 N=7168 K=2048, Zipf(1.2) split of 65536 tokens",
     7: "M-grouped contiguous FP8 NN GEMM (B [G, K, N]) G=8 N=4096 K=7168, tokens U[1024,8192] per group",
+    8: "K-grouped FP8 NT GEMM, fp32 D += A_g B_g^T, G=8 M=4096 N=7168, K_g = tokens U[1024,8192] rounded up to 128",
 }
 
 
@@ -313,6 +346,10 @@ def make_config(i: int, seed: int = 0) -> Problem:
     if i == 5:
         rng = np.random.default_rng(seed)
         return make_contiguous(zipf_counts(65536, 64, 1.2), 7168, 2048, rng=rng, name=CONFIGS[5])
+    if i == 8:
+        rng = np.random.default_rng(seed)
+        counts = rng.integers(1024, 8192, endpoint=True, size=8)
+        return make_k_grouped([align_up(int(c), SCALE_BLOCK) for c in counts], 4096, 7168, rng=rng, name=CONFIGS[8])
     if i == 7:
         rng = np.random.default_rng(seed)
         counts = rng.integers(1024, 8192, endpoint=True, size=8)
@@ -341,4 +378,8 @@ def to_torch(p: Problem, device="cuda"):
         out["m_indices"] = t(p.m_indices)
     if p.kind == "nopad":
         out["counts"] = t(p.counts)
+    if p.kind == "k_grouped":
+        out["ks"] = t(p.counts)
+        if p.c is not None:
+            out["c"] = t(p.c)
     return out

@@ -251,6 +251,50 @@ def test_nn_block_scale_orientation():
     np.testing.assert_allclose(moved[rows, :128] - base[rows, :128], contribution, rtol=1e-12, atol=1e-9)
 
 
+def test_k_grouped_equals_dense_products_of_each_k_segment():
+    """With B's row scales constant over each 128-row block, group g's K-grouped output equals C_g plus the
+    (separately pinned) dense block-scaled oracle on group g's K segment; an empty segment leaves C_g."""
+    ks = [256, 0, 384, 128]
+    p = synth.make_k_grouped(ks, M=136, N=256, seed=21)
+    nb = (p.N + 127) // 128
+    blocks = np.ones((nb, p.K // 128), np.float32)
+    for kb in range(p.K // 128):
+        for j in range(nb):
+            blocks[j, kb] = p.sfb[kb, 128 * j]
+            p.sfb[kb, 128 * j:128 * (j + 1)] = blocks[j, kb]
+    full = oracle.problem_full(p)
+    k0 = 0
+    for g, k in enumerate(ks):
+        if k == 0:
+            np.testing.assert_array_equal(full[g], p.c[g])
+            continue
+        seg = slice(k0, k0 + k)
+        sfa = np.ascontiguousarray(p.sfa[k0 // 128:(k0 + k) // 128])
+        dense = oracle.fp8_gemm_nt(np.ascontiguousarray(p.a[:, seg]), sfa, np.ascontiguousarray(p.b[:, seg]),
+                                   np.ascontiguousarray(blocks[:, k0 // 128:(k0 + k) // 128]))
+        np.testing.assert_allclose(full[g], p.c[g] + dense, rtol=1e-13, atol=1e-10)
+        k0 += k
+
+
+def test_k_grouped_row_scale_moves_one_column_of_one_group():
+    """Doubling B's scale of row n in K block kb changes only column n of the group whose segment holds kb,
+    by exactly that block's contribution; without C an empty group's output is zero."""
+    p = synth.make_k_grouped([128, 256, 0], M=64, N=200, seed=22, with_c=False)
+    base = oracle.problem_full(p)
+    assert (base[2] == 0).all()
+    kb, n = 2, 77  # K block 2 lies in group 1 (blocks 1..2)
+    p.sfb[kb, n] *= 2.0
+    moved = oracle.problem_full(p)
+    diff = moved - base
+    mask = np.zeros_like(diff, bool)
+    mask[1, :, n] = True
+    assert (diff[~mask] == 0).all()
+    blk = slice(128 * kb, 128 * kb + 128)
+    a = oracle.decode_e4m3(p.a[:, blk]) * p.sfa[kb, :64][:, None]
+    contribution = a @ oracle.decode_e4m3(p.b[n, blk]) * (p.sfb[kb, n] / 2.0)
+    np.testing.assert_allclose(diff[1, :, n], contribution, rtol=1e-12, atol=1e-9)
+
+
 def test_library_call_shapes_agree_with_problem_driver():
     p = synth.make_masked(G=3, M_max=64, N=128, K=128, masked_m=[3, 64, 0], seed=8)
     a = p.a.reshape(p.G, p.M, p.K)

@@ -75,6 +75,13 @@ def test_contiguous_nn_layout():
     assert np.array_equal(p.a, q.a) and np.array_equal(p.m_indices, q.m_indices)
 
 
+def test_k_grouped_layout():
+    p = synth.make_k_grouped([128, 0, 256], M=10, N=20, seed=1)
+    assert p.a.shape == (10, 384) and p.b.shape == (20, 384) and p.sfa.shape == (3, 12) and p.sfb.shape == (3, 20)
+    assert p.c.shape == (3, 10, 20) and p.out_shape() == (3, 10, 20)
+    assert p.flops() == 2 * 10 * 20 * 384
+
+
 def test_masked_layout():
     p = synth.make_masked(G=2, M_max=10, N=128, K=256, masked_m=[0, 10], seed=1)
     assert p.a.shape == (20, 256) and p.sfa.shape == (2, 2, 12) and p.sfb.shape == (2, 1, 2)
