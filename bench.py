@@ -38,7 +38,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7])
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7, 8])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
@@ -179,6 +179,8 @@ def call_library(p, t, out):
         dg.fp8_gemm_nt((t["a"], t["sfa"]), (t["b"], t["sfb"]), out)
     elif p.kind == "contiguous":
         dg.m_grouped_fp8_gemm_nt_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["m_indices"])
+    elif p.kind == "k_grouped":  # D = the products (no C)
+        dg.k_grouped_fp8_gemm_nt_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, p.counts.tolist(), t["ks"])
     elif p.kind == "contiguous_nn":
         dg.m_grouped_fp8_gemm_nn_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["m_indices"])
     elif p.kind == "nopad":
@@ -188,8 +190,13 @@ def call_library(p, t, out):
 
 
 def algorithmic_bytes(p):
-    """Each valid A row once, each active group's B once, the scales of those, each valid D row once."""
+    """Each valid A row once, each active group's B once, the scales of those, each valid D row once.
+    K-grouped: A and B once, their per-row scales, fp32 D once (no C in the timed call)."""
     import numpy as np
+
+    if p.kind == "k_grouped":
+        nkb = p.K // 128
+        return int((p.M + p.N) * p.K + (p.M + p.N) * nkb * 4 + p.G * p.M * p.N * 4)
 
     rows = p.valid_rows()
     nkb = p.K // 128
@@ -271,7 +278,8 @@ def run_ours(args, world, rank, local):
 
     p = synth.make_config(args.workload)
     t = synth.to_torch(p, f"cuda:{local}")
-    out = torch.empty(p.out_shape(), dtype=torch.bfloat16, device=f"cuda:{local}")
+    out_dtype = torch.float32 if p.kind == "k_grouped" else torch.bfloat16
+    out = torch.empty(p.out_shape(), dtype=out_dtype, device=f"cuda:{local}")
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.int32, device=f"cuda:{local}")
     stream = torch.cuda.current_stream()
     flops = p.flops()

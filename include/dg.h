@@ -124,6 +124,21 @@ DG_EXPORT int dg_m_grouped_fp8_gemm_nn_contiguous(const void *a, const float *sf
                                         void *d, const int *m_indices, int M_total, int N, int K, int G,
                                         dg_stream_t stream);
 
+/* K-grouped GEMM (MATE docs, 0.2.7 additions, `k_grouped_fp8_gemm_nt_contiguous`: recipe (1, 1, 128), host K
+ * extents, C accumulated into D), e.g. the per-expert weight gradient of an MoE layer.
+ *   a [M][sum ks] e4m3 and b [N][sum ks] e4m3, both K-major, the groups' K segments concatenated in group order;
+ *   sfa [sum ks / 128][ld(M)] and sfb [sum ks / 128][ld(N)] fp32: one scale per (row, 128-K block), MN-major;
+ *   ks: G host ints, each a multiple of 128 (0 allowed); ks_device: the same G values on the device (the kernel
+ *   reads these; they must equal ks);
+ *   d fp32 [G][M][N]:  D_g = C_g + sum over group g's 128-K blocks kb of sfa(m, kb) * sfb(n, kb) *
+ *   sum_{k in kb} A[m][k] * B[n][k].  c: NULL (D_g = the sum), another [G][M][N] fp32 buffer (copied into d
+ *   first), or d itself (accumulate in place).  A group with ks = 0 gives D_g = C_g (0 without C).
+ *   1 <= G <= 1024, N % 16 == 0, 16-byte aligned a, b, c, d.  Device values of ks_device that are negative or
+ *   not multiples of 128 are reported by dg_check_device_error() as DG_ERR_BAD_GROUP. */
+DG_EXPORT int dg_k_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
+                                        float *d, const float *c, const int *ks, const int *ks_device, int G, int M,
+                                        int N, dg_stream_t stream);
+
 /* M-grouped GEMM, no-padding layout (README "Grouped GEMMs (nopad layout)": a per-group token count replaces
  * the alignment of each group's rows to the M block).
  *   a [M_total][K] e4m3: group g's rows are off_g .. off_g + counts[g] - 1, off_g = counts[0] + ... +

@@ -15,7 +15,7 @@ from __future__ import annotations
 import ctypes
 import os
 import re
-from typing import Tuple
+from typing import Optional, Tuple
 
 import torch
 
@@ -56,6 +56,7 @@ _SIGNATURES = {
     "dg_m_grouped_fp8_gemm_nt_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_gemm_nt_nopad": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_gemm_nn_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "dg_k_grouped_fp8_gemm_nt_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_set_cta_pair_policy": (_I, [_I]),
     "dg_debug_bounded_wait": (_I, [ctypes.c_ulonglong, _I]),
@@ -258,6 +259,35 @@ def m_grouped_fp8_gemm_nn_contiguous(lhs, rhs, out: torch.Tensor, m_indices: tor
                                                     _ptr(m_indices), M, N, K, G, _stream()))
 
 
+def k_grouped_fp8_gemm_nt_contiguous(lhs, rhs, out: torch.Tensor, ks, ks_tensor: torch.Tensor,
+                                     c: Optional[torch.Tensor] = None) -> None:
+    """K-grouped (recipe (1, 1, 128)): lhs = (a [M, sum ks], sfa [sum ks/128, tma_aligned(M)]), rhs = (b [N, sum ks],
+    sfb [sum ks/128, tma_aligned(N)]); out fp32 [G, M, N] = c + per-group products (c None, another tensor, or out)."""
+    a, sfa = lhs
+    b, sfb = rhs
+    _check_operand("a", a, 2, _FP8_TYPES)
+    _check_operand("b", b, 2, _FP8_TYPES)
+    _check_operand("sfa", sfa, 2, (torch.float32,))
+    _check_operand("sfb", sfb, 2, (torch.float32,))
+    _check_operand("out", out, 3, (torch.float32,))
+    _check_operand("ks_tensor", ks_tensor, 1, (torch.int32,))
+    ks = [int(k) for k in ks]
+    G = len(ks)
+    M, Kt = a.shape
+    N = b.shape[0]
+    _need(b.shape[1] == Kt and sum(ks) == Kt and tuple(out.shape) == (G, M, N) and ks_tensor.shape[0] == G,
+          "shape mismatch")
+    _need(sfa.shape == (Kt // 128, get_tma_aligned_size(M, 4)), "sfa must be [sum ks/128, tma_aligned(M)]")
+    _need(sfb.shape == (Kt // 128, get_tma_aligned_size(N, 4)), "sfb must be [sum ks/128, tma_aligned(N)]")
+    if c is not None:
+        _check_operand("c", c, 3, (torch.float32,))
+        _need(tuple(c.shape) == (G, M, N), "c must be [G, M, N]")
+    ks_host = (ctypes.c_int * G)(*ks)
+    _check(_lib.dg_k_grouped_fp8_gemm_nt_contiguous(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(out), _ptr(c),
+                                                    ctypes.cast(ks_host, ctypes.c_void_p), _ptr(ks_tensor), G, M,
+                                                    N, _stream()))
+
+
 def m_grouped_fp8_gemm_nt_nopad(lhs, rhs, out: torch.Tensor, counts: torch.Tensor) -> None:
     """No-padding layout: group g's rows are off_g .. off_g + counts[g] - 1 (off_g = sum of the earlier counts);
     out rows of group g = lhs rows of group g @ rhs[g]^T; rows past sum(counts) are untouched."""
@@ -281,7 +311,7 @@ def m_grouped_fp8_gemm_nt_nopad(lhs, rhs, out: torch.Tensor, counts: torch.Tenso
 
 __all__ = [
     "DGError", "fp8_gemm_nt", "fp8_gemm_nt_noalloc", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
-    "m_grouped_fp8_gemm_nt_nopad", "m_grouped_fp8_gemm_nn_contiguous",
+    "m_grouped_fp8_gemm_nt_nopad", "m_grouped_fp8_gemm_nn_contiguous", "k_grouped_fp8_gemm_nt_contiguous",
     "get_m_alignment_for_contiguous_layout", "set_m_alignment_for_contiguous_layout", "get_tma_aligned_size", "set_num_sms", "get_num_sms", "num_tiles",
     "select_block_n", "set_cta_pair_policy", "check_device_error", "lib", "header_symbols", "last_error",
 ]

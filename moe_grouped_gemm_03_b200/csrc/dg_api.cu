@@ -118,6 +118,22 @@ int make_output_map(CUtensorMap &map, void *base, long long rows, int N) {
     return DG_OK;
 }
 
+// D fp32 [G][M][N] (K-grouped calls): a 3-D map so a box never crosses from one group's M rows into the next;
+// boxes of 32 rows x 16 columns (64-byte rows) with the 64-byte swizzle, like the bf16 chunks.
+int make_output_map_f32(CUtensorMap &map, float *base, int G, int M, int N) {
+    EncodeTiledFn encode;
+    if (int rc = get_encode_fn(encode)) return rc;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(G)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(N) * 4, static_cast<cuuint64_t>(M) * N * 4};
+    cuuint32_t box[3] = {16, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (fp32 output) failed (%d)", static_cast<int>(r));
+    return DG_OK;
+}
+
 // Packed scale atoms: rows of 128 32-bit words (512 bytes), boxes of `box_rows` atoms, no swizzle.
 int make_atom_map(CUtensorMap &map, const uint32_t *base, long long atoms, int box_rows) {
     EncodeTiledFn encode;
@@ -172,6 +188,7 @@ struct ScaleArgs {
     int sfa_ld;
     const float *sfb;
     bool sfb_kn = false;  // SFB stored [G][K/128][ceil(N/128)] (B in the NN orientation)
+    int sfb_ld = 0;       // K-grouped: one scale per row of B, [K/128][sfb_ld]
 };
 
 // Launch of the scale pre-pass: one warp per atom, spread over every SM (one block each), so that every SM is
@@ -204,6 +221,7 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
     pk.sfa_ld = sc.sfa_ld;
     pk.sfb = sc.sfb;
     pk.sfb_kn = sc.sfb_kn ? 1 : 0;
+    pk.sfb_ld = sc.sfb_ld;
     pk.N = p.N;
     pk.G = p.G;
     pk.bn = BN;
@@ -223,13 +241,14 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
         pk.rows_per_group = p.M;
         pk.blocks_per_group = CTAS * ((p.M + C::TILE_M - 1) / C::TILE_M + p.G);
         pk.sfa_groups = 1;
-    } else {
+    } else {  // dense, contiguous, K-grouped (the groups share A's rows)
         pk.rows_per_group = p.M;
         pk.blocks_per_group = (p.M + dg::BLOCK_M - 1) / dg::BLOCK_M;
         pk.sfa_groups = 1;
     }
     const long long sfa_atoms = static_cast<long long>(pk.sfa_groups) * pk.blocks_per_group * p.num_sf_groups;
-    const long long sfb_atoms = static_cast<long long>(p.G) * p.num_n_blocks * p.num_sf_groups * C::SFB_ATOMS;
+    const long long b_groups = p.mode == dg::MODE_KGROUPED ? 1 : p.G;  // K-grouped: one B for all groups
+    const long long sfb_atoms = b_groups * p.num_n_blocks * p.num_sf_groups * C::SFB_ATOMS;
     pk.sfa_words = sfa_atoms * dg::SF_ATOM_WORDS;
     pk.sfb_words = sfb_atoms * dg::SF_ATOM_WORDS;
     cudaMemPool_t pool;
@@ -243,7 +262,11 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
     do {
         // ---- tensor maps (all host work is done before the two launches, so they reach the GPU back to back)
         CUtensorMap ta, tb, tsfa, tsfb, td;
-        if ((rc = make_output_map(td, p.d, a_rows, p.N))) break;
+        if (p.out_mode == dg::OUT_BF16)
+            rc = make_output_map(td, p.d, a_rows, p.N);
+        else
+            rc = make_output_map_f32(td, p.d32, p.G, p.M, p.N);
+        if (rc) break;
         if ((rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M, KPS))) break;
         if ((rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS, KPS))) break;
         if ((rc = make_atom_map(tsfa, pk.sfa_out, sfa_atoms, 1))) break;
@@ -374,7 +397,8 @@ int plan_and_launch(dg::GemmParams p, const DeviceInfo &info, const Plan &plan, 
     p.num_n_blocks = (p.N + bn - 1) / bn;
     const bool device_windows = p.mode == dg::MODE_MASKED || p.mode == dg::MODE_NOPAD;  // counted by the kernel
     p.num_windows = static_cast<int>(device_windows ? 0 : (pair ? plan.windows2 : plan.windows1));
-    p.num_sf_groups = (p.K / dg::BLOCK_K + dg::SF_GROUP - 1) / dg::SF_GROUP;
+    if (p.num_sf_groups == 0)  // (the K-grouped call counts its groups' scale groups itself)
+        p.num_sf_groups = (p.K / dg::BLOCK_K + dg::SF_GROUP - 1) / dg::SF_GROUP;
     const long long tiles = (pair ? plan.bound2 : plan.bound1) * p.num_n_blocks;
     const int grid = static_cast<int>(tiles < units ? tiles : units);
     if (grid <= 0) return DG_OK;
@@ -441,6 +465,7 @@ int launch_cfg_noalloc(const void *a, long long a_rows, const void *b, long long
     pk.sfa_ld = sc.sfa_ld;
     pk.sfb = sc.sfb;
     pk.sfb_kn = sc.sfb_kn ? 1 : 0;
+    pk.sfb_ld = sc.sfb_ld;
     pk.N = p.N;
     pk.G = p.G;
     pk.bn = BN;
@@ -747,6 +772,58 @@ int dg_m_grouped_fp8_gemm_nt_nopad(const void *a, const float *sfa, const void *
     const Plan plan{w1 + G / 2, w2 + G / 2, w1 + G, w2 + G, 0, 0, true};
     return plan_and_launch(p, info, plan, a, M_total, b, static_cast<long long>(G) * N, sc,
                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dg_k_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb, float *d,
+                                        const float *c, const int *ks, const int *ks_device, int G, int M, int N,
+                                        dg_stream_t stream) {
+    if (!a || !sfa || !b || !sfb || !d || !ks || !ks_device) return fail(DG_ERR_INVALID_ARG, "null pointer argument");
+    if (G < 1 || G > dg::MAX_MASKED_GROUPS)
+        return fail(DG_ERR_INVALID_ARG, "G=%d must be in [1, %d]", G, dg::MAX_MASKED_GROUPS);
+    if (M < 0 || N <= 0) return fail(DG_ERR_INVALID_ARG, "M=%d must be non-negative and N=%d positive", M, N);
+    if (N % 16) return fail(DG_ERR_ALIGNMENT, "N=%d must be a multiple of 16", N);
+    if (!aligned(a, 16) || !aligned(b, 16) || !aligned(d, 16) || (c && !aligned(c, 16)))
+        return fail(DG_ERR_ALIGNMENT, "a, b, c and d must be 16-byte aligned");
+    if (!aligned(sfa, 4) || !aligned(sfb, 4) || !aligned(ks_device, 4))
+        return fail(DG_ERR_ALIGNMENT, "sfa, sfb and ks_device must be 4-byte aligned");
+    long long K_total = 0, sf_groups = 0;
+    for (int g = 0; g < G; ++g) {
+        if (ks[g] < 0 || ks[g] % dg::BLOCK_K)
+            return fail(DG_ERR_ALIGNMENT, "ks[%d]=%d must be a non-negative multiple of %d", g, ks[g], dg::BLOCK_K);
+        K_total += ks[g];
+        sf_groups += (ks[g] / dg::BLOCK_K + dg::SF_GROUP - 1) / dg::SF_GROUP;
+    }
+    if (K_total > 0x7fffff80LL) return fail(DG_ERR_INVALID_ARG, "the sum of ks exceeds 2^31");
+    if (static_cast<long long>(G) * M * N > 0x7fffffffLL) return fail(DG_ERR_INVALID_ARG, "G*M*N exceeds 2^31");
+    if (M == 0) return DG_OK;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t d_bytes = static_cast<size_t>(G) * M * N * sizeof(float);
+    // D = C + sum: a separate C is copied into D first and the products are added to D in place
+    cudaError_t e;
+    if (c && c != d && (e = cudaMemcpyAsync(d, c, d_bytes, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemcpyAsync (C into D)");
+    if (K_total == 0) {  // nothing to add
+        if (!c && (e = cudaMemsetAsync(d, 0, d_bytes, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (D)");
+        return DG_OK;
+    }
+    DeviceInfo info;
+    if (int rc = device_info(info)) return rc;
+    dg::GemmParams p{};
+    p.mode = dg::MODE_KGROUPED;
+    p.out_mode = c ? dg::OUT_F32_ADD : dg::OUT_F32_STORE;
+    p.M = M; p.N = N; p.K = static_cast<int>(K_total); p.G = G;
+    p.num_sf_groups = static_cast<int>(sf_groups);
+    p.d32 = d;
+    p.masked_m = ks_device;
+    p.err = device_error_word();
+    if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
+    ScaleArgs sc{sfa, dg_get_tma_aligned_size(M, 4), sfb};
+    sc.sfb_ld = dg_get_tma_aligned_size(N, 4);
+    // every group covers all M rows: G x ceil(M / rows per window) windows
+    const long long w1 = static_cast<long long>(G) * ((M + dg::BLOCK_M - 1) / dg::BLOCK_M);
+    const long long w2 = static_cast<long long>(G) * ((M + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M));
+    const Plan plan{w1, w2, w1, w2, w1, w2, true};
+    return plan_and_launch(p, info, plan, a, M, b, N, sc, s);
 }
 
 int dg_set_cta_pair_policy(int policy) {

@@ -52,7 +52,9 @@
 
 namespace dg {
 
-enum : int { MODE_DENSE = 0, MODE_CONTIGUOUS = 1, MODE_MASKED = 2, MODE_NOPAD = 3 };
+enum : int { MODE_DENSE = 0, MODE_CONTIGUOUS = 1, MODE_MASKED = 2, MODE_NOPAD = 3, MODE_KGROUPED = 4 };
+// output: bf16 D (the M-grouped and dense calls), fp32 D written, or fp32 D += the product (K-grouped call)
+enum : int { OUT_BF16 = 0, OUT_F32_STORE = 1, OUT_F32_ADD = 2 };
 
 constexpr int BLOCK_M = 128;  // rows per CTA
 constexpr int BLOCK_K = 128;  // = the scale block along K
@@ -75,15 +77,18 @@ constexpr unsigned ERR_BAD_GROUP = 2u;
 
 struct GemmParams {
     int mode;
-    int M;             // dense: M; contiguous / no padding: M_total; masked: M_max
+    int M;             // dense: M; contiguous / no padding: M_total; masked: M_max; K-grouped: M
+    int out_mode;      // OUT_*
     int N, K, G;
-    int num_windows;   // dense / contiguous: windows (128- or 256-row); masked / no padding: unused
+    int num_windows;   // dense / contiguous: windows (128- or 256-row); K-grouped: G x windows of M;
+                       // masked / no padding: unused
     int num_n_blocks;  // ceil(N / BN)
-    int num_sf_groups; // ceil(K / (128 * SF_GROUP))
+    int num_sf_groups; // ceil(K / (128 * SF_GROUP)); K-grouped: the sum over groups of ceil(K_g / (128 * SF_GROUP))
     int sfa_blocks;    // 128-row blocks per group of the packed SFA (masked layout)
     __nv_bfloat16 *d;
+    float *d32;        // fp32 output (out_mode != OUT_BF16): [G][M][N]
     const int *m_indices;
-    const int *masked_m;  // masked: masked_m; no padding: the groups' row counts
+    const int *masked_m;  // masked: masked_m; no padding: the groups' row counts; K-grouped: the groups' K extents
     unsigned *err;
     unsigned long long wait_limit_ns;  // limit of any single wait
     int skip_first_load;               // test hook: the first CTA (pair) never loads stage 0
@@ -151,9 +156,10 @@ struct Tile {
 
 struct SharedCtl {
     volatile int *abort;
-    const int *prefix;   // masked / no padding: window prefix per group; contiguous pairs: first block of each window
-    const int *mm;       // masked / no padding: the groups' clamped row counts
-    const int *off;      // no padding: first row of each group
+    const int *prefix;   // masked / no padding: window prefix per group; contiguous pairs: first block of each
+                         // window; K-grouped: first packed scale group of each group
+    const int *mm;       // masked / no padding: the groups' clamped row counts; K-grouped: 128-K blocks per group
+    const int *off;      // no padding: first row of each group; K-grouped: first 128-K block of each group
     const short *gblk;   // contiguous pairs, kernel prologue only: group of each 128-row block
 };
 
@@ -226,6 +232,12 @@ __device__ __forceinline__ bool decode_tile(const GemmParams &p, const SharedCtl
     if (p.mode == MODE_DENSE) {
         ti.g = 0;
         ti.row0 = ti.local_row0 = w * C::TILE_M;
+        return true;
+    }
+    if (p.mode == MODE_KGROUPED) {  // every group covers all M rows; windows of a group are consecutive
+        const int per_group = p.num_windows / p.G;
+        ti.g = w / per_group;
+        ti.row0 = ti.local_row0 = (w - ti.g * per_group) * C::TILE_M;
         return true;
     }
     if (p.mode == MODE_CONTIGUOUS) {
@@ -437,6 +449,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             s_mm[g] = m;
         }
+    } else if (p.mode == MODE_KGROUPED) {
+        for (int g = threadIdx.x; g < p.G; g += NUM_THREADS) {
+            const int k = __ldg(p.masked_m + g);  // a K extent: a non-negative multiple of 128
+            if (k < 0 || k % BLOCK_K) raise_error(p.err, ERR_BAD_GROUP);
+            s_mm[g] = k < 0 ? 0 : k / BLOCK_K;
+        }
     } else if (pair_contig) {
         // several independent loads in flight per thread (m_indices is usually cold in L2 here)
         constexpr int U = 8;
@@ -460,8 +478,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             build_group_rows(p.G, p.M, s_mm, s_off, p.err, lane);
             __syncwarp();
         }
-        if (p.mode == MODE_MASKED || p.mode == MODE_NOPAD) build_window_prefix(p.G, C::TILE_M, s_mm, s_prefix, lane);
-        else if (pair_contig) build_pair_windows(num_blocks, s_gblk, s_prefix, lane);
+        if (p.mode == MODE_KGROUPED) {
+            // each group's first 128-K block (clipped to K) and first packed scale group (SF_GROUP blocks each)
+            build_group_rows(p.G, p.K / BLOCK_K, s_mm, s_off, p.err, lane);
+            __syncwarp();
+            build_window_prefix(p.G, SF_GROUP, s_mm, s_prefix, lane);
+        } else if (p.mode == MODE_MASKED || p.mode == MODE_NOPAD) {
+            build_window_prefix(p.G, C::TILE_M, s_mm, s_prefix, lane);
+        } else if (pair_contig) {
+            build_pair_windows(num_blocks, s_gblk, s_prefix, lane);
+        }
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -535,8 +561,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int k = 0; k < my_tiles && ok; ++k) {
                 Tile ti;
                 if (!tile_at(k, ti)) continue;
+                // K-grouped: one B for all groups, each group contracts its own range of 128-K blocks and owns
+                // its own packed scale groups
+                const bool kgrouped = p.mode == MODE_KGROUPED;
+                const int gb = kgrouped ? 0 : ti.g;                       // B's group
+                const int tile_nkb = kgrouped ? ctl_main.mm[ti.g] : nkb;  // 128-K blocks of this tile
+                const int kbase = kgrouped ? ctl_main.off[ti.g] : 0;      // its first 128-K block
+                const int qbase = kgrouped ? ctl_main.prefix[ti.g] : 0;   // its first packed scale group
                 const int arow = ti.row0 + my_rows;
-                const int brow = ti.g * p.N + ti.n0 + static_cast<int>(rank) * C::B_ROWS;
+                const int brow = gb * p.N + ti.n0 + static_cast<int>(rank) * C::B_ROWS;
                 // packed scale atoms: SFA [block][group], SFB [g][n block][group][atom]
                 // (no padding: atoms of each group's windows, CTAS blocks per window, after the earlier groups')
                 int sfa_block = (ti.local_row0 + my_rows) / BLOCK_M;
@@ -546,16 +579,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     sfa_block += CTAS * ctl_main.prefix[ti.g];
                 else
                     sfa_block = (ti.row0 + my_rows) / BLOCK_M;
-                const int sfa_y0 = sfa_block * p.num_sf_groups;
-                const int sfb_y0 = (ti.g * p.num_n_blocks + ti.nb) * p.num_sf_groups * C::SFB_ATOMS;
-                for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
+                const int sfa_y0 = sfa_block * p.num_sf_groups + qbase;
+                const int sfb_y0 = ((gb * p.num_n_blocks + ti.nb) * p.num_sf_groups + qbase) * C::SFB_ATOMS;
+                for (int kb0 = 0; kb0 < tile_nkb; kb0 += C::KPS) {
                     const bool group_start = kb0 % SF_GROUP == 0;
                     if (issued == STAGES) wait_for_scales();  // the ring is full: the MMAs need the scales now
                     if (!wait_bounded(&empty[s], ph ^ 1u, s_abort, p.err, p.wait_limit_ns)) { ok = false; break; }
                     uint8_t *a_dst = sA + s * C::A_BYTES;
                     uint8_t *b_dst = sB + s * C::B_BYTES;
                     const int q = kb0 / SF_GROUP;
-                    // one 3-D box per operand brings KPS K blocks (a block past K arrives zero-filled and unused)
+                    // one 3-D box per operand brings KPS K blocks (a block past the tile's K range arrives zero-filled,
+                    // or from the next K group, and is unused)
                     const uint32_t bytes =
                         static_cast<uint32_t>(C::A_BYTES + C::B_BYTES + (group_start ? C::SF_BYTES : 0));
                     if constexpr (PAIR) {
@@ -564,12 +598,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         // transaction count dips below zero but the phase cannot complete before the arrival.
                         const uint32_t leader_full = full_leader0 + 8u * static_cast<uint32_t>(s);
                         if (rank == 0) mbar_arrive_expect_tx(&full[s], CTAS * bytes);
-                        tma_load_3d_pair(a_dst, &tmap_a, leader_full, 0, arow, kb0);
-                        tma_load_3d_pair(b_dst, &tmap_b, leader_full, 0, brow, kb0);
+                        tma_load_3d_pair(a_dst, &tmap_a, leader_full, 0, arow, kbase + kb0);
+                        tma_load_3d_pair(b_dst, &tmap_b, leader_full, 0, brow, kbase + kb0);
                     } else {
                         mbar_arrive_expect_tx(&full[s], bytes);
-                        tma_load_3d(a_dst, &tmap_a, &full[s], 0, arow, kb0);
-                        tma_load_3d(b_dst, &tmap_b, &full[s], 0, brow, kb0);
+                        tma_load_3d(a_dst, &tmap_a, &full[s], 0, arow, kbase + kb0);
+                        tma_load_3d(b_dst, &tmap_b, &full[s], 0, brow, kbase + kb0);
                     }
                     if (group_start) {
                         if (scales_ready) {
@@ -617,8 +651,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
                 uint32_t sf_tmem = 0;
-                for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
-                    const int nk = min(C::KPS, nkb - kb0);
+                // (K-grouped: a group with no K blocks issues no MMA; its epilogue writes zeros or nothing)
+                const int tile_nkb = p.mode == MODE_KGROUPED ? ctl_main.mm[ti.g] : nkb;
+                for (int kb0 = 0; kb0 < tile_nkb; kb0 += C::KPS) {
+                    const int nk = min(C::KPS, tile_nkb - kb0);
                     if (!wait_bounded(&full[s], ph, s_abort, p.err, p.wait_limit_ns)) { ok = false; break; }
                     tc_fence_after_sync();
                     if (kb0 % SF_GROUP == 0) {
@@ -680,56 +716,100 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!tile_at(k, ti)) continue;
             if (!warp_wait_bounded(&tmem_full[acc], acc_ph, s_abort, p.err, p.wait_limit_ns, lane)) break;
             tc_fence_after_sync();
-            const int r_local = my_rows + 32 * q + lane;
-            const int row = ti.row0 + r_local;
-            bool valid;
-            if (p.mode == MODE_DENSE)
-                valid = row < p.M;
-            else if (p.mode == MODE_CONTIGUOUS)
-                valid = row < p.M && __ldg(p.m_indices + row) == ti.g;
-            else
-                valid = ti.local_row0 + r_local < ctl.mm[ti.g];
-            // dense rows past M lie outside D and are clipped by the store
-            const bool tma_ok = p.mode == MODE_DENSE || __all_sync(0xffffffffu, valid);
-            __nv_bfloat16 *out = p.d + static_cast<size_t>(row) * p.N + ti.n0;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * BN);
+            if (p.out_mode != OUT_BF16) {
+                // fp32 D [G][M][N] through a 3-D map that clips rows past M: per 32-column TMEM load two 16-column
+                // chunks (64-byte rows, the same swizzled staging), each stored or added by one TMA operation.
+                const bool no_k = ctl.mm[ti.g] == 0;  // an empty K range: the accumulator holds nothing
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(t_row + 32 * c, r);
-                tmem_ld_wait_regs(r);
-                uint32_t h[16];
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + 32 * c, r);
+                    tmem_ld_wait_regs(r);
+                    if (no_k) {
+                        if (p.out_mode == OUT_F32_ADD) continue;  // adding zeros
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-                    h[j] = *reinterpret_cast<uint32_t *>(&v);
-                }
-                if (tma_ok) {
-                    uint8_t *buf = stage_buf + (chunk_count & 1) * EPI_CHUNK_BYTES;
-                    if (chunk_count >= 2) {
-                        if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
+                        for (int j = 0; j < 32; ++j) r[j] = 0u;
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint8_t *buf = stage_buf + (chunk_count & 1) * EPI_CHUNK_BYTES;
+                        if (chunk_count >= 2) {
+                            if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
+                            __syncwarp();
+                        }
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int sw = j ^ ((lane >> 1) & 3);
+                            *reinterpret_cast<uint4 *>(buf + lane * 64 + sw * 16) =
+                                make_uint4(r[16 * h + 4 * j], r[16 * h + 4 * j + 1], r[16 * h + 4 * j + 2],
+                                           r[16 * h + 4 * j + 3]);
+                        }
+                        fence_proxy_async_smem();
                         __syncwarp();
+                        if (lane == 0) {
+                            const int x = ti.n0 + 32 * c + 16 * h, y = ti.row0 + my_rows + 32 * q;
+                            if (p.out_mode == OUT_F32_ADD)
+                                tma_reduce_add_3d(&tmap_d, buf, x, y, ti.g);
+                            else
+                                tma_store_3d(&tmap_d, buf, x, y, ti.g);
+                            bulk_commit_group();
+                        }
+                        ++chunk_count;
                     }
+                }
+            } else {
+                const int r_local = my_rows + 32 * q + lane;
+                const int row = ti.row0 + r_local;
+                bool valid;
+                if (p.mode == MODE_DENSE)
+                    valid = row < p.M;
+                else if (p.mode == MODE_CONTIGUOUS)
+                    valid = row < p.M && __ldg(p.m_indices + row) == ti.g;
+                else
+                    valid = ti.local_row0 + r_local < ctl.mm[ti.g];
+                // dense rows past M lie outside D and are clipped by the store
+                const bool tma_ok = p.mode == MODE_DENSE || __all_sync(0xffffffffu, valid);
+                __nv_bfloat16 *out = p.d + static_cast<size_t>(row) * p.N + ti.n0;
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + 32 * c, r);
+                    tmem_ld_wait_regs(r);
+                    uint32_t h[16];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int sw = j ^ ((lane >> 1) & 3);
-                        *reinterpret_cast<uint4 *>(buf + lane * 64 + sw * 16) =
-                            make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+                    for (int j = 0; j < 16; ++j) {
+                        __nv_bfloat162 v =
+                            __floats2bfloat162_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                        h[j] = *reinterpret_cast<uint32_t *>(&v);
                     }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tmap_d, buf, ti.n0 + 32 * c, ti.row0 + my_rows + 32 * q);
-                        bulk_commit_group();
-                    }
-                    ++chunk_count;
-                } else if (valid) {
+                    if (tma_ok) {
+                        uint8_t *buf = stage_buf + (chunk_count & 1) * EPI_CHUNK_BYTES;
+                        if (chunk_count >= 2) {
+                            if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
+                            __syncwarp();
+                        }
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int col = ti.n0 + 32 * c + 8 * j;
-                        if (col < p.N)
-                            *reinterpret_cast<uint4 *>(out + 32 * c + 8 * j) =
+                        for (int j = 0; j < 4; ++j) {
+                            const int sw = j ^ ((lane >> 1) & 3);
+                            *reinterpret_cast<uint4 *>(buf + lane * 64 + sw * 16) =
                                 make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmap_d, buf, ti.n0 + 32 * c, ti.row0 + my_rows + 32 * q);
+                            bulk_commit_group();
+                        }
+                        ++chunk_count;
+                    } else if (valid) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int col = ti.n0 + 32 * c + 8 * j;
+                            if (col < p.N)
+                                *reinterpret_cast<uint4 *>(out + 32 * c + 8 * j) =
+                                    make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+                        }
                     }
                 }
             }

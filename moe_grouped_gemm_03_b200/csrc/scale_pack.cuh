@@ -33,6 +33,7 @@ struct PackParams {
     // SFB: fp32 [G][ceil(N/128)][K/128], or [G][K/128][ceil(N/128)] when sfb_kn (B in the NN orientation)
     const float *sfb;
     int sfb_kn;
+    int sfb_ld;           // K-grouped: row extent of the MN-major SFB [K/128][sfb_ld]
     int N, G, bn, n_tiles, sfb_atoms;
     int nkb, num_sf_groups;
     uint32_t *sfa_out;    // [sfa_groups * blocks_per_group][num_sf_groups][128]
@@ -49,22 +50,39 @@ constexpr int PACK_THREADS = 1024;
 // with one 16-byte store, so an atom is one coalesced 512-byte write.
 __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackParams p) {
     grid_launch_dependents();  // the GEMM may start its prologue; it waits for this grid before reading
-    // no padding: the groups' clamped counts, first rows and window prefix, as the GEMM derives them
+    // The group tables, as the GEMM derives them.  No padding: clamped row counts, first rows, window prefix.
+    // K-grouped: 128-K blocks per group, first 128-K block, prefix of packed scale groups (SF_GROUP blocks).
     __shared__ int s_cnt[MAX_MASKED_GROUPS], s_off[MAX_MASKED_GROUPS], s_wpre[MAX_MASKED_GROUPS + 1];
-    const bool nopad = p.mode == MODE_NOPAD;
-    if (nopad) {
+    const bool nopad = p.mode == MODE_NOPAD, kgrouped = p.mode == MODE_KGROUPED;
+    if (nopad || kgrouped) {
         for (int g = threadIdx.x; g < p.G; g += blockDim.x) {
             const int c = __ldg(p.counts + g);
-            s_cnt[g] = c < 0 ? 0 : c;
+            s_cnt[g] = c < 0 ? 0 : (kgrouped ? c / 128 : c);
         }
         __syncthreads();
         if (threadIdx.x < 32) {
-            build_group_rows(p.G, p.rows_per_group, s_cnt, s_off, nullptr, threadIdx.x);
+            build_group_rows(p.G, kgrouped ? p.nkb : p.rows_per_group, s_cnt, s_off, nullptr, threadIdx.x);
             __syncwarp();
-            build_window_prefix(p.G, p.tile_m, s_cnt, s_wpre, threadIdx.x);
+            build_window_prefix(p.G, kgrouped ? SF_GROUP : p.tile_m, s_cnt, s_wpre, threadIdx.x);
         }
         __syncthreads();
     }
+    // the 128-K blocks of packed scale group q: first block and how many exist (K-grouped: q counts the groups'
+    // scale groups one after another, each group's starting at its own first block)
+    auto k_blocks = [&](int q, int &kb_first, int &kb_count) {
+        if (!kgrouped) {
+            kb_first = SF_GROUP * q;
+            kb_count = p.nkb - kb_first;
+        } else if (q < s_wpre[p.G]) {
+            const int g = upper_index(s_wpre, p.G, q);
+            const int local = SF_GROUP * (q - s_wpre[g]);
+            kb_first = s_off[g] + local;
+            kb_count = s_cnt[g] - local;
+        } else {
+            kb_first = 0;
+            kb_count = 0;  // past the last scale group: never read
+        }
+    };
     const long long sfa_atoms = p.sfa_words / SF_ATOM_WORDS;
     const long long total = sfa_atoms + p.sfb_words / SF_ATOM_WORDS;
     const int lane = threadIdx.x & 31;
@@ -96,14 +114,16 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
                 rows = p.rows_per_group - first;
             }
             const float *base = p.sfa + group_base;
+            int kb_first, kb_count;
+            k_blocks(q, kb_first, kb_count);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int r = lane + 32 * j;
                 const int row = first + r;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int kb = 4 * q + i;
-                    const uint32_t code = (r < rows && row < p.sfa_ld && kb < p.nkb)
+                    const int kb = kb_first + i;
+                    const uint32_t code = (r < rows && row < p.sfa_ld && i < kb_count)
                                               ? ue8m0_code(__ldg(base + static_cast<size_t>(kb) * p.sfa_ld + row))
                                               : 0x7Fu;
                     word[j] |= code << (8 * i);
@@ -118,17 +138,29 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
             rest /= p.num_sf_groups;
             const int nt = static_cast<int>(rest % p.n_tiles);
             const int g = static_cast<int>(rest / p.n_tiles);
+            int kb_first, kb_count;
+            k_blocks(q, kb_first, kb_count);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int n = nt * p.bn + a * 128 + lane + 32 * j;
-                // SFB element (g, n/128, kb) sits at base + kb * stride_kb
-                const size_t stride_kb = p.sfb_kn ? static_cast<size_t>(nnb128) : 1;
-                const float *base = p.sfb_kn ? p.sfb + static_cast<size_t>(g) * p.nkb * nnb128 + n / 128
-                                             : p.sfb + (static_cast<size_t>(g) * nnb128 + n / 128) * p.nkb;
+                // SFB element of column n and K block kb sits at base + kb * stride_kb: 128x128 blocks
+                // [G][N/128][K/128] or, NN, [G][K/128][N/128]; K-grouped: one scale per row n, [K/128][sfb_ld]
+                size_t stride_kb;
+                const float *base;
+                if (kgrouped) {
+                    stride_kb = static_cast<size_t>(p.sfb_ld);
+                    base = p.sfb + n;
+                } else if (p.sfb_kn) {
+                    stride_kb = static_cast<size_t>(nnb128);
+                    base = p.sfb + static_cast<size_t>(g) * p.nkb * nnb128 + n / 128;
+                } else {
+                    stride_kb = 1;
+                    base = p.sfb + (static_cast<size_t>(g) * nnb128 + n / 128) * p.nkb;
+                }
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int kb = 4 * q + i;
-                    const uint32_t code = (n < p.N && kb < p.nkb) ? ue8m0_code(__ldg(base + kb * stride_kb)) : 0x7Fu;
+                    const int kb = kb_first + i;
+                    const uint32_t code = (n < p.N && i < kb_count) ? ue8m0_code(__ldg(base + kb * stride_kb)) : 0x7Fu;
                     word[j] |= code << (8 * i);
                 }
             }

@@ -78,7 +78,8 @@ class Problem:
 
     @property
     def rows(self) -> int:
-        return self.a.shape[0]
+        """Rows of the flattened output (= rows of ``a`` except for K-grouped problems, G x M)."""
+        return self.G * self.M if self.kind == "k_grouped" else self.a.shape[0]
 
     def valid_rows(self) -> np.ndarray:
         """Global row indices (into ``a`` / the flattened output) that the GEMM must produce."""
@@ -328,7 +329,7 @@ CONFIGS = {
     5: "M-grouped contiguous FP8 GEMM G=64 N=7168 K=2048, Zipf(1.2) split of 65536 tokens",
     6: "M-grouped no-padding FP8 GEMM G=64 N=7168 K=2048, Zipf(1.2) split of 65536 tokens",
     7: "M-grouped contiguous FP8 NN GEMM (B [G, K, N]) G=8 N=4096 K=7168, tokens U[1024,8192] per group",
-    8: "K-grouped FP8 NT GEMM, fp32 D += A_g B_g^T, G=8 M=4096 N=7168, K_g = tokens U[1024,8192] rounded up to 128",
+    8: "K-grouped FP8 NT GEMM, fp32 D_g = A_g B_g^T, G=8 M=4096 N=7168, K_g = tokens U[1024,8192] rounded up to 128",
 }
 
 
@@ -349,7 +350,8 @@ def make_config(i: int, seed: int = 0) -> Problem:
     if i == 8:
         rng = np.random.default_rng(seed)
         counts = rng.integers(1024, 8192, endpoint=True, size=8)
-        return make_k_grouped([align_up(int(c), SCALE_BLOCK) for c in counts], 4096, 7168, rng=rng, name=CONFIGS[8])
+        return make_k_grouped([align_up(int(c), SCALE_BLOCK) for c in counts], 4096, 7168, rng=rng, with_c=False,
+                              name=CONFIGS[8])
     if i == 7:
         rng = np.random.default_rng(seed)
         counts = rng.integers(1024, 8192, endpoint=True, size=8)

@@ -11,8 +11,13 @@ def run_problem(p, tensors=None, out=None, stream=None):
 
     t = tensors if tensors is not None else synth.to_torch(p)
     if out is None:
-        out = torch.empty(p.out_shape(), dtype=torch.bfloat16, device="cuda")
-        out.view(torch.int16).fill_(-1)  # 0xFFFF
+        dtype = torch.float32 if p.kind == "k_grouped" else torch.bfloat16
+        out = torch.empty(p.out_shape(), dtype=dtype, device="cuda")
+        out.view(torch.int16).fill_(-1)  # 0xFFFF (a NaN in either type)
+    if p.kind == "k_grouped":  # C, when the problem has one, is passed as a separate tensor
+        dg.k_grouped_fp8_gemm_nt_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, p.counts.tolist(),
+                                            t["ks"], t.get("c"))
+        return out
     if p.kind == "dense":
         dg.fp8_gemm_nt((t["a"], t["sfa"]), (t["b"], t["sfb"]), out)
     elif p.kind == "contiguous":
@@ -56,6 +61,6 @@ def assert_close(gpu: np.ndarray, ref: np.ndarray, what: str = ""):
 
 def untouched_rows_ok(out: torch.Tensor, rows_mask: np.ndarray) -> bool:
     """True if every row where rows_mask is False still holds the sentinel bits."""
-    bits = out.view(torch.int16).reshape(-1, out.shape[-1]).cpu().numpy().view(np.uint16)
+    bits = out.view(torch.int16).reshape(rows_mask.shape[0], -1).cpu().numpy().view(np.uint16)
     keep = ~rows_mask
     return bool((bits[keep] == SENTINEL_BITS).all())

@@ -113,6 +113,41 @@ def test_nn_equals_nt_on_the_transposed_b(policy):
     assert torch.equal(a[valid], b[valid])
 
 
+def _run_k_grouped(p, c_mode):
+    """c_mode: 'none' (D = products), 'separate' (C in its own tensor) or 'inplace' (D holds C on entry)."""
+    import moe_grouped_gemm_03_b200 as dg
+
+    t = synth.to_torch(p)
+    out = torch.full(p.out_shape(), float("nan"), dtype=torch.float32, device="cuda")
+    c = None
+    if c_mode == "separate":
+        c = t["c"]
+    elif c_mode == "inplace":
+        out.copy_(t["c"])
+        c = out
+    dg.k_grouped_fp8_gemm_nt_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, p.counts.tolist(), t["ks"], c)
+    dg.check_device_error()
+    return out.cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("ks,M,N", [
+    ([128, 256, 384], 256, 512),
+    ([0, 128, 640], 200, 272),    # an empty K range, M and N tails
+    ([512] * 4, 136, 1040),
+    ([128], 1, 16),               # one row, narrowest N
+    ([384, 128], 1000, 2048),     # several waves of tiles
+])
+@pytest.mark.parametrize("c_mode", ["none", "separate", "inplace"])
+def test_k_grouped_shapes(ks, M, N, c_mode, policy):
+    p = synth.make_k_grouped(ks, M, N, seed=sum(ks) + M + N, with_c=c_mode != "none")
+    got = _run_k_grouped(p, c_mode)
+    ref = oracle.problem_full(p)
+    assert_close(got.reshape(-1, N), ref.reshape(-1, N), p.name)
+    # fp32 output: far tighter than the bf16 tolerance (fp32 accumulation over at most 640 products per group)
+    rms = float(np.sqrt((ref * ref).mean()))
+    assert np.abs(got - ref).max() <= 1e-4 * rms + 1e-5 * np.abs(ref).max()
+
+
 @pytest.fixture
 def alignment_256():
     import moe_grouped_gemm_03_b200 as dg
