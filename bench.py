@@ -29,7 +29,8 @@ if ROOT not in sys.path:
 FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio (4.5 / 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["moe_grouped_gemm_03_b200/csrc/gemm_kernel.cuh", "moe_grouped_gemm_03_b200/csrc/ptx.cuh",
-                  "moe_grouped_gemm_03_b200/csrc/dg_api.cu"]
+                  "moe_grouped_gemm_03_b200/csrc/dg_api.cu", "moe_grouped_gemm_03_b200/csrc/scale_pack.cuh",
+                  "moe_grouped_gemm_03_b200/csrc/transpose.cuh"]
 
 
 def parse():
