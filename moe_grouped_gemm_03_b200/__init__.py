@@ -100,17 +100,21 @@ def _stream() -> int:
 _FP8_TYPES = (torch.uint8, torch.float8_e4m3fn)
 
 
-def _need(cond: bool, what: str):
+def _need(cond: bool, what) -> None:
+    """Raise DG_ERR_INVALID_ARG when cond is false; `what` is the message or a callable that builds it (messages
+    are only formatted on failure, which keeps a passing check cheap)."""
     if not cond:
-        raise DGError(-1, what)
+        raise DGError(-1, what() if callable(what) else what)
 
 
 def _check_operand(name, t, dims, dtypes):
-    _need(isinstance(t, torch.Tensor), f"{name} must be a torch.Tensor")
-    _need(t.dim() == dims, f"{name} must have {dims} dims, got {tuple(t.shape)}")
-    _need(t.dtype in dtypes, f"{name} has dtype {t.dtype}, expected one of {dtypes}")
-    _need(t.is_contiguous(), f"{name} must be contiguous")
-    _need(t.is_cuda, f"{name} must be a CUDA tensor")
+    if isinstance(t, torch.Tensor) and t.dim() == dims and t.dtype in dtypes and t.is_cuda and t.is_contiguous():
+        return
+    _need(isinstance(t, torch.Tensor), lambda: f"{name} must be a torch.Tensor")
+    _need(t.dim() == dims, lambda: f"{name} must have {dims} dims, got {tuple(t.shape)}")
+    _need(t.dtype in dtypes, lambda: f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    _need(t.is_contiguous(), lambda: f"{name} must be contiguous")
+    _need(t.is_cuda, lambda: f"{name} must be a CUDA tensor")
 
 
 # ------------------------------------------------------------------------------------------------ utilities
@@ -176,7 +180,7 @@ def fp8_gemm_nt(lhs: Tuple[torch.Tensor, torch.Tensor], rhs: Tuple[torch.Tensor,
     M, K = a.shape
     N = b.shape[0]
     _need(b.shape[1] == K and tuple(out.shape) == (M, N), "shape mismatch between a, b and out")
-    _need(sfa.shape == (K // 128, get_tma_aligned_size(M, 4)), f"sfa must be [{K // 128}, {get_tma_aligned_size(M, 4)}]")
+    _need(sfa.shape == (K // 128, get_tma_aligned_size(M, 4)), lambda: f"sfa must be [{K // 128}, {get_tma_aligned_size(M, 4)}]")
     _need(sfb.shape == ((N + 127) // 128, K // 128), "sfb must be [ceil(N/128), K/128]")
     _check(_lib.dg_fp8_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(out), M, N, K, _stream()))
 
@@ -196,7 +200,7 @@ def fp8_gemm_nt_noalloc(lhs: Tuple[torch.Tensor, torch.Tensor], rhs: Tuple[torch
     M, K = a.shape
     N = b.shape[0]
     _need(b.shape[1] == K and tuple(out.shape) == (M, N), "shape mismatch between a, b and out")
-    _need(sfa.shape == (K // 128, get_tma_aligned_size(M, 4)), f"sfa must be [{K // 128}, {get_tma_aligned_size(M, 4)}]")
+    _need(sfa.shape == (K // 128, get_tma_aligned_size(M, 4)), lambda: f"sfa must be [{K // 128}, {get_tma_aligned_size(M, 4)}]")
     _need(sfb.shape == ((N + 127) // 128, K // 128), "sfb must be [ceil(N/128), K/128]")
     _check(_lib.dg_fp8_gemm_nt_noalloc(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(out), M, N, K, _stream()))
 

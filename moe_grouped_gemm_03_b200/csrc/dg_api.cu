@@ -47,6 +47,12 @@ struct DeviceInfo {
 int device_info(DeviceInfo &info) {
     cudaError_t e = cudaGetDevice(&info.device);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    // the attributes of a device do not change: queried once per device
+    static DeviceInfo cache[64];
+    if (info.device >= 0 && info.device < 64 && cache[info.device].device == info.device) {
+        info = cache[info.device];
+        return DG_OK;
+    }
     if ((e = cudaDeviceGetAttribute(&info.num_sms, cudaDevAttrMultiProcessorCount, info.device)) != cudaSuccess)
         return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
     if ((e = cudaDeviceGetAttribute(&info.major, cudaDevAttrComputeCapabilityMajor, info.device)) != cudaSuccess)
@@ -56,6 +62,7 @@ int device_info(DeviceInfo &info) {
     if (info.major != 10 || info.minor != 0)
         return fail(DG_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a only", info.device,
                     info.major, info.minor);
+    if (info.device >= 0 && info.device < 64) cache[info.device] = info;
     return DG_OK;
 }
 
@@ -197,8 +204,8 @@ struct ScaleArgs {
 int launch_pack(const dg::PackParams &pk, int device, cudaStream_t stream) {
     const long long atoms = (pk.sfa_words + pk.sfb_words) / dg::SF_ATOM_WORDS;
     constexpr long long kMaxWarps = dg::PACK_THREADS / 32;
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms <= 0) sms = 1;
+    DeviceInfo info;  // (cached per device)
+    const int sms = device_info(info) == DG_OK && info.device == device && info.num_sms > 0 ? info.num_sms : 1;
     long long blocks = atoms < sms ? atoms : sms;
     if (blocks < 1) blocks = 1;
     long long warps = (atoms + blocks - 1) / blocks;
@@ -273,10 +280,14 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
         if ((rc = make_atom_map(tsfb, pk.sfb_out, sfb_atoms, C::SFB_ATOMS))) break;
         // ---- the GEMM, as a programmatic dependent of the pre-pass
         auto kernel = dg::fp8_gemm_kernel<C>;
-        if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) !=
-            cudaSuccess) {
-            rc = cuda_fail(e, "cudaFuncSetAttribute");
-            break;
+        static bool smem_set[64] = {false};  // per instantiation and device: the attribute persists
+        if (!(device >= 0 && device < 64 && smem_set[device])) {
+            if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) !=
+                cudaSuccess) {
+                rc = cuda_fail(e, "cudaFuncSetAttribute");
+                break;
+            }
+            if (device >= 0 && device < 64) smem_set[device] = true;
         }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(grid * CTAS), 1, 1);
@@ -406,8 +417,13 @@ int plan_and_launch(dg::GemmParams p, const DeviceInfo &info, const Plan &plan, 
 }
 
 unsigned *device_error_word() {
+    int device = 0;
+    if (cudaGetDevice(&device) != cudaSuccess) return nullptr;
+    static unsigned *cache[64] = {nullptr};  // the symbol's address on each device, looked up once
+    if (device >= 0 && device < 64 && cache[device]) return cache[device];
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
+    if (device >= 0 && device < 64) cache[device] = static_cast<unsigned *>(p);
     return static_cast<unsigned *>(p);
 }
 
