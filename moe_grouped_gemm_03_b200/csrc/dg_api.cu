@@ -90,19 +90,16 @@ int get_encode_fn(EncodeTiledFn &fn) {
 }
 
 // Row-major byte matrix [rows][K] (K-major e4m3 operand), boxes of box_rows x 128 bytes, 128-byte swizzle.
-// A or B, e4m3 K-major [rows][K], viewed as 3-D (128 bytes of a K block, row, K block) so that one box brings
-// `kps` K blocks of `box_rows` rows (laid out [K block][row][128 B] with the 128-byte swizzle, one swizzle
-// atom per 8 rows).  One request per operand per stage moves more bytes per SM than one 2-D box per K block.
-int make_operand_map(CUtensorMap &map, const void *base, long long rows, int K, int box_rows, int kps) {
+// A or B, e4m3 K-major [rows][K]: boxes of one 128-K block (128 bytes) x `box_rows` rows with the 128-byte
+// swizzle (one swizzle atom per 8 rows), the layout the MMA's shared-memory descriptors expect.
+int make_operand_map(CUtensorMap &map, const void *base, long long rows, int K, int box_rows) {
     EncodeTiledFn encode;
     if (int rc = get_encode_fn(encode)) return rc;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(dg::BLOCK_K), static_cast<cuuint64_t>(rows),
-                          static_cast<cuuint64_t>(K / dg::BLOCK_K)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(dg::BLOCK_K)};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(dg::BLOCK_K), static_cast<cuuint32_t>(box_rows),
-                         static_cast<cuuint32_t>(kps)};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(dg::BLOCK_K), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
@@ -274,8 +271,8 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
         else
             rc = make_output_map_f32(td, p.d32, p.G, p.M, p.N);
         if (rc) break;
-        if ((rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M, KPS))) break;
-        if ((rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS, KPS))) break;
+        if ((rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M))) break;
+        if ((rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS))) break;
         if ((rc = make_atom_map(tsfa, pk.sfa_out, sfa_atoms, 1))) break;
         if ((rc = make_atom_map(tsfb, pk.sfb_out, sfb_atoms, C::SFB_ATOMS))) break;
         // ---- the GEMM, as a programmatic dependent of the pre-pass
@@ -509,8 +506,8 @@ int launch_cfg_noalloc(const void *a, long long a_rows, const void *b, long long
     cudaError_t e;
     CUtensorMap ta, tb, tsfa, tsfb, td;
     if (int rc = make_output_map(td, p.d, a_rows, p.N)) return rc;
-    if (int rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M, KPS)) return rc;
-    if (int rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS, KPS)) return rc;
+    if (int rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M)) return rc;
+    if (int rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS)) return rc;
     if (int rc = make_atom_map(tsfa, pk.sfa_out, sfa_atoms, 1)) return rc;
     if (int rc = make_atom_map(tsfb, pk.sfb_out, sfb_atoms, C::SFB_ATOMS)) return rc;
     auto kernel = dg::fp8_gemm_kernel<C>;

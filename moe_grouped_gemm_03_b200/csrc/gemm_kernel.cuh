@@ -588,22 +588,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     uint8_t *a_dst = sA + s * C::A_BYTES;
                     uint8_t *b_dst = sB + s * C::B_BYTES;
                     const int q = kb0 / SF_GROUP;
-                    // one 3-D box per operand brings KPS K blocks (a block past the tile's K range arrives zero-filled,
-                    // or from the next K group, and is unused)
+                    const int nk = min(C::KPS, tile_nkb - kb0);  // K blocks in this stage
                     const uint32_t bytes =
-                        static_cast<uint32_t>(C::A_BYTES + C::B_BYTES + (group_start ? C::SF_BYTES : 0));
+                        static_cast<uint32_t>(nk * (C::A_BYTES1 + C::B_BYTES1) + (group_start ? C::SF_BYTES : 0));
                     if constexpr (PAIR) {
                         // Only the leader arms the barrier (with both CTAs' bytes); the peer's loads just count
                         // their bytes on it.  A peer load may land before the leader arms the phase: the
                         // transaction count dips below zero but the phase cannot complete before the arrival.
                         const uint32_t leader_full = full_leader0 + 8u * static_cast<uint32_t>(s);
                         if (rank == 0) mbar_arrive_expect_tx(&full[s], CTAS * bytes);
-                        tma_load_3d_pair(a_dst, &tmap_a, leader_full, 0, arow, kbase + kb0);
-                        tma_load_3d_pair(b_dst, &tmap_b, leader_full, 0, brow, kbase + kb0);
+                        for (int i = 0; i < nk; ++i) {
+                            const int x = (kbase + kb0 + i) * BLOCK_K;
+                            tma_load_2d_pair(a_dst + i * C::A_BYTES1, &tmap_a, leader_full, x, arow);
+                            tma_load_2d_pair(b_dst + i * C::B_BYTES1, &tmap_b, leader_full, x, brow);
+                        }
                     } else {
                         mbar_arrive_expect_tx(&full[s], bytes);
-                        tma_load_3d(a_dst, &tmap_a, &full[s], 0, arow, kbase + kb0);
-                        tma_load_3d(b_dst, &tmap_b, &full[s], 0, brow, kbase + kb0);
+                        for (int i = 0; i < nk; ++i) {
+                            const int x = (kbase + kb0 + i) * BLOCK_K;
+                            tma_load_2d(a_dst + i * C::A_BYTES1, &tmap_a, &full[s], x, arow);
+                            tma_load_2d(b_dst + i * C::B_BYTES1, &tmap_b, &full[s], x, brow);
+                        }
                     }
                     if (group_start) {
                         if (scales_ready) {
