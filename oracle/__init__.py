@@ -22,6 +22,11 @@ Grouped layouts (same README, "Grouped GEMMs (contiguous layout)" / "(masked lay
   both sides; D_g[m, n] = C_g[m, n] + sum over the 128-K blocks kb of group g of
   sfa(m, kb) * sfb(n, kb) * sum_{k in kb} dec(a[m, k]) * dec(b[n, k]).  Computed here with numpy in float64,
   one 128-K block at a time (each block's sum of 128 products of e4m3 values is exact in float64).
+* W4A8 (MATE docs, 0.2.7 additions: e4m3 A with packed E2M1 FP4 B, recipe_a (1, 128), recipe_b (1, 32)): the
+  contiguous layout with B_g stored as 4-bit E2M1 codes packed two per byte (element 2i in the low nibble) and
+  one B scale per (row n, 32-K block): D[m, n] = sum over 128-K blocks kb of sfa(m, kb) * sum over its four
+  32-K sub-blocks j of sfb(g, 4 kb + j, n) * sum_{k in the sub-block} dec(a[m, k]) * dec2(b_g[n, k]).
+  Computed with numpy in float64 one 32-K block at a time (each block's sum is exact in float64).
 * no padding (same README, "Grouped GEMMs (nopad layout)"): the groups' rows are concatenated in group order
   with no alignment; group g owns rows off_g .. off_g + counts[g] - 1 with off_g = counts[0] + ... +
   counts[g-1]; rows past the sum of the counts produce nothing.
@@ -71,6 +76,47 @@ def decode_e4m3(codes) -> np.ndarray:
     return out
 
 
+def decode_e2m1(codes) -> np.ndarray:
+    """4-bit OCP E2M1 codes (0..15) -> float64: sign bit 3, exponent bits 2..1 (bias 1), mantissa bit 0;
+    exponent 0 is subnormal (0 or 0.5); no Inf or NaN codes."""
+    c = np.asarray(codes, np.int64)
+    sign = np.where(c & 8, -1.0, 1.0)
+    e = (c >> 1) & 3
+    m = c & 1
+    mag = np.where(e == 0, 0.5 * m, np.ldexp(1.0 + 0.5 * m, e - 1))
+    return sign * mag
+
+
+def unpack_e2m1(packed) -> np.ndarray:
+    """Bytes [..., K/2] -> 4-bit codes [..., K]: element 2i from the low nibble of byte i, 2i + 1 from the high."""
+    b = np.asarray(packed, np.uint8)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), np.uint8)
+    out[..., 0::2] = b & 0x0F
+    out[..., 1::2] = b >> 4
+    return out
+
+
+def w4a8_rows(p, rows) -> np.ndarray:
+    """Rows of a contiguous W4A8 ``synth.Problem`` (rows of groups only)."""
+    rows = np.asarray(rows, np.int64)
+    groups = p.row_groups(rows)
+    out = np.zeros((len(rows), p.N))
+    for g in np.unique(groups):
+        sel = groups == g
+        r = rows[sel]
+        bdec = decode_e2m1(unpack_e2m1(p.b[g]))  # [N, K]
+        adec = decode_e4m3(p.a[r])                # [rows, K]
+        acc = np.zeros((len(r), p.N))
+        for kb in range(p.K // 128):
+            blk = np.zeros((len(r), p.N))
+            for j in range(4):
+                sub = slice(128 * kb + 32 * j, 128 * kb + 32 * j + 32)
+                blk += (adec[:, sub] @ bdec[:, sub].T) * p.sfb[g, 4 * kb + j, :p.N][None, :]
+            acc += blk * p.sfa[kb, r][:, None]
+        out[sel] = acc
+    return out
+
+
 def gemm_rows(a, sfa_row_off, sfa_kb_stride, sfa, b, sfb, rows, groups, N, K) -> np.ndarray:
     """Raw entry: listed rows of the fine-grained-scaled product, double [len(rows), N]."""
     a = np.ascontiguousarray(a, np.uint8)
@@ -108,6 +154,8 @@ def problem_rows(p, rows) -> np.ndarray:
             out[sel] = k_grouped_rows(p, int(g), rows[sel] - g * p.M)
         return out
     groups = p.row_groups(rows)
+    if p.kind == "contiguous_w4a8":
+        return w4a8_rows(p, rows)
     if p.kind == "contiguous_nn":
         # B_g[k, n] is the definition's b_g[n, k]; sfb_g[kb, nb] its s_b(g, nb, kb)
         b = np.ascontiguousarray(p.b.transpose(0, 2, 1))

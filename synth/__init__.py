@@ -46,11 +46,13 @@ def tma_aligned_rows(rows: int) -> int:
 class Problem:
     """One GEMM problem in the layouts the library takes.
 
-    kind       'dense' | 'contiguous' | 'masked' | 'nopad' | 'contiguous_nn' | 'k_grouped'
+    kind       'dense' | 'contiguous' | 'masked' | 'nopad' | 'contiguous_nn' | 'k_grouped' | 'contiguous_w4a8'
     a          uint8 e4m3 codes, [rows, K]; masked: [G * M_max, K] (= [G, M_max, K] flattened)
     sfa        fp32, dense/contiguous [K/128, align4(rows)]; masked [G, K/128, align4(M_max)]
-    b          uint8 e4m3 codes, [G, N, K] (G = 1 for dense); contiguous_nn: [G, K, N]
-    sfb        fp32, [G, ceil(N/128), K/128]; contiguous_nn: [G, K/128, ceil(N/128)]
+    b          uint8 e4m3 codes, [G, N, K] (G = 1 for dense); contiguous_nn: [G, K, N]; contiguous_w4a8: packed
+               E2M1 codes [G, N, K/2] (element 2i in the low nibble of byte i)
+    sfb        fp32, [G, ceil(N/128), K/128]; contiguous_nn: [G, K/128, ceil(N/128)]; contiguous_w4a8: one scale
+               per (row, 32-K block), [G, K/32, align4(N)] (recipe (1, 32))
     m_indices  int32 [rows] (contiguous only): group id of each row, -1 for padding rows
     masked_m   int32 [G] (masked only): number of valid rows of each group
     counts     int32 [G]: contiguous -- valid rows per group (metadata); nopad -- the call's per-group row counts;
@@ -87,7 +89,7 @@ class Problem:
             return np.arange(self.G * self.M, dtype=np.int64)  # rows of the flattened [G * M, N] output
         if self.kind == "dense":
             return np.arange(self.M, dtype=np.int64)
-        if self.kind in ("contiguous", "contiguous_nn"):
+        if self.kind in ("contiguous", "contiguous_nn", "contiguous_w4a8"):
             return np.nonzero(self.m_indices >= 0)[0].astype(np.int64)
         if self.kind == "nopad":
             return np.arange(int(np.sum(self.counts, dtype=np.int64)), dtype=np.int64)
@@ -99,7 +101,7 @@ class Problem:
             return (rows // self.M).astype(np.int32)
         if self.kind == "dense":
             return np.zeros(len(rows), np.int32)
-        if self.kind in ("contiguous", "contiguous_nn"):
+        if self.kind in ("contiguous", "contiguous_nn", "contiguous_w4a8"):
             return self.m_indices[rows].astype(np.int32)
         if self.kind == "nopad":
             ends = np.cumsum(np.asarray(self.counts, np.int64))
@@ -132,6 +134,46 @@ def pow2_scale_exponent(amax: np.ndarray) -> np.ndarray:
     f, ea = np.frexp(amax.astype(np.float64))
     e = ea.astype(np.int64) - 9 + (f > 0.875).astype(np.int64)
     return np.where(amax > 0, e, 0)
+
+
+E2M1_MAX = 6.0
+# magnitudes of the E2M1 codes 0..7 (OCP MX format: 1 sign, 2 exponent (bias 1), 1 mantissa bit, no Inf/NaN)
+_E2M1_MAGNITUDES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def pow2_scale_exponent_e2m1(amax: np.ndarray) -> np.ndarray:
+    """Smallest integer e with amax <= 6 * 2**e, exactly; amax == 0 -> 0.  With amax = f * 2**ea (f in [0.5, 1))
+    and 6 = 0.75 * 2**3: e >= ea - 3 when f <= 0.75, else e >= ea - 2."""
+    f, ea = np.frexp(amax.astype(np.float64))
+    e = ea.astype(np.int64) - 3 + (f > 0.75).astype(np.int64)
+    return np.where(amax > 0, e, 0)
+
+
+def _to_e2m1_codes(y: np.ndarray) -> np.ndarray:
+    """|y| <= 6 -> 4-bit E2M1 codes (uint8 0..15), round to nearest, ties to the even code (mantissa bit 0)."""
+    mag = np.abs(np.asarray(y, np.float64))
+    hi = np.clip(np.searchsorted(_E2M1_MAGNITUDES, mag, side="left"), 0, 7)
+    lo = np.clip(hi - 1, 0, 7)
+    d_lo = mag - _E2M1_MAGNITUDES[lo]
+    d_hi = _E2M1_MAGNITUDES[hi] - mag
+    code = np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, np.where(lo % 2 == 0, lo, hi)))
+    return (code | np.where(np.signbit(y) & (code != 0), 8, 0)).astype(np.uint8)
+
+
+def quantize_rows_e2m1(x: np.ndarray):
+    """x fp32 [R, K] -> (codes uint8 [R, K] in 0..15, scales fp32 [R, K/32]), one scale per (row, 32-K block)."""
+    R, K = x.shape
+    assert K % 32 == 0
+    xb = x.reshape(R, K // 32, 32)
+    e = pow2_scale_exponent_e2m1(np.abs(xb).max(axis=2))
+    q = np.ldexp(xb.astype(np.float64), -e[:, :, None])
+    return _to_e2m1_codes(q.reshape(R, K)), np.ldexp(np.ones_like(e, dtype=np.float32), e).astype(np.float32)
+
+
+def pack_e2m1(codes: np.ndarray) -> np.ndarray:
+    """4-bit codes [..., K] -> bytes [..., K/2]: element 2i in the low nibble, 2i + 1 in the high nibble."""
+    c = np.asarray(codes, np.uint8)
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
 
 
 def _to_e4m3_codes(x: np.ndarray) -> np.ndarray:
@@ -264,6 +306,25 @@ def make_k_grouped(ks: Sequence[int], M: int, N: int, seed: int = 0, with_c: boo
                    name=name or f"k-grouped G={G} M={M} N={N}")
 
 
+def make_contiguous_w4a8(counts: Sequence[int], N: int, K: int, seed: int = 0, name: str = "",
+                         rng: Optional[np.random.Generator] = None) -> Problem:
+    """The contiguous layout with B in E2M1 (FP4, packed two per byte) and one B scale per (row, 32-K block);
+    A as in ``make_contiguous`` (e4m3, one scale per (row, 128-K block))."""
+    rng = rng if rng is not None else np.random.default_rng(seed)
+    p = make_contiguous(counts, N, K, rng=rng)
+    G = p.G
+    b = np.empty((G, N, K // 2), np.uint8)
+    sfb = np.ones((G, K // 32, tma_aligned_rows(N)), np.float32)
+    for g in range(G):
+        codes, sb = quantize_rows_e2m1(_draw_normal(rng, (N, K)))
+        b[g] = pack_e2m1(codes)
+        sfb[g, :, :N] = sb.T
+    p.kind = "contiguous_w4a8"
+    p.b, p.sfb = b, sfb
+    p.name = name or f"contiguous W4A8 G={G} N={N} K={K}"
+    return p
+
+
 def make_nopad(counts: Sequence[int], N: int, K: int, seed: int = 0, extra_rows: int = 0, name: str = "",
                rng: Optional[np.random.Generator] = None) -> Problem:
     """Groups' rows concatenated with no padding, then ``extra_rows`` rows that no group owns (garbage)."""
@@ -320,7 +381,8 @@ def zipf_counts(total: int, G: int, s: float) -> np.ndarray:
 
 
 # The five workloads (all seed 0); 6: workload 5's token split in the no-padding layout; 7: workload 3 with B
-# in the NN orientation; 8: workload 3's token counts as the K extents of a K-grouped (weight-gradient) GEMM.
+# in the NN orientation; 8: workload 3's token counts as the K extents of a K-grouped (weight-gradient) GEMM;
+# 9: workload 3 with B in E2M1 (W4A8).
 CONFIGS = {
     1: "dense FP8 NT GEMM M=128 N=256 K=512",
     2: "dense FP8 NT GEMM M=4096 N=7168 K=7168",
@@ -330,6 +392,7 @@ CONFIGS = {
     6: "M-grouped no-padding FP8 GEMM G=64 N=7168 K=2048, Zipf(1.2) split of 65536 tokens",
     7: "M-grouped contiguous FP8 NN GEMM (B [G, K, N]) G=8 N=4096 K=7168, tokens U[1024,8192] per group",
     8: "K-grouped FP8 NT GEMM, fp32 D_g = A_g B_g^T, G=8 M=4096 N=7168, K_g = tokens U[1024,8192] rounded up to 128",
+    9: "M-grouped contiguous W4A8 GEMM (e4m3 A x E2M1 B) G=8 N=4096 K=7168, tokens U[1024,8192] per group",
 }
 
 
@@ -347,6 +410,10 @@ def make_config(i: int, seed: int = 0) -> Problem:
     if i == 5:
         rng = np.random.default_rng(seed)
         return make_contiguous(zipf_counts(65536, 64, 1.2), 7168, 2048, rng=rng, name=CONFIGS[5])
+    if i == 9:
+        rng = np.random.default_rng(seed)
+        counts = rng.integers(1024, 8192, endpoint=True, size=8)
+        return make_contiguous_w4a8(counts, 4096, 7168, rng=rng, name=CONFIGS[9])
     if i == 8:
         rng = np.random.default_rng(seed)
         counts = rng.integers(1024, 8192, endpoint=True, size=8)
@@ -376,7 +443,7 @@ def to_torch(p: Problem, device="cuda"):
     if p.kind == "masked":
         out["a"] = out["a"].view(p.G, p.M, p.K)
         out["masked_m"] = t(p.masked_m)
-    if p.kind in ("contiguous", "contiguous_nn"):
+    if p.kind in ("contiguous", "contiguous_nn", "contiguous_w4a8"):
         out["m_indices"] = t(p.m_indices)
     if p.kind == "nopad":
         out["counts"] = t(p.counts)

@@ -295,6 +295,55 @@ def test_k_grouped_row_scale_moves_one_column_of_one_group():
     np.testing.assert_allclose(diff[1, :, n], contribution, rtol=1e-12, atol=1e-9)
 
 
+def test_e2m1_decode_matches_the_format_table():
+    """All 16 E2M1 codes against the element table of the OCP Microscaling (MX) v1.0 specification (FP4 E2M1:
+    +-0, 0.5, 1, 1.5, 2, 3, 4, 6 in code order, sign in bit 3)."""
+    table = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    want = np.array(table + [-v for v in table])
+    np.testing.assert_array_equal(oracle.decode_e2m1(np.arange(16)), want)
+    # packing: element 2i in the low nibble
+    np.testing.assert_array_equal(oracle.unpack_e2m1(np.array([[0x21, 0xF7]], np.uint8)), [[1, 2, 7, 15]])
+
+
+def test_w4a8_bruteforce_integer_operands():
+    """Integer-valued e4m3 A times E2M1 B (values -6..6 on the E2M1 grid) with unit scales equals the exact
+    integer product (a misplaced nibble, sub-block or group fails it)."""
+    rng = np.random.default_rng(23)
+    p = synth.make_contiguous_w4a8([3, 130], N=48, K=256, seed=23)
+    grid = np.array([0, 1, 2, 3, 4, 6, -1, -2, -3, -4, -6])
+    codes_of = {0: 0, 1: 2, 2: 4, 3: 5, 4: 6, 6: 7, -1: 10, -2: 12, -3: 13, -4: 14, -6: 15}
+    ia = rng.integers(-8, 9, size=(p.rows, p.K))
+    ib = rng.choice(grid, size=(p.G, p.N, p.K))
+    p.a = _codes_for_values(ia.astype(np.float32))
+    p.b = synth.pack_e2m1(np.vectorize(codes_of.get)(ib).astype(np.uint8))
+    p.sfa[:] = 1.0
+    p.sfb[:] = 1.0
+    full = oracle.problem_full(p)
+    for g, start in enumerate([0, 128]):
+        c = int(p.counts[g])
+        exact = ia[start:start + c].astype(np.int64) @ ib[g].astype(np.int64).T
+        np.testing.assert_array_equal(full[start:start + c], exact.astype(np.float64))
+
+
+def test_w4a8_sub_block_scale_moves_one_column():
+    """Doubling B's scale of row n in one 32-K sub-block changes only column n of that group's rows, by exactly
+    that sub-block's contribution (scaled by A's 128-K block scale)."""
+    p = synth.make_contiguous_w4a8([130], N=64, K=256, seed=24)
+    base = oracle.problem_full(p)
+    j, n = 5, 17  # sub-block 5 = K 160..191, inside 128-K block 1
+    p.sfb[0, j, n] *= 2.0
+    moved = oracle.problem_full(p)
+    rows = np.arange(130)
+    diff = moved[rows] - base[rows]
+    others = np.ones(p.N, bool)
+    others[n] = False
+    assert (diff[:, others] == 0).all()
+    sub = slice(32 * j, 32 * j + 32)
+    a = oracle.decode_e4m3(p.a[:130, sub]) * p.sfa[1, :130][:, None]
+    b = oracle.decode_e2m1(oracle.unpack_e2m1(p.b[0, n]))[sub]
+    np.testing.assert_allclose(diff[:, n], (a @ b) * (p.sfb[0, j, n] / 2.0), rtol=1e-12, atol=1e-9)
+
+
 def test_library_call_shapes_agree_with_problem_driver():
     p = synth.make_masked(G=3, M_max=64, N=128, K=128, masked_m=[3, 64, 0], seed=8)
     a = p.a.reshape(p.G, p.M, p.K)

@@ -82,6 +82,16 @@ def test_k_grouped_layout():
     assert p.flops() == 2 * 10 * 20 * 384
 
 
+def test_e2m1_quantisation():
+    """The B quantiser of the W4A8 inputs: smallest power-of-two scale with amax <= 6 * scale, round to nearest
+    on the E2M1 grid with ties to the even code."""
+    np.testing.assert_array_equal(synth.pow2_scale_exponent_e2m1(np.array([6.0, 6.01, 3.0, 0.0, 12.0])), [0, 1, -1, 0, 1])
+    np.testing.assert_array_equal(synth._to_e2m1_codes(np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -6.0])),
+                                  [0, 2, 2, 4, 4, 6, 6, 15])
+    p = synth.make_contiguous_w4a8([3, 129], N=64, K=256, seed=1)
+    assert p.b.shape == (2, 64, 128) and p.sfb.shape == (2, 8, 64)
+
+
 def test_masked_layout():
     p = synth.make_masked(G=2, M_max=10, N=128, K=256, masked_m=[0, 10], seed=1)
     assert p.a.shape == (20, 256) and p.sfa.shape == (2, 2, 12) and p.sfb.shape == (2, 1, 2)
