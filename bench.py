@@ -39,7 +39,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7, 8])
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7, 8, 9])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
@@ -182,6 +182,8 @@ def call_library(p, t, out):
         dg.m_grouped_fp8_gemm_nt_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["m_indices"])
     elif p.kind == "k_grouped":  # D = the products (no C)
         dg.k_grouped_fp8_gemm_nt_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, p.counts.tolist(), t["ks"])
+    elif p.kind == "contiguous_w4a8":
+        dg.m_grouped_fp8_fp4_gemm_nt_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["m_indices"])
     elif p.kind == "contiguous_nn":
         dg.m_grouped_fp8_gemm_nn_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["m_indices"])
     elif p.kind == "nopad":
@@ -195,6 +197,12 @@ def algorithmic_bytes(p):
     K-grouped: A and B once, their per-row scales, fp32 D once (no C in the timed call)."""
     import numpy as np
 
+    if p.kind == "contiguous_w4a8":  # B is half a byte per element, with one 4-byte scale per row per 128 K
+        rows = p.valid_rows()
+        groups = np.unique(p.row_groups(rows)) if len(rows) else []
+        nkb = p.K // 128
+        return int(len(rows) * p.K + len(groups) * p.N * p.K // 2 + len(rows) * nkb * 4
+                   + len(groups) * p.N * nkb * 16 + len(rows) * p.N * 2)
     if p.kind == "k_grouped":
         nkb = p.K // 128
         return int((p.M + p.N) * p.K + (p.M + p.N) * nkb * 4 + p.G * p.M * p.N * 4)

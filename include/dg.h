@@ -124,6 +124,18 @@ DG_EXPORT int dg_m_grouped_fp8_gemm_nn_contiguous(const void *a, const float *sf
                                         void *d, const int *m_indices, int M_total, int N, int K, int G,
                                         dg_stream_t stream);
 
+/* M-grouped GEMM, contiguous layout, W4A8: e4m3 A times E2M1 (FP4) B (MATE docs, 0.2.7 additions,
+ * `m_grouped_fp8_fp4_gemm_nt_contiguous`: "FP8 E4M3 A plus packed E2M1 FP4 B", recipe_a (1, 128), recipe_b (1, 32)).
+ *   Same as dg_m_grouped_fp8_gemm_nt_contiguous except
+ *   b [G][N][K/2] bytes: E2M1 codes (sign, 2 exponent bits with bias 1, 1 mantissa bit) packed two per byte, code
+ *     k in the low nibble of byte k/2 when k is even, the high nibble when odd; 32-byte aligned;
+ *   sfb [G][K/32][ld(N)] fp32, MN-major: one power-of-two scale per (row n, 32-K block):
+ *   D[m][n] = sum over 128-K blocks kb of sfa(m, kb) * sum over its four 32-K sub-blocks j of sfb(g, 4 kb + j, n)
+ *             * sum_{k in the sub-block} A[m][k] * B_g[n][k]. */
+DG_EXPORT int dg_m_grouped_fp8_fp4_gemm_nt_contiguous(const void *a, const float *sfa, const void *b,
+                                            const float *sfb, void *d, const int *m_indices, int M_total, int N, int K,
+                                            int G, dg_stream_t stream);
+
 /* K-grouped GEMM (MATE docs, 0.2.7 additions, `k_grouped_fp8_gemm_nt_contiguous`: recipe (1, 1, 128), host K
  * extents, C accumulated into D), e.g. the per-expert weight gradient of an MoE layer.
  *   a [M][sum ks] e4m3 and b [N][sum ks] e4m3, both K-major, the groups' K segments concatenated in group order;

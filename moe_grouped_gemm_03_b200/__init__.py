@@ -56,6 +56,7 @@ _SIGNATURES = {
     "dg_m_grouped_fp8_gemm_nt_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_gemm_nt_nopad": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_gemm_nn_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "dg_m_grouped_fp8_fp4_gemm_nt_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_k_grouped_fp8_gemm_nt_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_set_cta_pair_policy": (_I, [_I]),
@@ -292,6 +293,26 @@ def k_grouped_fp8_gemm_nt_contiguous(lhs, rhs, out: torch.Tensor, ks, ks_tensor:
                                                     N, _stream()))
 
 
+def m_grouped_fp8_fp4_gemm_nt_contiguous(lhs, rhs, out: torch.Tensor, m_indices: torch.Tensor) -> None:
+    """W4A8 contiguous layout: rhs = (b packed E2M1 uint8 [G, N, K/2], sfb [G, K/32, tma_aligned(N)]), one B
+    scale per (row, 32-K block); lhs and out as for m_grouped_fp8_gemm_nt_contiguous."""
+    a, sfa = lhs
+    b, sfb = rhs
+    _check_operand("a", a, 2, _FP8_TYPES)
+    _check_operand("b", b, 3, (torch.uint8,))
+    _check_operand("sfa", sfa, 2, (torch.float32,))
+    _check_operand("sfb", sfb, 3, (torch.float32,))
+    _check_operand("out", out, 2, (torch.bfloat16,))
+    _check_operand("m_indices", m_indices, 1, (torch.int32,))
+    M, K = a.shape
+    G, N, half_k = b.shape
+    _need(half_k * 2 == K and tuple(out.shape) == (M, N) and m_indices.shape[0] == M, "shape mismatch")
+    _need(sfa.shape == (K // 128, get_tma_aligned_size(M, 4)), "sfa must be [K/128, tma_aligned(M)]")
+    _need(sfb.shape == (G, K // 32, get_tma_aligned_size(N, 4)), "sfb must be [G, K/32, tma_aligned(N)]")
+    _check(_lib.dg_m_grouped_fp8_fp4_gemm_nt_contiguous(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(out),
+                                                        _ptr(m_indices), M, N, K, G, _stream()))
+
+
 def m_grouped_fp8_gemm_nt_nopad(lhs, rhs, out: torch.Tensor, counts: torch.Tensor) -> None:
     """No-padding layout: group g's rows are off_g .. off_g + counts[g] - 1 (off_g = sum of the earlier counts);
     out rows of group g = lhs rows of group g @ rhs[g]^T; rows past sum(counts) are untouched."""
@@ -316,6 +337,7 @@ def m_grouped_fp8_gemm_nt_nopad(lhs, rhs, out: torch.Tensor, counts: torch.Tenso
 __all__ = [
     "DGError", "fp8_gemm_nt", "fp8_gemm_nt_noalloc", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
     "m_grouped_fp8_gemm_nt_nopad", "m_grouped_fp8_gemm_nn_contiguous", "k_grouped_fp8_gemm_nt_contiguous",
+    "m_grouped_fp8_fp4_gemm_nt_contiguous",
     "get_m_alignment_for_contiguous_layout", "set_m_alignment_for_contiguous_layout", "get_tma_aligned_size", "set_num_sms", "get_num_sms", "num_tiles",
     "select_block_n", "set_cta_pair_policy", "check_device_error", "lib", "header_symbols", "last_error",
 ]

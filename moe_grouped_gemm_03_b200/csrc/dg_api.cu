@@ -106,6 +106,24 @@ int make_operand_map(CUtensorMap &map, const void *base, long long rows, int K, 
     return DG_OK;
 }
 
+// B in E2M1, packed two codes per byte [rows][K/2]: the TMA's 16 x 4-bit type with 16-byte alignment stages each
+// 16 codes as 8 bytes followed by an 8-byte gap, so a box of 128 codes x `box_rows` rows fills 128-byte rows,
+// the footprint and 128-byte swizzle of an e4m3 box, which is how the MMA reads an E2M1 operand.  Requires a
+// 32-byte aligned base and K % 64 == 0 (the row stride K/2 a multiple of 32 bytes).
+int make_operand_map_fp4(CUtensorMap &map, const void *base, long long rows, int K, int box_rows) {
+    EncodeTiledFn encode;
+    if (int rc = get_encode_fn(encode)) return rc;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(dg::BLOCK_K), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void *>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (E2M1) failed (%d)", static_cast<int>(r));
+    return DG_OK;
+}
+
 // D, bf16 row-major [rows][N]: boxes of 32 rows x 32 columns (64-byte rows) with the 64-byte swizzle, the
 // layout the epilogue stages each chunk in.
 int make_output_map(CUtensorMap &map, void *base, long long rows, int N) {
@@ -192,7 +210,8 @@ struct ScaleArgs {
     int sfa_ld;
     const float *sfb;
     bool sfb_kn = false;  // SFB stored [G][K/128][ceil(N/128)] (B in the NN orientation)
-    int sfb_ld = 0;       // K-grouped: one scale per row of B, [K/128][sfb_ld]
+    bool sfb_fp4 = false; // B in E2M1 (packed two per byte) with SFB [G][K/32][sfb_ld]
+    int sfb_ld = 0;       // K-grouped: one scale per row of B, [K/128][sfb_ld]; FP4 B: [G][K/32][sfb_ld]
 };
 
 // Launch of the scale pre-pass: one warp per atom, spread over every SM (one block each), so that every SM is
@@ -214,10 +233,10 @@ int launch_pack(const dg::PackParams &pk, int device, cudaStream_t stream) {
     return DG_OK;
 }
 
-template <int BN, int CTAS, int KPS>
+template <int BN, int CTAS, int KPS, bool BF4 = false>
 int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows, const ScaleArgs &sc, dg::GemmParams p,
                int grid, int device, cudaStream_t stream) {
-    using C = dg::Cfg<BN, CTAS, KPS>;
+    using C = dg::Cfg<BN, CTAS, KPS, BF4>;
     // ---- packed scale atoms (pre-pass)
     const int nkb = p.K / dg::BLOCK_K;
     dg::PackParams pk{};
@@ -233,6 +252,11 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
     pk.sfb_atoms = C::SFB_ATOMS;
     pk.nkb = nkb;
     pk.num_sf_groups = p.num_sf_groups;
+    pk.sfb_kwords = p.num_sf_groups;
+    if (BF4) {  // B scale words: one per 128-K block
+        pk.sfb_fp4 = 1;
+        pk.sfb_kwords = nkb;
+    }
     pk.mode = p.mode;
     pk.counts = p.masked_m;
     pk.tile_m = C::TILE_M;
@@ -252,7 +276,7 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
     }
     const long long sfa_atoms = static_cast<long long>(pk.sfa_groups) * pk.blocks_per_group * p.num_sf_groups;
     const long long b_groups = p.mode == dg::MODE_KGROUPED ? 1 : p.G;  // K-grouped: one B for all groups
-    const long long sfb_atoms = b_groups * p.num_n_blocks * p.num_sf_groups * C::SFB_ATOMS;
+    const long long sfb_atoms = b_groups * p.num_n_blocks * pk.sfb_kwords * C::SFB_ATOMS;
     pk.sfa_words = sfa_atoms * dg::SF_ATOM_WORDS;
     pk.sfb_words = sfb_atoms * dg::SF_ATOM_WORDS;
     cudaMemPool_t pool;
@@ -272,9 +296,13 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
             rc = make_output_map_f32(td, p.d32, p.G, p.M, p.N);
         if (rc) break;
         if ((rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M))) break;
-        if ((rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS))) break;
+        if (BF4)
+            rc = make_operand_map_fp4(tb, b, b_rows, p.K, C::B_ROWS);
+        else
+            rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS);
+        if (rc) break;
         if ((rc = make_atom_map(tsfa, pk.sfa_out, sfa_atoms, 1))) break;
-        if ((rc = make_atom_map(tsfb, pk.sfb_out, sfb_atoms, C::SFB_ATOMS))) break;
+        if ((rc = make_atom_map(tsfb, pk.sfb_out, sfb_atoms, C::SFB_KB * C::SFB_ATOMS))) break;
         // ---- the GEMM, as a programmatic dependent of the pre-pass
         auto kernel = dg::fp8_gemm_kernel<C>;
         static bool smem_set[64] = {false};  // per instantiation and device: the attribute persists
@@ -336,26 +364,34 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
 // 512 TMEM columns (two BN-wide accumulators plus one scale slot per stage).
 constexpr int kCandidateBN[] = {224, 192, 160, 128};
 
-int launch_bn(int bn, int ctas, const void *a, long long a_rows, const void *b, long long b_rows,
-              const ScaleArgs &sc, const dg::GemmParams &p, int grid, int device, cudaStream_t stream) {
+template <bool BF4>
+int launch_bn_t(int bn, int ctas, const void *a, long long a_rows, const void *b, long long b_rows,
+                const ScaleArgs &sc, const dg::GemmParams &p, int grid, int device, cudaStream_t stream) {
     if (ctas == 2) {
         switch (bn) {
-            case 224: return launch_cfg<224, 2, 2>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            case 192: return launch_cfg<192, 2, 2>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            case 160: return launch_cfg<160, 2, 2>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            case 128: return launch_cfg<128, 2, 2>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 224: return launch_cfg<224, 2, 2, BF4>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 192: return launch_cfg<192, 2, 2, BF4>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 160: return launch_cfg<160, 2, 2, BF4>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 128: return launch_cfg<128, 2, 2, BF4>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
             default: break;
         }
     } else {
         switch (bn) {
-            case 224: return launch_cfg<224, 1, 1>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            case 192: return launch_cfg<192, 1, 1>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            case 160: return launch_cfg<160, 1, 1>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            case 128: return launch_cfg<128, 1, 1>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 224: return launch_cfg<224, 1, 1, BF4>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 192: return launch_cfg<192, 1, 1, BF4>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 160: return launch_cfg<160, 1, 1, BF4>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
+            case 128: return launch_cfg<128, 1, 1, BF4>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
             default: break;
         }
     }
     return fail(DG_ERR_UNSUPPORTED, "no kernel instantiated for BN=%d with %d CTA(s) per tile", bn, ctas);
+}
+
+// B e4m3, or (sc.sfb_fp4) B in E2M1 with 1x32 scales
+int launch_bn(int bn, int ctas, const void *a, long long a_rows, const void *b, long long b_rows,
+              const ScaleArgs &sc, const dg::GemmParams &p, int grid, int device, cudaStream_t stream) {
+    if (sc.sfb_fp4) return launch_bn_t<true>(bn, ctas, a, a_rows, b, b_rows, sc, p, grid, device, stream);
+    return launch_bn_t<false>(bn, ctas, a, a_rows, b, b_rows, sc, p, grid, device, stream);
 }
 
 // Tile width for `windows` row windows (128 rows per CTA, `ctas` CTAs per tile) of an N-wide output on
@@ -486,6 +522,7 @@ int launch_cfg_noalloc(const void *a, long long a_rows, const void *b, long long
     pk.sfb_atoms = C::SFB_ATOMS;
     pk.nkb = nkb;
     pk.num_sf_groups = p.num_sf_groups;
+    pk.sfb_kwords = p.num_sf_groups;
     pk.rows_per_group = p.M;
     pk.blocks_per_group = (p.M + dg::BLOCK_M - 1) / dg::BLOCK_M;
     pk.sfa_groups = 1;
@@ -584,12 +621,14 @@ int check_contiguous(const void *a, const float *sfa, const void *b, const float
 // The contiguous GEMM on checked arguments (M_total > 0); `sfb_kn` selects the NN orientation of SFB.
 int launch_contiguous(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
                       const int *m_indices, int M_total, int N, int K, int G, bool sfb_kn, const DeviceInfo &info,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, bool b_fp4 = false) {
     dg::GemmParams p{};
     p.mode = dg::MODE_CONTIGUOUS;
     p.M = M_total; p.N = N; p.K = K; p.G = G;
     ScaleArgs sc{sfa, dg_get_tma_aligned_size(M_total, 4), sfb};
     sc.sfb_kn = sfb_kn;
+    sc.sfb_fp4 = b_fp4;
+    if (b_fp4) sc.sfb_ld = dg_get_tma_aligned_size(N, 4);
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.m_indices = m_indices;
     p.err = device_error_word();
@@ -689,6 +728,18 @@ int dg_m_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const v
     if (int rc = device_info(info)) return rc;
     return launch_contiguous(a, sfa, b, sfb, d, m_indices, M_total, N, K, G, false, info,
                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dg_m_grouped_fp8_fp4_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
+                                            void *d, const int *m_indices, int M_total, int N, int K, int G,
+                                            dg_stream_t stream) {
+    if (int rc = check_contiguous(a, sfa, b, sfb, d, m_indices, M_total, N, K, G)) return rc;
+    if (!aligned(b, 32)) return fail(DG_ERR_ALIGNMENT, "b (packed E2M1) must be 32-byte aligned");
+    if (M_total == 0) return DG_OK;
+    DeviceInfo info;
+    if (int rc = device_info(info)) return rc;
+    return launch_contiguous(a, sfa, b, sfb, d, m_indices, M_total, N, K, G, false, info,
+                             reinterpret_cast<cudaStream_t>(stream), true);
 }
 
 int dg_m_grouped_fp8_gemm_nn_contiguous(const void *a, const float *sfa, const void *b, const float *sfb, void *d,

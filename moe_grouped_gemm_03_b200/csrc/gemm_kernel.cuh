@@ -94,21 +94,29 @@ struct GemmParams {
     int skip_first_load;               // test hook: the first CTA (pair) never loads stage 0
 };
 
-template <int BN_, int CTAS_, int KPS_>
+template <int BN_, int CTAS_, int KPS_, bool BF4_ = false>
 struct Cfg {
     static constexpr int BN = BN_;
     static constexpr int CTAS = CTAS_;
     static constexpr int KPS = KPS_;                              // 128-K blocks per pipeline stage
+    // B in E2M1 (W4A8): B's smem tiles keep the e4m3 footprint (TMA stages 4-bit codes one byte each) and B has
+    // one scale per (row, 32-K block), i.e. one 4-byte scale word per row per 128-K block, so a stage carries
+    // the B scale atoms of each of its K blocks (A's atom still packs SF_GROUP K blocks)
+    static constexpr bool BF4 = BF4_;
+    static constexpr int SFB_KB = BF4 ? KPS : 1;                  // K blocks whose B scale atoms a stage holds
     static constexpr int TILE_M = BLOCK_M * CTAS;
     static constexpr int B_ROWS = BN / CTAS;                      // B rows this CTA loads
     static constexpr int SFB_ATOMS = (BN + 127) / 128;            // 128-row scale atoms covering BN rows
     static constexpr int A_BYTES1 = BLOCK_M * BLOCK_K;            // one K block of A (e4m3: 1 byte each)
     static constexpr int B_BYTES1 = B_ROWS * BLOCK_K;             // one K block of this CTA's B rows
+    // transaction bytes of that load: an E2M1 box counts its packed bytes (half a byte per code), although
+    // shared memory receives one byte per code
+    static constexpr int B_TX1 = BF4_ ? B_ROWS * BLOCK_K / 2 : B_BYTES1;
     static constexpr int A_BYTES = KPS * A_BYTES1;                // per stage
     static constexpr int B_BYTES = KPS * B_BYTES1;
-    static constexpr int SF_BYTES = (1 + SFB_ATOMS) * SF_ATOM_WORDS * 4;  // SFA atom + SFB atoms
+    static constexpr int SF_BYTES = (1 + SFB_KB * SFB_ATOMS) * SF_ATOM_WORDS * 4;  // SFA atom + SFB atoms
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SF_BYTES;
-    static constexpr int SF_COLS = 4 + 4 * SFB_ATOMS;             // TMEM columns of one scale group's scales
+    static constexpr int SF_COLS = 4 + 4 * SFB_KB * SFB_ATOMS;    // TMEM columns of one scale slot
     static constexpr int SF_TMEM_BASE = 2 * BN;                   // after the two accumulators
     // scale slots in TMEM, used round-robin by successive scale groups (not by stages)
     static constexpr int SF_SLOTS_FIT = (TMEM_COLS - SF_TMEM_BASE) / SF_COLS;
@@ -580,9 +588,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 else
                     sfa_block = (ti.row0 + my_rows) / BLOCK_M;
                 const int sfa_y0 = sfa_block * p.num_sf_groups + qbase;
-                const int sfb_y0 = ((gb * p.num_n_blocks + ti.nb) * p.num_sf_groups + qbase) * C::SFB_ATOMS;
+                // B scale words along K per tile: one per scale group, or (FP4 B) one per 128-K block
+                const int sfb_words = C::BF4 ? nkb : p.num_sf_groups;
+                const int sfb_y0 = ((gb * p.num_n_blocks + ti.nb) * sfb_words + qbase) * C::SFB_ATOMS;
                 for (int kb0 = 0; kb0 < tile_nkb; kb0 += C::KPS) {
-                    const bool group_start = kb0 % SF_GROUP == 0;
+                    const bool group_start = C::BF4 || kb0 % SF_GROUP == 0;  // this stage carries scales
                     if (issued == STAGES) wait_for_scales();  // the ring is full: the MMAs need the scales now
                     if (!wait_bounded(&empty[s], ph ^ 1u, s_abort, p.err, p.wait_limit_ns)) { ok = false; break; }
                     uint8_t *a_dst = sA + s * C::A_BYTES;
@@ -590,7 +600,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const int q = kb0 / SF_GROUP;
                     const int nk = min(C::KPS, tile_nkb - kb0);  // K blocks in this stage
                     const uint32_t bytes =
-                        static_cast<uint32_t>(nk * (C::A_BYTES1 + C::B_BYTES1) + (group_start ? C::SF_BYTES : 0));
+                        static_cast<uint32_t>(nk * (C::A_BYTES1 + C::B_TX1) + (group_start ? C::SF_BYTES : 0));
                     if constexpr (PAIR) {
                         // Only the leader arms the barrier (with both CTAs' bytes); the peer's loads just count
                         // their bytes on it.  A peer load may land before the leader arms the phase: the
@@ -611,12 +621,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         }
                     }
                     if (group_start) {
+                        const int qb = C::BF4 ? kb0 : q;  // the stage's first B scale word
                         if (scales_ready) {
-                            load_scales(s, sfa_y0 + q, sfb_y0 + q * C::SFB_ATOMS);
+                            load_scales(s, sfa_y0 + q, sfb_y0 + qb * C::SFB_ATOMS);
                         } else {
                             def_stage[n_deferred] = s;
                             def_ya[n_deferred] = sfa_y0 + q;
-                            def_yb[n_deferred] = sfb_y0 + q * C::SFB_ATOMS;
+                            def_yb[n_deferred] = sfb_y0 + qb * C::SFB_ATOMS;
                             ++n_deferred;
                         }
                     }
@@ -642,7 +653,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer (leader CTA)
         if (lane == 0 && rank == 0) {
-            constexpr uint32_t IDESC = idesc_mxf8_e4m3(C::TILE_M, BN);
+            constexpr uint32_t IDESC = idesc_mxf8_e4m3(C::TILE_M, BN, C::BF4);
             int s = 0;
             uint32_t ph = 0;
             int acc = 0;
@@ -662,15 +673,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const int nk = min(C::KPS, tile_nkb - kb0);
                     if (!wait_bounded(&full[s], ph, s_abort, p.err, p.wait_limit_ns)) { ok = false; break; }
                     tc_fence_after_sync();
-                    if (kb0 % SF_GROUP == 0) {
-                        // the group's scales into the next TMEM slot (the slot's previous readers, the MMAs of
-                        // the group SF_SLOTS groups back, were issued earlier and the tensor pipe runs in order)
+                    if (C::BF4 || kb0 % SF_GROUP == 0) {
+                        // the group's (FP4 B: the stage's) scales into the next TMEM slot (the slot's previous
+                        // readers, SF_SLOTS slots back, were issued earlier and the tensor pipe runs in order)
                         sf_tmem = tmem_base + static_cast<uint32_t>(C::SF_TMEM_BASE + sf_slot * C::SF_COLS);
                         if (++sf_slot == C::SF_SLOTS) sf_slot = 0;
                         const uint32_t sf_smem = smem_u32(sSF + s * C::SF_BYTES);
                         tc_cp_32x128b_warpx4<CTAS>(sf_tmem, sdesc_rows16_noswizzle(sf_smem));
 #pragma unroll
-                        for (int a = 0; a < C::SFB_ATOMS; ++a)
+                        for (int a = 0; a < C::SFB_KB * C::SFB_ATOMS; ++a)
                             tc_cp_32x128b_warpx4<CTAS>(sf_tmem + 4 + 4 * a,
                                                        sdesc_rows16_noswizzle(sf_smem + 512 + 512 * a));
                     }
@@ -679,13 +690,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     for (int i = 0; i < nk; ++i) {
                         const int kb = kb0 + i;
                         const uint32_t sub = static_cast<uint32_t>(kb % SF_GROUP);  // byte of the packed scales
-                        const uint32_t idesc = IDESC | (sub << 29) | (sub << 4);
                         const uint32_t a_base = a_stage + i * C::A_BYTES1;
                         const uint32_t b_base = b_stage + i * C::B_BYTES1;
+                        // B's scales: the group's word (byte kb % 4) or, FP4 B, this K block's word in the slot,
+                        // whose byte k is the scale of the 32-K sub-block the k-th MMA contracts
+                        const uint32_t sf_b = sf_tmem + 4 + (C::BF4 ? static_cast<uint32_t>(4 * C::SFB_ATOMS * i) : 0u);
 #pragma unroll
                         for (int k = 0; k < BLOCK_K / MMA_K; ++k) {
+                            const uint32_t b_byte = C::BF4 ? static_cast<uint32_t>(k) : sub;
+                            const uint32_t idesc = IDESC | (sub << 29) | (b_byte << 4);
                             tc_mma_mxf8<CTAS>(d_tmem, sdesc_kmajor_sw128(a_base + k * MMA_K),
-                                              sdesc_kmajor_sw128(b_base + k * MMA_K), idesc, sf_tmem, sf_tmem + 4,
+                                              sdesc_kmajor_sw128(b_base + k * MMA_K), idesc, sf_tmem, sf_b,
                                               (kb | k) != 0);
                         }
                     }

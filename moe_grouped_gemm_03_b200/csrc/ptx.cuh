@@ -330,14 +330,14 @@ __device__ __forceinline__ uint64_t sdesc_rows16_noswizzle(uint32_t saddr) {
     return d;  // swizzle mode 0: none
 }
 
-// Instruction descriptor of kind::mxf8f6f4 with block scaling: A and B e4m3, both K-major, fp32
-// accumulator, UE8M0 scales, scale-factor byte 0 of each 32-bit TMEM scale word.
-__host__ __device__ constexpr uint32_t idesc_mxf8_e4m3(int M, int N) {
-    return (0u << 7)                                     // A format E4M3
-           | (0u << 10)                                  // B format E4M3
-           | (static_cast<uint32_t>(N >> 3) << 17)        // N / 8
-           | (1u << 23)                                  // scale format UE8M0
-           | (static_cast<uint32_t>(M >> 4) << 24);       // M / 16
+// Instruction descriptor of kind::mxf8f6f4 with block scaling: A e4m3, B e4m3 (or E2M1 when b_e2m1), both
+// K-major, fp32 accumulator, UE8M0 scales, scale-factor byte 0 of each 32-bit TMEM scale word.
+__host__ __device__ constexpr uint32_t idesc_mxf8_e4m3(int M, int N, bool b_e2m1 = false) {
+    return (0u << 7)                                          // A format E4M3
+           | ((b_e2m1 ? 5u : 0u) << 10)                       // B format E4M3 (0) or E2M1 (5)
+           | (static_cast<uint32_t>(N >> 3) << 17)             // N / 8
+           | (1u << 23)                                       // scale format UE8M0
+           | (static_cast<uint32_t>(M >> 4) << 24);            // M / 16
 }
 
 }  // namespace dg

@@ -33,7 +33,9 @@ struct PackParams {
     // SFB: fp32 [G][ceil(N/128)][K/128], or [G][K/128][ceil(N/128)] when sfb_kn (B in the NN orientation)
     const float *sfb;
     int sfb_kn;
-    int sfb_ld;           // K-grouped: row extent of the MN-major SFB [K/128][sfb_ld]
+    int sfb_ld;           // K-grouped: row extent of the MN-major SFB [K/128][sfb_ld]; FP4 B: of [G][K/32][sfb_ld]
+    int sfb_fp4;          // B in E2M1: one scale per (row, 32-K block); a B word holds a 128-K block's four
+    int sfb_kwords;       // B scale words along K per (group, N tile): num_sf_groups, or K/128 when sfb_fp4
     int N, G, bn, n_tiles, sfb_atoms;
     int nkb, num_sf_groups;
     uint32_t *sfa_out;    // [sfa_groups * blocks_per_group][num_sf_groups][128]
@@ -134,12 +136,29 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
             const long long b = atom - sfa_atoms;
             const int a = static_cast<int>(b % p.sfb_atoms);
             long long rest = b / p.sfb_atoms;
-            const int q = static_cast<int>(rest % p.num_sf_groups);
-            rest /= p.num_sf_groups;
+            const int q = static_cast<int>(rest % p.sfb_kwords);
+            rest /= p.sfb_kwords;
             const int nt = static_cast<int>(rest % p.n_tiles);
             const int g = static_cast<int>(rest / p.n_tiles);
             int kb_first, kb_count;
             k_blocks(q, kb_first, kb_count);
+            if (p.sfb_fp4) {  // the word of 128-K block q: bytes i = its 32-K sub-blocks 4q + i
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int n = nt * p.bn + a * 128 + lane + 32 * j;
+                    const float *base = p.sfb + static_cast<size_t>(g) * (4 * p.nkb) * p.sfb_ld + n;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t code = (n < p.N && q < p.nkb)
+                                                  ? ue8m0_code(__ldg(base + static_cast<size_t>(4 * q + i) * p.sfb_ld))
+                                                  : 0x7Fu;
+                        word[j] |= code << (8 * i);
+                    }
+                }
+                dst = p.sfb_out + b * SF_ATOM_WORDS;
+                *reinterpret_cast<uint4 *>(dst + 4 * lane) = make_uint4(word[0], word[1], word[2], word[3]);
+                continue;
+            }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int n = nt * p.bn + a * 128 + lane + 32 * j;

@@ -1,6 +1,6 @@
 """The workloads at full size on the GPU (the five of the method's benchmarks, workload 5's token split in the
-no-padding layout, workload 3 with B in the NN orientation, and workload 3's token counts as the K extents of a
-K-grouped GEMM), in the launch configuration the bench times.
+no-padding layout, workload 3 with B in the NN orientation, workload 3's token counts as the K extents of a
+K-grouped GEMM, and workload 3 with B in E2M1), in the launch configuration the bench times.
 
 Outputs are checked against the oracle on sampled rows (every group's first and last valid row, the rows
 on each side of every 128-row tile boundary of the sample's blocks, plus random rows), all N columns; the
@@ -33,7 +33,7 @@ def sample_rows(p, n_random=192, seed=0):
     return np.array(sorted(picks), np.int64)
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5, 6, 7, 8, 9])
 def test_full_config(cfg):
     import moe_grouped_gemm_03_b200 as dg
 

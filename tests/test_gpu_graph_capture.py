@@ -35,7 +35,8 @@ def _capture(fn):
     lambda: synth.make_nopad([130, 0, 257], 512, 256, seed=34),
     lambda: synth.make_contiguous_nn([129, 300], 512, 384, seed=35),
     lambda: synth.make_k_grouped([128, 384], 200, 512, seed=36, with_c=False),
-], ids=["dense", "contiguous", "masked", "nopad", "nn", "k_grouped"])
+    lambda: synth.make_contiguous_w4a8([129, 300], 512, 256, seed=38),
+], ids=["dense", "contiguous", "masked", "nopad", "nn", "k_grouped", "w4a8"])
 def test_captured_call_replays_to_eager_result(make):
     import moe_grouped_gemm_03_b200 as dg
 

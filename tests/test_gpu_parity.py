@@ -148,6 +148,17 @@ def test_k_grouped_shapes(ks, M, N, c_mode, policy):
     assert np.abs(got - ref).max() <= 1e-4 * rms + 1e-5 * np.abs(ref).max()
 
 
+@pytest.mark.parametrize("counts,N,K", [
+    ([0, 1, 127, 128, 129, 300], 512, 256),
+    ([513, 7, 260], 4096, 384),
+    ([1], 16, 128),
+    ([129, 1, 130, 255, 256, 257, 3], 640, 256),
+    ([300, 200], 7168, 1024),
+])
+def test_contiguous_w4a8_shapes(counts, N, K, policy):
+    _full_check(synth.make_contiguous_w4a8(counts, N, K, seed=sum(counts) + N + 4))
+
+
 @pytest.fixture
 def alignment_256():
     import moe_grouped_gemm_03_b200 as dg
