@@ -136,6 +136,13 @@ DG_EXPORT int dg_m_grouped_fp8_fp4_gemm_nt_contiguous(const void *a, const float
                                             const float *sfb, void *d, const int *m_indices, int M_total, int N, int K,
                                             int G, dg_stream_t stream);
 
+/* M-grouped GEMM, masked layout, W4A8 (`m_grouped_fp8_fp4_gemm_nt_masked`, same page): as
+ * dg_m_grouped_fp8_gemm_nt_masked except b [G][N][K/2] bytes of packed E2M1 codes (32-byte aligned) and
+ * sfb [G][K/32][ld(N)] fp32, one scale per (row n, 32-K block), as in dg_m_grouped_fp8_fp4_gemm_nt_contiguous. */
+DG_EXPORT int dg_m_grouped_fp8_fp4_gemm_nt_masked(const void *a, const float *sfa, const void *b, const float *sfb,
+                                        void *d, const int *masked_m, int G, int M_max, int N, int K, int expected_m,
+                                        dg_stream_t stream);
+
 /* K-grouped GEMM (MATE docs, 0.2.7 additions, `k_grouped_fp8_gemm_nt_contiguous`: recipe (1, 1, 128), host K
  * extents, C accumulated into D), e.g. the per-expert weight gradient of an MoE layer.
  *   a [M][sum ks] e4m3 and b [N][sum ks] e4m3, both K-major, the groups' K segments concatenated in group order;

@@ -57,6 +57,7 @@ _SIGNATURES = {
     "dg_m_grouped_fp8_gemm_nt_nopad": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_gemm_nn_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_m_grouped_fp8_fp4_gemm_nt_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "dg_m_grouped_fp8_fp4_gemm_nt_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "dg_k_grouped_fp8_gemm_nt_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_set_cta_pair_policy": (_I, [_I]),
@@ -313,6 +314,27 @@ def m_grouped_fp8_fp4_gemm_nt_contiguous(lhs, rhs, out: torch.Tensor, m_indices:
                                                         _ptr(m_indices), M, N, K, G, _stream()))
 
 
+def m_grouped_fp8_fp4_gemm_nt_masked(lhs, rhs, out: torch.Tensor, masked_m: torch.Tensor, expected_m: int) -> None:
+    """W4A8 masked layout: rhs = (b packed E2M1 uint8 [G, N, K/2], sfb [G, K/32, tma_aligned(N)]); lhs, out and
+    masked_m as for m_grouped_fp8_gemm_nt_masked."""
+    a, sfa = lhs
+    b, sfb = rhs
+    _check_operand("a", a, 3, _FP8_TYPES)
+    _check_operand("b", b, 3, (torch.uint8,))
+    _check_operand("sfa", sfa, 3, (torch.float32,))
+    _check_operand("sfb", sfb, 3, (torch.float32,))
+    _check_operand("out", out, 3, (torch.bfloat16,))
+    _check_operand("masked_m", masked_m, 1, (torch.int32,))
+    G, M_max, K = a.shape
+    N = b.shape[1]
+    _need(b.shape[0] == G and b.shape[2] * 2 == K and tuple(out.shape) == (G, M_max, N) and masked_m.shape[0] == G,
+          "shape mismatch")
+    _need(sfa.shape == (G, K // 128, get_tma_aligned_size(M_max, 4)), "sfa must be [G, K/128, tma_aligned(M_max)]")
+    _need(sfb.shape == (G, K // 32, get_tma_aligned_size(N, 4)), "sfb must be [G, K/32, tma_aligned(N)]")
+    _check(_lib.dg_m_grouped_fp8_fp4_gemm_nt_masked(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(out), _ptr(masked_m),
+                                                    G, M_max, N, K, int(expected_m), _stream()))
+
+
 def m_grouped_fp8_gemm_nt_nopad(lhs, rhs, out: torch.Tensor, counts: torch.Tensor) -> None:
     """No-padding layout: group g's rows are off_g .. off_g + counts[g] - 1 (off_g = sum of the earlier counts);
     out rows of group g = lhs rows of group g @ rhs[g]^T; rows past sum(counts) are untouched."""
@@ -337,7 +359,7 @@ def m_grouped_fp8_gemm_nt_nopad(lhs, rhs, out: torch.Tensor, counts: torch.Tenso
 __all__ = [
     "DGError", "fp8_gemm_nt", "fp8_gemm_nt_noalloc", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
     "m_grouped_fp8_gemm_nt_nopad", "m_grouped_fp8_gemm_nn_contiguous", "k_grouped_fp8_gemm_nt_contiguous",
-    "m_grouped_fp8_fp4_gemm_nt_contiguous",
+    "m_grouped_fp8_fp4_gemm_nt_contiguous", "m_grouped_fp8_fp4_gemm_nt_masked",
     "get_m_alignment_for_contiguous_layout", "set_m_alignment_for_contiguous_layout", "get_tma_aligned_size", "set_num_sms", "get_num_sms", "num_tiles",
     "select_block_n", "set_cta_pair_policy", "check_device_error", "lib", "header_symbols", "last_error",
 ]

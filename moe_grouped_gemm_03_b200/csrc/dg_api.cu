@@ -644,6 +644,45 @@ int launch_contiguous(const void *a, const float *sfa, const void *b, const floa
 
 }  // namespace
 
+namespace {
+
+// The masked calls: B e4m3, or (b_fp4) B in E2M1 with one scale per (row, 32-K block).
+int masked_call(const void *a, const float *sfa, const void *b, const float *sfb, void *d, const int *masked_m,
+                int G, int M_max, int N, int K, int expected_m, dg_stream_t stream, bool b_fp4) {
+    if (int rc = check_common(a, sfa, b, sfb, d, N, K)) return rc;
+    if (!masked_m) return fail(DG_ERR_INVALID_ARG, "masked_m is null");
+    if (!aligned(masked_m, 4)) return fail(DG_ERR_ALIGNMENT, "masked_m must be 4-byte aligned");
+    if (G < 1 || G > dg::MAX_MASKED_GROUPS)
+        return fail(DG_ERR_INVALID_ARG, "G=%d must be in [1, %d]", G, dg::MAX_MASKED_GROUPS);
+    if (M_max < 1) return fail(DG_ERR_INVALID_ARG, "M_max=%d must be positive", M_max);
+    if (static_cast<long long>(G) * M_max > 0x7fffffffLL || static_cast<long long>(G) * N > 0x7fffffffLL)
+        return fail(DG_ERR_INVALID_ARG, "G*M_max or G*N exceeds 2^31");
+    DeviceInfo info;
+    if (int rc = device_info(info)) return rc;
+    dg::GemmParams p{};
+    p.mode = dg::MODE_MASKED;
+    p.M = M_max; p.N = N; p.K = K; p.G = G;
+    ScaleArgs sc{sfa, dg_get_tma_aligned_size(M_max, 4), sfb};
+    sc.sfb_fp4 = b_fp4;
+    if (b_fp4) sc.sfb_ld = dg_get_tma_aligned_size(N, 4);
+    p.sfa_blocks = (M_max + dg::BLOCK_M - 1) / dg::BLOCK_M;
+    p.d = static_cast<__nv_bfloat16 *>(d);
+    p.masked_m = masked_m;
+    p.err = device_error_word();
+    if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
+    // tile shape from the caller's hint; the grid from the most tiles masked_m could ask for
+    const int hint = expected_m > 0 && expected_m < M_max ? expected_m : M_max;
+    const long long h1 = static_cast<long long>(G) * ((hint + dg::BLOCK_M - 1) / dg::BLOCK_M);
+    const long long h2 = static_cast<long long>(G) * ((hint + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M));
+    const long long max1 = static_cast<long long>(G) * ((M_max + dg::BLOCK_M - 1) / dg::BLOCK_M);
+    const long long max2 = static_cast<long long>(G) * ((M_max + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M));
+    const Plan plan{h1, h2, max1, max2, 0, 0, true};
+    return plan_and_launch(p, info, plan, a, static_cast<long long>(G) * M_max, b, static_cast<long long>(G) * N, sc,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
 extern "C" {
 
 int dg_get_m_alignment_for_contiguous_layout(void) { return g_m_alignment; }
@@ -772,35 +811,16 @@ int dg_m_grouped_fp8_gemm_nn_contiguous(const void *a, const float *sfa, const v
 int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
                                     const int *masked_m, int G, int M_max, int N, int K, int expected_m,
                                     dg_stream_t stream) {
-    if (int rc = check_common(a, sfa, b, sfb, d, N, K)) return rc;
-    if (!masked_m) return fail(DG_ERR_INVALID_ARG, "masked_m is null");
-    if (!aligned(masked_m, 4)) return fail(DG_ERR_ALIGNMENT, "masked_m must be 4-byte aligned");
-    if (G < 1 || G > dg::MAX_MASKED_GROUPS)
-        return fail(DG_ERR_INVALID_ARG, "G=%d must be in [1, %d]", G, dg::MAX_MASKED_GROUPS);
-    if (M_max < 1) return fail(DG_ERR_INVALID_ARG, "M_max=%d must be positive", M_max);
-    if (static_cast<long long>(G) * M_max > 0x7fffffffLL || static_cast<long long>(G) * N > 0x7fffffffLL)
-        return fail(DG_ERR_INVALID_ARG, "G*M_max or G*N exceeds 2^31");
-    DeviceInfo info;
-    if (int rc = device_info(info)) return rc;
-    dg::GemmParams p{};
-    p.mode = dg::MODE_MASKED;
-    p.M = M_max; p.N = N; p.K = K; p.G = G;
-    const ScaleArgs sc{sfa, dg_get_tma_aligned_size(M_max, 4), sfb};
-    p.sfa_blocks = (M_max + dg::BLOCK_M - 1) / dg::BLOCK_M;
-    p.d = static_cast<__nv_bfloat16 *>(d);
-    p.masked_m = masked_m;
-    p.err = device_error_word();
-    if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
-    // tile shape from the caller's hint; the grid from the most tiles masked_m could ask for
-    const int hint = expected_m > 0 && expected_m < M_max ? expected_m : M_max;
-    const long long h1 = static_cast<long long>(G) * ((hint + dg::BLOCK_M - 1) / dg::BLOCK_M);
-    const long long h2 = static_cast<long long>(G) * ((hint + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M));
-    const long long max1 = static_cast<long long>(G) * ((M_max + dg::BLOCK_M - 1) / dg::BLOCK_M);
-    const long long max2 = static_cast<long long>(G) * ((M_max + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M));
-    const Plan plan{h1, h2, max1, max2, 0, 0, true};
-    return plan_and_launch(p, info, plan, a, static_cast<long long>(G) * M_max, b, static_cast<long long>(G) * N, sc,
-                           reinterpret_cast<cudaStream_t>(stream));
+    return masked_call(a, sfa, b, sfb, d, masked_m, G, M_max, N, K, expected_m, stream, false);
 }
+
+int dg_m_grouped_fp8_fp4_gemm_nt_masked(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
+                                        const int *masked_m, int G, int M_max, int N, int K, int expected_m,
+                                        dg_stream_t stream) {
+    if (b && !aligned(b, 32)) return fail(DG_ERR_ALIGNMENT, "b (packed E2M1) must be 32-byte aligned");
+    return masked_call(a, sfa, b, sfb, d, masked_m, G, M_max, N, K, expected_m, stream, true);
+}
+
 
 int dg_debug_bounded_wait(unsigned long long limit_ns, int drop_first_stage) {
     if (limit_ns != 0 && (limit_ns < 1000000ull || limit_ns > dg::WAIT_LIMIT_NS))

@@ -97,7 +97,7 @@ def unpack_e2m1(packed) -> np.ndarray:
 
 
 def w4a8_rows(p, rows) -> np.ndarray:
-    """Rows of a contiguous W4A8 ``synth.Problem`` (rows of groups only)."""
+    """Rows of a W4A8 ``synth.Problem`` (contiguous or masked; rows of groups only)."""
     rows = np.asarray(rows, np.int64)
     groups = p.row_groups(rows)
     out = np.zeros((len(rows), p.N))
@@ -112,7 +112,8 @@ def w4a8_rows(p, rows) -> np.ndarray:
             for j in range(4):
                 sub = slice(128 * kb + 32 * j, 128 * kb + 32 * j + 32)
                 blk += (adec[:, sub] @ bdec[:, sub].T) * p.sfb[g, 4 * kb + j, :p.N][None, :]
-            acc += blk * p.sfa[kb, r][:, None]
+            sa = p.sfa[g, kb, r - g * p.M] if p.kind == "masked_w4a8" else p.sfa[kb, r]
+            acc += blk * sa[:, None]
         out[sel] = acc
     return out
 
@@ -154,7 +155,7 @@ def problem_rows(p, rows) -> np.ndarray:
             out[sel] = k_grouped_rows(p, int(g), rows[sel] - g * p.M)
         return out
     groups = p.row_groups(rows)
-    if p.kind == "contiguous_w4a8":
+    if p.kind in ("contiguous_w4a8", "masked_w4a8"):
         return w4a8_rows(p, rows)
     if p.kind == "contiguous_nn":
         # B_g[k, n] is the definition's b_g[n, k]; sfb_g[kb, nb] its s_b(g, nb, kb)

@@ -46,7 +46,8 @@ def tma_aligned_rows(rows: int) -> int:
 class Problem:
     """One GEMM problem in the layouts the library takes.
 
-    kind       'dense' | 'contiguous' | 'masked' | 'nopad' | 'contiguous_nn' | 'k_grouped' | 'contiguous_w4a8'
+    kind       'dense' | 'contiguous' | 'masked' | 'nopad' | 'contiguous_nn' | 'k_grouped' | 'contiguous_w4a8' |
+               'masked_w4a8'
     a          uint8 e4m3 codes, [rows, K]; masked: [G * M_max, K] (= [G, M_max, K] flattened)
     sfa        fp32, dense/contiguous [K/128, align4(rows)]; masked [G, K/128, align4(M_max)]
     b          uint8 e4m3 codes, [G, N, K] (G = 1 for dense); contiguous_nn: [G, K, N]; contiguous_w4a8: packed
@@ -116,7 +117,7 @@ class Problem:
     def out_shape(self):
         if self.kind == "k_grouped":
             return (self.G, self.M, self.N)
-        if self.kind == "masked":
+        if self.kind in ("masked", "masked_w4a8"):
             return (self.G, self.M, self.N)
         return (self.rows, self.N)
 
@@ -325,6 +326,23 @@ def make_contiguous_w4a8(counts: Sequence[int], N: int, K: int, seed: int = 0, n
     return p
 
 
+def make_masked_w4a8(G: int, M_max: int, N: int, K: int, masked_m: Optional[Sequence[int]] = None, seed: int = 0,
+                     expected_m: int = 0, name: str = "") -> Problem:
+    """The masked layout with B in E2M1 and one B scale per (row, 32-K block), as ``make_contiguous_w4a8``."""
+    p = make_masked(G, M_max, N, K, masked_m=masked_m, seed=seed, expected_m=expected_m)
+    rng = np.random.default_rng(seed + 1)
+    b = np.empty((G, N, K // 2), np.uint8)
+    sfb = np.ones((G, K // 32, tma_aligned_rows(N)), np.float32)
+    for g in range(G):
+        codes, sb = quantize_rows_e2m1(_draw_normal(rng, (N, K)))
+        b[g] = pack_e2m1(codes)
+        sfb[g, :, :N] = sb.T
+    p.kind = "masked_w4a8"
+    p.b, p.sfb = b, sfb
+    p.name = name or f"masked W4A8 G={G} M_max={M_max} N={N} K={K}"
+    return p
+
+
 def make_nopad(counts: Sequence[int], N: int, K: int, seed: int = 0, extra_rows: int = 0, name: str = "",
                rng: Optional[np.random.Generator] = None) -> Problem:
     """Groups' rows concatenated with no padding, then ``extra_rows`` rows that no group owns (garbage)."""
@@ -440,7 +458,7 @@ def to_torch(p: Problem, device="cuda"):
     if p.kind == "dense":
         out["b"] = out["b"].view(p.N, p.K)
         out["sfb"] = out["sfb"].view(p.sfb.shape[1], p.sfb.shape[2])
-    if p.kind == "masked":
+    if p.kind in ("masked", "masked_w4a8"):
         out["a"] = out["a"].view(p.G, p.M, p.K)
         out["masked_m"] = t(p.masked_m)
     if p.kind in ("contiguous", "contiguous_nn", "contiguous_w4a8"):

@@ -22,6 +22,8 @@ def run_problem(p, tensors=None, out=None, stream=None):
         dg.fp8_gemm_nt((t["a"], t["sfa"]), (t["b"], t["sfb"]), out)
     elif p.kind == "contiguous":
         dg.m_grouped_fp8_gemm_nt_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["m_indices"])
+    elif p.kind == "masked_w4a8":
+        dg.m_grouped_fp8_fp4_gemm_nt_masked((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["masked_m"], p.expected_m)
     elif p.kind == "contiguous_w4a8":
         dg.m_grouped_fp8_fp4_gemm_nt_contiguous((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["m_indices"])
     elif p.kind == "contiguous_nn":

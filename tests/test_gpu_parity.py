@@ -159,6 +159,15 @@ def test_contiguous_w4a8_shapes(counts, N, K, policy):
     _full_check(synth.make_contiguous_w4a8(counts, N, K, seed=sum(counts) + N + 4))
 
 
+@pytest.mark.parametrize("G,M_max,N,K,mm", [
+    (5, 200, 256, 512, [0, 1, 128, 200, 77]),
+    (3, 256, 7168, 256, [256, 0, 129]),
+    (40, 128, 384, 256, None),
+])
+def test_masked_w4a8_shapes(G, M_max, N, K, mm, policy):
+    _full_check(synth.make_masked_w4a8(G, M_max, N, K, masked_m=mm, seed=G + M_max + 4, expected_m=M_max // 2))
+
+
 @pytest.fixture
 def alignment_256():
     import moe_grouped_gemm_03_b200 as dg

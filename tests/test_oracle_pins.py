@@ -344,6 +344,22 @@ def test_w4a8_sub_block_scale_moves_one_column():
     np.testing.assert_allclose(diff[:, n], (a @ b) * (p.sfb[0, j, n] / 2.0), rtol=1e-12, atol=1e-9)
 
 
+def test_masked_w4a8_equals_contiguous_w4a8_of_the_same_rows():
+    """The masked W4A8 layout's owned rows equal the (separately pinned) contiguous W4A8 product of the same
+    rows, scales and B."""
+    q = synth.make_masked_w4a8(3, 128, 64, 256, masked_m=[128, 5, 0], seed=25)
+    c = synth.make_contiguous_w4a8([128, 128, 128], 64, 256, seed=25)
+    c.a = q.a.copy()
+    c.sfa = np.concatenate([q.sfa[g][:, :128] for g in range(3)], axis=1)
+    c.b, c.sfb = q.b.copy(), q.sfb.copy()
+    c.m_indices = np.repeat(np.arange(3, dtype=np.int32), 128)
+    full_q = oracle.problem_full(q).reshape(-1, 64)
+    full_c = oracle.problem_full(c)
+    rows = q.valid_rows()
+    np.testing.assert_array_equal(full_q[rows], full_c[rows])
+    assert np.isnan(full_q[np.setdiff1d(np.arange(384), rows)]).all()
+
+
 def test_library_call_shapes_agree_with_problem_driver():
     p = synth.make_masked(G=3, M_max=64, N=128, K=128, masked_m=[3, 64, 0], seed=8)
     a = p.a.reshape(p.G, p.M, p.K)
