@@ -192,6 +192,11 @@ def call_library(p, t, out):
         dg.m_grouped_fp8_gemm_nt_masked((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["masked_m"], p.expected_m)
 
 
+def launches_per_call(p):
+    """The library's kernels one call launches: the scale pre-pass and the GEMM (NN: the B transpose too)."""
+    return 3 if p.kind == "contiguous_nn" else 2
+
+
 def algorithmic_bytes(p):
     """Each valid A row once, each active group's B once, the scales of those, each valid D row once.
     K-grouped: A and B once, their per-row scales, fp32 D once (no C in the timed call)."""
@@ -365,7 +370,7 @@ def run_ours(args, world, rank, local):
         "roofline": roofline,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": K,
+        "gpu_launches": K * launches_per_call(p),
         "clocks": clocks.summary(),
     }
     if not args.no_cpu_baseline and world == 1:
