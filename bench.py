@@ -3,8 +3,9 @@
 
 One step = one call of the library's dense FP8 GEMM on the workload M=4096, N=7168, K=7168 (A and B e4m3
 with power-of-two 1x128 / 128x128 scales, bf16 out; seeded synthetic inputs), the configuration the
-headline metric is quoted on.  Other workloads can be timed with --workload (contiguous / masked grouped
-shapes) for reference; the default line is the contract line.
+headline metric is quoted on.  Other workloads can be timed with --workload for reference (the default line
+is the contract line): 1 dense 128x256x512; 3 and 5 contiguous grouped; 4 masked grouped; 6 no-padding grouped;
+7 contiguous with B in the NN orientation; 8 K-grouped with fp32 output; 9 contiguous W4A8 (B in E2M1).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 2]
 
