@@ -192,6 +192,43 @@ int scratch_pool(int device, cudaMemPool_t &pool) {
     return DG_OK;
 }
 
+}  // namespace
+
+// ------------------------------------------------------------------------------------------------------------
+// The fixed scratch buffer of the allocation-free dense GEMM (dg_fp8_gemm_nt_noalloc)
+//
+// Some callers may not allocate device memory at all during a call: code that runs while a stream is being
+// captured in the global capture mode (where allocation calls are refused), engines whose memory manager owns
+// every byte of HBM, or real-time paths that cannot afford an allocator call. For them the packed scales go to a
+// fixed buffer that exists for the lifetime of the library instead of the per-call pool allocation. All calls
+// share the buffer, so calls whose work overlaps on the GPU (different streams, no ordering between them) race on
+// it; calls on one stream are ordered and safe.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB of packed scale atoms
+static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoAllocScratchBytes / 4];
+
+// Device address of the static buffer, looked up once per device with that device current.  In host code the
+// name g_noalloc_scratch is only a host-side stand-in for the symbol, never a device address.
+int noalloc_scratch(int device, uint32_t **out) {
+    static std::mutex mu;
+    static uint32_t *ptrs[64] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (device < 0 || device >= 64) return fail(DG_ERR_UNSUPPORTED, "device index %d out of range", device);
+    if (!ptrs[device]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress (static scale buffer)");
+        ptrs[device] = static_cast<uint32_t *>(p);
+    }
+    *out = ptrs[device];
+    return DG_OK;
+}
+
+}  // namespace
+
+namespace {
+
 // ----------------------------------------------------------------------------------------------- launch
 int g_m_alignment = dg::BLOCK_M;  // contiguous layout: per-segment M padding (128 or 256)
 int g_pair_policy = -1;  // -1: library decides; 0: single CTAs only; 1: CTA pairs whenever supported
@@ -211,6 +248,7 @@ struct ScaleArgs {
     const float *sfb;
     bool sfb_kn = false;  // SFB stored [G][K/128][ceil(N/128)] (B in the NN orientation)
     bool sfb_fp4 = false; // B in E2M1 (packed two per byte) with SFB [G][K/32][sfb_ld]
+    bool fixed_scratch = false;  // packed scales in the library's fixed buffer (no allocation) instead of the pool
     int sfb_ld = 0;       // K-grouped: one scale per row of B, [K/128][sfb_ld]; FP4 B: [G][K/32][sfb_ld]
 };
 
@@ -279,11 +317,24 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
     const long long sfb_atoms = b_groups * p.num_n_blocks * pk.sfb_kwords * C::SFB_ATOMS;
     pk.sfa_words = sfa_atoms * dg::SF_ATOM_WORDS;
     pk.sfb_words = sfb_atoms * dg::SF_ATOM_WORDS;
-    cudaMemPool_t pool;
-    if (int rc = scratch_pool(device, pool)) return rc;
+    const size_t need = static_cast<size_t>(pk.sfa_words + pk.sfb_words) * 4;
     void *scratch = nullptr;
-    cudaError_t e = cudaMallocFromPoolAsync(&scratch, static_cast<size_t>(pk.sfa_words + pk.sfb_words) * 4, pool, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync (packed scales)");
+    cudaError_t e;
+    if (sc.fixed_scratch) {  // calls no allocator: every word of both regions is rewritten by the pre-pass
+        if (need > kNoAllocScratchBytes)
+            return fail(DG_ERR_UNSUPPORTED,
+                        "the packed scales of this shape need %zu bytes; the allocation-free call has a fixed %zu-byte "
+                        "buffer (use dg_fp8_gemm_nt)",
+                        need, kNoAllocScratchBytes);
+        uint32_t *fixed = nullptr;
+        if (int rc = noalloc_scratch(device, &fixed)) return rc;
+        scratch = fixed;
+    } else {
+        cudaMemPool_t pool;
+        if (int rc = scratch_pool(device, pool)) return rc;
+        if ((e = cudaMallocFromPoolAsync(&scratch, need, pool, stream)) != cudaSuccess)
+            return cuda_fail(e, "cudaMallocFromPoolAsync (packed scales)");
+    }
     pk.sfa_out = static_cast<uint32_t *>(scratch);
     pk.sfb_out = pk.sfa_out + pk.sfa_words;
     int rc = DG_OK;
@@ -355,8 +406,10 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
             break;
         }
     } while (false);
-    cudaError_t ef = cudaFreeAsync(scratch, stream);
-    if (rc == DG_OK && ef != cudaSuccess) rc = cuda_fail(ef, "cudaFreeAsync (packed scales)");
+    if (!sc.fixed_scratch) {
+        const cudaError_t ef = cudaFreeAsync(scratch, stream);
+        if (rc == DG_OK && ef != cudaSuccess) rc = cuda_fail(ef, "cudaFreeAsync (packed scales)");
+    }
     return rc;
 }
 
@@ -473,135 +526,6 @@ int check_common(const void *a, const float *sfa, const void *b, const float *sf
 
 }  // namespace
 
-// ------------------------------------------------------------------------------------------------------------
-// Allocation-free variant of the dense GEMM (dg_fp8_gemm_nt_noalloc)
-//
-// Some callers may not allocate device memory at all during a call: code that runs while a stream is being
-// captured in the global capture mode (where allocation calls are refused), engines whose memory manager owns
-// every byte of HBM, or real-time paths that cannot afford an allocator call. For them the packed scales go to a
-// fixed buffer that exists for the lifetime of the library instead of the per-call pool allocation. All calls
-// share the buffer, so calls whose work overlaps on the GPU (different streams, no ordering between them) race on
-// it; calls on one stream are ordered and safe.
-namespace {
-
-constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB of packed scale atoms
-static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoAllocScratchBytes / 4];
-
-// Device address of the static buffer, looked up once per device with that device current.  In host code the
-// name g_noalloc_scratch is only a host-side stand-in for the symbol, never a device address.
-int noalloc_scratch(int device, uint32_t **out) {
-    static std::mutex mu;
-    static uint32_t *ptrs[64] = {};
-    std::lock_guard<std::mutex> lock(mu);
-    if (device < 0 || device >= 64) return fail(DG_ERR_UNSUPPORTED, "device index %d out of range", device);
-    if (!ptrs[device]) {
-        void *p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress (static scale buffer)");
-        ptrs[device] = static_cast<uint32_t *>(p);
-    }
-    *out = ptrs[device];
-    return DG_OK;
-}
-
-template <int BN, int CTAS, int KPS>
-int launch_cfg_noalloc(const void *a, long long a_rows, const void *b, long long b_rows, const ScaleArgs &sc,
-                       dg::GemmParams p, int grid, int device, cudaStream_t stream) {
-    using C = dg::Cfg<BN, CTAS, KPS>;
-    const int nkb = p.K / dg::BLOCK_K;
-    dg::PackParams pk{};
-    pk.sfa = sc.sfa;
-    pk.sfa_ld = sc.sfa_ld;
-    pk.sfb = sc.sfb;
-    pk.sfb_kn = sc.sfb_kn ? 1 : 0;
-    pk.sfb_ld = sc.sfb_ld;
-    pk.N = p.N;
-    pk.G = p.G;
-    pk.bn = BN;
-    pk.n_tiles = p.num_n_blocks;
-    pk.sfb_atoms = C::SFB_ATOMS;
-    pk.nkb = nkb;
-    pk.num_sf_groups = p.num_sf_groups;
-    pk.sfb_kwords = p.num_sf_groups;
-    pk.rows_per_group = p.M;
-    pk.blocks_per_group = (p.M + dg::BLOCK_M - 1) / dg::BLOCK_M;
-    pk.sfa_groups = 1;
-    const long long sfa_atoms = static_cast<long long>(pk.blocks_per_group) * p.num_sf_groups;
-    const long long sfb_atoms = static_cast<long long>(p.G) * p.num_n_blocks * p.num_sf_groups * C::SFB_ATOMS;
-    pk.sfa_words = sfa_atoms * dg::SF_ATOM_WORDS;
-    pk.sfb_words = sfb_atoms * dg::SF_ATOM_WORDS;
-    const size_t need = static_cast<size_t>(pk.sfa_words + pk.sfb_words) * 4;
-    if (need > kNoAllocScratchBytes)
-        return fail(DG_ERR_UNSUPPORTED,
-                    "the packed scales of this shape need %zu bytes; the allocation-free call has a fixed %zu-byte "
-                    "buffer (use dg_fp8_gemm_nt)",
-                    need, kNoAllocScratchBytes);
-    uint32_t *scratch = nullptr;
-    if (int rc = noalloc_scratch(device, &scratch)) return rc;
-    pk.sfa_out = scratch;
-    pk.sfb_out = scratch + pk.sfa_words;  // every word of both regions is written by the pre-pass
-    cudaError_t e;
-    CUtensorMap ta, tb, tsfa, tsfb, td;
-    if (int rc = make_output_map(td, p.d, a_rows, p.N)) return rc;
-    if (int rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M)) return rc;
-    if (int rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS)) return rc;
-    if (int rc = make_atom_map(tsfa, pk.sfa_out, sfa_atoms, 1)) return rc;
-    if (int rc = make_atom_map(tsfb, pk.sfb_out, sfb_atoms, C::SFB_ATOMS)) return rc;
-    auto kernel = dg::fp8_gemm_kernel<C>;
-    if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) != cudaSuccess)
-        return cuda_fail(e, "cudaFuncSetAttribute");
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(grid * CTAS), 1, 1);
-    cfg.blockDim = dim3(dg::NUM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CTAS;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    if (CTAS > 1) {
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
-            cudaGetLastError();
-            n = grid;
-        }
-        if (grid > n) cfg.gridDim.x = static_cast<unsigned>(n * CTAS);
-    }
-    apply_wait_settings(p);
-    if (int rc = launch_pack(pk, device, stream)) return rc;
-    if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, tsfb, td, p)) != cudaSuccess)
-        return cuda_fail(e, "kernel launch");
-    return DG_OK;
-}
-
-int launch_bn_noalloc(int bn, int ctas, const void *a, long long a_rows, const void *b, long long b_rows,
-                      const ScaleArgs &sc, const dg::GemmParams &p, int grid, int device, cudaStream_t stream) {
-    if (ctas == 2) {
-        switch (bn) {
-            case 224: return launch_cfg_noalloc<224, 2, 2>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            case 192: return launch_cfg_noalloc<192, 2, 2>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            case 160: return launch_cfg_noalloc<160, 2, 2>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            case 128: return launch_cfg_noalloc<128, 2, 2>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            default: break;
-        }
-    } else {
-        switch (bn) {
-            case 224: return launch_cfg_noalloc<224, 1, 1>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            case 192: return launch_cfg_noalloc<192, 1, 1>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            case 160: return launch_cfg_noalloc<160, 1, 1>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            case 128: return launch_cfg_noalloc<128, 1, 1>(a, a_rows, b, b_rows, sc, p, grid, device, stream);
-            default: break;
-        }
-    }
-    return fail(DG_ERR_UNSUPPORTED, "no kernel instantiated for BN=%d with %d CTA(s) per tile", bn, ctas);
-}
-
-}  // namespace
 
 namespace {
 
@@ -640,6 +564,31 @@ int launch_contiguous(const void *a, const float *sfa, const void *b, const floa
     const bool pair_ok = (w1 + G) / 2 + 1 <= dg::MAX_PAIR_WINDOWS && G <= 32767;
     const Plan plan{w1, w2, w1, bound, w1, w2, pair_ok};
     return plan_and_launch(p, info, plan, a, M_total, b, static_cast<long long>(G) * N, sc, stream);
+}
+
+}  // namespace
+
+namespace {
+
+// The dense calls; `fixed_scratch`: the packed scales go to the library's fixed buffer (no allocation).
+int dense_call(const void *a, const float *sfa, const void *b, const float *sfb, void *d, int M, int N, int K,
+               dg_stream_t stream, bool fixed_scratch) {
+    if (M < 0) return fail(DG_ERR_INVALID_ARG, "M=%d must be non-negative", M);
+    if (int rc = check_common(a, sfa, b, sfb, d, N, K)) return rc;
+    if (M == 0) return DG_OK;
+    DeviceInfo info;
+    if (int rc = device_info(info)) return rc;
+    dg::GemmParams p{};
+    p.mode = dg::MODE_DENSE;
+    p.M = M; p.N = N; p.K = K; p.G = 1;
+    ScaleArgs sc{sfa, dg_get_tma_aligned_size(M, 4), sfb};
+    sc.fixed_scratch = fixed_scratch;
+    p.d = static_cast<__nv_bfloat16 *>(d);
+    p.err = device_error_word();
+    if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
+    const long long w1 = (M + dg::BLOCK_M - 1) / dg::BLOCK_M, w2 = (M + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M);
+    const Plan plan{w1, w2, w1, w2, w1, w2, true};
+    return plan_and_launch(p, info, plan, a, M, b, N, sc, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -741,21 +690,7 @@ int dg_check_device_error(dg_stream_t stream) {
 
 int dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const float *sfb, void *d, int M, int N, int K,
                    dg_stream_t stream) {
-    if (M < 0) return fail(DG_ERR_INVALID_ARG, "M=%d must be non-negative", M);
-    if (int rc = check_common(a, sfa, b, sfb, d, N, K)) return rc;
-    if (M == 0) return DG_OK;
-    DeviceInfo info;
-    if (int rc = device_info(info)) return rc;
-    dg::GemmParams p{};
-    p.mode = dg::MODE_DENSE;
-    p.M = M; p.N = N; p.K = K; p.G = 1;
-    const ScaleArgs sc{sfa, dg_get_tma_aligned_size(M, 4), sfb};
-    p.d = static_cast<__nv_bfloat16 *>(d);
-    p.err = device_error_word();
-    if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
-    const long long w1 = (M + dg::BLOCK_M - 1) / dg::BLOCK_M, w2 = (M + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M);
-    const Plan plan{w1, w2, w1, w2, w1, w2, true};
-    return plan_and_launch(p, info, plan, a, M, b, N, sc, reinterpret_cast<cudaStream_t>(stream));
+    return dense_call(a, sfa, b, sfb, d, M, N, K, stream, false);
 }
 
 
@@ -917,36 +852,7 @@ int dg_set_cta_pair_policy(int policy) {
 
 int dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void *b, const float *sfb, void *d, int M, int N,
                            int K, dg_stream_t stream) {
-    if (M < 0) return fail(DG_ERR_INVALID_ARG, "M=%d must be non-negative", M);
-    if (int rc = check_common(a, sfa, b, sfb, d, N, K)) return rc;
-    if (M == 0) return DG_OK;
-    DeviceInfo info;
-    if (int rc = device_info(info)) return rc;
-    dg::GemmParams p{};
-    p.mode = dg::MODE_DENSE;
-    p.M = M; p.N = N; p.K = K; p.G = 1;
-    const ScaleArgs sc{sfa, dg_get_tma_aligned_size(M, 4), sfb};
-    p.d = static_cast<__nv_bfloat16 *>(d);
-    p.err = device_error_word();
-    if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
-    // the same tile plan as dg_fp8_gemm_nt
-    const long long w1 = (M + dg::BLOCK_M - 1) / dg::BLOCK_M, w2 = (M + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M);
-    const int sms = effective_sms(info);
-    bool pair = sms >= 2;
-    if (g_pair_policy == 0) pair = false;
-    if (g_pair_policy < 0 && pair) {
-        const int bn2 = select_block_n(w2, N, sms / 2, 2);
-        pair = w2 * ((N + bn2 - 1) / bn2) >= sms / 2;
-    }
-    const int units = pair ? sms / 2 : sms;
-    const int bn = select_block_n(pair ? w2 : w1, N, units, pair ? 2 : 1);
-    p.num_n_blocks = (N + bn - 1) / bn;
-    p.num_windows = static_cast<int>(pair ? w2 : w1);
-    p.num_sf_groups = (K / dg::BLOCK_K + dg::SF_GROUP - 1) / dg::SF_GROUP;
-    const long long tiles = (pair ? w2 : w1) * p.num_n_blocks;
-    const int grid = static_cast<int>(tiles < units ? tiles : units);
-    return launch_bn_noalloc(bn, pair ? 2 : 1, a, M, b, N, sc, p, grid, info.device,
-                             reinterpret_cast<cudaStream_t>(stream));
+    return dense_call(a, sfa, b, sfb, d, M, N, K, stream, true);
 }
 
 }  // extern "C"
