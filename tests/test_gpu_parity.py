@@ -316,3 +316,34 @@ def test_expected_m_does_not_change_results():
     a = out1.reshape(-1, p.N)[torch.from_numpy(valid).cuda()]
     b = out2.reshape(-1, p.N)[torch.from_numpy(valid).cuda()]
     assert_close(bf16_to_f64(a), bf16_to_f64(b), "expected_m")
+
+
+def test_contiguous_many_groups_takes_the_single_cta_path():
+    """3000 one-block groups: more 128-row blocks than the pair window table holds (2048), so the call falls back
+    to single-CTA tiles; group ids above 2^11 exercise the tile list's group field.  Sampled rows vs the oracle."""
+    import moe_grouped_gemm_03_b200 as dg
+
+    rng = np.random.default_rng(41)
+    counts = rng.integers(1, 129, size=3000)
+    p = synth.make_contiguous(counts, 32, 128, seed=41)
+    out = run_problem(p)
+    dg.check_device_error()
+    valid = p.valid_rows()
+    rows = np.unique(np.concatenate([valid[:200], valid[-200:], rng.choice(valid, 400, replace=False)]))
+    ref = oracle.problem_rows(p, rows)
+    assert_close(bf16_to_f64(out[torch.from_numpy(rows).cuda()]), ref, "3000 groups")
+    mask = np.zeros(p.rows, bool)
+    mask[valid] = True
+    assert untouched_rows_ok(out, mask)
+
+
+def test_masked_and_nopad_at_the_group_limit(policy):
+    """1024 groups, the most the masked and no-padding calls accept."""
+    import moe_grouped_gemm_03_b200 as dg
+
+    rng = np.random.default_rng(42)
+    mm = rng.integers(0, 65, size=1024)
+    _full_check(synth.make_masked(1024, 64, 128, 128, masked_m=mm, seed=42, expected_m=32))
+    q = synth.make_nopad(rng.integers(0, 40, size=1024), 128, 128, seed=43, extra_rows=7)
+    _full_check(q)
+    dg.check_device_error()
