@@ -396,9 +396,9 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
         static const bool debug = getenv("DG_DEBUG") && getenv("DG_DEBUG")[0] == '1';
         if (debug)
             fprintf(stderr, "[dg] mode=%d M=%d N=%d K=%d G=%d BN=%d stages=%d x %d ctas=%d grid=%u smem=%d windows=%d"
-                            " scratch=%lld B\n",
+                            " raster=%d scratch=%lld B\n",
                     p.mode, p.M, p.N, p.K, p.G, BN, C::STAGES, KPS, CTAS, cfg.gridDim.x, C::SMEM_BYTES, p.num_windows,
-                    (pk.sfa_words + pk.sfb_words) * 4);
+                    p.raster_bands, (pk.sfa_words + pk.sfb_words) * 4);
         apply_wait_settings(p);
         if ((rc = launch_pack(pk, device, stream))) break;
         if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, tsfb, td, p)) != cudaSuccess) {
@@ -468,6 +468,21 @@ int select_block_n(long long windows, int N, int units, int ctas) {
     return best;
 }
 
+// Tile order of the dense and K-grouped layouts: raster groups of this many row windows, swept down the windows
+// first.  The CTAs running at one time then share a few B column blocks, and the group's A rows (at most about
+// kRasterBytes, so they stay in the 126 MB L2 beside the B blocks in flight and the D tiles written back) serve
+// every column block of the group.  On the dense 4096 x 7168 x 7168 GEMM this order measured 2.7% faster than
+// sweeping the columns first, which re-streams all of B every ~2 windows.
+constexpr long long kRasterBytes = 40ll << 20;
+int raster_bands(const dg::GemmParams &p, int ctas) {
+    const long long windows = p.mode == dg::MODE_KGROUPED ? p.num_windows / p.G : p.num_windows;
+    const long long k = p.mode == dg::MODE_KGROUPED ? p.K / p.G : p.K;  // a group's mean K extent
+    const long long window_bytes = static_cast<long long>(dg::BLOCK_M) * ctas * (k > 0 ? k : 1);
+    long long bands = kRasterBytes / window_bytes;
+    if (bands > windows) bands = windows;
+    return static_cast<int>(bands < 1 ? 1 : bands);
+}
+
 // Shape and launch: picks single CTAs or CTA pairs, the tile width, and the persistent grid.
 //   sel1 / sel2:     128-row / 256-row windows the tile shape is chosen for (a hint for the masked layout)
 //   bound1 / bound2: the most 128-row / 256-row tiles the device may find (sizes the grid)
@@ -496,6 +511,8 @@ int plan_and_launch(dg::GemmParams p, const DeviceInfo &info, const Plan &plan, 
     p.num_windows = static_cast<int>(device_windows ? 0 : (pair ? plan.windows2 : plan.windows1));
     if (p.num_sf_groups == 0)  // (the K-grouped call counts its groups' scale groups itself)
         p.num_sf_groups = (p.K / dg::BLOCK_K + dg::SF_GROUP - 1) / dg::SF_GROUP;
+    if (p.mode == dg::MODE_DENSE || p.mode == dg::MODE_KGROUPED)
+        p.raster_bands = raster_bands(p, pair ? 2 : 1);
     const long long tiles = (pair ? plan.bound2 : plan.bound1) * p.num_n_blocks;
     const int grid = static_cast<int>(tiles < units ? tiles : units);
     if (grid <= 0) return DG_OK;

@@ -85,6 +85,7 @@ struct GemmParams {
     int num_n_blocks;  // ceil(N / BN)
     int num_sf_groups; // ceil(K / (128 * SF_GROUP)); K-grouped: the sum over groups of ceil(K_g / (128 * SF_GROUP))
     int sfa_blocks;    // 128-row blocks per group of the packed SFA (masked layout)
+    int raster_bands;  // dense / K-grouped: row windows per raster group (the tile order); 0: columns first
     __nv_bfloat16 *d;
     float *d32;        // fp32 output (out_mode != OUT_BF16): [G][M][N]
     const int *m_indices;
@@ -232,22 +233,46 @@ __device__ __forceinline__ int upper_index(const int *table, int n, int v) {
     return lo;
 }
 
+// Order of the tiles of a grid of `windows` row windows x `nblocks` column blocks: tile t -> (window, *nb).
+// The windows are cut into raster groups of `bands` consecutive windows; inside a group the tiles walk down
+// the windows first, then across the columns, so the CTAs running at one time share a few B column blocks
+// and the group's A rows, which stay in L2 while the group's columns are swept.  bands <= 0: columns first.
+__device__ __forceinline__ int raster_tile(int t, int windows, int nblocks, int bands, int &nb) {
+    if (bands <= 0) {
+        const int w = t / nblocks;
+        nb = t - w * nblocks;
+        return w;
+    }
+    const int span = bands * nblocks;  // tiles of one full raster group
+    const int grp = t / span;
+    const int w0 = grp * bands;
+    const int gm = min(bands, windows - w0);  // the last group may be narrower
+    const int local = t - grp * span;
+    nb = local / gm;
+    return w0 + (local - nb * gm);
+}
+
 template <class C>
 __device__ __forceinline__ bool decode_tile(const GemmParams &p, const SharedCtl &ctl, int t, Tile &ti) {
-    const int w = t / p.num_n_blocks;  // window-tile index
-    ti.nb = t - w * p.num_n_blocks;
-    ti.n0 = ti.nb * C::BN;
     if (p.mode == MODE_DENSE) {
+        const int w = raster_tile(t, p.num_windows, p.num_n_blocks, p.raster_bands, ti.nb);
+        ti.n0 = ti.nb * C::BN;
         ti.g = 0;
         ti.row0 = ti.local_row0 = w * C::TILE_M;
         return true;
     }
-    if (p.mode == MODE_KGROUPED) {  // every group covers all M rows; windows of a group are consecutive
+    if (p.mode == MODE_KGROUPED) {  // every group covers all M rows; a group's tiles are consecutive
         const int per_group = p.num_windows / p.G;
-        ti.g = w / per_group;
-        ti.row0 = ti.local_row0 = (w - ti.g * per_group) * C::TILE_M;
+        const int group_tiles = per_group * p.num_n_blocks;
+        ti.g = t / group_tiles;
+        const int w = raster_tile(t - ti.g * group_tiles, per_group, p.num_n_blocks, p.raster_bands, ti.nb);
+        ti.n0 = ti.nb * C::BN;
+        ti.row0 = ti.local_row0 = w * C::TILE_M;
         return true;
     }
+    const int w = t / p.num_n_blocks;  // window-tile index
+    ti.nb = t - w * p.num_n_blocks;
+    ti.n0 = ti.nb * C::BN;
     if (p.mode == MODE_CONTIGUOUS) {
         if constexpr (C::CTAS == 1) {
             ti.row0 = ti.local_row0 = w * BLOCK_M;
