@@ -386,6 +386,17 @@ def make_masked(G: int, M_max: int, N: int, K: int, masked_m: Optional[Sequence[
                    expected_m=expected_m or M_max, name=name or f"masked G={G} M_max={M_max} N={N} K={K}")
 
 
+def with_fp32_scales(p: Problem, seed: int = 0) -> Problem:
+    """The same problem with every A and B scale multiplied by its own seeded factor drawn uniformly from [1, 2)
+    (fp32): scales that are no longer powers of two (each 128-K block and 128x128 block gets its own mantissa).
+    The e4m3 codes are unchanged.  Input for the fp32 scale-promotion path."""
+    rng = np.random.default_rng(seed + 0x5CA1E)
+    p.sfa = (p.sfa * rng.uniform(1.0, 2.0, size=p.sfa.shape)).astype(np.float32)
+    p.sfb = (p.sfb * rng.uniform(1.0, 2.0, size=p.sfb.shape)).astype(np.float32)
+    p.name = p.name + " (fp32 scales)"
+    return p
+
+
 def zipf_counts(total: int, G: int, s: float) -> np.ndarray:
     """Deterministic Zipf(s) split of ``total`` tokens over G groups: w_g = (g+1)^-s, floor(total * w / sum w)
     plus largest-remainder rounding so that the counts sum to ``total`` (ties go to the lower group id)."""

@@ -68,6 +68,33 @@ def test_bruteforce_integer_operands(M, N, K):
     np.testing.assert_array_equal(got, exact.astype(np.float64))
 
 
+def test_fp32_scales_against_exact_rational_arithmetic():
+    """Arbitrary fp32 scales (no powers of two) on integer-valued operands: the oracle's fp64 result equals the
+    exact rational value of sum_kb sfa * sfb * (integer dot product), computed with fractions.Fraction, to
+    within fp64 rounding of the sum."""
+    from fractions import Fraction
+
+    rng = np.random.default_rng(11)
+    M, N, K = 3, 130, 384  # two 128-column scale blocks (the second ragged), three K blocks
+    nkb, nnb = K // 128, 2
+    ia = rng.integers(-8, 9, size=(M, K))
+    ib = rng.integers(-8, 9, size=(N, K))
+    a = _codes_for_values(ia.astype(np.float32))
+    b = _codes_for_values(ib.astype(np.float32))
+    sfa = rng.uniform(0.01, 3.0, size=(nkb, synth.tma_aligned_rows(M))).astype(np.float32)
+    sfb = rng.uniform(0.01, 3.0, size=(nnb, nkb)).astype(np.float32)
+    got = oracle.fp8_gemm_nt(a, sfa, b, sfb)
+    for m in range(M):
+        for n in range(N):
+            exact, mag = Fraction(0), 0.0
+            for kb in range(nkb):
+                dot = int(ia[m, 128 * kb:128 * (kb + 1)] @ ib[n, 128 * kb:128 * (kb + 1)])
+                term = Fraction(float(sfa[kb, m])) * Fraction(float(sfb[n // 128, kb])) * dot
+                exact += term
+                mag += abs(float(term))
+            assert abs(got[m, n] - float(exact)) <= 1e-15 * (mag + 1.0), (m, n)
+
+
 def _random_finite_codes(rng, shape):
     c = rng.integers(0, 256, size=shape, dtype=np.uint8)
     return np.where((c & 0x7F) == 0x7F, c ^ 0x01, c).astype(np.uint8)
@@ -83,8 +110,10 @@ def test_unit_scales_reduce_to_numpy_matmul():
     np.testing.assert_allclose(got, ref, rtol=1e-13, atol=0)
 
 
-def test_blockwise_definition_equals_dequantise_then_matmul():
-    """With arbitrary power-of-two scales the blockwise sum equals the matmul of the dequantised operands."""
+@pytest.mark.parametrize("scales", ["pow2", "fp32"])
+def test_blockwise_definition_equals_dequantise_then_matmul(scales):
+    """With arbitrary power-of-two (or arbitrary fp32) scales the blockwise sum equals the matmul of the
+    dequantised operands."""
     rng = np.random.default_rng(2)
     M, N, K = 19, 300, 512  # N not a multiple of 128: ragged last scale block
     nkb = K // 128
@@ -92,11 +121,17 @@ def test_blockwise_definition_equals_dequantise_then_matmul():
     b = _random_finite_codes(rng, (N, K))
     sfa = np.ldexp(1.0, rng.integers(-6, 7, size=(nkb, 20))).astype(np.float32)
     sfb = np.ldexp(1.0, rng.integers(-6, 7, size=(3, nkb))).astype(np.float32)
+    if scales == "fp32":
+        sfa = (sfa * rng.uniform(1, 2, size=sfa.shape)).astype(np.float32)
+        sfb = (sfb * rng.uniform(1, 2, size=sfb.shape)).astype(np.float32)
     got = oracle.fp8_gemm_nt(a, sfa, b, sfb)
     A = torch_decode(a) * np.repeat(sfa[:, :M].T, 128, axis=1)
     sb_full = np.repeat(np.repeat(sfb, 128, axis=0)[:N], 128, axis=1)
     B = torch_decode(b) * sb_full
-    np.testing.assert_allclose(got, A @ B.T, rtol=1e-12, atol=1e-9)
+    # fp64 rounding of the two summation orders, bounded by the sum of the products' magnitudes (with fp32 scales a
+    # dequantised product carries up to 56 significant bits, so cancelling sums differ by more than 1e-12 relative)
+    mag = np.abs(A) @ np.abs(B).T
+    assert (np.abs(got - A @ B.T) <= 1e-13 * mag + 1e-12).all()
 
 
 def test_dropped_or_misindexed_scale_is_detected():

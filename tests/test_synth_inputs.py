@@ -103,3 +103,16 @@ def test_seeded_determinism():
     a = synth.make_dense(16, 128, 256, seed=3)
     b = synth.make_dense(16, 128, 256, seed=3)
     assert np.array_equal(a.a, b.a) and np.array_equal(a.b, b.b) and np.array_equal(a.sfa, b.sfa)
+
+
+def test_with_fp32_scales_gives_each_block_its_own_mantissa():
+    base = synth.make_contiguous([130, 0, 257], 272, 384, seed=5)
+    p = synth.with_fp32_scales(synth.make_contiguous([130, 0, 257], 272, 384, seed=5), seed=5)
+    again = synth.with_fp32_scales(synth.make_contiguous([130, 0, 257], 272, 384, seed=5), seed=5)
+    assert np.array_equal(p.a, base.a) and np.array_equal(p.b, base.b)  # codes unchanged
+    for new, old in ((p.sfa, base.sfa), (p.sfb, base.sfb)):
+        ratio = new.astype(np.float64) / old
+        assert ((ratio >= 1.0) & (ratio < 2.0)).all()
+        mantissa = new.view(np.uint32) & 0x7FFFFF
+        assert (mantissa != 0).mean() > 0.99  # (almost) no power of two left
+    assert np.array_equal(p.sfa, again.sfa) and np.array_equal(p.sfb, again.sfb)  # seeded
