@@ -14,12 +14,18 @@
  *   sfa  fp32, MN-major: [K/128][ld] with ld = dg_get_tma_aligned_size(rows, 4) (rows rounded up to a
  *        multiple of 4 so every K block's column starts on 16 bytes).  Masked layout: [G][K/128][ld(M_max)].
  *   sfb  fp32, [G][ceil(N/128)][K/128] (G = 1 for the dense call).
- * Every scale must be a positive power of two in [2^-127, 2^127] (a UE8M0 value): the tensor cores apply
- * the scales as exponents.  Other values give wrong results; the library does not check them.
+ * Scale values.  By default every scale must be a power of two in [2^-126, 2^127] (a UE8M0 value): the
+ * block-scaled tensor-core MMA applies the scales as exponents.  The scale pre-pass checks every scale the
+ * call reads (the A scales of rows the call owns, all B scales) and reports one with a sign, mantissa bits,
+ * Inf or NaN as DG_ERR_BAD_SCALE through dg_check_device_error(); the results of that call are then wrong.
+ * A zero scale is taken as 2^-127.  After dg_set_fp32_scale_promotion(1) the calls with bf16 output take any
+ * finite fp32 scales: every 128-K block's partial product is multiplied by sfa * sfb and added in fp32 (the
+ * "promotion operations" of the DeepGEMM-for-PPU README, "Optimizations"), at a lower speed.
  *
  * Common conventions
- *   - All array arguments are device pointers owned by the caller.  The library allocates nothing per
- *     call and keeps no reference after the call returns.
+ *   - All array arguments are device pointers owned by the caller.  The library keeps no reference after the
+ *     call returns; its only per-call memory is stream-ordered scratch (packed scales, the NN call's transposed
+ *     B) taken from and returned to a device memory pool on `stream` (dg_fp8_gemm_nt_noalloc takes none).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).  m_indices and
  *     masked_m are read only on the device, so the host never synchronises.
  *   - Arguments are validated before anything is launched; a bad argument returns a negative dg_status,
@@ -29,7 +35,8 @@
  *   - Pointer alignment: a, b, d, sfa, sfb 16-byte aligned; m_indices, masked_m 4-byte aligned.
  *   - Shapes: K % 128 == 0, N % 16 == 0, N, K > 0, all extents below 2^31 elements per dimension.
  *   - Device-side faults are not expected.  Every wait inside the kernel is bounded; a kernel that gives
- *     up records a code that dg_check_device_error() returns (DG_ERR_DEVICE_TIMEOUT or DG_ERR_BAD_GROUP).
+ *     up records a code that dg_check_device_error() returns (DG_ERR_DEVICE_TIMEOUT, DG_ERR_BAD_GROUP or
+ *     DG_ERR_BAD_SCALE).
  */
 #ifndef DG_H_
 #define DG_H_
@@ -53,8 +60,9 @@ typedef enum {
     DG_ERR_UNSUPPORTED = -3,   /* device is not sm_100, or a shape outside the supported set */
     DG_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed */
     DG_ERR_DEVICE_TIMEOUT = -5,/* (device error word) a bounded wait inside the kernel ran out */
-    DG_ERR_BAD_GROUP = -6      /* (device error word) a group id outside [-1, G), masked_m outside [0, M_max],
+    DG_ERR_BAD_GROUP = -6,     /* (device error word) a group id outside [-1, G), masked_m outside [0, M_max],
                                   or no-padding counts that are negative or sum past M_total */
+    DG_ERR_BAD_SCALE = -7      /* (device error word) a scale read by a block-scaled call is not a power of two */
 } dg_status;
 
 /* Per-segment M padding of the contiguous layout: each group's rows start on a multiple of this (128 unless
@@ -188,6 +196,17 @@ DG_EXPORT int dg_m_grouped_fp8_gemm_nt_nopad(const void *a, const float *sfa, co
 DG_EXPORT int dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
                                      int M, int N, int K, dg_stream_t stream);
 
+/* Scale handling for the next calls on any thread ("promotion operations", DeepGEMM-for-PPU README,
+ * "Optimizations"; the wrapper's disable_ue8m0_cast option).  0 (default): scales must be powers of two and are
+ * applied by the block-scaled MMA (kind::mxf8f6f4, UE8M0 scales in tensor memory).  1: any finite fp32 scales;
+ * dg_fp8_gemm_nt, dg_fp8_gemm_nt_noalloc, dg_m_grouped_fp8_gemm_nt_contiguous, _masked, _nopad and
+ * dg_m_grouped_fp8_gemm_nn_contiguous then run plain kind::f8f6f4 MMAs into one tensor-memory buffer per
+ * 128-K block, and the epilogue warps accumulate buffer * sfa(m, kb) * sfb(g, n/128, kb) in fp32 registers
+ * (128-column tiles; the scales are read from the caller's arrays, no scale pre-pass).  While it is on, the
+ * K-grouped and W4A8 calls return DG_ERR_UNSUPPORTED.  Returns the setting now in force. */
+DG_EXPORT int dg_set_fp32_scale_promotion(int enable);
+DG_EXPORT int dg_get_fp32_scale_promotion(void);
+
 /* Tile-shape policy for the next calls on any thread: -1 (default) lets the library choose between one
  * CTA per 128-row tile and CTA pairs (2-CTA clusters, tcgen05 cta_group::2) computing 256-row tiles;
  * 0 forces single CTAs; 1 uses pairs wherever the layout allows.  Results agree within the tolerance of
@@ -211,7 +230,8 @@ DG_EXPORT int dg_debug_bounded_wait(unsigned long long limit_ns, int drop_first_
 DG_EXPORT const char *dg_last_error(void);
 
 /* Synchronises `stream`, then returns and clears the device error word of the current device:
- * DG_OK, DG_ERR_DEVICE_TIMEOUT or DG_ERR_BAD_GROUP (DG_ERR_CUDA if the synchronisation failed). */
+ * DG_OK, DG_ERR_DEVICE_TIMEOUT, DG_ERR_BAD_GROUP or DG_ERR_BAD_SCALE (DG_ERR_CUDA if the synchronisation
+ * failed).  The first error recorded since the last check wins. */
 DG_EXPORT int dg_check_device_error(dg_stream_t stream);
 
 #ifdef __cplusplus

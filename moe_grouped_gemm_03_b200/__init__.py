@@ -8,7 +8,8 @@ kernels; there is no fallback of any kind.
 Operands follow the NT convention of the DeepGEMM family ("Interfaces / Notices" of the DeepGEMM-for-PPU
 README): ``lhs = (a, sfa)`` with ``a`` [M, K] e4m3 and ``sfa`` fp32 [K/128, tma_aligned(M)] (MN-major, one
 scale per row and 128-K block); ``rhs = (b, sfb)`` with ``b`` [N, K] e4m3 (grouped: [G, N, K]) and ``sfb``
-fp32 [ceil(N/128), K/128] (grouped: [G, ...]), one scale per 128x128 block.  Scales must be powers of two.
+fp32 [ceil(N/128), K/128] (grouped: [G, ...]), one scale per 128x128 block.  Scales must be powers of two
+unless ``set_fp32_scale_promotion(True)`` is in force (any finite fp32 scales, promoted per 128-K block).
 """
 from __future__ import annotations
 
@@ -25,7 +26,8 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "dg.h")
 
 DG_OK = 0
 STATUS_NAMES = {0: "DG_OK", -1: "DG_ERR_INVALID_ARG", -2: "DG_ERR_ALIGNMENT", -3: "DG_ERR_UNSUPPORTED",
-                -4: "DG_ERR_CUDA", -5: "DG_ERR_DEVICE_TIMEOUT", -6: "DG_ERR_BAD_GROUP"}
+                -4: "DG_ERR_CUDA", -5: "DG_ERR_DEVICE_TIMEOUT", -6: "DG_ERR_BAD_GROUP",
+                -7: "DG_ERR_BAD_SCALE"}
 
 
 class DGError(RuntimeError):
@@ -61,6 +63,8 @@ _SIGNATURES = {
     "dg_k_grouped_fp8_gemm_nt_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_set_cta_pair_policy": (_I, [_I]),
+    "dg_set_fp32_scale_promotion": (_I, [_I]),
+    "dg_get_fp32_scale_promotion": (_I, []),
     "dg_debug_bounded_wait": (_I, [ctypes.c_ulonglong, _I]),
     "dg_last_error": (ctypes.c_char_p, []),
     "dg_check_device_error": (_I, [_P]),
@@ -154,6 +158,17 @@ def select_block_n(num_m_blocks: int, N: int, num_sms: int) -> int:
 def set_cta_pair_policy(policy: int) -> int:
     """-1: library decides; 0: single-CTA 128-row tiles only; 1: 2-CTA 256-row tiles wherever possible."""
     return _lib.dg_set_cta_pair_policy(policy)
+
+
+def set_fp32_scale_promotion(enable: bool) -> bool:
+    """False (default): scales must be powers of two (applied as UE8M0 exponents by the block-scaled MMA; others
+    are reported as DG_ERR_BAD_SCALE by check_device_error).  True: any finite fp32 scales, applied by fp32
+    promotion of every 128-K block's partial product (the bf16-output calls; K-grouped and W4A8 refuse)."""
+    return bool(_lib.dg_set_fp32_scale_promotion(1 if enable else 0))
+
+
+def get_fp32_scale_promotion() -> bool:
+    return bool(_lib.dg_get_fp32_scale_promotion())
 
 
 def debug_bounded_wait(limit_ns: int = 0, drop_first_stage: bool = False) -> None:

@@ -232,6 +232,7 @@ namespace {
 // ----------------------------------------------------------------------------------------------- launch
 int g_m_alignment = dg::BLOCK_M;  // contiguous layout: per-segment M padding (128 or 256)
 int g_pair_policy = -1;  // -1: library decides; 0: single CTAs only; 1: CTA pairs whenever supported
+bool g_fp32_promotion = false;  // true: any fp32 scales, applied by promotion; false: power-of-two scales (UE8M0)
 unsigned long long g_wait_limit_ns = dg::WAIT_LIMIT_NS;  // limit of every in-kernel wait
 bool g_drop_first_stage = false;  // testing aid: the next GEMM launch leaves one stage unloaded
 
@@ -297,6 +298,8 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
     }
     pk.mode = p.mode;
     pk.counts = p.masked_m;
+    pk.m_indices = p.m_indices;
+    pk.err = p.err;
     pk.tile_m = C::TILE_M;
     if (p.mode == dg::MODE_MASKED) {
         pk.rows_per_group = p.M;
@@ -413,6 +416,71 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
     return rc;
 }
 
+// The fp32 scale-promotion GEMM (any finite fp32 scales): 128-wide tiles, plain kind::f8f6f4 MMAs, the epilogue
+// warps read the caller's scales directly, so there is no pre-pass and no scratch.  The launch is an ordinary
+// stream-ordered one (the kernel's first loads may not run ahead of the previous kernel on the stream).
+template <int CTAS>
+int launch_promo(const void *a, long long a_rows, const void *b, long long b_rows, const ScaleArgs &sc,
+                 dg::GemmParams p, int grid, int device, cudaStream_t stream) {
+    using C = dg::Cfg<128, CTAS, CTAS == 2 ? 2 : 1, false, true>;  // (a single CTA fits more stages of one K block)
+    const int nkb = p.K / dg::BLOCK_K;
+    const int nnb = (p.N + 127) / 128;
+    p.sfa32 = sc.sfa;
+    p.sfa_ld = sc.sfa_ld;
+    p.sfb32 = sc.sfb;
+    p.sfb_sg = nkb * nnb;
+    p.sfb_sn = sc.sfb_kn ? 1 : nkb;  // NN: [G][K/128][ceil(N/128)]; NT: [G][ceil(N/128)][K/128]
+    p.sfb_sk = sc.sfb_kn ? nnb : 1;
+    CUtensorMap ta, tb, td;
+    int rc;
+    if ((rc = make_output_map(td, p.d, a_rows, p.N))) return rc;
+    if ((rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M))) return rc;
+    if ((rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS))) return rc;
+    auto kernel = dg::fp8_gemm_kernel<C>;
+    cudaError_t e;
+    static bool smem_set[64] = {false};
+    if (!(device >= 0 && device < 64 && smem_set[device])) {
+        if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) !=
+            cudaSuccess)
+            return cuda_fail(e, "cudaFuncSetAttribute");
+        if (device >= 0 && device < 64) smem_set[device] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid * CTAS), 1, 1);
+    cfg.blockDim = dim3(dg::NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CTAS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (CTAS > 1) {
+        static int max_clusters[64] = {0};
+        int &cached = max_clusters[device & 63];
+        if (cached == 0) {
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+                cudaGetLastError();
+                n = grid;
+            }
+            cached = n;
+        }
+        if (grid > cached) cfg.gridDim.x = static_cast<unsigned>(cached * CTAS);
+    }
+    static const bool debug = getenv("DG_DEBUG") && getenv("DG_DEBUG")[0] == '1';
+    if (debug)
+        fprintf(stderr, "[dg] fp32 promotion: mode=%d M=%d N=%d K=%d G=%d BN=128 stages=%d x %d ctas=%d grid=%u smem=%d\n",
+                p.mode, p.M, p.N, p.K, p.G, C::STAGES, C::KPS, CTAS, cfg.gridDim.x, C::SMEM_BYTES);
+    apply_wait_settings(p);
+    // the kernel takes five maps; the two scale-atom maps are unused on this path
+    if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, ta, ta, td, p)) != cudaSuccess)
+        return cuda_fail(e, "kernel launch");
+    return DG_OK;
+}
+
 // Tile widths the library is built with, and the pipeline depth each fits in 227 KB of shared memory and
 // 512 TMEM columns (two BN-wide accumulators plus one scale slot per stage).
 constexpr int kCandidateBN[] = {224, 192, 160, 128};
@@ -503,6 +571,21 @@ int plan_and_launch(dg::GemmParams p, const DeviceInfo &info, const Plan &plan, 
         pair = plan.sel2 * ((p.N + bn - 1) / bn) >= sms / 2;
     }
     const int units = pair ? sms / 2 : sms;
+    if (g_fp32_promotion) {
+        if (sc.sfb_fp4 || p.mode == dg::MODE_KGROUPED || p.out_mode != dg::OUT_BF16)
+            return fail(DG_ERR_UNSUPPORTED,
+                        "fp32 scale promotion covers the bf16-output FP8 calls (dense, contiguous, masked, no-padding, "
+                        "NN); switch it off for the K-grouped and W4A8 calls");
+        p.num_n_blocks = (p.N + 127) / 128;
+        const bool device_windows = p.mode == dg::MODE_MASKED || p.mode == dg::MODE_NOPAD;
+        p.num_windows = static_cast<int>(device_windows ? 0 : (pair ? plan.windows2 : plan.windows1));
+        if (p.mode == dg::MODE_DENSE) p.raster_bands = raster_bands(p, pair ? 2 : 1);
+        const long long tiles = (pair ? plan.bound2 : plan.bound1) * p.num_n_blocks;
+        const int grid = static_cast<int>(tiles < units ? tiles : units);
+        if (grid <= 0) return DG_OK;
+        if (pair) return launch_promo<2>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
+        return launch_promo<1>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
+    }
     int bn = select_block_n(pair ? plan.sel2 : plan.sel1, p.N, units, pair ? 2 : 1);
     static const int forced_bn = getenv("DG_BLOCK_N") ? atoi(getenv("DG_BLOCK_N")) : 0;  // tuning override
     if (forced_bn > 0) bn = forced_bn;
@@ -701,6 +784,10 @@ int dg_check_device_error(dg_stream_t stream) {
     if (word == dg::ERR_TIMEOUT) return fail(DG_ERR_DEVICE_TIMEOUT, "a bounded wait inside the kernel ran out");
     if (word == dg::ERR_BAD_GROUP)
         return fail(DG_ERR_BAD_GROUP, "a group id or masked_m value was out of range; those rows were skipped");
+    if (word == dg::ERR_BAD_SCALE)
+        return fail(DG_ERR_BAD_SCALE,
+                    "a scale was not a power of two; the block-scaled path applies only the exponent "
+                    "(dg_set_fp32_scale_promotion(1) takes any fp32 scales)");
     if (word != 0) return fail(DG_ERR_CUDA, "unknown device error word %u", word);
     return DG_OK;
 }
@@ -861,6 +948,13 @@ int dg_k_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const v
     const Plan plan{w1, w2, w1, w2, w1, w2, true};
     return plan_and_launch(p, info, plan, a, M, b, N, sc, s);
 }
+
+int dg_set_fp32_scale_promotion(int enable) {
+    g_fp32_promotion = enable != 0;
+    return g_fp32_promotion ? 1 : 0;
+}
+
+int dg_get_fp32_scale_promotion(void) { return g_fp32_promotion ? 1 : 0; }
 
 int dg_set_cta_pair_policy(int policy) {
     g_pair_policy = policy < 0 ? -1 : (policy > 0 ? 1 : 0);

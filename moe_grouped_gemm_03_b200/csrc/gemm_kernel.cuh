@@ -74,6 +74,7 @@ constexpr int SMEM_LIMIT = 232448;                  // 227 KB of dynamic shared 
 // device error word codes
 constexpr unsigned ERR_TIMEOUT = 1u;
 constexpr unsigned ERR_BAD_GROUP = 2u;
+constexpr unsigned ERR_BAD_SCALE = 3u;  // a scale the block-scaled MMA cannot represent (not a power of two)
 
 struct GemmParams {
     int mode;
@@ -93,9 +94,14 @@ struct GemmParams {
     unsigned *err;
     unsigned long long wait_limit_ns;  // limit of any single wait
     int skip_first_load;               // test hook: the first CTA (pair) never loads stage 0
+    // fp32 scale promotion (Cfg::PROMO): the caller's scales, read by the epilogue warps
+    const float *sfa32;  // MN-major [K/128][sfa_ld] (masked: [G][K/128][sfa_ld])
+    const float *sfb32;  // scale of (group g, 128-column block nb, K block kb) at g * sfb_sg + nb * sfb_sn + kb * sfb_sk
+    int sfa_ld;
+    int sfb_sg, sfb_sn, sfb_sk;
 };
 
-template <int BN_, int CTAS_, int KPS_, bool BF4_ = false>
+template <int BN_, int CTAS_, int KPS_, bool BF4_ = false, bool PROMO_ = false>
 struct Cfg {
     static constexpr int BN = BN_;
     static constexpr int CTAS = CTAS_;
@@ -104,6 +110,11 @@ struct Cfg {
     // one scale per (row, 32-K block), i.e. one 4-byte scale word per row per 128-K block, so a stage carries
     // the B scale atoms of each of its K blocks (A's atom still packs SF_GROUP K blocks)
     static constexpr bool BF4 = BF4_;
+    // fp32 scale promotion: plain kind::f8f6f4 MMAs write each 128-K block's partial product to its own TMEM
+    // buffer (two partial stages of KPS blocks, 2 * KPS * BN columns), and the epilogue warps accumulate
+    // partial * sfa * sfb in registers.  No scale atoms travel with the stages.  BN = 128: a tile's columns are
+    // exactly one 128-column block of B's scales.
+    static constexpr bool PROMO = PROMO_;
     static constexpr int SFB_KB = BF4 ? KPS : 1;                  // K blocks whose B scale atoms a stage holds
     static constexpr int TILE_M = BLOCK_M * CTAS;
     static constexpr int B_ROWS = BN / CTAS;                      // B rows this CTA loads
@@ -115,7 +126,7 @@ struct Cfg {
     static constexpr int B_TX1 = BF4_ ? B_ROWS * BLOCK_K / 2 : B_BYTES1;
     static constexpr int A_BYTES = KPS * A_BYTES1;                // per stage
     static constexpr int B_BYTES = KPS * B_BYTES1;
-    static constexpr int SF_BYTES = (1 + SFB_KB * SFB_ATOMS) * SF_ATOM_WORDS * 4;  // SFA atom + SFB atoms
+    static constexpr int SF_BYTES = PROMO ? 0 : (1 + SFB_KB * SFB_ATOMS) * SF_ATOM_WORDS * 4;  // SFA + SFB atoms
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SF_BYTES;
     static constexpr int SF_COLS = 4 + 4 * SFB_KB * SFB_ATOMS;    // TMEM columns of one scale slot
     static constexpr int SF_TMEM_BASE = 2 * BN;                   // after the two accumulators
@@ -143,6 +154,7 @@ struct Cfg {
     static constexpr int OFF_TILES = (OFF_MM + 4 * MAX_MASKED_GROUPS + 15) / 16 * 16;  // uint2[TILE_LIST_CAP]
     static constexpr int SMEM_BYTES = OFF_TILES + 8 * TILE_LIST_CAP + 1024;     // + alignment slack
     static_assert(CTAS == 1 || CTAS == 2, "single CTA or CTA pair");
+    static_assert(!PROMO || (BN == 128 && !BF4 && 2 * KPS * BN <= TMEM_COLS), "promotion: 128-wide tiles, e4m3 B");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32, 256]");
     static_assert(B_ROWS % 8 == 0, "B tile rows must fill whole 8-row swizzle atoms");
     static_assert(STAGES >= 3, "pipeline too shallow");
@@ -617,7 +629,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int sfb_words = C::BF4 ? nkb : p.num_sf_groups;
                 const int sfb_y0 = ((gb * p.num_n_blocks + ti.nb) * sfb_words + qbase) * C::SFB_ATOMS;
                 for (int kb0 = 0; kb0 < tile_nkb; kb0 += C::KPS) {
-                    const bool group_start = C::BF4 || kb0 % SF_GROUP == 0;  // this stage carries scales
+                    // this stage carries scale atoms (the promotion path reads fp32 scales directly)
+                    const bool group_start = !C::PROMO && (C::BF4 || kb0 % SF_GROUP == 0);
                     if (issued == STAGES) wait_for_scales();  // the ring is full: the MMAs need the scales now
                     if (!wait_bounded(&empty[s], ph ^ 1u, s_abort, p.err, p.wait_limit_ns)) { ok = false; break; }
                     uint8_t *a_dst = sA + s * C::A_BYTES;
@@ -677,7 +690,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer (leader CTA)
-        if (lane == 0 && rank == 0) {
+        if (C::PROMO && lane == 0 && rank == 0) {
+            // fp32 scale promotion: each 128-K block's partial product goes to its own TMEM buffer of the current
+            // partial stage (KPS buffers of BN columns); the epilogue warps release a partial stage once they have
+            // read it, so the MMAs run up to two stages ahead of the promotion
+            constexpr uint32_t IDESC_P = idesc_f8f6f4_e4m3(C::TILE_M, BN);
+            int s = 0;
+            uint32_t ph = 0;
+            int pb = 0;  // partial stage
+            uint32_t pb_ph = 0;
+            bool ok = true;
+            for (int k = 0; k < my_tiles && ok; ++k) {
+                Tile ti;
+                if (!tile_at(k, ti)) continue;
+                for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
+                    const int nk = min(C::KPS, nkb - kb0);
+                    if (!wait_bounded(&full[s], ph, s_abort, p.err, p.wait_limit_ns)) { ok = false; break; }
+                    if (!wait_bounded(&tmem_empty[pb], pb_ph ^ 1u, s_abort, p.err, p.wait_limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_stage = smem_u32(sA + s * C::A_BYTES);
+                    const uint32_t b_stage = smem_u32(sB + s * C::B_BYTES);
+                    for (int i = 0; i < nk; ++i) {
+                        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((pb * C::KPS + i) * BN);
+#pragma unroll
+                        for (int kk = 0; kk < BLOCK_K / MMA_K; ++kk)
+                            tc_mma_f8<CTAS>(d_tmem, sdesc_kmajor_sw128(a_stage + i * C::A_BYTES1 + kk * MMA_K),
+                                            sdesc_kmajor_sw128(b_stage + i * C::B_BYTES1 + kk * MMA_K), IDESC_P,
+                                            kk != 0);
+                    }
+                    tc_commit<CTAS>(&empty[s]);
+                    tc_commit<CTAS>(&tmem_full[pb]);
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                    pb ^= 1;
+                    if (pb == 0) pb_ph ^= 1u;
+                }
+            }
+            tc_commit<CTAS>(drain);
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < p.wait_limit_ns) {
+            }
+        } else if (!C::PROMO && lane == 0 && rank == 0) {
             constexpr uint32_t IDESC = idesc_mxf8_e4m3(C::TILE_M, BN, C::BF4);
             int s = 0;
             uint32_t ph = 0;
@@ -756,9 +811,141 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int acc = 0;
         uint32_t acc_ph = 0;
         int chunk_count = 0;  // chunks this warp has staged (selects the staging buffer)
-        for (int k = 0; k < my_tiles; ++k) {
+        // Does this lane's row of the tile belong to the call (the rows D may be written at)?
+        auto row_owned = [&](const Tile &ti, int row, int r_local) -> bool {
+            if (p.mode == MODE_DENSE) return row < p.M;
+            if (p.mode == MODE_CONTIGUOUS) return row < p.M && __ldg(p.m_indices + row) == ti.g;
+            return ti.local_row0 + r_local < ctl.mm[ti.g];
+        };
+        // One 32-column bf16 chunk of this lane's row (h: 16 packed pairs): staged and written by one TMA tensor
+        // store when all 32 rows of the warp belong to the call (tma_ok), else stored by the owning lanes.
+        auto emit_bf16 = [&](const Tile &ti, int row, int c, const uint32_t(&h)[16], bool tma_ok, bool valid) {
+            if (tma_ok) {
+                uint8_t *buf = stage_buf + (chunk_count & 1) * EPI_CHUNK_BYTES;
+                if (chunk_count >= 2) {
+                    if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
+                    __syncwarp();
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int sw = j ^ ((lane >> 1) & 3);
+                    *reinterpret_cast<uint4 *>(buf + lane * 64 + sw * 16) =
+                        make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmap_d, buf, ti.n0 + 32 * c, ti.row0 + my_rows + 32 * q);
+                    bulk_commit_group();
+                }
+                ++chunk_count;
+            } else if (valid) {
+                __nv_bfloat16 *out = p.d + static_cast<size_t>(row) * p.N + ti.n0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int col = ti.n0 + 32 * c + 8 * j;
+                    if (col < p.N)
+                        *reinterpret_cast<uint4 *>(out + 32 * c + 8 * j) =
+                            make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+                }
+            }
+        };
+        int pb = 0;  // promotion: the partial stage read next
+        uint32_t pb_ph = 0;
+        // fp32 scale promotion of one tile: this lane's row accumulates partial(kb) * sfa[row, kb] * sfb[g, nb, kb]
+        // over the K blocks in registers (BN = 128 columns: one 128-column block of B's scales), then it is
+        // written as bf16.  The scales are read from the caller's arrays one partial stage ahead.  false = gave up.
+        auto promote_tile = [&](const Tile &ti) -> bool {
+            const int r_local = my_rows + 32 * q + lane;
+            const int row = ti.row0 + r_local;
+            bool row_in;          // the row exists in the A scale array (rows past it read no scale)
+            long long sa_base;    // element of (row, K block 0); K block kb at sa_base + kb * sfa_ld
+            if (p.mode == MODE_MASKED) {
+                const int lrow = ti.local_row0 + r_local;
+                row_in = lrow < p.M;
+                sa_base = static_cast<long long>(ti.g) * nkb * p.sfa_ld + lrow;
+            } else {
+                row_in = row < p.M;
+                sa_base = row;
+            }
+            const float *sfb_t = p.sfb32 + static_cast<long long>(ti.g) * p.sfb_sg +
+                                 static_cast<long long>(ti.n0 / 128) * p.sfb_sn;
+            float acc_r[BN];
+#pragma unroll
+            for (int j = 0; j < BN; ++j) acc_r[j] = 0.f;
+            float sa_n[C::KPS], sb_n[C::KPS];
+            auto load_scales = [&](int kb0) {
+#pragma unroll
+                for (int i = 0; i < C::KPS; ++i) {
+                    const int kb = kb0 + i;
+                    const bool in = kb < nkb;
+                    sa_n[i] = (in && row_in) ? __ldg(p.sfa32 + sa_base + static_cast<long long>(kb) * p.sfa_ld) : 0.f;
+                    sb_n[i] = in ? __ldg(sfb_t + static_cast<long long>(kb) * p.sfb_sk) : 0.f;
+                }
+            };
+            load_scales(0);
+            for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
+                const int nk = min(C::KPS, nkb - kb0);
+                float sc[C::KPS];
+#pragma unroll
+                for (int i = 0; i < C::KPS; ++i) sc[i] = sa_n[i] * sb_n[i];
+                if (kb0 + C::KPS < nkb) load_scales(kb0 + C::KPS);
+                if (!warp_wait_bounded(&tmem_full[pb], pb_ph, s_abort, p.err, p.wait_limit_ns, lane)) return false;
+                tc_fence_after_sync();
+                const uint32_t t_part =
+                    tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(pb * C::KPS * BN);
+#pragma unroll
+                for (int i = 0; i < C::KPS; ++i) {
+                    if (i < nk) {
+#pragma unroll
+                        for (int c = 0; c < BN / 32; c += 2) {
+                            uint32_t r0[32], r1[32];
+                            tmem_ld_32x32b_x32(t_part + static_cast<uint32_t>(i * BN + 32 * c), r0);
+                            tmem_ld_32x32b_x32(t_part + static_cast<uint32_t>(i * BN + 32 * c + 32), r1);
+                            tmem_ld_wait_regs(r0);
+                            tmem_ld_wait_regs(r1);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                acc_r[32 * c + j] = fmaf(__uint_as_float(r0[j]), sc[i], acc_r[32 * c + j]);
+                                acc_r[32 * c + 32 + j] = fmaf(__uint_as_float(r1[j]), sc[i], acc_r[32 * c + 32 + j]);
+                            }
+                        }
+                    }
+                }
+                // the partial stage has been read: the MMAs may overwrite it
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (PAIR)
+                        mbar_arrive_cluster(tmem_empty_leader0 + 8u * static_cast<uint32_t>(pb));
+                    else
+                        mbar_arrive(&tmem_empty[pb]);
+                }
+                pb ^= 1;
+                if (pb == 0) pb_ph ^= 1u;
+            }
+            const bool valid = row_owned(ti, row, r_local);
+            const bool tma_ok = p.mode == MODE_DENSE || __all_sync(0xffffffffu, valid);
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t h[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    __nv_bfloat162 v = __floats2bfloat162_rn(acc_r[32 * c + 2 * j], acc_r[32 * c + 2 * j + 1]);
+                    h[j] = *reinterpret_cast<uint32_t *>(&v);
+                }
+                emit_bf16(ti, row, c, h, tma_ok, valid);
+            }
+            return true;
+        };
+        bool promo_ok = true;
+        for (int k = 0; k < my_tiles && promo_ok; ++k) {
             Tile ti;
             if (!tile_at(k, ti)) continue;
+            if constexpr (C::PROMO) {
+                promo_ok = promote_tile(ti);
+                continue;
+            }
             if (!warp_wait_bounded(&tmem_full[acc], acc_ph, s_abort, p.err, p.wait_limit_ns, lane)) break;
             tc_fence_after_sync();
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * BN);
@@ -806,16 +993,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             } else {
                 const int r_local = my_rows + 32 * q + lane;
                 const int row = ti.row0 + r_local;
-                bool valid;
-                if (p.mode == MODE_DENSE)
-                    valid = row < p.M;
-                else if (p.mode == MODE_CONTIGUOUS)
-                    valid = row < p.M && __ldg(p.m_indices + row) == ti.g;
-                else
-                    valid = ti.local_row0 + r_local < ctl.mm[ti.g];
+                const bool valid = row_owned(ti, row, r_local);
                 // dense rows past M lie outside D and are clipped by the store
                 const bool tma_ok = p.mode == MODE_DENSE || __all_sync(0xffffffffu, valid);
-                __nv_bfloat16 *out = p.d + static_cast<size_t>(row) * p.N + ti.n0;
 #pragma unroll 1
                 for (int c = 0; c < BN / 32; ++c) {
                     uint32_t r[32];
@@ -828,34 +1008,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             __floats2bfloat162_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
                         h[j] = *reinterpret_cast<uint32_t *>(&v);
                     }
-                    if (tma_ok) {
-                        uint8_t *buf = stage_buf + (chunk_count & 1) * EPI_CHUNK_BYTES;
-                        if (chunk_count >= 2) {
-                            if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
-                            __syncwarp();
-                        }
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int sw = j ^ ((lane >> 1) & 3);
-                            *reinterpret_cast<uint4 *>(buf + lane * 64 + sw * 16) =
-                                make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d(&tmap_d, buf, ti.n0 + 32 * c, ti.row0 + my_rows + 32 * q);
-                            bulk_commit_group();
-                        }
-                        ++chunk_count;
-                    } else if (valid) {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int col = ti.n0 + 32 * c + 8 * j;
-                            if (col < p.N)
-                                *reinterpret_cast<uint4 *>(out + 32 * c + 8 * j) =
-                                    make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
-                        }
-                    }
+                    emit_bf16(ti, row, c, h, tma_ok, valid);
                 }
             }
             tc_fence_before_sync();

@@ -276,6 +276,27 @@ __device__ __forceinline__ void tc_mma_mxf8(uint32_t d_tmem, uint64_t a_desc, ui
             : "memory");
 }
 
+// D (+)= A * B with e4m3 operands and no scale factors (kind::f8f6f4): one 128-K block's partial product for
+// the fp32 scale-promotion path.
+template <int CTAS>
+__device__ __forceinline__ void tc_mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    if constexpr (CTAS == 1)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
+}
+
 // Each thread of the warp reads 32 consecutive 32-bit columns of its own TMEM lane.
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
@@ -338,6 +359,15 @@ __host__ __device__ constexpr uint32_t idesc_mxf8_e4m3(int M, int N, bool b_e2m1
            | (static_cast<uint32_t>(N >> 3) << 17)             // N / 8
            | (1u << 23)                                       // scale format UE8M0
            | (static_cast<uint32_t>(M >> 4) << 24);            // M / 16
+}
+
+// Instruction descriptor of kind::f8f6f4 (no block scaling): fp32 accumulator (bits 4-5 = 1), A and B E4M3,
+// both K-major, N / 8 and M / 16 (the bit layout of CUTLASS's UMMA::InstrDescriptor).
+__host__ __device__ constexpr uint32_t idesc_f8f6f4_e4m3(int M, int N) {
+    return (1u << 4)                                           // accumulator F32
+           | (0u << 7) | (0u << 10)                            // A and B E4M3
+           | (static_cast<uint32_t>(N >> 3) << 17)              // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);             // M / 16
 }
 
 }  // namespace dg

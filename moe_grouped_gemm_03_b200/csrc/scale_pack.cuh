@@ -38,12 +38,21 @@ struct PackParams {
     int sfb_kwords;       // B scale words along K per (group, N tile): num_sf_groups, or K/128 when sfb_fp4
     int N, G, bn, n_tiles, sfb_atoms;
     int nkb, num_sf_groups;
+    const int *m_indices; // contiguous: row -> group (-1 = padding); only rows of a group have their scales checked
+    unsigned *err;        // device error word: ERR_BAD_SCALE for a scale the call reads that is not a power of two
     uint32_t *sfa_out;    // [sfa_groups * blocks_per_group][num_sf_groups][128]
     uint32_t *sfb_out;    // [G][n_tiles][num_sf_groups][sfb_atoms][128]
     long long sfa_words, sfb_words;
 };
 
 __device__ __forceinline__ uint32_t ue8m0_code(float s) { return (__float_as_uint(s) >> 23) & 0xFFu; }
+
+// A scale the exponent code represents exactly: +0 (taken as 2^-127) or a positive normal power of two
+// (no sign, no mantissa bits, not Inf / NaN).
+__device__ __forceinline__ bool ue8m0_exact(float s) {
+    const uint32_t b = __float_as_uint(s);
+    return (b & 0x807FFFFFu) == 0u && (b >> 23) != 0xFFu;
+}
 
 // Most threads per block of the pre-pass (the host launches at most one block per SM).
 constexpr int PACK_THREADS = 1024;
@@ -91,6 +100,7 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
     const int warps_per_block = blockDim.x >> 5;
     const long long num_warps = static_cast<long long>(gridDim.x) * warps_per_block;
     const int nnb128 = (p.N + 127) / 128;
+    bool bad_scale = false;  // this lane read a scale the block-scaled MMA cannot represent
     for (long long atom = static_cast<long long>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5); atom < total;
          atom += num_warps) {
         uint32_t word[4] = {0u, 0u, 0u, 0u};
@@ -118,16 +128,28 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
             const float *base = p.sfa + group_base;
             int kb_first, kb_count;
             k_blocks(q, kb_first, kb_count);
+            // rows whose scales the call uses: masked, below the group's masked_m; contiguous, rows of a group
+            int owned = rows;
+            if (p.mode == MODE_MASKED) {
+                const int m = __ldg(p.counts + block / p.blocks_per_group);
+                owned = min(max(m, 0), p.rows_per_group) - first;
+            }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int r = lane + 32 * j;
                 const int row = first + r;
+                const bool in = r < rows && row < p.sfa_ld;
+                const bool check =
+                    in && r < owned && (p.mode != MODE_CONTIGUOUS || __ldg(p.m_indices + row) >= 0);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int kb = kb_first + i;
-                    const uint32_t code = (r < rows && row < p.sfa_ld && i < kb_count)
-                                              ? ue8m0_code(__ldg(base + static_cast<size_t>(kb) * p.sfa_ld + row))
-                                              : 0x7Fu;
+                    uint32_t code = 0x7Fu;
+                    if (in && i < kb_count) {
+                        const float v = __ldg(base + static_cast<size_t>(kb) * p.sfa_ld + row);
+                        code = ue8m0_code(v);
+                        if (check && !ue8m0_exact(v)) bad_scale = true;
+                    }
                     word[j] |= code << (8 * i);
                 }
             }
@@ -149,9 +171,12 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
                     const float *base = p.sfb + static_cast<size_t>(g) * (4 * p.nkb) * p.sfb_ld + n;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const uint32_t code = (n < p.N && q < p.nkb)
-                                                  ? ue8m0_code(__ldg(base + static_cast<size_t>(4 * q + i) * p.sfb_ld))
-                                                  : 0x7Fu;
+                        uint32_t code = 0x7Fu;
+                        if (n < p.N && q < p.nkb) {
+                            const float v = __ldg(base + static_cast<size_t>(4 * q + i) * p.sfb_ld);
+                            code = ue8m0_code(v);
+                            if (!ue8m0_exact(v)) bad_scale = true;
+                        }
                         word[j] |= code << (8 * i);
                     }
                 }
@@ -179,7 +204,12 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int kb = kb_first + i;
-                    const uint32_t code = (n < p.N && i < kb_count) ? ue8m0_code(__ldg(base + kb * stride_kb)) : 0x7Fu;
+                    uint32_t code = 0x7Fu;
+                    if (n < p.N && i < kb_count) {
+                        const float v = __ldg(base + kb * stride_kb);
+                        code = ue8m0_code(v);
+                        if (!ue8m0_exact(v)) bad_scale = true;
+                    }
                     word[j] |= code << (8 * i);
                 }
             }
@@ -187,6 +217,7 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
         }
         *reinterpret_cast<uint4 *>(dst + 4 * lane) = make_uint4(word[0], word[1], word[2], word[3]);
     }
+    if (__any_sync(0xffffffffu, bad_scale) && lane == 0) raise_error(p.err, ERR_BAD_SCALE);
 }
 
 }  // namespace dg
