@@ -5,7 +5,8 @@ One step = one call of the library's dense FP8 GEMM on the workload M=4096, N=71
 with power-of-two 1x128 / 128x128 scales, bf16 out; seeded synthetic inputs), the configuration the
 headline metric is quoted on.  Other workloads can be timed with --workload for reference (the default line
 is the contract line): 1 dense 128x256x512; 3 and 5 contiguous grouped; 4 masked grouped; 6 no-padding grouped;
-7 contiguous with B in the NN orientation; 8 K-grouped with fp32 output; 9 contiguous W4A8 (B in E2M1).
+7 contiguous with B in the NN orientation; 8 K-grouped with fp32 output; 9 contiguous W4A8 (B in E2M1);
+10 workload 2 with fp32 (non-power-of-two) scales, through the fp32 scale-promotion path.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 2]
 
@@ -44,7 +45,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7, 8, 9])
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7, 8, 9, 10])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
@@ -197,9 +198,13 @@ def call_library(p, t, out):
         dg.m_grouped_fp8_gemm_nt_masked((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["masked_m"], p.expected_m)
 
 
-def launches_per_call(p):
-    """The library's kernels one call launches: the scale pre-pass and the GEMM (NN: the B transpose too)."""
-    return 3 if p.kind == "contiguous_nn" else 2
+PROMOTION_WORKLOADS = (10,)  # run with fp32 scale promotion (their scales are not powers of two)
+
+
+def launches_per_call(p, promotion=False):
+    """The library's kernels one call launches: the scale pre-pass and the GEMM (NN: the B transpose too); the
+    fp32 scale-promotion GEMM has no pre-pass."""
+    return (2 if p.kind == "contiguous_nn" else 1) + (0 if promotion else 1)
 
 
 def algorithmic_bytes(p):
@@ -296,6 +301,8 @@ def run_ours(args, world, rank, local):
     import synth
 
     p = synth.make_config(args.workload)
+    promotion = args.workload in PROMOTION_WORKLOADS
+    dg.set_fp32_scale_promotion(promotion)
     t = synth.to_torch(p, f"cuda:{local}")
     out_dtype = torch.float32 if p.kind == "k_grouped" else torch.bfloat16
     out = torch.empty(p.out_shape(), dtype=out_dtype, device=f"cuda:{local}")
@@ -396,16 +403,17 @@ def run_ours(args, world, rank, local):
         "steps": K, "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3", "data": "synthetic",
         "config": {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "G": p.G,
-                   "block_n": dg.select_block_n(
+                   "block_n": 128 if promotion else dg.select_block_n(
                        p.G * ((p.expected_m + 127) // 128) if p.kind == "masked" else (p.rows + 127) // 128,
                        p.N, dg.get_num_sms()),
+                   "scales": "fp32, promoted per 128-K block" if promotion else "powers of two (UE8M0, block-scaled MMA)",
                    "l2": "flushed between steps (512 MB write outside the timed events)",
                    "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU",
                    "tflops_frac_of_fp8_peak": achieved / fp8_peak},
         "roofline": roofline,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": K * launches_per_call(p),
+        "gpu_launches": K * launches_per_call(p, promotion),
         "clocks": clocks.summary(),
     }
     if not args.no_cpu_baseline and world == 1:

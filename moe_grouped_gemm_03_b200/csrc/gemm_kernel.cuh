@@ -854,7 +854,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t pb_ph = 0;
         // fp32 scale promotion of one tile: this lane's row accumulates partial(kb) * sfa[row, kb] * sfb[g, nb, kb]
         // over the K blocks in registers (BN = 128 columns: one 128-column block of B's scales), then it is
-        // written as bf16.  The scales are read from the caller's arrays one partial stage ahead.  false = gave up.
+        // written as bf16.  The scales are read from the caller's arrays one partial stage ahead: the loads go out
+        // right after a stage is released and are used after the next stage's wait, so they are complete before
+        // the next release (a release orders every earlier memory access of the thread, and would otherwise wait
+        // for loads still in flight).  false = gave up.
         auto promote_tile = [&](const Tile &ti) -> bool {
             const int r_local = my_rows + 32 * q + lane;
             const int row = ti.row0 + r_local;
@@ -886,12 +889,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             load_scales(0);
             for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
                 const int nk = min(C::KPS, nkb - kb0);
+                if (!warp_wait_bounded(&tmem_full[pb], pb_ph, s_abort, p.err, p.wait_limit_ns, lane)) return false;
+                tc_fence_after_sync();
                 float sc[C::KPS];
 #pragma unroll
                 for (int i = 0; i < C::KPS; ++i) sc[i] = sa_n[i] * sb_n[i];
-                if (kb0 + C::KPS < nkb) load_scales(kb0 + C::KPS);
-                if (!warp_wait_bounded(&tmem_full[pb], pb_ph, s_abort, p.err, p.wait_limit_ns, lane)) return false;
-                tc_fence_after_sync();
                 const uint32_t t_part =
                     tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(pb * C::KPS * BN);
 #pragma unroll
@@ -917,12 +919,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 __syncwarp();
                 if (lane == 0) {
                     if constexpr (PAIR)
-                        mbar_arrive_cluster(tmem_empty_leader0 + 8u * static_cast<uint32_t>(pb));
+                        mbar_arrive_remote(tmem_empty_leader0 + 8u * static_cast<uint32_t>(pb));
                     else
                         mbar_arrive(&tmem_empty[pb]);
                 }
                 pb ^= 1;
                 if (pb == 0) pb_ph ^= 1u;
+                if (kb0 + C::KPS < nkb) load_scales(kb0 + C::KPS);
             }
             const bool valid = row_owned(ti, row, r_local);
             const bool tma_ok = p.mode == MODE_DENSE || __all_sync(0xffffffffu, valid);
@@ -1015,7 +1018,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             __syncwarp();
             if (lane == 0) {
                 if constexpr (PAIR)
-                    mbar_arrive_cluster(tmem_empty_leader0 + 8u * static_cast<uint32_t>(acc));
+                    mbar_arrive_remote(tmem_empty_leader0 + 8u * static_cast<uint32_t>(acc));
                 else
                     mbar_arrive(&tmem_empty[acc]);
             }

@@ -108,23 +108,13 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// 32-bit store to the shared memory of a CTA of this cluster (shared::cluster address).
-__device__ __forceinline__ void st_shared_cluster(uint32_t cluster_addr, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-
-// Orders this thread's generic-proxy writes to shared memory of any CTA of the cluster before later
-// async-proxy accesses.
-__device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
-
-// Arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_addr, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_addr),
-                 "r"(bytes)
-                 : "memory");
+// Arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA), with release semantics
+// at CTA scope (the default).  Used to hand a tensor-memory buffer back to the MMA issuer: the arriving thread's
+// TMEM reads have completed (tcgen05.wait::ld) and are ordered by the tcgen05 fences around the handoff, and a
+// cluster-scope release here cost the promotion epilogue a memory-barrier stall per partial stage (the
+// promotion call ran 1.6x slower with it).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // ------------------------------------------------------------------------------------------------

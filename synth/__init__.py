@@ -422,6 +422,7 @@ CONFIGS = {
     7: "M-grouped contiguous FP8 NN GEMM (B [G, K, N]) G=8 N=4096 K=7168, tokens U[1024,8192] per group",
     8: "K-grouped FP8 NT GEMM, fp32 D_g = A_g B_g^T, G=8 M=4096 N=7168, K_g = tokens U[1024,8192] rounded up to 128",
     9: "M-grouped contiguous W4A8 GEMM (e4m3 A x E2M1 B) G=8 N=4096 K=7168, tokens U[1024,8192] per group",
+    10: "dense FP8 NT GEMM M=4096 N=7168 K=7168 with fp32 (non-power-of-two) scales",
 }
 
 
@@ -455,6 +456,10 @@ def make_config(i: int, seed: int = 0) -> Problem:
     if i == 6:
         rng = np.random.default_rng(seed)
         return make_nopad(zipf_counts(65536, 64, 1.2), 7168, 2048, rng=rng, name=CONFIGS[6])
+    if i == 10:
+        p = with_fp32_scales(make_dense(4096, 7168, 7168, seed), seed)
+        p.name = CONFIGS[10]
+        return p
     raise ValueError(f"unknown config {i}")
 
 
