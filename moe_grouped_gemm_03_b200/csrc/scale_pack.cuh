@@ -45,14 +45,12 @@ struct PackParams {
     long long sfa_words, sfb_words;
 };
 
-__device__ __forceinline__ uint32_t ue8m0_code(float s) { return (__float_as_uint(s) >> 23) & 0xFFu; }
-
-// A scale the exponent code represents exactly: +0 (taken as 2^-127) or a positive normal power of two
-// (no sign, no mantissa bits, not Inf / NaN).
-__device__ __forceinline__ bool ue8m0_exact(float s) {
-    const uint32_t b = __float_as_uint(s);
-    return (b & 0x807FFFFFu) == 0u && (b >> 23) != 0xFFu;
+// Nonzero unless the scale's fp32 bits are ones the exponent code represents exactly: +0 (taken as 2^-127) or
+// a positive normal power of two (no sign, no mantissa bits, not Inf / NaN).
+__device__ __forceinline__ uint32_t ue8m0_inexact_bits(uint32_t b) {
+    return (b & 0x807FFFFFu) | (((b >> 23) & 0xFFu) == 0xFFu ? 1u : 0u);
 }
+constexpr uint32_t ONE_F32_BITS = 0x3F800000u;  // 1.0f: the code 0x7F written for entries past the problem
 
 // Most threads per block of the pre-pass (the host launches at most one block per SM).
 constexpr int PACK_THREADS = 1024;
@@ -100,7 +98,7 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
     const int warps_per_block = blockDim.x >> 5;
     const long long num_warps = static_cast<long long>(gridDim.x) * warps_per_block;
     const int nnb128 = (p.N + 127) / 128;
-    bool bad_scale = false;  // this lane read a scale the block-scaled MMA cannot represent
+    uint32_t bad_bits = 0;  // nonzero once this lane read a scale the block-scaled MMA cannot represent
     for (long long atom = static_cast<long long>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5); atom < total;
          atom += num_warps) {
         uint32_t word[4] = {0u, 0u, 0u, 0u};
@@ -141,16 +139,18 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
                 const bool in = r < rows && row < p.sfa_ld;
                 const bool check =
                     in && r < owned && (p.mode != MODE_CONTIGUOUS || __ldg(p.m_indices + row) >= 0);
+                uint32_t bits[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int kb = kb_first + i;
-                    uint32_t code = 0x7Fu;
-                    if (in && i < kb_count) {
-                        const float v = __ldg(base + static_cast<size_t>(kb) * p.sfa_ld + row);
-                        code = ue8m0_code(v);
-                        if (check && !ue8m0_exact(v)) bad_scale = true;
-                    }
-                    word[j] |= code << (8 * i);
+                    bits[i] = (in && i < kb_count)
+                                  ? __float_as_uint(__ldg(base + static_cast<size_t>(kb) * p.sfa_ld + row))
+                                  : ONE_F32_BITS;
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    word[j] |= ((bits[i] >> 23) & 0xFFu) << (8 * i);
+                    if (check) bad_bits |= ue8m0_inexact_bits(bits[i]);
                 }
             }
             dst = p.sfa_out + atom * SF_ATOM_WORDS;
@@ -171,13 +171,11 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
                     const float *base = p.sfb + static_cast<size_t>(g) * (4 * p.nkb) * p.sfb_ld + n;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        uint32_t code = 0x7Fu;
-                        if (n < p.N && q < p.nkb) {
-                            const float v = __ldg(base + static_cast<size_t>(4 * q + i) * p.sfb_ld);
-                            code = ue8m0_code(v);
-                            if (!ue8m0_exact(v)) bad_scale = true;
-                        }
-                        word[j] |= code << (8 * i);
+                        const uint32_t bits = (n < p.N && q < p.nkb)
+                                                  ? __float_as_uint(__ldg(base + static_cast<size_t>(4 * q + i) * p.sfb_ld))
+                                                  : ONE_F32_BITS;
+                        word[j] |= ((bits >> 23) & 0xFFu) << (8 * i);
+                        bad_bits |= ue8m0_inexact_bits(bits);
                     }
                 }
                 dst = p.sfb_out + b * SF_ATOM_WORDS;
@@ -204,20 +202,17 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int kb = kb_first + i;
-                    uint32_t code = 0x7Fu;
-                    if (n < p.N && i < kb_count) {
-                        const float v = __ldg(base + kb * stride_kb);
-                        code = ue8m0_code(v);
-                        if (!ue8m0_exact(v)) bad_scale = true;
-                    }
-                    word[j] |= code << (8 * i);
+                    const uint32_t bits =
+                        (n < p.N && i < kb_count) ? __float_as_uint(__ldg(base + kb * stride_kb)) : ONE_F32_BITS;
+                    word[j] |= ((bits >> 23) & 0xFFu) << (8 * i);
+                    bad_bits |= ue8m0_inexact_bits(bits);
                 }
             }
             dst = p.sfb_out + b * SF_ATOM_WORDS;
         }
         *reinterpret_cast<uint4 *>(dst + 4 * lane) = make_uint4(word[0], word[1], word[2], word[3]);
     }
-    if (__any_sync(0xffffffffu, bad_scale) && lane == 0) raise_error(p.err, ERR_BAD_SCALE);
+    if (__any_sync(0xffffffffu, bad_bits != 0) && lane == 0) raise_error(p.err, ERR_BAD_SCALE);
 }
 
 }  // namespace dg
