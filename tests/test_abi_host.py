@@ -124,3 +124,26 @@ def test_contiguous_alignment_setting():
     finally:
         assert dg.set_m_alignment_for_contiguous_layout(128) == 128
     assert L.dg_m_grouped_fp8_gemm_nt_contiguous(*ok.values(), P(256), 200, 256, 512, 2, None) == -2
+
+
+def test_fp32_scale_promotion_setting_roundtrip():
+    assert dg.get_fp32_scale_promotion() is False  # power-of-two scales (UE8M0) by default
+    try:
+        assert L.dg_set_fp32_scale_promotion(7) == 1  # any nonzero value switches it on
+        assert dg.get_fp32_scale_promotion() is True
+        # argument checks still come first on the promotion path (nothing is launched)
+        z = ctypes.c_void_p(16)
+        assert L.dg_fp8_gemm_nt(z, z, z, z, z, 128, 256, 100, None) == -2
+        assert L.dg_fp8_gemm_nt(z, z, z, z, z, 0, 256, 128, None) == 0  # empty: a no-op, no device needed
+    finally:
+        assert dg.set_fp32_scale_promotion(False) is False
+    assert L.dg_get_fp32_scale_promotion() == 0
+
+
+def test_status_names_cover_the_header():
+    import re
+
+    text = open(dg.HEADER_PATH).read()
+    declared = {int(v): name for name, v in re.findall(r"\b(DG_(?:OK|ERR_[A-Z_]+))\s*=\s*(-?\d+)", text)}
+    assert declared[0] == "DG_OK" and declared[-7] == "DG_ERR_BAD_SCALE"
+    assert declared == dg.STATUS_NAMES
