@@ -13,6 +13,11 @@
 // the scale-factor ids of the instruction descriptor for all four 32-wide K sub-blocks, which applies the
 // 1x128 / 128x128 recipe exactly.
 //
+// Cfg::PROMO (any finite fp32 scales): the promotion runs in the epilogue warps instead.  Plain kind::f8f6f4
+// MMAs write each 128-K block's partial product into its own TMEM buffer (two partial stages of KPS buffers),
+// and the epilogue warps accumulate partial * sfa * sfb in fp32 registers over 128-wide tiles, reading the
+// caller's fp32 scales directly (no pre-pass).
+//
 // CTAS = 1: one CTA computes a 128 x BN output tile.  CTAS = 2: a cluster of two CTAs (a CTA pair) computes
 // a 256 x BN tile with tcgen05.mma.cta_group::2: each CTA loads its own 128 rows of A and its own BN/2 rows
 // of B (no multicast), the leader CTA issues the MMAs, and each CTA's TMEM holds its 128 rows of D.  All
@@ -21,15 +26,17 @@
 // Per CTA, 192 threads:
 //   warp 0      TMA producer: per pipeline stage KPS 128-K blocks of A [128 x 128 B] and B [BN/CTAS x 128 B]
 //               (128-byte swizzle) and, at the first stage of each group of four K blocks, the packed scale
-//               atoms of the group (SFA of this CTA's rows, SFB of the whole tile).
+//               atoms of the group (SFA of this CTA's rows, SFB of the whole tile; none with PROMO).
 //   warp 1      TMEM owner (both CTAs) and MMA issuer (one thread of the leader CTA): copies a group's scale
 //               atoms shared -> TMEM (tcgen05.cp), then issues four tcgen05.mma (K = 32 each) per 128-K
 //               block into one of two TMEM accumulators (BN fp32 columns).
 //   warps 2..5  epilogue: TMEM -> registers -> bf16 (RNE) -> global, only for rows the GEMM owns, while the
-//               MMA already fills the other accumulator with the next tile.
+//               MMA already fills the other accumulator with the next tile (with PROMO: the fp32 promotion of
+//               each partial product, then the same bf16 stores).
 //
-// Tile scheduler (every role walks the same sequence): windows of 128*CTAS rows x BN columns, N fastest,
-// handed round-robin to the persistent CTAs (pairs).
+// Tile scheduler (every role walks the same sequence): windows of 128*CTAS rows x BN columns handed
+// round-robin to the persistent CTAs (pairs); dense and K-grouped tiles go down the windows first inside raster
+// groups of windows (see raster_tile), the other layouts across the columns first.
 //   dense       ceil(M / 128*CTAS) windows.
 //   contiguous  CTAS = 1: M_total/128 blocks, group = m_indices[first row], -1 skips the block.
 //               CTAS = 2: 256-row windows starting at each group's first block (two blocks of one group; the
