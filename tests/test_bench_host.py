@@ -1,0 +1,43 @@
+"""Host-side pieces of bench.py that need no GPU: the kernel-source hash that ties recorded ncu traffic to the
+code it was captured on, and the per-call launch count."""
+import os
+
+import bench
+import synth
+
+
+def test_strip_comments_keeps_code_and_literals():
+    src = ('asm volatile("mbarrier.try_wait // kept-1");  // gone-1\n'
+           "/* gone-2\n   gone-3 */ int x = '/';\n\n   \n"
+           'const char *s = "a \\" quote /* kept */";\n')
+    out = bench.strip_comments(src)
+    assert "gone" not in out
+    assert '"mbarrier.try_wait // kept-1"' in out
+    assert '"a \\" quote /* kept */"' in out and "int x = '/';" in out
+    assert "\n\n" not in out  # blank lines dropped
+
+
+def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    f = tmp_path / "k.cuh"
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", ["k.cuh"])
+    f.write_text("int a = 1;  // one\n")
+    h1 = bench.kernel_source_hash()
+    f.write_text("// header\nint a = 1;  /* still one */\n\n")
+    assert bench.kernel_source_hash() == h1
+    f.write_text("int a = 2;\n")
+    assert bench.kernel_source_hash() != h1
+
+
+def test_recorded_traffic_matches_the_tree():
+    """profiles/traffic.json holds counters of the kernels as they are now (else the bench reports null)."""
+    assert os.path.exists(os.path.join(bench.ROOT, "profiles", "traffic.json"))
+    assert bench.recorded_traffic(2) is not None and bench.recorded_traffic(5) is not None
+
+
+def test_launches_per_call():
+    dense = synth.make_dense(128, 256, 512)
+    nn = synth.make_contiguous_nn([129], 256, 256)
+    assert bench.launches_per_call(dense) == 2  # scale pre-pass + GEMM
+    assert bench.launches_per_call(nn) == 3  # + the B transpose
+    assert bench.launches_per_call(dense, promotion=True) == 1  # the promotion GEMM has no pre-pass
