@@ -139,6 +139,23 @@ def get_tma_aligned_size(mn: int, element_size: int) -> int:
     return _lib.dg_get_tma_aligned_size(mn, element_size)
 
 
+def get_mn_major_tma_aligned_tensor(sf: torch.Tensor) -> torch.Tensor:
+    """Per-row scales [M, K/128] (masked layout: [G, M, K/128]) -> the layout the GEMMs take for sfa: fp32,
+    MN-major and TMA-aligned, [K/128, tma_aligned(M)] (or [G, K/128, tma_aligned(M)]), contiguous, on the same
+    device; the padding columns hold 1.0.  ("Utilities" and "Notices" of the DeepGEMM-for-PPU README: the LHS
+    scale factor tensor is TMA-aligned and transposed.)  Input preparation by a tensor copy, outside any GEMM
+    call."""
+    _need(isinstance(sf, torch.Tensor) and sf.dim() in (2, 3), "sf must be a [M, K/128] or [G, M, K/128] tensor")
+    x = sf.unsqueeze(0) if sf.dim() == 2 else sf
+    G, M, nkb = x.shape
+    out = torch.ones((G, nkb, get_tma_aligned_size(M, 4)), dtype=torch.float32, device=sf.device)
+    out[:, :, :M] = x.transpose(1, 2)
+    return out[0] if sf.dim() == 2 else out
+
+
+get_col_major_tma_aligned_tensor = get_mn_major_tma_aligned_tensor  # the pages' other name for it
+
+
 def set_num_sms(n: int) -> int:
     return _lib.dg_set_num_sms(n)
 

@@ -147,3 +147,22 @@ def test_status_names_cover_the_header():
     declared = {int(v): name for name, v in re.findall(r"\b(DG_(?:OK|ERR_[A-Z_]+))\s*=\s*(-?\d+)", text)}
     assert declared[0] == "DG_OK" and declared[-7] == "DG_ERR_BAD_SCALE"
     assert declared == dg.STATUS_NAMES
+
+
+def test_mn_major_tma_aligned_scale_layout():
+    import numpy as np
+    import torch
+
+    import synth
+
+    sf = torch.arange(1, 1 + 13 * 3, dtype=torch.float32).reshape(13, 3)  # [M, K/128], M = 13 -> aligned 16
+    out = dg.get_mn_major_tma_aligned_tensor(sf)
+    assert out.shape == (3, 16) and out.is_contiguous() and out.dtype == torch.float32
+    assert torch.equal(out[:, :13], sf.t()) and torch.equal(out[:, 13:], torch.ones(3, 3))
+    g = torch.rand(2, 5, 4)
+    og = dg.get_col_major_tma_aligned_tensor(g)
+    assert og.shape == (2, 4, 8) and torch.equal(og[:, :, :5], g.transpose(1, 2))
+    # the generator's dense-call sfa is exactly this layout of its per-row scales
+    p = synth.make_dense(37, 128, 384, seed=3)
+    per_row = torch.from_numpy(np.ascontiguousarray(p.sfa[:, :37].T))
+    assert torch.equal(dg.get_mn_major_tma_aligned_tensor(per_row), torch.from_numpy(p.sfa))
