@@ -128,6 +128,11 @@ def get_m_alignment_for_contiguous_layout() -> int:
     return _lib.dg_get_m_alignment_for_contiguous_layout()
 
 
+def get_mk_alignment_for_contiguous_layout() -> int:
+    """The MATE wrapper's name for get_m_alignment_for_contiguous_layout (same value)."""
+    return _lib.dg_get_m_alignment_for_contiguous_layout()
+
+
 def set_m_alignment_for_contiguous_layout(alignment: int) -> int:
     """128 (default) or 256: the per-segment M padding the contiguous calls expect from here on."""
     rc = _lib.dg_set_m_alignment_for_contiguous_layout(int(alignment))

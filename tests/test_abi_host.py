@@ -118,6 +118,7 @@ def test_contiguous_alignment_setting():
     try:
         assert dg.set_m_alignment_for_contiguous_layout(256) == 256
         assert dg.get_m_alignment_for_contiguous_layout() == 256
+        assert dg.get_mk_alignment_for_contiguous_layout() == 256  # the MATE name, same value
         # 384 rows are 128-aligned but not 256-aligned
         assert L.dg_m_grouped_fp8_gemm_nt_contiguous(*ok.values(), P(256), 384, 256, 512, 2, None) == -2
         assert L.dg_m_grouped_fp8_gemm_nt_contiguous(*ok.values(), P(256), 0, 256, 512, 2, None) == 0
