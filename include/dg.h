@@ -139,14 +139,17 @@ DG_EXPORT int dg_m_grouped_fp8_gemm_nn_contiguous(const void *a, const float *sf
  *     k in the low nibble of byte k/2 when k is even, the high nibble when odd; 32-byte aligned;
  *   sfb [G][K/32][ld(N)] fp32, MN-major: one power-of-two scale per (row n, 32-K block):
  *   D[m][n] = sum over 128-K blocks kb of sfa(m, kb) * sum over its four 32-K sub-blocks j of sfb(g, 4 kb + j, n)
- *             * sum_{k in the sub-block} A[m][k] * B_g[n][k]. */
+ *             * sum_{k in the sub-block} A[m][k] * B_g[n][k].
+ *   Scales must be powers of two (others: DG_ERR_BAD_SCALE); returns DG_ERR_UNSUPPORTED while fp32 scale
+ *   promotion is on (dg_set_fp32_scale_promotion). */
 DG_EXPORT int dg_m_grouped_fp8_fp4_gemm_nt_contiguous(const void *a, const float *sfa, const void *b,
                                             const float *sfb, void *d, const int *m_indices, int M_total, int N, int K,
                                             int G, dg_stream_t stream);
 
 /* M-grouped GEMM, masked layout, W4A8 (`m_grouped_fp8_fp4_gemm_nt_masked`, same page): as
  * dg_m_grouped_fp8_gemm_nt_masked except b [G][N][K/2] bytes of packed E2M1 codes (32-byte aligned) and
- * sfb [G][K/32][ld(N)] fp32, one scale per (row n, 32-K block), as in dg_m_grouped_fp8_fp4_gemm_nt_contiguous. */
+ * sfb [G][K/32][ld(N)] fp32, one scale per (row n, 32-K block), as in dg_m_grouped_fp8_fp4_gemm_nt_contiguous
+ * (powers of two; DG_ERR_UNSUPPORTED while fp32 scale promotion is on). */
 DG_EXPORT int dg_m_grouped_fp8_fp4_gemm_nt_masked(const void *a, const float *sfa, const void *b, const float *sfb,
                                         void *d, const int *masked_m, int G, int M_max, int N, int K, int expected_m,
                                         dg_stream_t stream);
@@ -161,7 +164,8 @@ DG_EXPORT int dg_m_grouped_fp8_fp4_gemm_nt_masked(const void *a, const float *sf
  *   sum_{k in kb} A[m][k] * B[n][k].  c: NULL (D_g = the sum), another [G][M][N] fp32 buffer (copied into d
  *   first), or d itself (accumulate in place).  A group with ks = 0 gives D_g = C_g (0 without C).
  *   1 <= G <= 1024, N % 16 == 0, 16-byte aligned a, b, c, d.  Device values of ks_device that are negative or
- *   not multiples of 128 are reported by dg_check_device_error() as DG_ERR_BAD_GROUP. */
+ *   not multiples of 128 are reported by dg_check_device_error() as DG_ERR_BAD_GROUP.  Scales must be powers of
+ *   two (others: DG_ERR_BAD_SCALE); returns DG_ERR_UNSUPPORTED while fp32 scale promotion is on. */
 DG_EXPORT int dg_k_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
                                         float *d, const float *c, const int *ks, const int *ks_device, int G, int M,
                                         int N, dg_stream_t stream);
@@ -188,7 +192,8 @@ DG_EXPORT int dg_m_grouped_fp8_gemm_nt_nopad(const void *a, const float *sfa, co
  * one).  It never calls cudaMalloc, cudaFree or any allocating routine.
  *   - Limit: the packed scales take at most (ceil(M/128) + 2*ceil(N/BN)) * ceil(K/512) * 512 bytes (BN is the
  *     chosen tile width, 128..224); a shape needing more than 16 MiB returns DG_ERR_UNSUPPORTED and launches
- *     nothing (M = N = K = 16384 needs about 4.5 MB).
+ *     nothing (M = N = K = 16384 needs about 4.5 MB).  With fp32 scale promotion on, the call reads the caller's
+ *     scales directly and uses no buffer at all (no limit).
  *   - The first call on each device looks up the buffer's device address with that device current; make that
  *     first call before any stream capture.
  *   - All calls share the buffer and each call rewrites every word it uses: calls whose work overlaps on the GPU
