@@ -862,9 +862,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // fp32 scale promotion of one tile: this lane's row accumulates partial(kb) * sfa[row, kb] * sfb[g, nb, kb]
         // over the K blocks in registers (BN = 128 columns: one 128-column block of B's scales), then it is
         // written as bf16.  The scales are read from the caller's arrays one partial stage ahead: the loads go out
-        // right after a stage is released and are used after the next stage's wait, so they are complete before
-        // the next release (a release orders every earlier memory access of the thread, and would otherwise wait
-        // for loads still in flight).  false = gave up.
+        // right after a stage is released and are used after the next stage's wait.  false = gave up.
         auto promote_tile = [&](const Tile &ti) -> bool {
             const int r_local = my_rows + 32 * q + lane;
             const int row = ti.row0 + r_local;
