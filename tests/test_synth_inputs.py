@@ -116,3 +116,13 @@ def test_with_fp32_scales_gives_each_block_its_own_mantissa():
         mantissa = new.view(np.uint32) & 0x7FFFFF
         assert (mantissa != 0).mean() > 0.99  # (almost) no power of two left
     assert np.array_equal(p.sfa, again.sfa) and np.array_equal(p.sfb, again.sfb)  # seeded
+
+
+def test_workload_10_is_workload_2_with_fp32_scales():
+    w2, w10 = synth.make_config(2), synth.make_config(10)
+    assert (w10.kind, w10.M, w10.N, w10.K) == ("dense", 4096, 7168, 7168)
+    assert np.array_equal(w10.a, w2.a) and np.array_equal(w10.b, w2.b)
+    for s10, s2 in ((w10.sfa, w2.sfa), (w10.sfb, w2.sfb)):
+        ratio = s10.astype(np.float64) / s2
+        assert ((ratio >= 1.0) & (ratio < 2.0)).all()
+    assert ((w10.sfb.view(np.uint32) & 0x7FFFFF) != 0).all()  # no B scale is a power of two
