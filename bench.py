@@ -33,6 +33,12 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio (4.5 / 2.25 PFLOP/s)
+# Dense FP8 tensor FLOPs per SM per clock: a 128 x 224 x 32 block-scaled MMA issues every 112 cycles when nothing
+# else holds it (an issue-loop micro-benchmark on this GPU); twice the 8192 of BF16 (the measured cuBLAS BF16 peak
+# equals 148 x 8192 x the SM clock it ran at).
+FP8_FLOP_PER_SM_CLOCK = 16384
+METRIC = "FP8 GEMM TFLOPS (dense and M-grouped)"
+GROUPED_WORKLOADS = (3, 4, 5)  # the M-grouped half of the metric, timed beside the dense headline
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["moe_grouped_gemm_03_b200/csrc/gemm_kernel.cuh", "moe_grouped_gemm_03_b200/csrc/ptx.cuh",
                   "moe_grouped_gemm_03_b200/csrc/dg_api.cu", "moe_grouped_gemm_03_b200/csrc/scale_pack.cuh",
@@ -48,6 +54,11 @@ def parse():
     ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5, 6, 7, 8, 9, 10])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--grouped", default="auto",
+                    help="comma-separated workloads timed after the main one and reported under 'grouped' "
+                         "(auto: 3,4,5 when the main workload is 2 on one GPU; none: skip)")
+    ap.add_argument("--ref-seconds", type=float, default=30.0,
+                    help="reference arm: wall time of all warm-up and timed oracle steps together")
     return ap.parse_args()
 
 
@@ -280,8 +291,18 @@ def oracle_sample(p, seconds, rng_seed=0):
                       f"{dt:.2f} s wall for {flops / 1e9:.1f} GFLOP in fp64"}
 
 
+def workload_config(p, world, promotion):
+    """The `config` object of both arms: the workload, its scales and the timing protocol."""
+    return {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "G": p.G,
+            "scales": "fp32, promoted per 128-K block" if promotion else "powers of two (UE8M0, block-scaled MMA)",
+            "l2": "flushed between steps (512 MB write outside the timed events)",
+            "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"}
+
+
 def run_reference(args, world, rank):
-    """Reference arm: the CPU oracle, as it stands, on bounded samples of the same workload."""
+    """Reference arm: the CPU oracle, as it stands, on bounded samples of the same workload.  It runs the requested
+    --warmup and --steps; every step times the oracle on a fresh random sample of valid rows (all columns), sized so
+    that all warm-up and timed steps together take about --ref-seconds of wall time."""
     import synth
 
     if rank != 0:
@@ -296,9 +317,9 @@ def run_reference(args, world, rank):
     probe = time.perf_counter()
     oracle.problem_rows(p, np.sort(rng.choice(valid, 2, replace=False)))
     per_row = (time.perf_counter() - probe) / 2
-    rows_per_step = int(max(1, min(len(valid), 3.0 / max(per_row, 1e-9))))  # ~3 s per step
-    steps = max(1, min(args.steps, 10))
-    warm = min(args.warmup, 1)
+    steps, warm = max(1, args.steps), max(0, args.warmup)
+    per_step = min(3.0, max(0.01, args.ref_seconds / (steps + warm)))
+    rows_per_step = int(max(1, min(len(valid), per_step / max(per_row, 1e-9))))
     for _ in range(warm):
         oracle.problem_rows(p, np.sort(rng.choice(valid, rows_per_step, replace=False)))
     times = []
@@ -310,15 +331,113 @@ def run_reference(args, world, rank):
     flops = 2.0 * rows_per_step * p.N * p.K
     value = flops / statistics.mean(times) / 1e12
     line = {
-        "impl": "reference", "metric": "FP8 GEMM TFLOPS (dense and M-grouped)", "value": value, "unit": "TFLOP/s",
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": steps, "warmup": warm, "ms_per_step": 1e3 * statistics.mean(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "G": p.G},
+        "config": workload_config(p, world, args.workload in PROMOTION_WORKLOADS),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": f"{rows_per_step} random valid rows x all {p.N} columns per step"},
+                         "sample": f"{rows_per_step} random valid rows x all {p.N} columns per step "
+                                   f"({2 * rows_per_step * p.N * p.K / 1e9:.1f} GFLOP in fp64)"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def time_steps(p, t, out, flush, steps, warmup, world, promotion):
+    """Warm up, then time `steps` calls, each bracketed by CUDA events on the launching stream with an L2 flush
+    between them (outside the events).  NVML samples clocks during the timed loop, and the library's clock record
+    gives the SM clock the GEMM launches themselves ran at (the board's power limit holds it below the maximum
+    while the tensor cores are busy, a drop NVML's 10 ms samples mostly miss between the short launches)."""
+    import torch
+
+    import moe_grouped_gemm_03_b200 as dg
+
+    stream = torch.cuda.current_stream()
+    for _ in range(max(warmup, 3)):
+        call_library(p, t, out)
+    torch.cuda.synchronize()
+    dg.check_device_error()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    dg.debug_clock_read(reset=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    dg.debug_clock_record(True)
+    with clocks:
+        for i in range(steps):
+            flush.fill_(i)
+            starts[i].record(stream)
+            call_library(p, t, out)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    dg.debug_clock_record(False)
+    barrier(world)
+    dg.check_device_error()
+    cycles, ns, launches = dg.debug_clock_read(reset=True)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    summary = clocks.summary()
+    summary["sm_mhz_in_kernel"] = 1e3 * cycles / ns if ns else None
+    summary["in_kernel_launches"] = launches
+    return step_ms, summary
+
+
+def roofline_for(p, workload, mean_ms, peaks, peak_src, clocks, num_sms):
+    """Roofline of one workload's GEMM.  `peak` is the contract's: the measured bf16 burst peak x the nominal
+    FP8/BF16 ratio 2.  `clock_consistent` restates it from the SM clock the GEMM ran at (the library's clock
+    record) and from the maximum clock, at FP8_FLOP_PER_SM_CLOCK."""
+    flops = p.flops()
+    achieved = flops / (mean_ms * 1e-3) / 1e12
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    nbytes = algorithmic_bytes(p)
+    hbm_gbs = nbytes / (mean_ms * 1e-3) / 1e9
+    mhz = clocks.get("sm_mhz_in_kernel")
+    max_mhz = clocks.get("sm_max_mhz") or peaks.get("sm_max_mhz")
+    at_clock = num_sms * FP8_FLOP_PER_SM_CLOCK * mhz / 1e6 if mhz else None
+    at_max = num_sms * FP8_FLOP_PER_SM_CLOCK * max_mhz / 1e6 if max_mhz else None
+    roof = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+            "frac": achieved / fp8_peak, "traffic": recorded_traffic(workload),
+            "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x nominal fp8/bf16 ratio 2",
+            "clock_consistent": {
+                "fp8_flop_per_sm_clock": FP8_FLOP_PER_SM_CLOCK, "sms": num_sms,
+                "sm_mhz_in_kernel": mhz, "peak_at_kernel_clock": at_clock,
+                "frac_at_kernel_clock": achieved / at_clock if at_clock else None,
+                "sm_max_mhz": max_mhz, "peak_at_max_clock": at_max,
+                "frac_at_max_clock": achieved / at_max if at_max else None},
+            "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": nbytes,
+            "hbm_gbs_achieved": hbm_gbs, "hbm_peak_gbs": peaks["hbm_gbs"]}
+    if p.kind in ("masked", "masked_w4a8"):
+        roof.update(bound="hbm", achieved=hbm_gbs, peak=peaks["hbm_gbs"], unit="GB/s", frac=hbm_gbs / peaks["hbm_gbs"],
+                    peak_source=f"{peak_src} HBM copy bandwidth", tflops_achieved=achieved)
+    return roof
+
+
+def run_grouped(workloads, args, world, local, flush, peaks, peak_src, num_sms):
+    """The M-grouped half of the metric, timed in the same process with the same protocol as the main line."""
+    import torch
+
+    import synth
+
+    res = {}
+    for w in workloads:
+        p = synth.make_config(w)
+        promotion = w in PROMOTION_WORKLOADS
+        import moe_grouped_gemm_03_b200 as dg
+
+        dg.set_fp32_scale_promotion(promotion)
+        t = synth.to_torch(p, f"cuda:{local}")
+        out = torch.empty(p.out_shape(), dtype=torch.float32 if p.kind == "k_grouped" else torch.bfloat16,
+                          device=f"cuda:{local}")
+        step_ms, clocks = time_steps(p, t, out, flush, args.steps, args.warmup, world, promotion)
+        ms, value = whole_job_throughput(p.flops(), statistics.mean(step_ms), world)
+        res[str(w)] = {"workload": p.name, "value": value, "unit": "TFLOP/s", "ms_per_step": ms,
+                       "steps": args.steps, "warmup": max(args.warmup, 3),
+                       "roofline": roofline_for(p, w, statistics.mean(step_ms), peaks, peak_src, clocks, num_sms),
+                       "clocks": clocks, "gpu_launches": args.steps * launches_per_call(p, promotion),
+                       "config": workload_config(p, world, promotion)}
+        del t, out
+        torch.cuda.empty_cache()
+    return res
 
 
 def run_ours(args, world, rank, local):
@@ -336,28 +455,10 @@ def run_ours(args, world, rank, local):
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.int32, device=f"cuda:{local}")
     stream = torch.cuda.current_stream()
     flops = p.flops()
-
-    for _ in range(max(args.warmup, 3)):
-        call_library(p, t, out)
-    torch.cuda.synchronize()
-    dg.check_device_error()
+    num_sms = torch.cuda.get_device_properties(local).multi_processor_count
 
     K = args.steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    clocks = ClockSampler(torch.cuda.current_device())
-    barrier(world)
-    torch.cuda.synchronize()
-    with clocks:
-        for i in range(K):
-            flush.fill_(i)
-            starts[i].record(stream)
-            call_library(p, t, out)
-            ends[i].record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    dg.check_device_error()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    step_ms, clocks = time_steps(p, t, out, flush, K, args.warmup, world, promotion)
     ms, value = whole_job_throughput(flops, statistics.mean(step_ms), world)
 
     # End to end through the public API: every step copies its inputs from pinned host memory to the device,
@@ -409,43 +510,39 @@ def run_ours(args, world, rank, local):
     # the results read back equal the device-timed result bit for bit (same inputs, same kernels)
     if not all(torch.equal(h.view(torch.uint8), ref_bytes) for h in host_outs):
         raise RuntimeError("end-to-end results differ from the device-timed result")
+    del bufs, host, host_outs, t, out, ref_bytes
+    torch.cuda.empty_cache()
 
-    if rank != 0:
-        return
     peaks, peak_src = load_peaks()
-    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
-    achieved = flops / (statistics.mean(step_ms) * 1e-3) / 1e12
-    nbytes = algorithmic_bytes(p)
-    traffic = recorded_traffic(args.workload)
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
-                "frac": achieved / fp8_peak, "traffic": traffic,
-                "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x nominal fp8/bf16 ratio 2",
-                "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": nbytes,
-                "hbm_gbs_achieved": nbytes / (statistics.mean(step_ms) * 1e-3) / 1e9, "hbm_peak_gbs": peaks["hbm_gbs"]}
-    if p.kind == "masked":
-        roofline.update(bound="hbm", achieved=roofline["hbm_gbs_achieved"], peak=peaks["hbm_gbs"], unit="GB/s",
-                        frac=roofline["hbm_gbs_achieved"] / peaks["hbm_gbs"])
+    roofline = roofline_for(p, args.workload, statistics.mean(step_ms), peaks, peak_src, clocks, num_sms)
     line = {
-        "metric": "FP8 GEMM TFLOPS (dense and M-grouped)", "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": K, "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3", "data": "synthetic",
-        "config": {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "G": p.G,
-                   "block_n": 128 if promotion else dg.select_block_n(
-                       p.G * ((p.expected_m + 127) // 128) if p.kind == "masked" else (p.rows + 127) // 128,
-                       p.N, dg.get_num_sms()),
-                   "scales": "fp32, promoted per 128-K block" if promotion else "powers of two (UE8M0, block-scaled MMA)",
-                   "l2": "flushed between steps (512 MB write outside the timed events)",
-                   "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU",
-                   "tflops_frac_of_fp8_peak": achieved / fp8_peak},
+        "config": workload_config(p, world, promotion),
+        "plan": {"block_n": 128 if promotion else dg.select_block_n(
+                     p.G * ((p.expected_m + 127) // 128) if p.kind == "masked" else (p.rows + 127) // 128,
+                     p.N, dg.get_num_sms()),
+                 "tflops_frac_of_fp8_peak": roofline["achieved"] / roofline["peak"] if roofline["unit"] == "TFLOP/s"
+                 else None},
         "roofline": roofline,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": K * launches_per_call(p, promotion),
-        "clocks": clocks.summary(),
+        "clocks": clocks,
     }
-    if not args.no_cpu_baseline and world == 1:
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = oracle_sample(p, args.cpu_seconds)
-    print(json.dumps(line), flush=True)
+    grouped = args.grouped
+    if grouped == "auto":
+        grouped = ",".join(str(w) for w in GROUPED_WORKLOADS) if args.workload == 2 and world == 1 else ""
+    workloads = [int(w) for w in grouped.split(",") if w.strip() and w.strip() != "none"]
+    if workloads:
+        del p
+        line["grouped"] = run_grouped(workloads, args, world, local, flush, peaks, peak_src, num_sms)
+    dg.set_fp32_scale_promotion(False)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def main():

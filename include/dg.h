@@ -37,6 +37,16 @@
  *   - Device-side faults are not expected.  Every wait inside the kernel is bounded; a kernel that gives
  *     up records a code that dg_check_device_error() returns (DG_ERR_DEVICE_TIMEOUT, DG_ERR_BAD_GROUP or
  *     DG_ERR_BAD_SCALE).
+ *   - Settings (dg_set_m_alignment_for_contiguous_layout, dg_set_num_sms, dg_set_cta_pair_policy,
+ *     dg_set_fp32_scale_promotion, dg_debug_bounded_wait, dg_debug_clock_record) are process-wide, not
+ *     per thread or per stream.  Setting one while another thread calls the library is defined (each value is
+ *     an atomic) but that call sees whichever value was in force when it read it, so two users of one process
+ *     that want different settings must serialise their calls.  The M alignment also changes how every
+ *     later contiguous call's M_total is validated.
+ *   - The first call on a device, and the first call of each kernel configuration (tile width, CTA pair or
+ *     single CTA, layout) on it, does one-time set-up that is not a stream operation: device attribute
+ *     queries, symbol address look-ups, the kernel's shared-memory attribute and its cluster occupancy.  Make
+ *     one eager call of each shape class before capturing a stream into a CUDA graph.
  */
 #ifndef DG_H_
 #define DG_H_
@@ -70,8 +80,7 @@ typedef enum {
  * MATE docs "Contiguous Grouped GEMM Alignment": the alignment is 128 by default, 256 on request, nothing else. */
 DG_EXPORT int dg_get_m_alignment_for_contiguous_layout(void);
 
-/* Sets that alignment for the contiguous calls that follow (process-wide; not thread-safe against concurrent
- * calls).  128 or 256; returns the value set, or DG_ERR_INVALID_ARG (nothing changes) for any other value.
+/* Sets that alignment for the contiguous calls that follow (process-wide, see "Common conventions").  128 or 256; returns the value set, or DG_ERR_INVALID_ARG (nothing changes) for any other value.
  * With 256 every group owns whole 256-row windows, so the 2-CTA tiles never straddle two groups; results do
  * not depend on the alignment, only M_total's validation does (M_total % alignment == 0). */
 DG_EXPORT int dg_set_m_alignment_for_contiguous_layout(int alignment);
@@ -194,8 +203,9 @@ DG_EXPORT int dg_m_grouped_fp8_gemm_nt_nopad(const void *a, const float *sfa, co
  *     chosen tile width, 128..224); a shape needing more than 16 MiB returns DG_ERR_UNSUPPORTED and launches
  *     nothing (M = N = K = 16384 needs about 4.5 MB).  With fp32 scale promotion on, the call reads the caller's
  *     scales directly and uses no buffer at all (no limit).
- *   - The first call on each device looks up the buffer's device address with that device current; make that
- *     first call before any stream capture.
+ *   - The first call on each device looks up the buffer's device address with that device current, and the
+ *     first call of each tile configuration does the one-time kernel set-up listed under "Common conventions";
+ *     make one eager call of the same shape class on each device before any stream capture.
  *   - All calls share the buffer and each call rewrites every word it uses: calls whose work overlaps on the GPU
  *     (unordered streams) race; calls ordered on one stream are safe. */
 DG_EXPORT int dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
@@ -228,8 +238,19 @@ DG_EXPORT int dg_set_cta_pair_policy(int policy);
  *                     comes.  Its wait runs out after limit_ns, the CTA abandons its tiles (their rows of D are
  *                     left unwritten), the other CTAs finish, and dg_check_device_error() returns
  *                     DG_ERR_DEVICE_TIMEOUT.  The CUDA context stays usable.
- * Process-wide, not thread-safe; call it between launches.  Returns DG_OK or DG_ERR_INVALID_ARG. */
+ * Process-wide (see "Common conventions"); call it between launches.  Returns DG_OK or DG_ERR_INVALID_ARG. */
 DG_EXPORT int dg_debug_bounded_wait(unsigned long long limit_ns, int drop_first_stage);
+
+/* Measurement aid (no counterpart in the method; it exists so that a benchmark can state the SM clock its GEMM
+ * launches actually ran at, which under the board's power limit is below the maximum clock).
+ *   dg_debug_clock_record(1): every later GEMM launch (any entry point, any device) makes its first CTA add
+ *     the SM clock cycles (clock64) and the nanoseconds (globaltimer) it spent from start to exit, and 1, to a
+ *     per-device accumulator of three 64-bit counters; 0 switches it off (the default).  Returns the setting.
+ *   dg_debug_clock_read(out, reset): synchronises the current device, copies its three counters (cycles,
+ *     nanoseconds, launches) to the host array out[3] and, when reset != 0, clears them.  The mean SM clock of
+ *     the recorded launches is out[0] / out[1] GHz.  Returns DG_OK, DG_ERR_INVALID_ARG or DG_ERR_CUDA. */
+DG_EXPORT int dg_debug_clock_record(int enable);
+DG_EXPORT int dg_debug_clock_read(unsigned long long *out, int reset);
 
 /* Message for the last non-OK status returned on this thread ("" if none). */
 DG_EXPORT const char *dg_last_error(void);

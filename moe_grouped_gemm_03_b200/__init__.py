@@ -66,6 +66,8 @@ _SIGNATURES = {
     "dg_set_fp32_scale_promotion": (_I, [_I]),
     "dg_get_fp32_scale_promotion": (_I, []),
     "dg_debug_bounded_wait": (_I, [ctypes.c_ulonglong, _I]),
+    "dg_debug_clock_record": (_I, [_I]),
+    "dg_debug_clock_read": (_I, [_P, _I]),
     "dg_last_error": (ctypes.c_char_p, []),
     "dg_check_device_error": (_I, [_P]),
 }
@@ -197,6 +199,20 @@ def debug_bounded_wait(limit_ns: int = 0, drop_first_stage: bool = False) -> Non
     """Testing aid: set the in-kernel wait limit (0 = default 2 s) and, optionally, make the next GEMM launch
     leave one operand stage unloaded so a wait runs out and DG_ERR_DEVICE_TIMEOUT is recorded."""
     _check(_lib.dg_debug_bounded_wait(int(limit_ns), 1 if drop_first_stage else 0))
+
+
+def debug_clock_record(enable: bool) -> None:
+    """Measurement aid: while on, every GEMM launch's first CTA adds its SM cycles and nanoseconds to a per-device
+    accumulator (dg_debug_clock_record)."""
+    _lib.dg_debug_clock_record(1 if enable else 0)
+
+
+def debug_clock_read(reset: bool = True):
+    """(cycles, nanoseconds, launches) recorded on the current device since the last reset (dg_debug_clock_read);
+    cycles / nanoseconds is the mean SM clock of those launches in GHz."""
+    out = (ctypes.c_ulonglong * 3)()
+    _check(_lib.dg_debug_clock_read(ctypes.cast(out, _P), 1 if reset else 0))
+    return int(out[0]), int(out[1]), int(out[2])
 
 
 def check_device_error(stream=None) -> None:

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
@@ -18,9 +19,11 @@
 namespace {
 
 thread_local std::string g_last_error;
-int g_num_sms_cap = 0;  // 0: every SM of the device
+std::atomic<int> g_num_sms_cap{0};  // 0: every SM of the device
 
 __device__ unsigned g_device_error_word;  // first device-side error code since the last check
+// measurement aid (dg_debug_clock_record): SM cycles, nanoseconds and launches summed over recorded launches
+__device__ unsigned long long g_clock_acc[3];
 
 int fail(int code, const char *fmt, ...) {
     char buf[512];
@@ -67,7 +70,8 @@ int device_info(DeviceInfo &info) {
 }
 
 int effective_sms(const DeviceInfo &info) {
-    return (g_num_sms_cap > 0 && g_num_sms_cap < info.num_sms) ? g_num_sms_cap : info.num_sms;
+    const int cap = g_num_sms_cap.load(std::memory_order_relaxed);
+    return (cap > 0 && cap < info.num_sms) ? cap : info.num_sms;
 }
 
 // ----------------------------------------------------------------------------------------------- TMA
@@ -230,17 +234,37 @@ int noalloc_scratch(int device, uint32_t **out) {
 namespace {
 
 // ----------------------------------------------------------------------------------------------- launch
-int g_m_alignment = dg::BLOCK_M;  // contiguous layout: per-segment M padding (128 or 256)
-int g_pair_policy = -1;  // -1: library decides; 0: single CTAs only; 1: CTA pairs whenever supported
-bool g_fp32_promotion = false;  // true: any fp32 scales, applied by promotion; false: power-of-two scales (UE8M0)
-unsigned long long g_wait_limit_ns = dg::WAIT_LIMIT_NS;  // limit of every in-kernel wait
-bool g_drop_first_stage = false;  // testing aid: the next GEMM launch leaves one stage unloaded
+// Process-wide settings (atomics: reading one while another thread sets it is defined, but a call sees whichever
+// value was in force when it read it).
+std::atomic<int> g_m_alignment{dg::BLOCK_M};  // contiguous layout: per-segment M padding (128 or 256)
+std::atomic<int> g_pair_policy{-1};  // -1: library decides; 0: single CTAs only; 1: CTA pairs whenever supported
+std::atomic<bool> g_fp32_promotion{false};  // true: any fp32 scales, applied by promotion; false: powers of two
+std::atomic<unsigned long long> g_wait_limit_ns{dg::WAIT_LIMIT_NS};  // limit of every in-kernel wait
+std::atomic<bool> g_drop_first_stage{false};  // testing aid: the next GEMM launch leaves one stage unloaded
+std::atomic<bool> g_clock_record{false};      // measurement aid: launches add their clock record
 
-// Per-launch wait settings; the dropped stage applies to one launch only.
+// Device address of a __device__ symbol of this library (given by its host-side stand-in) on the current
+// device, looked up once per device with that device current.
+void *symbol_address(const void *symbol, void *(&cache)[64]) {
+    int device = 0;
+    if (cudaGetDevice(&device) != cudaSuccess) return nullptr;
+    if (device >= 0 && device < 64 && cache[device]) return cache[device];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess) return nullptr;
+    if (device >= 0 && device < 64) cache[device] = p;
+    return p;
+}
+
+unsigned long long *clock_accumulator() {
+    static void *cache[64] = {nullptr};
+    return static_cast<unsigned long long *>(symbol_address(g_clock_acc, cache));
+}
+
+// Per-launch settings: the wait limit, the dropped stage (one launch only) and the clock record.
 void apply_wait_settings(dg::GemmParams &p) {
-    p.wait_limit_ns = g_wait_limit_ns;
-    p.skip_first_load = g_drop_first_stage ? 1 : 0;
-    g_drop_first_stage = false;
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    p.skip_first_load = g_drop_first_stage.exchange(false) ? 1 : 0;
+    p.clock_acc = g_clock_record.load() ? clock_accumulator() : nullptr;
 }
 
 struct ScaleArgs {
@@ -250,6 +274,7 @@ struct ScaleArgs {
     bool sfb_kn = false;  // SFB stored [G][K/128][ceil(N/128)] (B in the NN orientation)
     bool sfb_fp4 = false; // B in E2M1 (packed two per byte) with SFB [G][K/32][sfb_ld]
     bool fixed_scratch = false;  // packed scales in the library's fixed buffer (no allocation) instead of the pool
+    bool swap = false;    // masked layout with swapped operands (B's rows on the MMA's M side, tokens on its N side)
     int sfb_ld = 0;       // K-grouped: one scale per row of B, [K/128][sfb_ld]; FP4 B: [G][K/32][sfb_ld]
 };
 
@@ -272,10 +297,10 @@ int launch_pack(const dg::PackParams &pk, int device, cudaStream_t stream) {
     return DG_OK;
 }
 
-template <int BN, int CTAS, int KPS, bool BF4 = false>
+template <int BN, int CTAS, int KPS, bool BF4 = false, bool SWAP = false>
 int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows, const ScaleArgs &sc, dg::GemmParams p,
                int grid, int device, cudaStream_t stream) {
-    using C = dg::Cfg<BN, CTAS, KPS, BF4>;
+    using C = dg::Cfg<BN, CTAS, KPS, BF4, false, SWAP>;
     // ---- packed scale atoms (pre-pass)
     const int nkb = p.K / dg::BLOCK_K;
     dg::PackParams pk{};
@@ -315,9 +340,17 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
         pk.blocks_per_group = (p.M + dg::BLOCK_M - 1) / dg::BLOCK_M;
         pk.sfa_groups = 1;
     }
-    const long long sfa_atoms = static_cast<long long>(pk.sfa_groups) * pk.blocks_per_group * p.num_sf_groups;
+    long long sfa_atoms = static_cast<long long>(pk.sfa_groups) * pk.blocks_per_group * p.num_sf_groups;
     const long long b_groups = p.mode == dg::MODE_KGROUPED ? 1 : p.G;  // K-grouped: one B for all groups
-    const long long sfb_atoms = b_groups * p.num_n_blocks * pk.sfb_kwords * C::SFB_ATOMS;
+    long long sfb_atoms = b_groups * p.num_n_blocks * pk.sfb_kwords * C::SFB_ATOMS;
+    if (SWAP) {  // B-side atoms per 128-row block of B, token-side atoms per chunk of each group
+        pk.swap = 1;
+        pk.b_blocks = p.sfa_blocks;
+        pk.chunks = p.swap_chunks;
+        pk.rows_per_group = p.M;
+        sfa_atoms = static_cast<long long>(p.G) * p.sfa_blocks * p.num_sf_groups;
+        sfb_atoms = static_cast<long long>(p.G) * p.swap_chunks * p.num_sf_groups * C::SFB_ATOMS;
+    }
     pk.sfa_words = sfa_atoms * dg::SF_ATOM_WORDS;
     pk.sfb_words = sfb_atoms * dg::SF_ATOM_WORDS;
     const size_t need = static_cast<size_t>(pk.sfa_words + pk.sfb_words) * 4;
@@ -349,11 +382,12 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
         else
             rc = make_output_map_f32(td, p.d32, p.G, p.M, p.N);
         if (rc) break;
-        if ((rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M))) break;
+        // (swapped operands: the 128-row boxes of the MMA's M side come from B, the N side's from A)
+        if ((rc = make_operand_map(ta, SWAP ? b : a, SWAP ? b_rows : a_rows, p.K, dg::BLOCK_M))) break;
         if (BF4)
             rc = make_operand_map_fp4(tb, b, b_rows, p.K, C::B_ROWS);
         else
-            rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS);
+            rc = make_operand_map(tb, SWAP ? a : b, SWAP ? a_rows : b_rows, p.K, C::B_ROWS);
         if (rc) break;
         if ((rc = make_atom_map(tsfa, pk.sfa_out, sfa_atoms, 1))) break;
         if ((rc = make_atom_map(tsfb, pk.sfb_out, sfb_atoms, C::SFB_KB * C::SFB_ATOMS))) break;
@@ -398,10 +432,10 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
         }
         static const bool debug = getenv("DG_DEBUG") && getenv("DG_DEBUG")[0] == '1';
         if (debug)
-            fprintf(stderr, "[dg] mode=%d M=%d N=%d K=%d G=%d BN=%d stages=%d x %d ctas=%d grid=%u smem=%d windows=%d"
+            fprintf(stderr, "[dg] mode=%d%s M=%d N=%d K=%d G=%d BN=%d stages=%d x %d ctas=%d grid=%u smem=%d windows=%d"
                             " raster=%d scratch=%lld B\n",
-                    p.mode, p.M, p.N, p.K, p.G, BN, C::STAGES, KPS, CTAS, cfg.gridDim.x, C::SMEM_BYTES, p.num_windows,
-                    p.raster_bands, (pk.sfa_words + pk.sfb_words) * 4);
+                    p.mode, SWAP ? " (swapped operands)" : "", p.M, p.N, p.K, p.G, BN, C::STAGES, KPS, CTAS,
+                    cfg.gridDim.x, C::SMEM_BYTES, p.num_windows, p.raster_bands, (pk.sfa_words + pk.sfb_words) * 4);
         apply_wait_settings(p);
         if ((rc = launch_pack(pk, device, stream))) break;
         if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, tsfa, tsfb, td, p)) != cudaSuccess) {
@@ -564,14 +598,15 @@ int plan_and_launch(dg::GemmParams p, const DeviceInfo &info, const Plan &plan, 
                     const void *b, long long b_rows, const ScaleArgs &sc, cudaStream_t stream) {
     const int sms = effective_sms(info);
     bool pair = plan.pair_supported && sms >= 2;
-    if (g_pair_policy == 0) pair = false;
-    if (g_pair_policy < 0 && pair) {
+    const int policy = g_pair_policy.load();
+    if (policy == 0) pair = false;
+    if (policy < 0 && pair) {
         // pairs pay once there is at least a wave of them
         const int bn = select_block_n(plan.sel2, p.N, sms / 2, 2);
         pair = plan.sel2 * ((p.N + bn - 1) / bn) >= sms / 2;
     }
     const int units = pair ? sms / 2 : sms;
-    if (g_fp32_promotion) {
+    if (g_fp32_promotion.load()) {
         if (sc.sfb_fp4 || p.mode == dg::MODE_KGROUPED || p.out_mode != dg::OUT_BF16)
             return fail(DG_ERR_UNSUPPORTED,
                         "fp32 scale promotion covers the bf16-output FP8 calls (dense, contiguous, masked, no-padding, "
@@ -603,14 +638,8 @@ int plan_and_launch(dg::GemmParams p, const DeviceInfo &info, const Plan &plan, 
 }
 
 unsigned *device_error_word() {
-    int device = 0;
-    if (cudaGetDevice(&device) != cudaSuccess) return nullptr;
-    static unsigned *cache[64] = {nullptr};  // the symbol's address on each device, looked up once
-    if (device >= 0 && device < 64 && cache[device]) return cache[device];
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
-    if (device >= 0 && device < 64) cache[device] = static_cast<unsigned *>(p);
-    return static_cast<unsigned *>(p);
+    static void *cache[64] = {nullptr};  // the symbol's address on each device, looked up once
+    return static_cast<unsigned *>(symbol_address(&g_device_error_word, cache));
 }
 
 int check_common(const void *a, const float *sfa, const void *b, const float *sfb, const void *d, long long N,
@@ -636,8 +665,9 @@ int check_contiguous(const void *a, const float *sfa, const void *b, const float
     if (!aligned(m_indices, 4)) return fail(DG_ERR_ALIGNMENT, "m_indices must be 4-byte aligned");
     if (G < 1 || G > 65534) return fail(DG_ERR_INVALID_ARG, "G=%d must be in [1, 65534]", G);
     if (M_total < 0) return fail(DG_ERR_INVALID_ARG, "M_total=%d must be non-negative", M_total);
-    if (M_total % g_m_alignment)
-        return fail(DG_ERR_ALIGNMENT, "M_total=%d must be a multiple of %d", M_total, g_m_alignment);
+    const int alignment = g_m_alignment.load();
+    if (M_total % alignment)
+        return fail(DG_ERR_ALIGNMENT, "M_total=%d must be a multiple of %d", M_total, alignment);
     if (static_cast<long long>(G) * N > 0x7fffffffLL) return fail(DG_ERR_INVALID_ARG, "G*N exceeds 2^31");
     return DG_OK;
 }
@@ -719,8 +749,35 @@ int masked_call(const void *a, const float *sfa, const void *b, const float *sfb
     p.masked_m = masked_m;
     p.err = device_error_word();
     if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
-    // tile shape from the caller's hint; the grid from the most tiles masked_m could ask for
     const int hint = expected_m > 0 && expected_m < M_max ? expected_m : M_max;
+    static const bool swap_off = getenv("DG_MASKED_SWAP") && getenv("DG_MASKED_SWAP")[0] == '0';  // A/B timing
+    if (!b_fp4 && !g_fp32_promotion.load() && !swap_off) {
+        // Swapped operands: tiles of TILE_M rows of B x one chunk (at most kSwapTokens) of a group's tokens; a
+        // group of m tokens costs ceil(m / 16) * 16 rows of MMA work instead of whole 128-row blocks.
+        constexpr int kSwapTokens = 224;
+        const int sms = effective_sms(info);
+        const long long chunks_max = (M_max + kSwapTokens - 1) / kSwapTokens;
+        const long long hint_chunks = (hint + kSwapTokens - 1) / kSwapTokens;
+        const int policy = g_pair_policy.load();
+        bool pair = sms >= 2 && policy != 0;
+        if (pair && policy < 0)  // pairs pay once there is at least a wave of them
+            pair = static_cast<long long>(G) * hint_chunks * ((N + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M)) >= sms / 2;
+        const int tile_m = pair ? 2 * dg::BLOCK_M : dg::BLOCK_M;
+        p.num_n_blocks = (N + tile_m - 1) / tile_m;
+        p.sfa_blocks = p.num_n_blocks * (pair ? 2 : 1);
+        p.swap_chunks = static_cast<int>(chunks_max);
+        p.num_windows = 0;
+        p.num_sf_groups = (K / dg::BLOCK_K + dg::SF_GROUP - 1) / dg::SF_GROUP;
+        sc.swap = true;
+        const long long tiles = static_cast<long long>(G) * chunks_max * p.num_n_blocks;
+        const int units = pair ? sms / 2 : sms;
+        const int grid = static_cast<int>(tiles < units ? tiles : units);
+        const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        const long long a_rows = static_cast<long long>(G) * M_max, b_rows = static_cast<long long>(G) * N;
+        if (pair) return launch_cfg<kSwapTokens, 2, 2, false, true>(a, a_rows, b, b_rows, sc, p, grid, info.device, s);
+        return launch_cfg<kSwapTokens, 1, 1, false, true>(a, a_rows, b, b_rows, sc, p, grid, info.device, s);
+    }
+    // tile shape from the caller's hint; the grid from the most tiles masked_m could ask for
     const long long h1 = static_cast<long long>(G) * ((hint + dg::BLOCK_M - 1) / dg::BLOCK_M);
     const long long h2 = static_cast<long long>(G) * ((hint + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M));
     const long long max1 = static_cast<long long>(G) * ((M_max + dg::BLOCK_M - 1) / dg::BLOCK_M);
@@ -734,12 +791,12 @@ int masked_call(const void *a, const float *sfa, const void *b, const float *sfb
 
 extern "C" {
 
-int dg_get_m_alignment_for_contiguous_layout(void) { return g_m_alignment; }
+int dg_get_m_alignment_for_contiguous_layout(void) { return g_m_alignment.load(); }
 
 int dg_set_m_alignment_for_contiguous_layout(int alignment) {
     if (alignment != 128 && alignment != 256)
         return fail(DG_ERR_INVALID_ARG, "alignment=%d must be 128 or 256", alignment);
-    g_m_alignment = alignment;
+    g_m_alignment.store(alignment);
     return alignment;
 }
 
@@ -750,7 +807,7 @@ int dg_get_tma_aligned_size(int mn, int elem_bytes) {
 }
 
 int dg_set_num_sms(int n) {
-    g_num_sms_cap = n > 0 ? n : 0;
+    g_num_sms_cap.store(n > 0 ? n : 0);
     return dg_get_num_sms();
 }
 
@@ -759,9 +816,10 @@ int dg_get_num_sms(void) {
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
         cudaGetLastError();
-        return g_num_sms_cap;  // no device: report the cap alone
+        return g_num_sms_cap.load();  // no device: report the cap alone
     }
-    return (g_num_sms_cap > 0 && g_num_sms_cap < sms) ? g_num_sms_cap : sms;
+    const int cap = g_num_sms_cap.load();
+    return (cap > 0 && cap < sms) ? cap : sms;
 }
 
 long long dg_num_tiles(long long M, long long N, int block_m, int block_n) {
@@ -864,8 +922,27 @@ int dg_m_grouped_fp8_fp4_gemm_nt_masked(const void *a, const float *sfa, const v
 int dg_debug_bounded_wait(unsigned long long limit_ns, int drop_first_stage) {
     if (limit_ns != 0 && (limit_ns < 1000000ull || limit_ns > dg::WAIT_LIMIT_NS))
         return fail(DG_ERR_INVALID_ARG, "limit_ns=%llu must be 0 or within [1 ms, 2 s]", limit_ns);
-    g_wait_limit_ns = limit_ns == 0 ? dg::WAIT_LIMIT_NS : limit_ns;
-    g_drop_first_stage = drop_first_stage != 0;
+    g_wait_limit_ns.store(limit_ns == 0 ? dg::WAIT_LIMIT_NS : limit_ns);
+    g_drop_first_stage.store(drop_first_stage != 0);
+    return DG_OK;
+}
+
+int dg_debug_clock_record(int enable) {
+    g_clock_record.store(enable != 0);
+    return enable != 0 ? 1 : 0;
+}
+
+int dg_debug_clock_read(unsigned long long *out, int reset) {
+    if (!out) return fail(DG_ERR_INVALID_ARG, "out is null");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    if ((e = cudaMemcpyFromSymbol(out, g_clock_acc, sizeof(g_clock_acc))) != cudaSuccess)
+        return cuda_fail(e, "reading the clock record");
+    if (reset) {
+        const unsigned long long zero[3] = {0, 0, 0};
+        if ((e = cudaMemcpyToSymbol(g_clock_acc, zero, sizeof(zero))) != cudaSuccess)
+            return cuda_fail(e, "clearing the clock record");
+    }
     return DG_OK;
 }
 
@@ -950,15 +1027,16 @@ int dg_k_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const v
 }
 
 int dg_set_fp32_scale_promotion(int enable) {
-    g_fp32_promotion = enable != 0;
-    return g_fp32_promotion ? 1 : 0;
+    g_fp32_promotion.store(enable != 0);
+    return enable != 0 ? 1 : 0;
 }
 
-int dg_get_fp32_scale_promotion(void) { return g_fp32_promotion ? 1 : 0; }
+int dg_get_fp32_scale_promotion(void) { return g_fp32_promotion.load() ? 1 : 0; }
 
 int dg_set_cta_pair_policy(int policy) {
-    g_pair_policy = policy < 0 ? -1 : (policy > 0 ? 1 : 0);
-    return g_pair_policy;
+    const int v = policy < 0 ? -1 : (policy > 0 ? 1 : 0);
+    g_pair_policy.store(v);
+    return v;
 }
 
 int dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void *b, const float *sfb, void *d, int M, int N,

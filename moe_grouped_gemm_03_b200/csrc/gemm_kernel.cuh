@@ -92,7 +92,8 @@ struct GemmParams {
                        // masked / no padding: unused
     int num_n_blocks;  // ceil(N / BN)
     int num_sf_groups; // ceil(K / (128 * SF_GROUP)); K-grouped: the sum over groups of ceil(K_g / (128 * SF_GROUP))
-    int sfa_blocks;    // 128-row blocks per group of the packed SFA (masked layout)
+    int sfa_blocks;    // 128-row blocks per group of the packed SFA (masked layout; swapped operands: of B's rows)
+    int swap_chunks;   // swapped operands: token chunks per group in the packed token-side scales
     int raster_bands;  // dense / K-grouped: row windows per raster group (the tile order); 0: columns first
     __nv_bfloat16 *d;
     float *d32;        // fp32 output (out_mode != OUT_BF16): [G][M][N]
@@ -106,9 +107,11 @@ struct GemmParams {
     const float *sfb32;  // scale of (group g, 128-column block nb, K block kb) at g * sfb_sg + nb * sfb_sn + kb * sfb_sk
     int sfa_ld;
     int sfb_sg, sfb_sn, sfb_sk;
+    // measurement aid (null: off): CTA 0 adds its SM cycles, nanoseconds and 1 to clock_acc[0..2] at exit
+    unsigned long long *clock_acc;
 };
 
-template <int BN_, int CTAS_, int KPS_, bool BF4_ = false, bool PROMO_ = false>
+template <int BN_, int CTAS_, int KPS_, bool BF4_ = false, bool PROMO_ = false, bool SWAP_ = false>
 struct Cfg {
     static constexpr int BN = BN_;
     static constexpr int CTAS = CTAS_;
@@ -122,6 +125,12 @@ struct Cfg {
     // partial * sfa * sfb in registers.  No scale atoms travel with the stages.  BN = 128: a tile's columns are
     // exactly one 128-column block of B's scales.
     static constexpr bool PROMO = PROMO_;
+    // Swapped operands (masked layout): the MMA's M side runs over B's rows (D's columns, TILE_M per tile) and
+    // its N side over up to BN of one group's tokens (D's rows).  The A-side tile of shared memory then holds 128
+    // rows of B and the B-side tile up to BN/CTAS tokens of A; the MMA's N is set per tile to the tile's token
+    // count rounded up to 16, so a group is padded to 16 rows instead of TILE_M.  Same buffers, barriers and
+    // TMEM layout as the unswapped configuration.
+    static constexpr bool SWAP = SWAP_;
     static constexpr int SFB_KB = BF4 ? KPS : 1;                  // K blocks whose B scale atoms a stage holds
     static constexpr int TILE_M = BLOCK_M * CTAS;
     static constexpr int B_ROWS = BN / CTAS;                      // B rows this CTA loads
@@ -162,6 +171,7 @@ struct Cfg {
     static constexpr int SMEM_BYTES = OFF_TILES + 8 * TILE_LIST_CAP + 1024;     // + alignment slack
     static_assert(CTAS == 1 || CTAS == 2, "single CTA or CTA pair");
     static_assert(!PROMO || (BN == 128 && !BF4 && 2 * KPS * BN <= TMEM_COLS), "promotion: 128-wide tiles, e4m3 B");
+    static_assert(!SWAP || (!PROMO && !BF4 && BN % 16 == 0), "swapped operands: block-scaled e4m3 only");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32, 256]");
     static_assert(B_ROWS % 8 == 0, "B tile rows must fill whole 8-row swizzle atoms");
     static_assert(STAGES >= 3, "pipeline too shallow");
@@ -271,6 +281,14 @@ __device__ __forceinline__ int raster_tile(int t, int windows, int nblocks, int 
     return w0 + (local - nb * gm);
 }
 
+// Swapped operands: a group of m tokens is cut into ceil(m / bn) chunks of equal size, rounded up to 16 rows (the
+// MMA's N granularity), so no chunk exceeds bn.  Rows of one chunk: chunk_rows(m, bn); the last may hold fewer.
+__host__ __device__ __forceinline__ int chunk_rows(int m, int bn) {
+    if (m <= 0) return bn;
+    const int chunks = (m + bn - 1) / bn;
+    return ((m + chunks - 1) / chunks + 15) & ~15;
+}
+
 template <class C>
 __device__ __forceinline__ bool decode_tile(const GemmParams &p, const SharedCtl &ctl, int t, Tile &ti) {
     if (p.mode == MODE_DENSE) {
@@ -291,7 +309,14 @@ __device__ __forceinline__ bool decode_tile(const GemmParams &p, const SharedCtl
     }
     const int w = t / p.num_n_blocks;  // window-tile index
     ti.nb = t - w * p.num_n_blocks;
-    ti.n0 = ti.nb * C::BN;
+    ti.n0 = ti.nb * (C::SWAP ? C::TILE_M : C::BN);
+    if constexpr (C::SWAP) {  // masked: window w = one chunk of one group's tokens
+        const int g = upper_index(ctl.prefix, p.G, w);
+        ti.g = g;
+        ti.local_row0 = (w - ctl.prefix[g]) * chunk_rows(ctl.mm[g], C::BN);
+        ti.row0 = g * p.M + ti.local_row0;
+        return true;
+    }
     if (p.mode == MODE_CONTIGUOUS) {
         if constexpr (C::CTAS == 1) {
             ti.row0 = ti.local_row0 = w * BLOCK_M;
@@ -325,7 +350,7 @@ __device__ __forceinline__ bool unpack_tile(const GemmParams &p, const SharedCtl
     if (g1 == 0) return false;
     ti.g = g1 - 1;
     ti.nb = static_cast<int>(e.y >> 16);
-    ti.n0 = ti.nb * C::BN;
+    ti.n0 = ti.nb * (C::SWAP ? C::TILE_M : C::BN);
     ti.row0 = static_cast<int>(e.x);
     if (p.mode == MODE_MASKED)
         ti.local_row0 = ti.row0 - ti.g * p.M;
@@ -462,6 +487,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t rank = PAIR ? cluster_cta_rank() : 0u;
     const int cluster_id = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
     const int num_clusters = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+    const bool clock_rec = p.clock_acc != nullptr && blockIdx.x == 0 && threadIdx.x == 0;
+    const unsigned long long clk0 = clock_rec ? clock64() : 0ull, ns0 = clock_rec ? global_timer_ns() : 0ull;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -536,7 +563,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             __syncwarp();
             build_window_prefix(p.G, SF_GROUP, s_mm, s_prefix, lane);
         } else if (p.mode == MODE_MASKED || p.mode == MODE_NOPAD) {
-            build_window_prefix(p.G, C::TILE_M, s_mm, s_prefix, lane);
+            build_window_prefix(p.G, C::SWAP ? C::BN : C::TILE_M, s_mm, s_prefix, lane);
         } else if (pair_contig) {
             build_pair_windows(num_blocks, s_gblk, s_prefix, lane);
         }
@@ -620,21 +647,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int tile_nkb = kgrouped ? ctl_main.mm[ti.g] : nkb;  // 128-K blocks of this tile
                 const int kbase = kgrouped ? ctl_main.off[ti.g] : 0;      // its first 128-K block
                 const int qbase = kgrouped ? ctl_main.prefix[ti.g] : 0;   // its first packed scale group
-                const int arow = ti.row0 + my_rows;
-                const int brow = gb * p.N + ti.n0 + static_cast<int>(rank) * C::B_ROWS;
-                // packed scale atoms: SFA [block][group], SFB [g][n block][group][atom]
-                // (no padding: atoms of each group's windows, CTAS blocks per window, after the earlier groups')
-                int sfa_block = (ti.local_row0 + my_rows) / BLOCK_M;
-                if (p.mode == MODE_MASKED)
-                    sfa_block += ti.g * p.sfa_blocks;
-                else if (p.mode == MODE_NOPAD)
-                    sfa_block += CTAS * ctl_main.prefix[ti.g];
-                else
-                    sfa_block = (ti.row0 + my_rows) / BLOCK_M;
-                const int sfa_y0 = sfa_block * p.num_sf_groups + qbase;
-                // B scale words along K per tile: one per scale group, or (FP4 B) one per 128-K block
-                const int sfb_words = C::BF4 ? nkb : p.num_sf_groups;
-                const int sfb_y0 = ((gb * p.num_n_blocks + ti.nb) * sfb_words + qbase) * C::SFB_ATOMS;
+                int arow, brow, sfa_y0, sfb_y0;  // rows loaded through tmap_a / tmap_b, first scale atoms
+                if constexpr (C::SWAP) {
+                    // tmap_a covers B's rows (the MMA's M side), tmap_b the tokens (its N side); this CTA brings
+                    // its 128 rows of B and its half of the tile's tokens (the MMA's N rounded to 16, split in two)
+                    const int m = ctl_main.mm[ti.g];
+                    const int cs = chunk_rows(m, C::BN);
+                    const int nmma = (min(cs, m - ti.local_row0) + 15) & ~15;
+                    arow = ti.g * p.N + ti.n0 + my_rows;
+                    brow = ti.row0 + static_cast<int>(rank) * (nmma / CTAS);
+                    // packed scale atoms: B side [g][128-row block of B][group] (every row of an atom holds the
+                    // block's scale), token side [g][chunk][group][atom]
+                    sfa_y0 = (ti.g * p.sfa_blocks + (ti.n0 + my_rows) / BLOCK_M) * p.num_sf_groups;
+                    sfb_y0 = (ti.g * p.swap_chunks + ti.local_row0 / cs) * p.num_sf_groups * C::SFB_ATOMS;
+                } else {
+                    arow = ti.row0 + my_rows;
+                    brow = gb * p.N + ti.n0 + static_cast<int>(rank) * C::B_ROWS;
+                    // packed scale atoms: SFA [block][group], SFB [g][n block][group][atom]
+                    // (no padding: atoms of each group's windows, CTAS blocks per window, after the earlier groups')
+                    int sfa_block = (ti.local_row0 + my_rows) / BLOCK_M;
+                    if (p.mode == MODE_MASKED)
+                        sfa_block += ti.g * p.sfa_blocks;
+                    else if (p.mode == MODE_NOPAD)
+                        sfa_block += CTAS * ctl_main.prefix[ti.g];
+                    else
+                        sfa_block = (ti.row0 + my_rows) / BLOCK_M;
+                    sfa_y0 = sfa_block * p.num_sf_groups + qbase;
+                    // B scale words along K per tile: one per scale group, or (FP4 B) one per 128-K block
+                    const int sfb_words = C::BF4 ? nkb : p.num_sf_groups;
+                    sfb_y0 = ((gb * p.num_n_blocks + ti.nb) * sfb_words + qbase) * C::SFB_ATOMS;
+                }
                 for (int kb0 = 0; kb0 < tile_nkb; kb0 += C::KPS) {
                     // this stage carries scale atoms (the promotion path reads fp32 scales directly)
                     const bool group_start = !C::PROMO && (C::BF4 || kb0 % SF_GROUP == 0);
@@ -740,7 +782,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < p.wait_limit_ns) {
             }
         } else if (!C::PROMO && lane == 0 && rank == 0) {
-            constexpr uint32_t IDESC = idesc_mxf8_e4m3(C::TILE_M, BN, C::BF4);
+            // (swapped operands: N is the tile's token count rounded up to 16, set per tile below)
+            constexpr uint32_t IDESC = idesc_mxf8_e4m3(C::TILE_M, C::SWAP ? 0 : BN, C::BF4);
             int s = 0;
             uint32_t ph = 0;
             int acc = 0;
@@ -754,6 +797,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
                 uint32_t sf_tmem = 0;
+                uint32_t idesc_n = 0;  // N / 8 in bits 17..22 (swapped operands only)
+                if constexpr (C::SWAP) {
+                    const int m = ctl_main.mm[ti.g];
+                    const int nmma = (min(chunk_rows(m, BN), m - ti.local_row0) + 15) & ~15;
+                    idesc_n = static_cast<uint32_t>(nmma >> 3) << 17;
+                }
                 // (K-grouped: a group with no K blocks issues no MMA; its epilogue writes zeros or nothing)
                 const int tile_nkb = p.mode == MODE_KGROUPED ? ctl_main.mm[ti.g] : nkb;
                 for (int kb0 = 0; kb0 < tile_nkb; kb0 += C::KPS) {
@@ -785,7 +834,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                         for (int k = 0; k < BLOCK_K / MMA_K; ++k) {
                             const uint32_t b_byte = C::BF4 ? static_cast<uint32_t>(k) : sub;
-                            const uint32_t idesc = IDESC | (sub << 29) | (b_byte << 4);
+                            const uint32_t idesc = IDESC | idesc_n | (sub << 29) | (b_byte << 4);
                             tc_mma_mxf8<CTAS>(d_tmem, sdesc_kmajor_sw128(a_base + k * MMA_K),
                                               sdesc_kmajor_sw128(b_base + k * MMA_K), idesc, sf_tmem, sf_b,
                                               (kb | k) != 0);
@@ -957,7 +1006,65 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!warp_wait_bounded(&tmem_full[acc], acc_ph, s_abort, p.err, p.wait_limit_ns, lane)) break;
             tc_fence_after_sync();
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * BN);
-            if (p.out_mode != OUT_BF16) {
+            if constexpr (C::SWAP) {
+                // Swapped operands: TMEM lane = a column of D (this CTA's rows of B), TMEM column j = the tile's
+                // token j (row row0 + j of D).  Each 32-token chunk is converted to bf16, turned around with one
+                // exchange between neighbouring lanes (a lane then holds two adjacent columns of one token row),
+                // staged as 32 token rows of 64 bytes (the 64-byte-swizzle box layout) and written by one TMA
+                // store when all 32 tokens belong to the call; the chunk with the tile's last tokens is stored by
+                // the lanes, row by row.
+                const int m = ctl.mm[ti.g];
+                const int cnt = min(chunk_rows(m, BN), m - ti.local_row0);
+                const int col0 = ti.n0 + my_rows + 32 * q;  // this warp's first column of D
+                const bool odd = (lane & 1) != 0;
+                const int pair_col = col0 + (lane & ~1);    // first of the two columns of this lane's words
+                const int cb = 2 * (lane & ~1);             // their byte offset in a 64-byte token row
+#pragma unroll 1
+                for (int c = 0; c < (cnt + 31) / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + 32 * c, r);
+                    tmem_ld_wait_regs(r);
+                    // w[i]: token row 2i (even lane) or 2i + 1 (odd lane), columns pair_col and pair_col + 1
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        __nv_bfloat162 v =
+                            __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                        const uint32_t own = *reinterpret_cast<uint32_t *>(&v);  // this column, tokens 2i, 2i + 1
+                        const uint32_t other = __shfl_xor_sync(0xffffffffu, own, 1);
+                        w[i] = odd ? ((other >> 16) | (own & 0xFFFF0000u)) : ((own & 0xFFFFu) | (other << 16));
+                    }
+                    const int tok0 = 32 * c;
+                    if (tok0 + 32 <= cnt) {
+                        uint8_t *buf = stage_buf + (chunk_count & 1) * EPI_CHUNK_BYTES;
+                        if (chunk_count >= 2) {
+                            if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
+                            __syncwarp();
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int tr = 2 * i + (odd ? 1 : 0);
+                            const int sw = (cb >> 4) ^ ((tr >> 1) & 3);
+                            *reinterpret_cast<uint32_t *>(buf + tr * 64 + sw * 16 + (cb & 15)) = w[i];
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmap_d, buf, col0, ti.row0 + tok0);
+                            bulk_commit_group();
+                        }
+                        ++chunk_count;
+                    } else if (pair_col < p.N) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int tok = tok0 + 2 * i + (odd ? 1 : 0);
+                            if (tok < cnt)
+                                *reinterpret_cast<uint32_t *>(p.d + static_cast<size_t>(ti.row0 + tok) * p.N +
+                                                              pair_col) = w[i];
+                        }
+                    }
+                }
+            } else if (p.out_mode != OUT_BF16) {
                 // fp32 D [G][M][N] through a 3-D map that clips rows past M: per 32-column TMEM load two 16-column
                 // chunks (64-byte rows, the same swizzled staging), each stored or added by one TMA operation.
                 const bool no_k = ctl.mm[ti.g] == 0;  // an empty K range: the accumulator holds nothing
@@ -1037,6 +1144,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_before_sync();
     __syncthreads();
     if constexpr (PAIR) cluster_sync();  // neither CTA leaves while the pair may still touch its memory
+    if (clock_rec) {
+        atomicAdd(p.clock_acc, static_cast<unsigned long long>(clock64()) - clk0);
+        atomicAdd(p.clock_acc + 1, global_timer_ns() - ns0);
+        atomicAdd(p.clock_acc + 2, 1ull);
+    }
     if (warp == 1) {
         __syncwarp();
         tc_fence_after_sync();

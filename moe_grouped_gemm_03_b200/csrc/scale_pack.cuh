@@ -12,6 +12,9 @@
 //   SFB atoms: [g][N tile][group][atom a]   rows a*128 .. a*128+127 of the BN-wide N tile (tile-aligned,
 //                                           so a tile whose start is not a multiple of 128 still gets one
 //                                           word per output column in the right TMEM lane)
+// Swapped operands (masked layout; the MMA's M side runs over B's rows, its N side over a group's tokens):
+//   B-side atoms:     [g][128-row block of B][group]   every row holds the 128x128 block's scale
+//   token-side atoms: [g][chunk][group][atom a]        rows a*128 .. a*128+127 of the chunk's tokens
 // Entries past the problem (rows >= the scale extent, K blocks >= K/128, columns >= N) hold 0x7F (2^0).
 #pragma once
 #include <cstdint>
@@ -40,6 +43,9 @@ struct PackParams {
     int nkb, num_sf_groups;
     const int *m_indices; // contiguous: row -> group (-1 = padding); only rows of a group have their scales checked
     unsigned *err;        // device error word: ERR_BAD_SCALE for a scale the call reads that is not a power of two
+    int swap;             // swapped operands (masked layout): sfa_out holds B's atoms, sfb_out the tokens'
+    int b_blocks;         // swapped: 128-row blocks of B per group in sfa_out (past N: 2^0)
+    int chunks;           // swapped: token chunks per group in sfb_out (chunk size chunk_rows(masked_m, bn))
     uint32_t *sfa_out;    // [sfa_groups * blocks_per_group][num_sf_groups][128]
     uint32_t *sfb_out;    // [G][n_tiles][num_sf_groups][sfb_atoms][128]
     long long sfa_words, sfb_words;
@@ -103,7 +109,54 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
          atom += num_warps) {
         uint32_t word[4] = {0u, 0u, 0u, 0u};
         uint32_t *dst;
-        if (atom < sfa_atoms) {
+        if (p.swap) {
+            if (atom < sfa_atoms) {  // B side: the block scales of 128 rows of B, the same word in every row
+                const int q = static_cast<int>(atom % p.num_sf_groups);
+                const long long rest = atom / p.num_sf_groups;
+                const int blk = static_cast<int>(rest % p.b_blocks);
+                const long long g = rest / p.b_blocks;
+                uint32_t wv = 0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int kb = SF_GROUP * q + i;
+                    const bool in = blk < nnb128 && kb < p.nkb;
+                    const uint32_t bits =
+                        in ? __float_as_uint(__ldg(p.sfb + (g * nnb128 + blk) * p.nkb + kb)) : ONE_F32_BITS;
+                    wv |= ((bits >> 23) & 0xFFu) << (8 * i);
+                    if (in) bad_bits |= ue8m0_inexact_bits(bits);
+                }
+                word[0] = word[1] = word[2] = word[3] = wv;
+                dst = p.sfa_out + atom * SF_ATOM_WORDS;
+            } else {  // token side: the per-row scales of 256 tokens of one chunk of one group
+                const long long b = atom - sfa_atoms;
+                const int a = static_cast<int>(b % p.sfb_atoms);
+                long long rest = b / p.sfb_atoms;
+                const int q = static_cast<int>(rest % p.num_sf_groups);
+                rest /= p.num_sf_groups;
+                const int c = static_cast<int>(rest % p.chunks);
+                const long long g = rest / p.chunks;
+                const int m = min(max(__ldg(p.counts + g), 0), p.rows_per_group);
+                const int cs = chunk_rows(m, p.bn);
+                const float *base = p.sfa + g * p.nkb * p.sfa_ld;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int r = a * 128 + lane + 32 * j;
+                    const long long tok = static_cast<long long>(c) * cs + r;
+                    const bool in = tok < p.sfa_ld;
+                    const bool check = tok < m && r < cs;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int kb = SF_GROUP * q + i;
+                        const uint32_t bits = (in && kb < p.nkb)
+                                                  ? __float_as_uint(__ldg(base + static_cast<size_t>(kb) * p.sfa_ld + tok))
+                                                  : ONE_F32_BITS;
+                        word[j] |= ((bits >> 23) & 0xFFu) << (8 * i);
+                        if (check && kb < p.nkb) bad_bits |= ue8m0_inexact_bits(bits);
+                    }
+                }
+                dst = p.sfb_out + b * SF_ATOM_WORDS;
+            }
+        } else if (atom < sfa_atoms) {
             const int q = static_cast<int>(atom % p.num_sf_groups);
             const long long block = atom / p.num_sf_groups;
             long long group_base = 0;  // masked: the group's scale array

@@ -191,7 +191,7 @@ def quantize_rows(x: np.ndarray):
     nkb = K // SCALE_BLOCK
     xb = x.reshape(R, nkb, SCALE_BLOCK)
     e = pow2_scale_exponent(np.abs(xb).max(axis=2))  # [R, nkb]
-    q = np.ldexp(xb, -e[:, :, None]).astype(np.float32)
+    q = np.ldexp(xb, -e[:, :, None]).astype(np.float32, copy=False)  # exact: a power-of-two scaling
     codes = _to_e4m3_codes(q.reshape(R, K))
     return codes, np.ldexp(np.ones_like(e, dtype=np.float32), e).astype(np.float32)
 
@@ -206,7 +206,7 @@ def quantize_blocks(x: np.ndarray):
     xp = np.pad(x, ((0, pad), (0, 0))) if pad else x
     xb = xp.reshape(nnb, SCALE_BLOCK, nkb, SCALE_BLOCK)
     e = pow2_scale_exponent(np.abs(xb).max(axis=(1, 3)))  # [nnb, nkb]
-    q = np.ldexp(xb, -e[:, None, :, None]).astype(np.float32).reshape(nnb * SCALE_BLOCK, K)[:N]
+    q = np.ldexp(xb, -e[:, None, :, None]).astype(np.float32, copy=False).reshape(nnb * SCALE_BLOCK, K)[:N]
     return _to_e4m3_codes(q), np.ldexp(np.ones_like(e, dtype=np.float32), e).astype(np.float32)
 
 

@@ -85,6 +85,10 @@ def test_contiguous_shapes(counts, N, K, policy):
     (3, 256, 7168, 256, [256, 0, 129]),
     (4, 64, 160, 128, [64, 63, 0, 1]),
     (40, 128, 384, 256, None),
+    # groups cut into several token chunks (a chunk holds at most 224 tokens; 1000 -> 5 chunks of 208 rows),
+    # N not a multiple of 256, a partial scale group along K (5 K blocks)
+    (6, 700, 304, 640, [700, 225, 224, 449, 15, 0]),
+    (2, 1000, 7168, 256, [1000, 31]),
 ])
 def test_masked_shapes(G, M_max, N, K, mm, policy):
     _full_check(synth.make_masked(G, M_max, N, K, masked_m=mm, seed=G + M_max, expected_m=M_max // 2))

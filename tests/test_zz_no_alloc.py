@@ -2,14 +2,18 @@
 
 It exists for callers that may not allocate device memory during a call (for example code running under a
 global-mode stream capture, where allocation calls are refused, or engines whose memory manager owns all of
-device memory).  It must give the same results as dg_fp8_gemm_nt; two calls in a row on different inputs check
-that the shared static buffer holds nothing stale from the previous call.  This file is collected last.
+device memory).  It runs the same kernels on the same tile plan as dg_fp8_gemm_nt, with its packed scales in a
+fixed buffer instead of per-call scratch, so its results must equal dg_fp8_gemm_nt's bit for bit; one call is also
+checked against the oracle.  Calls in a row on different inputs and scales, a large call followed by a small one
+included, check that the shared buffer holds nothing stale from an earlier call.  This file is collected last.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 from _helpers import assert_close, bf16_to_f64
 
@@ -22,20 +26,45 @@ def _call(fn, t, out, p):
               P(out.data_ptr()), p.M, p.N, p.K, P(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("M,N,K", [(512, 2048, 1024), (300, 7168, 384), (4096, 7168, 7168)])
-def test_noalloc_matches_allocating_entry_point_on_two_calls(M, N, K):
+def _both(p):
+    """(allocation-free result, dg_fp8_gemm_nt result) on the same inputs, D pre-filled with NaN bits."""
     import moe_grouped_gemm_03_b200 as dg
 
     L = dg.lib()
+    t = synth.to_torch(p)
+    out = torch.full((p.M, p.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    assert _call(L.dg_fp8_gemm_nt_noalloc, t, out, p) == 0, dg.last_error()
+    ref = torch.full((p.M, p.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    assert _call(L.dg_fp8_gemm_nt, t, ref, p) == 0, dg.last_error()
+    dg.check_device_error()
+    return out, ref
+
+
+def _rescaled(p, ja, jb):
+    """The same problem with every A scale multiplied by 2^ja and every B scale by 2^jb (still powers of two)."""
+    p.sfa = (p.sfa * np.float32(2.0 ** ja)).astype(np.float32)
+    p.sfb = (p.sfb * np.float32(2.0 ** jb)).astype(np.float32)
+    return p
+
+
+@pytest.mark.parametrize("M,N,K", [(512, 2048, 1024), (300, 7168, 384), (4096, 7168, 7168)])
+def test_noalloc_equals_allocating_entry_point_bit_for_bit_on_two_calls(M, N, K):
     for call, seed in enumerate((M + 1, M + 2)):  # two calls in a row, different inputs and scales
         p = synth.make_dense(M, N, K, seed=seed)
-        t = synth.to_torch(p)
-        ref = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
-        assert _call(L.dg_fp8_gemm_nt, t, ref, p) == 0, dg.last_error()
-        out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
-        assert _call(L.dg_fp8_gemm_nt_noalloc, t, out, p) == 0, dg.last_error()
-        dg.check_device_error()
-        assert_close(bf16_to_f64(out), bf16_to_f64(ref), f"call {call} of {M}x{N}x{K}")
+        out, ref = _both(p)
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), f"call {call} of {M}x{N}x{K}"
+
+
+def test_noalloc_large_then_small_call_matches_oracle():
+    """A large call fills much of the shared buffer; the small call after it, with other scales, must read only its
+    own packed scales: bit-identical to dg_fp8_gemm_nt and within the tolerance of the oracle."""
+    big = _rescaled(synth.make_dense(2048, 7168, 4096, seed=31), 2, -3)
+    out, ref = _both(big)
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), "large call"
+    small = _rescaled(synth.make_dense(300, 640, 384, seed=32), -4, 5)
+    out, ref = _both(small)
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), "small call after the large one"
+    assert_close(bf16_to_f64(out), oracle.problem_full(small).reshape(small.M, small.N), "small call vs oracle")
 
 
 def test_noalloc_rejects_shapes_beyond_its_buffer():
