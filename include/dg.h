@@ -37,7 +37,7 @@
  *   - Device-side faults are not expected.  Every wait inside the kernel is bounded; a kernel that gives
  *     up records a code that dg_check_device_error() returns (DG_ERR_DEVICE_TIMEOUT, DG_ERR_BAD_GROUP or
  *     DG_ERR_BAD_SCALE).
- *   - Settings (dg_set_m_alignment_for_contiguous_layout, dg_set_num_sms, dg_set_cta_pair_policy,
+ *   - Settings (dg_set_m_alignment_for_contiguous_layout, dg_set_num_sms, dg_set_cta_pair_policy, dg_set_swap_policy,
  *     dg_set_fp32_scale_promotion, dg_debug_bounded_wait, dg_debug_clock_record) are process-wide, not
  *     per thread or per stream.  Setting one while another thread calls the library is defined (each value is
  *     an atomic) but that call sees whichever value was in force when it read it, so two users of one process
@@ -135,8 +135,10 @@ DG_EXPORT int dg_m_grouped_fp8_gemm_nt_masked(const void *a, const float *sfa, c
  *   Same as dg_m_grouped_fp8_gemm_nt_contiguous except
  *   b [G][K][N] e4m3 (N contiguous) and sfb [G][K/128][ceil(N/128)] (B's 128x128 block scales in B's
  *   orientation): D[m][n] = sum_k A[m][k] * B_g[k][n] with the block scales as in the NT call.
- *   The library transposes B into stream-ordered scratch of G*N*K bytes (one HBM read and write of B) and runs
- *   the NT kernel on it; the scratch is released in stream order when the call's work is done. */
+ *   With swapped-operand tiles (dg_set_swap_policy; used whenever the policy allows and M_total / 128 <= 1024) the
+ *   kernel reads B in place: each K block of 128 of B's columns is loaded as an MN-major tile (128 K-rows of 128
+ *   bytes).  Otherwise the library transposes B into stream-ordered scratch of G*N*K bytes (one HBM read and write
+ *   of B) and runs the NT kernel on it; the scratch is released in stream order when the call's work is done. */
 DG_EXPORT int dg_m_grouped_fp8_gemm_nn_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
                                         void *d, const int *m_indices, int M_total, int N, int K, int G,
                                         dg_stream_t stream);
@@ -228,6 +230,18 @@ DG_EXPORT int dg_get_fp32_scale_promotion(void);
  * fp32 accumulation either way.  Returns the policy now in force.  (README "Optimizations": larger block
  * sizes up to 256x256.) */
 DG_EXPORT int dg_set_cta_pair_policy(int policy);
+
+/* Operand order of the grouped tiles for the next calls on any thread: -1 (default) lets the library choose, 0
+ * never swaps, 1 swaps wherever supported.  Swapped operands put B's rows (D's columns) on the tensor core's M
+ * side and a group's tokens (D's rows) on its N side, which the MMA sizes per tile in steps of 16, so a group of
+ * m tokens costs ceil(m / 16) * 16 rows of MMA work instead of whole 128- or 256-row windows; each tile covers
+ * 256 (CTA pair) or 128 columns of D and up to 224 of one group's tokens.  Supported for the masked, no-padding
+ * and contiguous FP8 calls (the contiguous ones while M_total / 128 <= 1024) with block-scaled (power-of-two)
+ * scales.  The library swaps the masked calls and the NN call, and the no-padding and contiguous calls whose groups
+ * hold at most 512 rows on average or whose N fills 256-wide tiles better than the unswapped tile width.  Results
+ * agree within the tolerance of fp32 accumulation either way.  Returns the policy
+ * now in force.  (README "Grouped GEMMs (masked layout)": decode-time groups of a few tokens.) */
+DG_EXPORT int dg_set_swap_policy(int policy);
 
 /* Testing aid for the bounded waits (no counterpart in the method; it exists so that the timeout path can be
  * exercised without faulting or hanging a GPU).

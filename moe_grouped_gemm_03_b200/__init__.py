@@ -63,6 +63,7 @@ _SIGNATURES = {
     "dg_k_grouped_fp8_gemm_nt_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_set_cta_pair_policy": (_I, [_I]),
+    "dg_set_swap_policy": (_I, [_I]),
     "dg_set_fp32_scale_promotion": (_I, [_I]),
     "dg_get_fp32_scale_promotion": (_I, []),
     "dg_debug_bounded_wait": (_I, [ctypes.c_ulonglong, _I]),
@@ -182,6 +183,12 @@ def select_block_n(num_m_blocks: int, N: int, num_sms: int) -> int:
 def set_cta_pair_policy(policy: int) -> int:
     """-1: library decides; 0: single-CTA 128-row tiles only; 1: 2-CTA 256-row tiles wherever possible."""
     return _lib.dg_set_cta_pair_policy(policy)
+
+
+def set_swap_policy(policy: int) -> int:
+    """-1: library decides; 0: never; 1: swapped operands (B's rows on the MMA's M side, a group's tokens on its
+    N side) wherever supported."""
+    return _lib.dg_set_swap_policy(policy)
 
 
 def set_fp32_scale_promotion(enable: bool) -> bool:

@@ -128,6 +128,22 @@ int make_operand_map_fp4(CUtensorMap &map, const void *base, long long rows, int
     return DG_OK;
 }
 
+// B in the NN orientation, e4m3 [rows = G*K][N] (N contiguous): boxes of 128 columns x 128 K-rows with the 128-byte
+// swizzle, an MN-major operand tile of one 128-K block (8 K-rows per 1024-byte swizzle atom).
+int make_operand_map_nn(CUtensorMap &map, const void *base, long long rows, int N) {
+    EncodeTiledFn encode;
+    if (int rc = get_encode_fn(encode)) return rc;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(dg::BLOCK_M), static_cast<cuuint32_t>(dg::BLOCK_K)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (NN operand) failed (%d)", static_cast<int>(r));
+    return DG_OK;
+}
+
 // D, bf16 row-major [rows][N]: boxes of 32 rows x 32 columns (64-byte rows) with the 64-byte swizzle, the
 // layout the epilogue stages each chunk in.
 int make_output_map(CUtensorMap &map, void *base, long long rows, int N) {
@@ -242,6 +258,7 @@ std::atomic<bool> g_fp32_promotion{false};  // true: any fp32 scales, applied by
 std::atomic<unsigned long long> g_wait_limit_ns{dg::WAIT_LIMIT_NS};  // limit of every in-kernel wait
 std::atomic<bool> g_drop_first_stage{false};  // testing aid: the next GEMM launch leaves one stage unloaded
 std::atomic<bool> g_clock_record{false};      // measurement aid: launches add their clock record
+std::atomic<int> g_swap_policy{-1};  // -1: library decides; 0: never swapped operands; 1: wherever supported
 
 // Device address of a __device__ symbol of this library (given by its host-side stand-in) on the current
 // device, looked up once per device with that device current.
@@ -297,10 +314,10 @@ int launch_pack(const dg::PackParams &pk, int device, cudaStream_t stream) {
     return DG_OK;
 }
 
-template <int BN, int CTAS, int KPS, bool BF4 = false, bool SWAP = false>
+template <int BN, int CTAS, int KPS, bool BF4 = false, bool SWAP = false, bool BNN = false>
 int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows, const ScaleArgs &sc, dg::GemmParams p,
                int grid, int device, cudaStream_t stream) {
-    using C = dg::Cfg<BN, CTAS, KPS, BF4, false, SWAP>;
+    using C = dg::Cfg<BN, CTAS, KPS, BF4, false, SWAP, BNN>;
     // ---- packed scale atoms (pre-pass)
     const int nkb = p.K / dg::BLOCK_K;
     dg::PackParams pk{};
@@ -343,13 +360,13 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
     long long sfa_atoms = static_cast<long long>(pk.sfa_groups) * pk.blocks_per_group * p.num_sf_groups;
     const long long b_groups = p.mode == dg::MODE_KGROUPED ? 1 : p.G;  // K-grouped: one B for all groups
     long long sfb_atoms = b_groups * p.num_n_blocks * pk.sfb_kwords * C::SFB_ATOMS;
-    if (SWAP) {  // B-side atoms per 128-row block of B, token-side atoms per chunk of each group
+    if (SWAP) {  // B-side atoms per 128-row block of B, token-side atoms per chunk (all groups' chunks in order)
         pk.swap = 1;
         pk.b_blocks = p.sfa_blocks;
         pk.chunks = p.swap_chunks;
         pk.rows_per_group = p.M;
         sfa_atoms = static_cast<long long>(p.G) * p.sfa_blocks * p.num_sf_groups;
-        sfb_atoms = static_cast<long long>(p.G) * p.swap_chunks * p.num_sf_groups * C::SFB_ATOMS;
+        sfb_atoms = static_cast<long long>(p.swap_chunks) * p.num_sf_groups * C::SFB_ATOMS;
     }
     pk.sfa_words = sfa_atoms * dg::SF_ATOM_WORDS;
     pk.sfb_words = sfb_atoms * dg::SF_ATOM_WORDS;
@@ -383,7 +400,11 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
             rc = make_output_map_f32(td, p.d32, p.G, p.M, p.N);
         if (rc) break;
         // (swapped operands: the 128-row boxes of the MMA's M side come from B, the N side's from A)
-        if ((rc = make_operand_map(ta, SWAP ? b : a, SWAP ? b_rows : a_rows, p.K, dg::BLOCK_M))) break;
+        if (BNN)  // (b_rows = G * K rows of N bytes)
+            rc = make_operand_map_nn(ta, b, b_rows, p.N);
+        else
+            rc = make_operand_map(ta, SWAP ? b : a, SWAP ? b_rows : a_rows, p.K, dg::BLOCK_M);
+        if (rc) break;
         if (BF4)
             rc = make_operand_map_fp4(tb, b, b_rows, p.K, C::B_ROWS);
         else
@@ -658,6 +679,67 @@ int check_common(const void *a, const float *sfa, const void *b, const float *sf
 
 namespace {
 
+// Swapped operands (masked, no-padding and contiguous layouts, e4m3 B, block-scaled): tiles of TILE_M rows of B
+// (D's columns) x one chunk of at most kSwapTokens of a group's tokens (D's rows), the MMA's N set per tile to the
+// chunk's rows rounded up to 16, so a group of m tokens costs ceil(m / 16) * 16 rows of MMA work instead of whole
+// 128-row windows.  hint_chunks: the chunks the caller expects (picks single CTAs or pairs); max_chunks: the most the
+// device can find (sizes the grid and the packed scales).
+constexpr int kSwapTokens = 224;
+constexpr int kSwapDefaultRows = 512;  // contiguous / no padding: swapped by default up to this mean group size
+
+int select_block_n(long long windows, int N, int units, int ctas);
+
+// The library's default for the contiguous and no-padding layouts (measured, interleaved in one process): the
+// swapped tiles pay where groups are small (a group costs its rows rounded up to 16 instead of whole 256-row
+// windows) or where the unswapped plan's tile width leaves part of its last column block empty and 256-wide swapped
+// tiles do not (N = 4096: 19 blocks of 224 columns hold 4256; 0.984 of the unswapped time on G=8, K=7168).  With
+// large groups and N a multiple of both widths they measured 1.03-1.04x slower (G=64, N=7168, K=2048: every group
+// ends in a partial chunk, and a tile loads its whole 224-token box whatever its width).
+bool swap_by_default(long long M_total, int G, int N, int sms) {
+    if (M_total <= static_cast<long long>(G) * kSwapDefaultRows) return true;
+    const long long windows = (M_total + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M);
+    const int bn = select_block_n(windows, N, sms / 2 > 0 ? sms / 2 : 1, 2);
+    const double unswapped = static_cast<double>(N) / (static_cast<double>((N + bn - 1) / bn) * bn);
+    const double swapped = static_cast<double>(N) / (static_cast<double>((N + 255) / 256) * 256);
+    return swapped >= unswapped + 0.02;
+}
+
+// Swapped operands for this call?  by_default: the library's own choice for the layout and shape.
+bool swap_enabled(bool by_default) {
+    if (g_fp32_promotion.load()) return false;
+    const int policy = g_swap_policy.load();
+    return policy < 0 ? by_default : policy > 0;
+}
+
+int launch_swapped(dg::GemmParams p, const DeviceInfo &info, const void *a, long long a_rows, const void *b,
+                   long long b_rows, ScaleArgs sc, long long hint_chunks, long long max_chunks, cudaStream_t stream,
+                   bool b_nn = false) {
+    const int sms = effective_sms(info);
+    const int policy = g_pair_policy.load();
+    bool pair = sms >= 2 && policy != 0;
+    if (pair && policy < 0)  // pairs pay once there is at least a wave of them
+        pair = hint_chunks * ((p.N + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M)) >= sms / 2;
+    const int tile_m = pair ? 2 * dg::BLOCK_M : dg::BLOCK_M;
+    p.num_n_blocks = (p.N + tile_m - 1) / tile_m;
+    p.sfa_blocks = p.num_n_blocks * (pair ? 2 : 1);
+    if (max_chunks > 0x7fffffffLL / 16) return fail(DG_ERR_INVALID_ARG, "too many token chunks");
+    p.swap_chunks = static_cast<int>(max_chunks);
+    p.num_windows = 0;
+    p.num_sf_groups = (p.K / dg::BLOCK_K + dg::SF_GROUP - 1) / dg::SF_GROUP;
+    sc.swap = true;
+    const long long tiles = max_chunks * p.num_n_blocks;
+    const int units = pair ? sms / 2 : sms;
+    const int grid = static_cast<int>(tiles < units ? tiles : units);
+    if (grid <= 0) return DG_OK;
+    if (b_nn) {  // B [G][K][N] read as MN-major tiles, no transposed copy
+        if (pair)
+            return launch_cfg<kSwapTokens, 2, 2, false, true, true>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
+        return launch_cfg<kSwapTokens, 1, 1, false, true, true>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
+    }
+    if (pair) return launch_cfg<kSwapTokens, 2, 2, false, true>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
+    return launch_cfg<kSwapTokens, 1, 1, false, true>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
+}
+
 int check_contiguous(const void *a, const float *sfa, const void *b, const float *sfb, const void *d,
                      const int *m_indices, int M_total, int N, int K, int G) {
     if (int rc = check_common(a, sfa, b, sfb, d, N, K)) return rc;
@@ -675,7 +757,7 @@ int check_contiguous(const void *a, const float *sfa, const void *b, const float
 // The contiguous GEMM on checked arguments (M_total > 0); `sfb_kn` selects the NN orientation of SFB.
 int launch_contiguous(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
                       const int *m_indices, int M_total, int N, int K, int G, bool sfb_kn, const DeviceInfo &info,
-                      cudaStream_t stream, bool b_fp4 = false) {
+                      cudaStream_t stream, bool b_fp4 = false, bool b_nn = false) {
     dg::GemmParams p{};
     p.mode = dg::MODE_CONTIGUOUS;
     p.M = M_total; p.N = N; p.K = K; p.G = G;
@@ -688,6 +770,15 @@ int launch_contiguous(const void *a, const float *sfa, const void *b, const floa
     p.err = device_error_word();
     if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
     const long long w1 = M_total / dg::BLOCK_M, w2 = (w1 + 1) / 2;
+    // Swapped operands while the device's tables hold every 128-row block: runs of blocks of one group, each cut
+    // into token chunks; at most ceil(M_total / kSwapTokens) full chunks plus one partial chunk per run.
+    // b_nn: B is [G][K][N], read directly by the swapped tiles (the caller has checked they apply)
+    if (b_nn || (!b_fp4 && swap_enabled(swap_by_default(M_total, G, N, effective_sms(info))) &&
+                 w1 <= dg::MAX_MASKED_GROUPS)) {
+        const long long full = (M_total + kSwapTokens - 1) / kSwapTokens;
+        return launch_swapped(p, info, a, M_total, b, static_cast<long long>(G) * (b_nn ? K : N), sc,
+                              full + (G < w1 ? G : w1) / 2, full + w1, stream, b_nn);
+    }
     // a 256-row window holds at most two tiles (its halves may belong to two groups)
     const long long bound = w2 + (w2 < G ? w2 : G);
     // pairs need the device-built window list to fit (at most NB/2 + G/2 windows) and group ids below 2^15
@@ -750,32 +841,10 @@ int masked_call(const void *a, const float *sfa, const void *b, const float *sfb
     p.err = device_error_word();
     if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
     const int hint = expected_m > 0 && expected_m < M_max ? expected_m : M_max;
-    static const bool swap_off = getenv("DG_MASKED_SWAP") && getenv("DG_MASKED_SWAP")[0] == '0';  // A/B timing
-    if (!b_fp4 && !g_fp32_promotion.load() && !swap_off) {
-        // Swapped operands: tiles of TILE_M rows of B x one chunk (at most kSwapTokens) of a group's tokens; a
-        // group of m tokens costs ceil(m / 16) * 16 rows of MMA work instead of whole 128-row blocks.
-        constexpr int kSwapTokens = 224;
-        const int sms = effective_sms(info);
-        const long long chunks_max = (M_max + kSwapTokens - 1) / kSwapTokens;
-        const long long hint_chunks = (hint + kSwapTokens - 1) / kSwapTokens;
-        const int policy = g_pair_policy.load();
-        bool pair = sms >= 2 && policy != 0;
-        if (pair && policy < 0)  // pairs pay once there is at least a wave of them
-            pair = static_cast<long long>(G) * hint_chunks * ((N + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M)) >= sms / 2;
-        const int tile_m = pair ? 2 * dg::BLOCK_M : dg::BLOCK_M;
-        p.num_n_blocks = (N + tile_m - 1) / tile_m;
-        p.sfa_blocks = p.num_n_blocks * (pair ? 2 : 1);
-        p.swap_chunks = static_cast<int>(chunks_max);
-        p.num_windows = 0;
-        p.num_sf_groups = (K / dg::BLOCK_K + dg::SF_GROUP - 1) / dg::SF_GROUP;
-        sc.swap = true;
-        const long long tiles = static_cast<long long>(G) * chunks_max * p.num_n_blocks;
-        const int units = pair ? sms / 2 : sms;
-        const int grid = static_cast<int>(tiles < units ? tiles : units);
-        const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-        const long long a_rows = static_cast<long long>(G) * M_max, b_rows = static_cast<long long>(G) * N;
-        if (pair) return launch_cfg<kSwapTokens, 2, 2, false, true>(a, a_rows, b, b_rows, sc, p, grid, info.device, s);
-        return launch_cfg<kSwapTokens, 1, 1, false, true>(a, a_rows, b, b_rows, sc, p, grid, info.device, s);
+    if (!b_fp4 && swap_enabled(true)) {
+        const long long per = (M_max + kSwapTokens - 1) / kSwapTokens, hint_per = (hint + kSwapTokens - 1) / kSwapTokens;
+        return launch_swapped(p, info, a, static_cast<long long>(G) * M_max, b, static_cast<long long>(G) * N, sc,
+                              G * hint_per, G * per, reinterpret_cast<cudaStream_t>(stream));
     }
     // tile shape from the caller's hint; the grid from the most tiles masked_m could ask for
     const long long h1 = static_cast<long long>(G) * ((hint + dg::BLOCK_M - 1) / dg::BLOCK_M);
@@ -885,7 +954,10 @@ int dg_m_grouped_fp8_gemm_nn_contiguous(const void *a, const float *sfa, const v
     DeviceInfo info;
     if (int rc = device_info(info)) return rc;
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // B [G][K][N] -> K-major [G][N][K] in stream-ordered scratch, then the NT path
+    // Swapped-operand tiles read B [G][K][N] as MN-major tiles: no transposed copy
+    if (swap_enabled(true) && M_total / dg::BLOCK_M <= dg::MAX_MASKED_GROUPS)
+        return launch_contiguous(a, sfa, b, sfb, d, m_indices, M_total, N, K, G, true, info, s, false, true);
+    // Otherwise B [G][K][N] -> K-major [G][N][K] in stream-ordered scratch, then the NT path
     cudaMemPool_t pool;
     if (int rc = scratch_pool(info.device, pool)) return rc;
     const size_t bytes = static_cast<size_t>(G) * N * K;
@@ -961,11 +1033,18 @@ int dg_m_grouped_fp8_gemm_nt_nopad(const void *a, const float *sfa, const void *
     dg::GemmParams p{};
     p.mode = dg::MODE_NOPAD;
     p.M = M_total; p.N = N; p.K = K; p.G = G;
-    const ScaleArgs sc{sfa, dg_get_tma_aligned_size(M_total, 4), sfb};
+    ScaleArgs sc{sfa, dg_get_tma_aligned_size(M_total, 4), sfb};
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.masked_m = counts;
     p.err = device_error_word();
     if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");
+    // chunks: each group adds at most one partial chunk to ceil(M_total / kSwapTokens) (by default only for small
+    // groups, as for the contiguous layout)
+    if (swap_enabled(swap_by_default(M_total, G, N, effective_sms(info)))) {
+        const long long full = (M_total + kSwapTokens - 1) / kSwapTokens;
+        return launch_swapped(p, info, a, M_total, b, static_cast<long long>(G) * N, sc, full + G / 2, full + G,
+                              reinterpret_cast<cudaStream_t>(stream));
+    }
     // Windows: each group adds at most one partial window to ceil(M_total / rows per window); the tile shape
     // is chosen for half a partial window per group.
     const long long w1 = (M_total + dg::BLOCK_M - 1) / dg::BLOCK_M, w2 = (M_total + 2 * dg::BLOCK_M - 1) / (2 * dg::BLOCK_M);
@@ -1032,6 +1111,12 @@ int dg_set_fp32_scale_promotion(int enable) {
 }
 
 int dg_get_fp32_scale_promotion(void) { return g_fp32_promotion.load() ? 1 : 0; }
+
+int dg_set_swap_policy(int policy) {
+    const int v = policy < 0 ? -1 : (policy > 0 ? 1 : 0);
+    g_swap_policy.store(v);
+    return v;
+}
 
 int dg_set_cta_pair_policy(int policy) {
     const int v = policy < 0 ? -1 : (policy > 0 ? 1 : 0);

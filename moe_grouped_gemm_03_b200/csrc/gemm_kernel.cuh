@@ -93,7 +93,7 @@ struct GemmParams {
     int num_n_blocks;  // ceil(N / BN)
     int num_sf_groups; // ceil(K / (128 * SF_GROUP)); K-grouped: the sum over groups of ceil(K_g / (128 * SF_GROUP))
     int sfa_blocks;    // 128-row blocks per group of the packed SFA (masked layout; swapped operands: of B's rows)
-    int swap_chunks;   // swapped operands: token chunks per group in the packed token-side scales
+    int swap_chunks;   // swapped operands: token chunks (all groups) the packed token-side scales have room for
     int raster_bands;  // dense / K-grouped: row windows per raster group (the tile order); 0: columns first
     __nv_bfloat16 *d;
     float *d32;        // fp32 output (out_mode != OUT_BF16): [G][M][N]
@@ -111,7 +111,8 @@ struct GemmParams {
     unsigned long long *clock_acc;
 };
 
-template <int BN_, int CTAS_, int KPS_, bool BF4_ = false, bool PROMO_ = false, bool SWAP_ = false>
+template <int BN_, int CTAS_, int KPS_, bool BF4_ = false, bool PROMO_ = false, bool SWAP_ = false,
+          bool BNN_ = false>
 struct Cfg {
     static constexpr int BN = BN_;
     static constexpr int CTAS = CTAS_;
@@ -131,6 +132,10 @@ struct Cfg {
     // count rounded up to 16, so a group is padded to 16 rows instead of TILE_M.  Same buffers, barriers and
     // TMEM layout as the unswapped configuration.
     static constexpr bool SWAP = SWAP_;
+    // With swapped operands, B in the NN orientation ([G][K][N], N contiguous): each K block of the M-side tile is
+    // loaded as 128 K-rows of 128 N-bytes, an MN-major operand (the 128-byte swizzle atom of 8 K-rows x 128 B), so
+    // no transposed copy of B is made.
+    static constexpr bool BNN = BNN_;
     static constexpr int SFB_KB = BF4 ? KPS : 1;                  // K blocks whose B scale atoms a stage holds
     static constexpr int TILE_M = BLOCK_M * CTAS;
     static constexpr int B_ROWS = BN / CTAS;                      // B rows this CTA loads
@@ -153,8 +158,8 @@ struct Cfg {
     static constexpr int TABLE_INTS =
         MAX_PAIR_WINDOWS + 1 > 2 * (MAX_MASKED_GROUPS + 1) ? MAX_PAIR_WINDOWS + 1 : 2 * (MAX_MASKED_GROUPS + 1);
     static constexpr int EPI_BYTES = 4 * 2 * EPI_CHUNK_BYTES;    // per epilogue warp: two staging chunks
-    static constexpr int FIXED_BYTES =
-        EPI_BYTES + 4 * TABLE_INTS + 4 * MAX_MASKED_GROUPS + 16 + 8 * TILE_LIST_CAP + 16 + 8 * 16 + 1024;
+    static constexpr int FIXED_BYTES = EPI_BYTES + 4 * TABLE_INTS + 4 * MAX_MASKED_GROUPS + 2 * MAX_MASKED_GROUPS + 16 +
+                                       8 * TILE_LIST_CAP + 16 + 8 * 16 + 1024;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES - 8 * 2 * 8) / STAGE_BYTES;
     static constexpr int STAGES_MAX = STAGES_FIT;
     static constexpr int STAGES = STAGES_MAX > 8 ? 8 : STAGES_MAX;
@@ -167,11 +172,13 @@ struct Cfg {
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARRIERS * 8;   // tmem base, abort flag
     static constexpr int OFF_PREFIX = OFF_MISC + 16;               // int[TABLE_INTS]
     static constexpr int OFF_MM = OFF_PREFIX + 4 * TABLE_INTS;     // masked: clamped masked_m
-    static constexpr int OFF_TILES = (OFF_MM + 4 * MAX_MASKED_GROUPS + 15) / 16 * 16;  // uint2[TILE_LIST_CAP]
+    static constexpr int OFF_RG = OFF_MM + 4 * MAX_MASKED_GROUPS;  // short[]: group of each run (contiguous, swapped)
+    static constexpr int OFF_TILES = (OFF_RG + 2 * MAX_MASKED_GROUPS + 15) / 16 * 16;  // uint2[TILE_LIST_CAP]
     static constexpr int SMEM_BYTES = OFF_TILES + 8 * TILE_LIST_CAP + 1024;     // + alignment slack
     static_assert(CTAS == 1 || CTAS == 2, "single CTA or CTA pair");
     static_assert(!PROMO || (BN == 128 && !BF4 && 2 * KPS * BN <= TMEM_COLS), "promotion: 128-wide tiles, e4m3 B");
     static_assert(!SWAP || (!PROMO && !BF4 && BN % 16 == 0), "swapped operands: block-scaled e4m3 only");
+    static_assert(!BNN || SWAP, "B in the NN orientation is read through swapped operands");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32, 256]");
     static_assert(B_ROWS % 8 == 0, "B tile rows must fill whole 8-row swizzle atoms");
     static_assert(STAGES >= 3, "pipeline too shallow");
@@ -195,10 +202,15 @@ struct Tile {
 struct SharedCtl {
     volatile int *abort;
     const int *prefix;   // masked / no padding: window prefix per group; contiguous pairs: first block of each
-                         // window; K-grouped: first packed scale group of each group
-    const int *mm;       // masked / no padding: the groups' clamped row counts; K-grouped: 128-K blocks per group
-    const int *off;      // no padding: first row of each group; K-grouped: first 128-K block of each group
+                         // window; K-grouped: first packed scale group of each group; swapped operands: chunk
+                         // prefix per group (contiguous: per run)
+    const int *mm;       // masked / no padding: the groups' clamped row counts; K-grouped: 128-K blocks per group;
+                         // contiguous with swapped operands: rows of each run
+    const int *off;      // no padding: first row of each group; K-grouped: first 128-K block of each group;
+                         // contiguous with swapped operands: first row of each run
     const short *gblk;   // contiguous pairs, kernel prologue only: group of each 128-row block
+    const short *rg;     // contiguous with swapped operands: group of each run
+    int ntab;            // entries of prefix / mm / off: G, or the runs (contiguous with swapped operands)
 };
 
 __device__ __forceinline__ void raise_error(unsigned *err, unsigned code) { atomicCAS(err, 0u, code); }
@@ -310,11 +322,11 @@ __device__ __forceinline__ bool decode_tile(const GemmParams &p, const SharedCtl
     const int w = t / p.num_n_blocks;  // window-tile index
     ti.nb = t - w * p.num_n_blocks;
     ti.n0 = ti.nb * (C::SWAP ? C::TILE_M : C::BN);
-    if constexpr (C::SWAP) {  // masked: window w = one chunk of one group's tokens
-        const int g = upper_index(ctl.prefix, p.G, w);
+    if constexpr (C::SWAP) {  // window w = one chunk of one group's (contiguous: one run's) tokens
+        const int g = upper_index(ctl.prefix, ctl.ntab, w);
         ti.g = g;
         ti.local_row0 = (w - ctl.prefix[g]) * chunk_rows(ctl.mm[g], C::BN);
-        ti.row0 = g * p.M + ti.local_row0;
+        ti.row0 = (p.mode == MODE_MASKED ? g * p.M : ctl.off[g]) + ti.local_row0;
         return true;
     }
     if (p.mode == MODE_CONTIGUOUS) {
@@ -354,7 +366,7 @@ __device__ __forceinline__ bool unpack_tile(const GemmParams &p, const SharedCtl
     ti.row0 = static_cast<int>(e.x);
     if (p.mode == MODE_MASKED)
         ti.local_row0 = ti.row0 - ti.g * p.M;
-    else if (p.mode == MODE_NOPAD)
+    else if (p.mode == MODE_NOPAD || (C::SWAP && p.mode == MODE_CONTIGUOUS))
         ti.local_row0 = ti.row0 - ctl.off[ti.g];
     else
         ti.local_row0 = ti.row0;
@@ -454,6 +466,61 @@ __device__ void build_pair_windows(int num_blocks, const short *gblk, int *list,
     if (lane == 0) list[MAX_PAIR_WINDOWS] = min(total, MAX_PAIR_WINDOWS);
 }
 
+// Contiguous layout with swapped operands, step 1 (one warp; gblk[b] = the group of 128-row block b or -1): runs of
+// consecutive blocks of one group.  off[r] = run r's first block, mm[r] = its last block, rg[r] = its group, in row
+// order; returns the run count (at most num_blocks).
+__device__ int build_run_heads(int num_blocks, const short *gblk, int *off, int *mm, short *rg, int lane) {
+    const int chunk = (num_blocks + 31) / 32;
+    const int begin = min(lane * chunk, num_blocks), end = min(begin + chunk, num_blocks);
+    auto head = [&](int b) { return gblk[b] >= 0 && (b == 0 || gblk[b - 1] != gblk[b]); };
+    auto tail = [&](int b) { return gblk[b] >= 0 && (b + 1 == num_blocks || gblk[b + 1] != gblk[b]); };
+    int nh = 0, nt = 0;
+    for (int b = begin; b < end; ++b) {
+        nh += head(b) ? 1 : 0;
+        nt += tail(b) ? 1 : 0;
+    }
+    int runs, tails;
+    int ph = warp_exclusive_sum(nh, lane, &runs);
+    int pt = warp_exclusive_sum(nt, lane, &tails);
+    for (int b = begin; b < end; ++b) {
+        if (head(b)) {
+            off[ph] = b;
+            rg[ph] = gblk[b];
+            ++ph;
+        }
+        if (tail(b)) mm[pt++] = b;
+    }
+    return runs;
+}
+
+// Step 2 (warp `warp` of `nwarps`, after step 1): run r's rows go from its first block's first row to the last row
+// of its last block that belongs to its group (the layout pads a segment at its end); off[r] becomes that first row
+// and mm[r] the row count.  Rows inside the run that belong to no group are computed and never stored.
+__device__ void finish_runs(const int *m_indices, int M, int runs, int *off, int *mm, const short *rg, int warp,
+                            int nwarps, int lane) {
+    for (int r = warp; r < runs; r += nwarps) {
+        const int last_blk = mm[r], first_blk = off[r], g = rg[r];
+        const int base = last_blk * BLOCK_M;
+        int v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int row = base + 32 * j + lane;
+            v[j] = row < M ? __ldg(m_indices + row) : -1;
+        }
+        int last = 0;  // the block's first row belongs to g, so some row does
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const unsigned bal = __ballot_sync(0xffffffffu, v[j] == g);
+            if (bal) last = 32 * j + 31 - __clz(bal);
+        }
+        __syncwarp();
+        if (lane == 0) {
+            off[r] = first_blk * BLOCK_M;
+            mm[r] = (last_blk - first_blk) * BLOCK_M + last + 1;
+        }
+    }
+}
+
 template <class C>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -516,8 +583,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // Scheduler tables.  Loads first, by all threads (independent loads in flight together), into shared
     // memory: masked_m, or the group of every 128-row block (staged in the A ring, unused until the producer
     // starts); then one warp scans them.
-    const bool pair_contig = PAIR && p.mode == MODE_CONTIGUOUS;
+    const bool pair_contig = PAIR && p.mode == MODE_CONTIGUOUS && !C::SWAP;
+    const bool swap_contig = C::SWAP && p.mode == MODE_CONTIGUOUS;
     short *s_gblk = reinterpret_cast<short *>(sA);
+    short *s_rg = reinterpret_cast<short *>(smem + C::OFF_RG);
+    int *s_ntab = reinterpret_cast<int *>(smem + C::OFF_MISC + 8);
     const int num_blocks = p.M / BLOCK_M;
     if (p.mode == MODE_MASKED || p.mode == MODE_NOPAD) {
         for (int g = threadIdx.x; g < p.G; g += NUM_THREADS) {
@@ -534,7 +604,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (k < 0 || k % BLOCK_K) raise_error(p.err, ERR_BAD_GROUP);
             s_mm[g] = k < 0 ? 0 : k / BLOCK_K;
         }
-    } else if (pair_contig) {
+    } else if (pair_contig || swap_contig) {
         // several independent loads in flight per thread (m_indices is usually cold in L2 here)
         constexpr int U = 8;
         for (int b0 = threadIdx.x; b0 < num_blocks; b0 += NUM_THREADS * U) {
@@ -566,7 +636,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             build_window_prefix(p.G, C::SWAP ? C::BN : C::TILE_M, s_mm, s_prefix, lane);
         } else if (pair_contig) {
             build_pair_windows(num_blocks, s_gblk, s_prefix, lane);
+        } else if (swap_contig) {
+            const int runs = build_run_heads(num_blocks, s_gblk, s_off, s_mm, s_rg, lane);
+            if (lane == 0) *s_ntab = runs;
         }
+        if (!swap_contig && lane == 0) *s_ntab = p.G;
+    }
+    if (swap_contig) {  // the runs' row ranges (every warp), then their chunk prefix
+        __syncthreads();
+        finish_runs(p.m_indices, p.M, *s_ntab, s_off, s_mm, s_rg, warp, NUM_THREADS / 32, lane);
+        __syncthreads();
+        if (warp == EPI_WARP0) build_window_prefix(*s_ntab, C::BN, s_mm, s_prefix, lane);
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -574,11 +654,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after_sync();
     const uint32_t tmem_base = *s_tmem_base;
 
-    const SharedCtl ctl{s_abort, s_prefix, s_mm, s_off, s_gblk};
+    const int ntab = *s_ntab;
+    const SharedCtl ctl{s_abort, s_prefix, s_mm, s_off, s_gblk, s_rg, ntab};
     const int nkb = p.K / BLOCK_K;
     int total_windows;
-    if (p.mode == MODE_MASKED || p.mode == MODE_NOPAD)
-        total_windows = s_prefix[p.G];
+    if (p.mode == MODE_MASKED || p.mode == MODE_NOPAD || swap_contig)
+        total_windows = s_prefix[ntab];
     else if (pair_contig)
         total_windows = s_prefix[MAX_PAIR_WINDOWS];
     else
@@ -595,7 +676,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         s_tiles[k] = pack_tile(valid, ti);
     }
     __syncthreads();
-    const SharedCtl ctl_main{s_abort, s_prefix, s_mm, s_off, nullptr};  // the A ring is operand data from here on
+    const SharedCtl ctl_main{s_abort, s_prefix, s_mm, s_off, nullptr, s_rg, ntab};  // the A ring holds operands now
     auto tile_at = [&](int k, Tile &ti) -> bool {
         if (k < TILE_LIST_CAP) return unpack_tile<C>(p, ctl_main, s_tiles[k], ti);
         return decode_tile<C>(p, ctl_main, cluster_id + k * num_clusters, ti);
@@ -648,18 +729,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int kbase = kgrouped ? ctl_main.off[ti.g] : 0;      // its first 128-K block
                 const int qbase = kgrouped ? ctl_main.prefix[ti.g] : 0;   // its first packed scale group
                 int arow, brow, sfa_y0, sfb_y0;  // rows loaded through tmap_a / tmap_b, first scale atoms
+                int a_k_rows = 0;  // B in the NN orientation: the first K row of the group in tmap_a (rows G*K)
                 if constexpr (C::SWAP) {
                     // tmap_a covers B's rows (the MMA's M side), tmap_b the tokens (its N side); this CTA brings
                     // its 128 rows of B and its half of the tile's tokens (the MMA's N rounded to 16, split in two)
                     const int m = ctl_main.mm[ti.g];
                     const int cs = chunk_rows(m, C::BN);
                     const int nmma = (min(cs, m - ti.local_row0) + 15) & ~15;
-                    arow = ti.g * p.N + ti.n0 + my_rows;
+                    const int gB = swap_contig ? ctl_main.rg[ti.g] : ti.g;  // (contiguous: ti.g is a run)
+                    arow = gB * p.N + ti.n0 + my_rows;
+                    a_k_rows = gB * p.K;
                     brow = ti.row0 + static_cast<int>(rank) * (nmma / CTAS);
                     // packed scale atoms: B side [g][128-row block of B][group] (every row of an atom holds the
-                    // block's scale), token side [g][chunk][group][atom]
-                    sfa_y0 = (ti.g * p.sfa_blocks + (ti.n0 + my_rows) / BLOCK_M) * p.num_sf_groups;
-                    sfb_y0 = (ti.g * p.swap_chunks + ti.local_row0 / cs) * p.num_sf_groups * C::SFB_ATOMS;
+                    // block's scale), token side [chunk][group][atom] over all groups' chunks in order
+                    sfa_y0 = (gB * p.sfa_blocks + (ti.n0 + my_rows) / BLOCK_M) * p.num_sf_groups;
+                    sfb_y0 = (ctl_main.prefix[ti.g] + ti.local_row0 / cs) * p.num_sf_groups * C::SFB_ATOMS;
                 } else {
                     arow = ti.row0 + my_rows;
                     brow = gb * p.N + ti.n0 + static_cast<int>(rank) * C::B_ROWS;
@@ -696,14 +780,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         if (rank == 0) mbar_arrive_expect_tx(&full[s], CTAS * bytes);
                         for (int i = 0; i < nk; ++i) {
                             const int x = (kbase + kb0 + i) * BLOCK_K;
-                            tma_load_2d_pair(a_dst + i * C::A_BYTES1, &tmap_a, leader_full, x, arow);
+                            if constexpr (C::BNN)  // 128 N columns x 128 K rows of B [G*K][N]
+                                tma_load_2d_pair(a_dst + i * C::A_BYTES1, &tmap_a, leader_full, ti.n0 + my_rows,
+                                                 a_k_rows + x);
+                            else
+                                tma_load_2d_pair(a_dst + i * C::A_BYTES1, &tmap_a, leader_full, x, arow);
                             tma_load_2d_pair(b_dst + i * C::B_BYTES1, &tmap_b, leader_full, x, brow);
                         }
                     } else {
                         mbar_arrive_expect_tx(&full[s], bytes);
                         for (int i = 0; i < nk; ++i) {
                             const int x = (kbase + kb0 + i) * BLOCK_K;
-                            tma_load_2d(a_dst + i * C::A_BYTES1, &tmap_a, &full[s], x, arow);
+                            if constexpr (C::BNN)
+                                tma_load_2d(a_dst + i * C::A_BYTES1, &tmap_a, &full[s], ti.n0, a_k_rows + x);
+                            else
+                                tma_load_2d(a_dst + i * C::A_BYTES1, &tmap_a, &full[s], x, arow);
                             tma_load_2d(b_dst + i * C::B_BYTES1, &tmap_b, &full[s], x, brow);
                         }
                     }
@@ -783,7 +874,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
         } else if (!C::PROMO && lane == 0 && rank == 0) {
             // (swapped operands: N is the tile's token count rounded up to 16, set per tile below)
-            constexpr uint32_t IDESC = idesc_mxf8_e4m3(C::TILE_M, C::SWAP ? 0 : BN, C::BF4);
+            // (B in the NN orientation: the M-side operand is MN-major, bit 15 of the instruction descriptor)
+            constexpr uint32_t IDESC = idesc_mxf8_e4m3(C::TILE_M, C::SWAP ? 0 : BN, C::BF4) | (C::BNN ? 1u << 15 : 0u);
             int s = 0;
             uint32_t ph = 0;
             int acc = 0;
@@ -835,9 +927,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         for (int k = 0; k < BLOCK_K / MMA_K; ++k) {
                             const uint32_t b_byte = C::BF4 ? static_cast<uint32_t>(k) : sub;
                             const uint32_t idesc = IDESC | idesc_n | (sub << 29) | (b_byte << 4);
-                            tc_mma_mxf8<CTAS>(d_tmem, sdesc_kmajor_sw128(a_base + k * MMA_K),
-                                              sdesc_kmajor_sw128(b_base + k * MMA_K), idesc, sf_tmem, sf_b,
-                                              (kb | k) != 0);
+                            // K step of an MN-major tile: 32 K-rows of 128 bytes
+                            const uint64_t a_desc = C::BNN ? sdesc_mnmajor_sw128(a_base + k * MMA_K * 128)
+                                                           : sdesc_kmajor_sw128(a_base + k * MMA_K);
+                            tc_mma_mxf8<CTAS>(d_tmem, a_desc, sdesc_kmajor_sw128(b_base + k * MMA_K), idesc, sf_tmem,
+                                              sf_b, (kb | k) != 0);
                         }
                     }
                     tc_commit<CTAS>(&empty[s]);
@@ -1015,6 +1109,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 // the lanes, row by row.
                 const int m = ctl.mm[ti.g];
                 const int cnt = min(chunk_rows(m, BN), m - ti.local_row0);
+                const int gB = swap_contig ? ctl.rg[ti.g] : ti.g;
                 const int col0 = ti.n0 + my_rows + 32 * q;  // this warp's first column of D
                 const bool odd = (lane & 1) != 0;
                 const int pair_col = col0 + (lane & ~1);    // first of the two columns of this lane's words
@@ -1035,7 +1130,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         w[i] = odd ? ((other >> 16) | (own & 0xFFFF0000u)) : ((own & 0xFFFFu) | (other << 16));
                     }
                     const int tok0 = 32 * c;
-                    if (tok0 + 32 <= cnt) {
+                    // token rows of this chunk the call owns (contiguous: m_indices[row] == the group)
+                    unsigned own;
+                    if (swap_contig) {
+                        const int row = ti.row0 + tok0 + lane;
+                        own = __ballot_sync(0xffffffffu, tok0 + lane < cnt && row < p.M && __ldg(p.m_indices + row) == gB);
+                    } else {
+                        own = tok0 + 32 <= cnt ? 0xffffffffu : (1u << (cnt - tok0)) - 1u;
+                    }
+                    if (own == 0xffffffffu) {
                         uint8_t *buf = stage_buf + (chunk_count & 1) * EPI_CHUNK_BYTES;
                         if (chunk_count >= 2) {
                             if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
@@ -1057,9 +1160,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     } else if (pair_col < p.N) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const int tok = tok0 + 2 * i + (odd ? 1 : 0);
-                            if (tok < cnt)
-                                *reinterpret_cast<uint32_t *>(p.d + static_cast<size_t>(ti.row0 + tok) * p.N +
+                            const int t = 2 * i + (odd ? 1 : 0);
+                            if ((own >> t) & 1u)
+                                *reinterpret_cast<uint32_t *>(p.d + static_cast<size_t>(ti.row0 + tok0 + t) * p.N +
                                                               pair_col) = w[i];
                         }
                     }

@@ -330,6 +330,20 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
     return d;
 }
 
+// Shared-memory matrix descriptor, MN-major operand tile stored by TMA with the 128-byte swizzle: K-rows of 128
+// bytes (128 e4m3 elements along M/N), 8-K-row (1024-byte) swizzle atoms stacked along K (stride byte offset).
+// The tile is one swizzle atom wide along M/N (128 elements), so the leading byte offset (the stride between
+// 128-byte M/N chunks) is never used.  A K step is taken by advancing the start address by whole 8-row atoms.
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);  // [0,14)  start address >> 4
+    d |= static_cast<uint64_t>(16384 >> 4) << 16;          // [16,30) leading byte offset (unused: one M/N chunk)
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;           // [32,46) stride byte offset: 8 K-rows x 128 B
+    d |= static_cast<uint64_t>(1) << 46;                   // [46,48) descriptor version for sm_100
+    d |= static_cast<uint64_t>(2) << 61;                   // [61,64) swizzle mode: 128 B
+    return d;
+}
+
 // Descriptor of a 32-row x 16-byte block stored densely (row r at byte 16 r), no swizzle: the source of
 // tcgen05.cp .32x128b.  Core matrices of 8 rows x 16 bytes are 128 bytes apart along the rows.
 __device__ __forceinline__ uint64_t sdesc_rows16_noswizzle(uint32_t saddr) {

@@ -14,7 +14,9 @@
 //                                           word per output column in the right TMEM lane)
 // Swapped operands (masked layout; the MMA's M side runs over B's rows, its N side over a group's tokens):
 //   B-side atoms:     [g][128-row block of B][group]   every row holds the 128x128 block's scale
-//   token-side atoms: [g][chunk][group][atom a]        rows a*128 .. a*128+127 of the chunk's tokens
+//   token-side atoms: [chunk][group][atom a]           rows a*128 .. a*128+127 of the chunk's tokens, the
+//                                                      chunks of all groups in order (group g's first chunk
+//                                                      is the sum of the earlier groups' chunk counts)
 // Entries past the problem (rows >= the scale extent, K blocks >= K/128, columns >= N) hold 0x7F (2^0).
 #pragma once
 #include <cstdint>
@@ -45,7 +47,7 @@ struct PackParams {
     unsigned *err;        // device error word: ERR_BAD_SCALE for a scale the call reads that is not a power of two
     int swap;             // swapped operands (masked layout): sfa_out holds B's atoms, sfb_out the tokens'
     int b_blocks;         // swapped: 128-row blocks of B per group in sfa_out (past N: 2^0)
-    int chunks;           // swapped: token chunks per group in sfb_out (chunk size chunk_rows(masked_m, bn))
+    int chunks;           // swapped: token chunks sfb_out has room for (chunk size chunk_rows(group rows, bn))
     uint32_t *sfa_out;    // [sfa_groups * blocks_per_group][num_sf_groups][128]
     uint32_t *sfb_out;    // [G][n_tiles][num_sf_groups][sfb_atoms][128]
     long long sfa_words, sfb_words;
@@ -67,18 +69,44 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
     grid_launch_dependents();  // the GEMM may start its prologue; it waits for this grid before reading
     // The group tables, as the GEMM derives them.  No padding: clamped row counts, first rows, window prefix.
     // K-grouped: 128-K blocks per group, first 128-K block, prefix of packed scale groups (SF_GROUP blocks).
-    __shared__ int s_cnt[MAX_MASKED_GROUPS], s_off[MAX_MASKED_GROUPS], s_wpre[MAX_MASKED_GROUPS + 1];
+    // Contiguous layout with swapped operands: the runs of blocks of one group (s_cnt: rows, s_off: first row,
+    // s_rg: group), built as the GEMM builds them.
+    __shared__ int s_cnt[MAX_MASKED_GROUPS], s_off[MAX_MASKED_GROUPS + 1], s_wpre[MAX_MASKED_GROUPS + 1];
+    __shared__ short s_rg[MAX_MASKED_GROUPS], s_gb[MAX_MASKED_GROUPS];
+    __shared__ int s_runs;
     const bool nopad = p.mode == MODE_NOPAD, kgrouped = p.mode == MODE_KGROUPED;
-    if (nopad || kgrouped) {
-        for (int g = threadIdx.x; g < p.G; g += blockDim.x) {
-            const int c = __ldg(p.counts + g);
-            s_cnt[g] = c < 0 ? 0 : (kgrouped ? c / 128 : c);
+    const bool swap_contig = p.swap && p.mode == MODE_CONTIGUOUS;
+    int ntab = p.G;  // entries of the tables
+    if (swap_contig) {
+        const int num_blocks = p.rows_per_group / 128;  // (at most MAX_MASKED_GROUPS: checked by the host)
+        for (int b = threadIdx.x; b < num_blocks; b += blockDim.x) {
+            const int g = __ldg(p.m_indices + static_cast<size_t>(b) * 128);
+            s_gb[b] = static_cast<short>(g >= 0 && g < p.G ? g : -1);
         }
         __syncthreads();
         if (threadIdx.x < 32) {
-            build_group_rows(p.G, kgrouped ? p.nkb : p.rows_per_group, s_cnt, s_off, nullptr, threadIdx.x);
+            const int runs = build_run_heads(num_blocks, s_gb, s_off, s_cnt, s_rg, threadIdx.x);
+            if (threadIdx.x == 0) s_runs = runs;
+        }
+        __syncthreads();
+        ntab = s_runs;
+        finish_runs(p.m_indices, p.rows_per_group, ntab, s_off, s_cnt, s_rg, threadIdx.x >> 5, blockDim.x >> 5,
+                    threadIdx.x & 31);
+        __syncthreads();
+        if (threadIdx.x < 32) build_window_prefix(ntab, p.bn, s_cnt, s_wpre, threadIdx.x);
+        __syncthreads();
+    } else if (nopad || kgrouped || p.swap) {
+        for (int g = threadIdx.x; g < p.G; g += blockDim.x) {
+            const int c = __ldg(p.counts + g);
+            s_cnt[g] = c < 0 ? 0 : (kgrouped ? c / 128 : (p.mode == MODE_MASKED ? min(c, p.rows_per_group) : c));
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            if (p.mode != MODE_MASKED)
+                build_group_rows(p.G, kgrouped ? p.nkb : p.rows_per_group, s_cnt, s_off, nullptr, threadIdx.x);
             __syncwarp();
-            build_window_prefix(p.G, kgrouped ? SF_GROUP : p.tile_m, s_cnt, s_wpre, threadIdx.x);
+            // chunks (swapped operands), windows (no padding) or packed scale groups (K-grouped) per group
+            build_window_prefix(p.G, p.swap ? p.bn : (kgrouped ? SF_GROUP : p.tile_m), s_cnt, s_wpre, threadIdx.x);
         }
         __syncthreads();
     }
@@ -120,8 +148,9 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
                 for (int i = 0; i < 4; ++i) {
                     const int kb = SF_GROUP * q + i;
                     const bool in = blk < nnb128 && kb < p.nkb;
-                    const uint32_t bits =
-                        in ? __float_as_uint(__ldg(p.sfb + (g * nnb128 + blk) * p.nkb + kb)) : ONE_F32_BITS;
+                    // [G][N/128][K/128], or [G][K/128][N/128] for B in the NN orientation
+                    const long long idx = p.sfb_kn ? (g * p.nkb + kb) * nnb128 + blk : (g * nnb128 + blk) * p.nkb + kb;
+                    const uint32_t bits = in ? __float_as_uint(__ldg(p.sfb + idx)) : ONE_F32_BITS;
                     wv |= ((bits >> 23) & 0xFFu) << (8 * i);
                     if (in) bad_bits |= ue8m0_inexact_bits(bits);
                 }
@@ -130,20 +159,26 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
             } else {  // token side: the per-row scales of 256 tokens of one chunk of one group
                 const long long b = atom - sfa_atoms;
                 const int a = static_cast<int>(b % p.sfb_atoms);
-                long long rest = b / p.sfb_atoms;
+                const long long rest = b / p.sfb_atoms;
                 const int q = static_cast<int>(rest % p.num_sf_groups);
-                rest /= p.num_sf_groups;
-                const int c = static_cast<int>(rest % p.chunks);
-                const long long g = rest / p.chunks;
-                const int m = min(max(__ldg(p.counts + g), 0), p.rows_per_group);
+                const int w = static_cast<int>(rest / p.num_sf_groups);  // chunk over all groups (runs)
+                if (w >= s_wpre[ntab]) continue;  // past the last chunk: never read
+                const int g = upper_index(s_wpre, ntab, w);  // group, or run (contiguous)
+                const int m = s_cnt[g];
                 const int cs = chunk_rows(m, p.bn);
-                const float *base = p.sfa + g * p.nkb * p.sfa_ld;
+                const int c = w - s_wpre[g];
+                const long long first = p.mode == MODE_MASKED ? 0 : s_off[g];  // the group's first token row
+                const int gid = swap_contig ? s_rg[g] : g;
+                const float *base = p.sfa + (p.mode == MODE_MASKED ? static_cast<long long>(g) * p.nkb * p.sfa_ld : 0);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int r = a * 128 + lane + 32 * j;
-                    const long long tok = static_cast<long long>(c) * cs + r;
+                    const long long local = static_cast<long long>(c) * cs + r;  // token within the group
+                    const long long tok = first + local;
                     const bool in = tok < p.sfa_ld;
-                    const bool check = tok < m && r < cs;
+                    // scales of rows the call owns are checked (contiguous: rows whose m_indices is the group)
+                    const bool check = in && local < m && r < cs &&
+                                       (!swap_contig || __ldg(p.m_indices + tok) == gid);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int kb = SF_GROUP * q + i;

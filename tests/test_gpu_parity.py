@@ -24,6 +24,16 @@ def policy(request):
     dg.set_cta_pair_policy(-1)
 
 
+@pytest.fixture(params=[0, 1], ids=["unswapped", "swapped"])
+def swap(request):
+    """Tiles with the operands in their own order, or swapped (B's rows on the MMA's M side, tokens on N)."""
+    import moe_grouped_gemm_03_b200 as dg
+
+    dg.set_swap_policy(request.param)
+    yield request.param
+    dg.set_swap_policy(-1)
+
+
 def _full_check(p):
     out = run_problem(p)
     import moe_grouped_gemm_03_b200 as dg
@@ -76,8 +86,14 @@ def test_dense_shapes(M, N, K, policy):
     ([129, 1, 130, 255, 256, 257, 3], 640, 256),  # odd block counts: 256-row windows straddle groups
     ([128] * 9, 256, 128),                        # nine one-block groups: every pair window holds two groups
 ])
-def test_contiguous_shapes(counts, N, K, policy):
+def test_contiguous_shapes(counts, N, K, policy, swap):
     _full_check(synth.make_contiguous(counts, N, K, seed=sum(counts) + N))
+
+
+def test_contiguous_beyond_the_swapped_tables(policy):
+    """More 128-row blocks (1105) than the device tables of the swapped-operand tiles hold (1024): the call runs
+    the unswapped 128- or 256-row windows instead."""
+    _full_check(synth.make_contiguous([15000, 1, 129, 30000, 95000, 127, 256, 255, 70], 256, 128, seed=77))
 
 
 @pytest.mark.parametrize("G,M_max,N,K,mm", [
@@ -90,7 +106,7 @@ def test_contiguous_shapes(counts, N, K, policy):
     (6, 700, 304, 640, [700, 225, 224, 449, 15, 0]),
     (2, 1000, 7168, 256, [1000, 31]),
 ])
-def test_masked_shapes(G, M_max, N, K, mm, policy):
+def test_masked_shapes(G, M_max, N, K, mm, policy, swap):
     _full_check(synth.make_masked(G, M_max, N, K, masked_m=mm, seed=G + M_max, expected_m=M_max // 2))
 
 
@@ -100,7 +116,7 @@ def test_masked_shapes(G, M_max, N, K, mm, policy):
     ([1], 16, 128),
     ([129, 1, 130, 255, 256, 257, 3], 640, 256),
 ])
-def test_contiguous_nn_shapes(counts, N, K, policy):
+def test_contiguous_nn_shapes(counts, N, K, policy, swap):
     _full_check(synth.make_contiguous_nn(counts, N, K, seed=sum(counts) + N))
 
 
@@ -186,7 +202,7 @@ def alignment_256():
     ([129, 1, 130, 255, 256, 257, 3], 640, 384),
     ([256] * 5, 256, 128),
 ])
-def test_contiguous_alignment_256(counts, N, K, policy, alignment_256):
+def test_contiguous_alignment_256(counts, N, K, policy, alignment_256, swap):
     """Segments padded to 256 rows (the optional alignment): every 256-row window holds one group."""
     _full_check(synth.make_contiguous(counts, N, K, seed=sum(counts) + 256, alignment=256))
 
@@ -199,11 +215,11 @@ def test_contiguous_alignment_256(counts, N, K, policy, alignment_256):
     ([37] * 40, 384, 256, 0),                          # forty small groups: every window is partial
     ([0, 0, 0], 256, 128, 40),                         # no group owns a row: nothing is written
 ])
-def test_nopad_shapes(counts, N, K, extra, policy):
+def test_nopad_shapes(counts, N, K, extra, policy, swap):
     _full_check(synth.make_nopad(counts, N, K, seed=sum(counts) + N + extra, extra_rows=extra))
 
 
-def test_nopad_counts_past_m_total_are_clipped_and_reported(policy):
+def test_nopad_counts_past_m_total_are_clipped_and_reported(policy, swap):
     """Counts summing past M_total: the rows up to M_total are computed as the clipped layout says, and the
     device error word reports it; a negative count owns no row."""
     import moe_grouped_gemm_03_b200 as dg
@@ -255,7 +271,7 @@ def test_nopad_equals_contiguous_call_on_the_padded_layout(policy):
         src += c
 
 
-def test_masked_all_groups_empty_writes_nothing(policy):
+def test_masked_all_groups_empty_writes_nothing(policy, swap):
     p = synth.make_masked(3, 128, 256, 256, masked_m=[0, 0, 0], seed=1)
     out = run_problem(p)
     assert untouched_rows_ok(out, np.zeros(3 * 128, bool))
@@ -292,7 +308,7 @@ def test_contiguous_groups_equal_dense_calls(policy):
         start += seg
 
 
-def test_bad_group_id_is_reported_and_skipped(policy):
+def test_bad_group_id_is_reported_and_skipped(policy, swap):
     import moe_grouped_gemm_03_b200 as dg
 
     p = synth.make_contiguous([128, 128], 256, 256, seed=13)
@@ -341,7 +357,7 @@ def test_contiguous_many_groups_takes_the_single_cta_path():
     assert untouched_rows_ok(out, mask)
 
 
-def test_masked_and_nopad_at_the_group_limit(policy):
+def test_masked_and_nopad_at_the_group_limit(policy, swap):
     """1024 groups, the most the masked and no-padding calls accept."""
     import moe_grouped_gemm_03_b200 as dg
 

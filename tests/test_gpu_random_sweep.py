@@ -65,17 +65,19 @@ def test_random_shape(case):
     import moe_grouped_gemm_03_b200 as dg
 
     p = _draw(case)
-    policy = int(np.random.default_rng(case).choice([-1, 0, 1]))
+    policy, swap = (int(v) for v in np.random.default_rng(case).choice([-1, 0, 1], size=2))
     dg.set_cta_pair_policy(policy)
+    dg.set_swap_policy(swap)
     try:
         out = run_problem(p)
         dg.check_device_error()
     finally:
         dg.set_cta_pair_policy(-1)
+        dg.set_swap_policy(-1)
     ref = oracle.problem_full(p).reshape(-1, p.N)
     got = bf16_to_f64(out).reshape(-1, p.N)
     valid = ~np.isnan(ref[:, 0])
-    assert_close(got[valid], ref[valid], f"{p.name} policy {policy}")
+    assert_close(got[valid], ref[valid], f"{p.name} policy {policy} swap {swap}")
     assert untouched_rows_ok(out, valid), f"{p.name}: rows outside the groups were written"
 
 
