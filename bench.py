@@ -240,9 +240,11 @@ PROMOTION_WORKLOADS = (10,)  # run with fp32 scale promotion (their scales are n
 
 
 def launches_per_call(p, promotion=False):
-    """The library's kernels one call launches: the scale pre-pass and the GEMM (NN: the B transpose too); the
-    fp32 scale-promotion GEMM has no pre-pass."""
-    return (2 if p.kind == "contiguous_nn" else 1) + (0 if promotion else 1)
+    """The library's kernels one call launches: the scale pre-pass and the GEMM (the fp32 scale-promotion GEMM has no
+    pre-pass).  The NN call reads B in place through the swapped-operand tiles when its 128-row blocks fit their
+    tables (M_total / 128 <= 1024) and promotion is off; otherwise it transposes B first (one more launch)."""
+    transpose = p.kind == "contiguous_nn" and (promotion or p.rows // 128 > 1024)
+    return (2 if transpose else 1) + (0 if promotion else 1)
 
 
 def algorithmic_bytes(p):

@@ -53,5 +53,6 @@ def test_launches_per_call():
     dense = synth.make_dense(128, 256, 512)
     nn = synth.make_contiguous_nn([129], 256, 256)
     assert bench.launches_per_call(dense) == 2  # scale pre-pass + GEMM
-    assert bench.launches_per_call(nn) == 3  # + the B transpose
+    assert bench.launches_per_call(nn) == 2  # B read in place by the swapped-operand tiles
+    assert bench.launches_per_call(nn, promotion=True) == 2  # transpose + the promotion GEMM
     assert bench.launches_per_call(dense, promotion=True) == 1  # the promotion GEMM has no pre-pass
