@@ -241,10 +241,12 @@ PROMOTION_WORKLOADS = (10,)  # run with fp32 scale promotion (their scales are n
 
 def launches_per_call(p, promotion=False):
     """The library's kernels one call launches: the scale pre-pass and the GEMM (the fp32 scale-promotion GEMM has no
-    pre-pass).  The NN call reads B in place through the swapped-operand tiles when its 128-row blocks fit their
+    pre-pass; a short dense call -- K <= 2048 and 2MNK <= 2^34 -- runs that GEMM alone on its power-of-two
+    scales).  The NN call reads B in place through the swapped-operand tiles when its 128-row blocks fit their
     tables (M_total / 128 <= 1024) and promotion is off; otherwise it transposes B first (one more launch)."""
     transpose = p.kind == "contiguous_nn" and (promotion or p.rows // 128 > 1024)
-    return (2 if transpose else 1) + (0 if promotion else 1)
+    short_dense = p.kind == "dense" and p.K <= 2048 and 2 * p.M * p.N * p.K <= 1 << 34
+    return (2 if transpose else 1) + (0 if promotion or short_dense else 1)
 
 
 def algorithmic_bytes(p):
@@ -295,8 +297,13 @@ def oracle_sample(p, seconds, rng_seed=0):
 
 def workload_config(p, world, promotion):
     """The `config` object of both arms: the workload, its scales and the timing protocol."""
-    return {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "G": p.G,
-            "scales": "fp32, promoted per 128-K block" if promotion else "powers of two (UE8M0, block-scaled MMA)",
+    if promotion:
+        scales = "fp32, promoted per 128-K block"
+    elif launches_per_call(p) == 1:  # a short dense call: one kernel
+        scales = "powers of two, applied per 128-K block by the promotion GEMM (short call: no pre-pass)"
+    else:
+        scales = "powers of two (UE8M0, block-scaled MMA)"
+    return {"workload": p.name, "M": p.M, "N": p.N, "K": p.K, "G": p.G, "scales": scales,
             "l2": "flushed between steps (512 MB write outside the timed events)",
             "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"}
 

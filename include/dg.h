@@ -18,9 +18,9 @@
  * block-scaled tensor-core MMA applies the scales as exponents.  The scale pre-pass checks every scale the
  * call reads (the A scales of rows the call owns, all B scales) and reports one with a sign, mantissa bits,
  * Inf or NaN as DG_ERR_BAD_SCALE through dg_check_device_error(); the results of that call are then wrong.
- * A zero scale is taken as 2^-127.  After dg_set_fp32_scale_promotion(1) the calls with bf16 output take any
- * finite fp32 scales: every 128-K block's partial product is multiplied by sfa * sfb and added in fp32 (the
- * "promotion operations" of the DeepGEMM-for-PPU README, "Optimizations"), at a lower speed.
+ * A zero scale is taken as 2^-127.  After dg_set_fp32_scale_promotion(1) every call takes any finite fp32
+ * scales: every 128-K block's partial product (W4A8: every 32-K sub-block's) is multiplied by sfa * sfb and
+ * added in fp32 (the "promotion operations" of the DeepGEMM-for-PPU README, "Optimizations"), at a lower speed.
  *
  * Common conventions
  *   - All array arguments are device pointers owned by the caller.  The library keeps no reference after the
@@ -105,7 +105,11 @@ DG_EXPORT int dg_select_block_n(long long num_m_blocks, int N, int num_sms);
 
 /* Dense NT GEMM (README "Normal dense GEMMs", gemm_fp8_fp8_bf16_nt).
  *   a [M][K] e4m3, sfa [K/128][ld(M)] fp32, b [N][K] e4m3, sfb [ceil(N/128)][K/128] fp32,
- *   d [M][N] bf16 row-major (written in full).  M == 0 is a no-op. */
+ *   d [M][N] bf16 row-major (written in full).  M == 0 is a no-op.
+ *   Short calls (K <= 2048 and 2*M*N*K <= 2^34) launch one kernel instead of the scale pre-pass and the
+ *   block-scaled GEMM: the fp32-promotion GEMM, which reads the scales directly and still requires them to be
+ *   powers of two (DG_ERR_BAD_SCALE), reading a zero scale as 2^-127.  Results agree with the block-scaled path
+ *   within the tolerance of fp32 accumulation, not bit for bit. */
 DG_EXPORT int dg_fp8_gemm_nt(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
                    int M, int N, int K, dg_stream_t stream);
 
@@ -151,8 +155,8 @@ DG_EXPORT int dg_m_grouped_fp8_gemm_nn_contiguous(const void *a, const float *sf
  *   sfb [G][K/32][ld(N)] fp32, MN-major: one power-of-two scale per (row n, 32-K block):
  *   D[m][n] = sum over 128-K blocks kb of sfa(m, kb) * sum over its four 32-K sub-blocks j of sfb(g, 4 kb + j, n)
  *             * sum_{k in the sub-block} A[m][k] * B_g[n][k].
- *   Scales must be powers of two (others: DG_ERR_BAD_SCALE); returns DG_ERR_UNSUPPORTED while fp32 scale
- *   promotion is on (dg_set_fp32_scale_promotion). */
+ *   Scales must be powers of two (others: DG_ERR_BAD_SCALE) unless fp32 scale promotion is on
+ *   (dg_set_fp32_scale_promotion), which takes any finite scales and then needs sfb 16-byte aligned. */
 DG_EXPORT int dg_m_grouped_fp8_fp4_gemm_nt_contiguous(const void *a, const float *sfa, const void *b,
                                             const float *sfb, void *d, const int *m_indices, int M_total, int N, int K,
                                             int G, dg_stream_t stream);
@@ -160,7 +164,7 @@ DG_EXPORT int dg_m_grouped_fp8_fp4_gemm_nt_contiguous(const void *a, const float
 /* M-grouped GEMM, masked layout, W4A8 (`m_grouped_fp8_fp4_gemm_nt_masked`, same page): as
  * dg_m_grouped_fp8_gemm_nt_masked except b [G][N][K/2] bytes of packed E2M1 codes (32-byte aligned) and
  * sfb [G][K/32][ld(N)] fp32, one scale per (row n, 32-K block), as in dg_m_grouped_fp8_fp4_gemm_nt_contiguous
- * (powers of two; DG_ERR_UNSUPPORTED while fp32 scale promotion is on). */
+ * (powers of two, or any finite scales with sfb 16-byte aligned while fp32 scale promotion is on). */
 DG_EXPORT int dg_m_grouped_fp8_fp4_gemm_nt_masked(const void *a, const float *sfa, const void *b, const float *sfb,
                                         void *d, const int *masked_m, int G, int M_max, int N, int K, int expected_m,
                                         dg_stream_t stream);
@@ -176,7 +180,8 @@ DG_EXPORT int dg_m_grouped_fp8_fp4_gemm_nt_masked(const void *a, const float *sf
  *   first), or d itself (accumulate in place).  A group with ks = 0 gives D_g = C_g (0 without C).
  *   1 <= G <= 1024, N % 16 == 0, 16-byte aligned a, b, c, d.  Device values of ks_device that are negative or
  *   not multiples of 128 are reported by dg_check_device_error() as DG_ERR_BAD_GROUP.  Scales must be powers of
- *   two (others: DG_ERR_BAD_SCALE); returns DG_ERR_UNSUPPORTED while fp32 scale promotion is on. */
+ *   two (others: DG_ERR_BAD_SCALE) unless fp32 scale promotion is on, which takes any finite scales and then
+ *   needs sfb 16-byte aligned (else DG_ERR_ALIGNMENT). */
 DG_EXPORT int dg_k_grouped_fp8_gemm_nt_contiguous(const void *a, const float *sfa, const void *b, const float *sfb,
                                         float *d, const float *c, const int *ks, const int *ks_device, int G, int M,
                                         int N, dg_stream_t stream);
@@ -203,8 +208,8 @@ DG_EXPORT int dg_m_grouped_fp8_gemm_nt_nopad(const void *a, const float *sfa, co
  * one).  It never calls cudaMalloc, cudaFree or any allocating routine.
  *   - Limit: the packed scales take at most (ceil(M/128) + 2*ceil(N/BN)) * ceil(K/512) * 512 bytes (BN is the
  *     chosen tile width, 128..224); a shape needing more than 16 MiB returns DG_ERR_UNSUPPORTED and launches
- *     nothing (M = N = K = 16384 needs about 4.5 MB).  With fp32 scale promotion on, the call reads the caller's
- *     scales directly and uses no buffer at all (no limit).
+ *     nothing (M = N = K = 16384 needs about 4.5 MB).  Short calls (one kernel, see dg_fp8_gemm_nt) and calls
+ *     with fp32 scale promotion on read the caller's scales directly and use no buffer at all (no limit).
  *   - The first call on each device looks up the buffer's device address with that device current, and the
  *     first call of each tile configuration does the one-time kernel set-up listed under "Common conventions";
  *     make one eager call of the same shape class on each device before any stream capture.
@@ -216,11 +221,14 @@ DG_EXPORT int dg_fp8_gemm_nt_noalloc(const void *a, const float *sfa, const void
 /* Scale handling for the next calls on any thread ("promotion operations", DeepGEMM-for-PPU README,
  * "Optimizations"; the wrapper's disable_ue8m0_cast option).  0 (default): scales must be powers of two and are
  * applied by the block-scaled MMA (kind::mxf8f6f4, UE8M0 scales in tensor memory).  1: any finite fp32 scales;
- * dg_fp8_gemm_nt, dg_fp8_gemm_nt_noalloc, dg_m_grouped_fp8_gemm_nt_contiguous, _masked, _nopad and
- * dg_m_grouped_fp8_gemm_nn_contiguous then run plain kind::f8f6f4 MMAs into one tensor-memory buffer per
- * 128-K block, and the epilogue warps accumulate buffer * sfa(m, kb) * sfb(g, n/128, kb) in fp32 registers
- * (128-column tiles; the scales are read from the caller's arrays, no scale pre-pass).  While it is on, the
- * K-grouped and W4A8 calls return DG_ERR_UNSUPPORTED.  Returns the setting now in force. */
+ * every call then runs plain kind::f8f6f4 MMAs into one tensor-memory buffer per 128-K block, and the epilogue
+ * warps accumulate buffer * sfa(m, kb) * sfb in fp32 registers (the scales are read from the caller's arrays, no
+ * scale pre-pass):
+ *   - e4m3 B (dense, allocation-free, contiguous, masked, no-padding, NN): 128-column tiles, sfb(g, n/128, kb);
+ *   - K-grouped: 128-column tiles, the per-column sfb(n, kb), fp32 D stored or added as without promotion;
+ *   - W4A8 (E2M1 B): 64-column tiles, one buffer per 32-K sub-block j, sfb(g, j, n).
+ * The calls with per-column B scales (K-grouped, W4A8) need sfb 16-byte aligned (else DG_ERR_ALIGNMENT).
+ * Returns the setting now in force. */
 DG_EXPORT int dg_set_fp32_scale_promotion(int enable);
 DG_EXPORT int dg_get_fp32_scale_promotion(void);
 

@@ -194,7 +194,7 @@ def set_swap_policy(policy: int) -> int:
 def set_fp32_scale_promotion(enable: bool) -> bool:
     """False (default): scales must be powers of two (applied as UE8M0 exponents by the block-scaled MMA; others
     are reported as DG_ERR_BAD_SCALE by check_device_error).  True: any finite fp32 scales, applied by fp32
-    promotion of every 128-K block's partial product (the bf16-output calls; K-grouped and W4A8 refuse)."""
+    promotion of every 128-K block's partial product (W4A8: of every 32-K sub-block's), on every call."""
     return bool(_lib.dg_set_fp32_scale_promotion(1 if enable else 0))
 
 

@@ -291,6 +291,7 @@ struct ScaleArgs {
     bool sfb_kn = false;  // SFB stored [G][K/128][ceil(N/128)] (B in the NN orientation)
     bool sfb_fp4 = false; // B in E2M1 (packed two per byte) with SFB [G][K/32][sfb_ld]
     bool fixed_scratch = false;  // packed scales in the library's fixed buffer (no allocation) instead of the pool
+    bool single_kernel = false;  // power-of-two scales applied by the promotion GEMM (one launch, no pre-pass)
     bool swap = false;    // masked layout with swapped operands (B's rows on the MMA's M side, tokens on its N side)
     int sfb_ld = 0;       // K-grouped: one scale per row of B, [K/128][sfb_ld]; FP4 B: [G][K/32][sfb_ld]
 };
@@ -471,26 +472,45 @@ int launch_cfg(const void *a, long long a_rows, const void *b, long long b_rows,
     return rc;
 }
 
-// The fp32 scale-promotion GEMM (any finite fp32 scales): 128-wide tiles, plain kind::f8f6f4 MMAs, the epilogue
-// warps read the caller's scales directly, so there is no pre-pass and no scratch.  The launch is an ordinary
-// stream-ordered one (the kernel's first loads may not run ahead of the previous kernel on the stream).
-template <int CTAS>
+// The fp32 scale-promotion GEMM (any finite fp32 scales): plain kind::f8f6f4 MMAs, the epilogue warps read the
+// caller's scales directly, so there is no pre-pass and no scratch.  e4m3 B: 128-wide tiles (one 128-column
+// block of B's scales); K-grouped (per-column B scales, fp32 D): 64-wide tiles, which keep the accumulators and
+// the fp32 epilogue within the registers; E2M1 B: 64-wide tiles, one partial per 32-K MMA.
+// The launch is an ordinary stream-ordered one (the kernel's first loads may not run ahead of the previous
+// kernel on the stream).
+template <int BN, int CTAS, int KPS, bool BF4, bool PCOL = false>
 int launch_promo(const void *a, long long a_rows, const void *b, long long b_rows, const ScaleArgs &sc,
                  dg::GemmParams p, int grid, int device, cudaStream_t stream) {
-    using C = dg::Cfg<128, CTAS, CTAS == 2 ? 2 : 1, false, true>;  // (a single CTA fits more stages of one K block)
+    using C = dg::Cfg<BN, CTAS, KPS, BF4, true, false, false, PCOL>;
     const int nkb = p.K / dg::BLOCK_K;
     const int nnb = (p.N + 127) / 128;
     p.sfa32 = sc.sfa;
     p.sfa_ld = sc.sfa_ld;
     p.sfb32 = sc.sfb;
-    p.sfb_sg = nkb * nnb;
-    p.sfb_sn = sc.sfb_kn ? 1 : nkb;  // NN: [G][K/128][ceil(N/128)]; NT: [G][ceil(N/128)][K/128]
-    p.sfb_sk = sc.sfb_kn ? nnb : 1;
+    if (BF4) {  // [G][K/32][sfb_ld]: per column and 32-K sub-block
+        p.sfb_sg = static_cast<int>(static_cast<long long>(p.K / 32) * sc.sfb_ld);
+        p.sfb_sk = sc.sfb_ld;
+    } else if (PCOL) {  // K-grouped, [sum ks / 128][sfb_ld]: per column and K block, one B for all groups
+        p.sfb_sg = 0;
+        p.sfb_sk = sc.sfb_ld;
+    } else {
+        p.sfb_sg = nkb * nnb;
+        p.sfb_sn = sc.sfb_kn ? 1 : nkb;  // NN: [G][K/128][ceil(N/128)]; NT: [G][ceil(N/128)][K/128]
+        p.sfb_sk = sc.sfb_kn ? nnb : 1;
+    }
     CUtensorMap ta, tb, td;
     int rc;
-    if ((rc = make_output_map(td, p.d, a_rows, p.N))) return rc;
+    if (p.out_mode == dg::OUT_BF16)
+        rc = make_output_map(td, p.d, a_rows, p.N);
+    else
+        rc = make_output_map_f32(td, p.d32, p.G, p.M, p.N);
+    if (rc) return rc;
     if ((rc = make_operand_map(ta, a, a_rows, p.K, dg::BLOCK_M))) return rc;
-    if ((rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS))) return rc;
+    if (BF4)
+        rc = make_operand_map_fp4(tb, b, b_rows, p.K, C::B_ROWS);
+    else
+        rc = make_operand_map(tb, b, b_rows, p.K, C::B_ROWS);
+    if (rc) return rc;
     auto kernel = dg::fp8_gemm_kernel<C>;
     cudaError_t e;
     static bool smem_set[64] = {false};
@@ -527,8 +547,8 @@ int launch_promo(const void *a, long long a_rows, const void *b, long long b_row
     }
     static const bool debug = getenv("DG_DEBUG") && getenv("DG_DEBUG")[0] == '1';
     if (debug)
-        fprintf(stderr, "[dg] fp32 promotion: mode=%d M=%d N=%d K=%d G=%d BN=128 stages=%d x %d ctas=%d grid=%u smem=%d\n",
-                p.mode, p.M, p.N, p.K, p.G, C::STAGES, C::KPS, CTAS, cfg.gridDim.x, C::SMEM_BYTES);
+        fprintf(stderr, "[dg] fp32 promotion: mode=%d M=%d N=%d K=%d G=%d BN=%d stages=%d x %d ctas=%d grid=%u smem=%d\n",
+                p.mode, p.M, p.N, p.K, p.G, BN, C::STAGES, C::KPS, CTAS, cfg.gridDim.x, C::SMEM_BYTES);
     apply_wait_settings(p);
     // the kernel takes five maps; the two scale-atom maps are unused on this path
     if ((e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, ta, ta, td, p)) != cudaSuccess)
@@ -627,20 +647,31 @@ int plan_and_launch(dg::GemmParams p, const DeviceInfo &info, const Plan &plan, 
         pair = plan.sel2 * ((p.N + bn - 1) / bn) >= sms / 2;
     }
     const int units = pair ? sms / 2 : sms;
-    if (g_fp32_promotion.load()) {
-        if (sc.sfb_fp4 || p.mode == dg::MODE_KGROUPED || p.out_mode != dg::OUT_BF16)
-            return fail(DG_ERR_UNSUPPORTED,
-                        "fp32 scale promotion covers the bf16-output FP8 calls (dense, contiguous, masked, no-padding, "
-                        "NN); switch it off for the K-grouped and W4A8 calls");
-        p.num_n_blocks = (p.N + 127) / 128;
+    const bool promotion = g_fp32_promotion.load();
+    if (promotion || sc.single_kernel) {
+        p.check_scales = promotion ? 0 : 1;
+        // per-column B scales (K-grouped, E2M1 B) are copied 16 bytes at a time
+        if ((sc.sfb_fp4 || p.mode == dg::MODE_KGROUPED) && !aligned(sc.sfb, 16))
+            return fail(DG_ERR_ALIGNMENT, "with fp32 scale promotion, sfb must be 16-byte aligned");
+        const int bn = sc.sfb_fp4 || p.mode == dg::MODE_KGROUPED ? 64 : 128;  // (per-column scales: 64 wide)
+        p.num_n_blocks = (p.N + bn - 1) / bn;
         const bool device_windows = p.mode == dg::MODE_MASKED || p.mode == dg::MODE_NOPAD;
         p.num_windows = static_cast<int>(device_windows ? 0 : (pair ? plan.windows2 : plan.windows1));
-        if (p.mode == dg::MODE_DENSE) p.raster_bands = raster_bands(p, pair ? 2 : 1);
+        if (p.mode == dg::MODE_DENSE || p.mode == dg::MODE_KGROUPED) p.raster_bands = raster_bands(p, pair ? 2 : 1);
         const long long tiles = (pair ? plan.bound2 : plan.bound1) * p.num_n_blocks;
         const int grid = static_cast<int>(tiles < units ? tiles : units);
         if (grid <= 0) return DG_OK;
-        if (pair) return launch_promo<2>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
-        return launch_promo<1>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
+        // (a single CTA fits more stages of one K block)
+        if (sc.sfb_fp4) {
+            if (pair) return launch_promo<64, 2, 1, true>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
+            return launch_promo<64, 1, 1, true>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
+        }
+        if (p.mode == dg::MODE_KGROUPED) {
+            if (pair) return launch_promo<64, 2, 2, false, true>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
+            return launch_promo<64, 1, 1, false, true>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
+        }
+        if (pair) return launch_promo<128, 2, 2, false>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
+        return launch_promo<128, 1, 1, false>(a, a_rows, b, b_rows, sc, p, grid, info.device, stream);
     }
     int bn = select_block_n(pair ? plan.sel2 : plan.sel1, p.N, units, pair ? 2 : 1);
     static const int forced_bn = getenv("DG_BLOCK_N") ? atoi(getenv("DG_BLOCK_N")) : 0;  // tuning override
@@ -791,6 +822,19 @@ int launch_contiguous(const void *a, const float *sfa, const void *b, const floa
 
 namespace {
 
+// Dense calls this short run as one kernel -- the promotion GEMM, reading the caller's scales -- instead of the
+// scale pre-pass and the block-scaled GEMM: their time is then mostly the second launch and the GEMM's wait for
+// the pre-pass (about 6 us), which the promotion's costlier per-K-block epilogue does not spend back while K is
+// short.  Measured on B200 (L2 flushed between calls, CUDA events), one kernel / two: 0.66 at 128 x 256 x 512,
+// 0.85-0.88 from 0.5 to 8.6 GFLOP with K <= 2048, 0.92 at 1024 x 4096 x 2048; 1.05-1.10 with K = 7168 and 1.29 at
+// 2048 x 4096 x 4096.  The scales must still be powers of two: the promotion epilogue checks each one it reads
+// (DG_ERR_BAD_SCALE) and reads a zero scale as 2^-127, as the block-scaled path does.
+constexpr int kSingleKernelMaxK = 2048;
+constexpr long long kSingleKernelMaxFlops = 1ll << 34;
+bool dense_single_kernel(long long M, long long N, long long K) {
+    return K <= kSingleKernelMaxK && 2 * M * N * K <= kSingleKernelMaxFlops;
+}
+
 // The dense calls; `fixed_scratch`: the packed scales go to the library's fixed buffer (no allocation).
 int dense_call(const void *a, const float *sfa, const void *b, const float *sfb, void *d, int M, int N, int K,
                dg_stream_t stream, bool fixed_scratch) {
@@ -804,6 +848,7 @@ int dense_call(const void *a, const float *sfa, const void *b, const float *sfb,
     p.M = M; p.N = N; p.K = K; p.G = 1;
     ScaleArgs sc{sfa, dg_get_tma_aligned_size(M, 4), sfb};
     sc.fixed_scratch = fixed_scratch;
+    sc.single_kernel = dense_single_kernel(M, N, K);
     p.d = static_cast<__nv_bfloat16 *>(d);
     p.err = device_error_word();
     if (!p.err) return fail(DG_ERR_CUDA, "device error word is not available");

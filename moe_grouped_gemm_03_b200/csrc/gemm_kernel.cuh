@@ -104,15 +104,21 @@ struct GemmParams {
     int skip_first_load;               // test hook: the first CTA (pair) never loads stage 0
     // fp32 scale promotion (Cfg::PROMO): the caller's scales, read by the epilogue warps
     const float *sfa32;  // MN-major [K/128][sfa_ld] (masked: [G][K/128][sfa_ld])
-    const float *sfb32;  // scale of (group g, 128-column block nb, K block kb) at g * sfb_sg + nb * sfb_sn + kb * sfb_sk
+    // Cfg::PCOL = false: scale of (group g, 128-column block nb, K block kb) at g * sfb_sg + nb * sfb_sn + kb * sfb_sk;
+    // Cfg::PCOL: one scale per column n (K-grouped: per K block kb of the whole K range; W4A8: per 32-K sub-block
+    // j) at g * sfb_sg + kb (or j) * sfb_sk + n, the address of each 4 columns 16-byte aligned
+    const float *sfb32;
     int sfa_ld;
     int sfb_sg, sfb_sn, sfb_sk;
+    // 1: the scales must be powers of two (the block-scaled calls' rule, applied by the promotion GEMM when a dense
+    // call runs as one kernel): each one read is checked (ERR_BAD_SCALE) and a zero scale is read as 2^-127
+    int check_scales;
     // measurement aid (null: off): CTA 0 adds its SM cycles, nanoseconds and 1 to clock_acc[0..2] at exit
     unsigned long long *clock_acc;
 };
 
 template <int BN_, int CTAS_, int KPS_, bool BF4_ = false, bool PROMO_ = false, bool SWAP_ = false,
-          bool BNN_ = false>
+          bool BNN_ = false, bool PCOL_ = false>
 struct Cfg {
     static constexpr int BN = BN_;
     static constexpr int CTAS = CTAS_;
@@ -123,9 +129,15 @@ struct Cfg {
     static constexpr bool BF4 = BF4_;
     // fp32 scale promotion: plain kind::f8f6f4 MMAs write each 128-K block's partial product to its own TMEM
     // buffer (two partial stages of KPS blocks, 2 * KPS * BN columns), and the epilogue warps accumulate
-    // partial * sfa * sfb in registers.  No scale atoms travel with the stages.  BN = 128: a tile's columns are
-    // exactly one 128-column block of B's scales.
+    // partial * sfa * sfb in registers.  No scale atoms travel with the stages.  e4m3 B: BN = 128, a tile's
+    // columns are exactly one 128-column block of B's scales (K-grouped: 64 columns of per-column scales).  E2M1 B
+    // (one scale per column and 32-K sub-block): each of a K block's four 32-K MMAs writes its own partial
+    // (PSUB = 4), so BN = 64 and one K block per stage fill the 512 TMEM columns.
     static constexpr bool PROMO = PROMO_;
+    static constexpr int PSUB = PROMO && BF4_ ? 4 : 1;  // partial buffers per 128-K block
+    // promotion with one B scale per column (the K-grouped calls' configuration, fp32 D; E2M1 B always): the
+    // epilogue stages each partial stage's column scales in shared memory
+    static constexpr bool PCOL = PROMO && (PCOL_ || BF4_);
     // Swapped operands (masked layout): the MMA's M side runs over B's rows (D's columns, TILE_M per tile) and
     // its N side over up to BN of one group's tokens (D's rows).  The A-side tile of shared memory then holds 128
     // rows of B and the B-side tile up to BN/CTAS tokens of A; the MMA's N is set per tile to the tile's token
@@ -158,7 +170,10 @@ struct Cfg {
     static constexpr int TABLE_INTS =
         MAX_PAIR_WINDOWS + 1 > 2 * (MAX_MASKED_GROUPS + 1) ? MAX_PAIR_WINDOWS + 1 : 2 * (MAX_MASKED_GROUPS + 1);
     static constexpr int EPI_BYTES = 4 * 2 * EPI_CHUNK_BYTES;    // per epilogue warp: two staging chunks
-    static constexpr int FIXED_BYTES = EPI_BYTES + 4 * TABLE_INTS + 4 * MAX_MASKED_GROUPS + 2 * MAX_MASKED_GROUPS + 16 +
+    // promotion with per-column B scales: per epilogue warp, two partial stages' worth (KPS * PSUB rows of BN)
+    static constexpr int PSB_FLOATS = KPS * PSUB * BN;
+    static constexpr int PSB_BYTES = PCOL ? 4 * 2 * PSB_FLOATS * 4 : 0;
+    static constexpr int FIXED_BYTES = EPI_BYTES + PSB_BYTES + 4 * TABLE_INTS + 4 * MAX_MASKED_GROUPS + 2 * MAX_MASKED_GROUPS + 16 +
                                        8 * TILE_LIST_CAP + 16 + 8 * 16 + 1024;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES - 8 * 2 * 8) / STAGE_BYTES;
     static constexpr int STAGES_MAX = STAGES_FIT;
@@ -168,7 +183,8 @@ struct Cfg {
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_EPI = OFF_SF + STAGES * SF_BYTES;    // 1024-aligned (64-byte swizzle atoms)
-    static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
+    static constexpr int OFF_PSB = OFF_EPI + EPI_BYTES;
+    static constexpr int OFF_BAR = OFF_PSB + PSB_BYTES;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARRIERS * 8;   // tmem base, abort flag
     static constexpr int OFF_PREFIX = OFF_MISC + 16;               // int[TABLE_INTS]
     static constexpr int OFF_MM = OFF_PREFIX + 4 * TABLE_INTS;     // masked: clamped masked_m
@@ -176,7 +192,12 @@ struct Cfg {
     static constexpr int OFF_TILES = (OFF_RG + 2 * MAX_MASKED_GROUPS + 15) / 16 * 16;  // uint2[TILE_LIST_CAP]
     static constexpr int SMEM_BYTES = OFF_TILES + 8 * TILE_LIST_CAP + 1024;     // + alignment slack
     static_assert(CTAS == 1 || CTAS == 2, "single CTA or CTA pair");
-    static_assert(!PROMO || (BN == 128 && !BF4 && 2 * KPS * BN <= TMEM_COLS), "promotion: 128-wide tiles, e4m3 B");
+    static_assert(!PROMO || ((BF4 ? BN == 64 && KPS == 1 : (BN == 128 || (PCOL && BN == 64))) &&
+                             2 * KPS * PSUB * BN <= TMEM_COLS),
+                  "promotion: 128-wide tiles (e4m3 B; 64 with per-column scales) or 64-wide tiles of one K block "
+                  "(E2M1 B)");
+    static_assert(!PCOL || (PSB_FLOATS % 64 == 0 && OFF_PSB % 16 == 0), "per-column scale staging");
+    static_assert(!PCOL_ || PROMO_, "per-column B scales are a promotion variant");
     static_assert(!SWAP || (!PROMO && !BF4 && BN % 16 == 0), "swapped operands: block-scaled e4m3 only");
     static_assert(!BNN || SWAP, "B in the NN orientation is read through swapped operands");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32, 256]");
@@ -214,6 +235,13 @@ struct SharedCtl {
 };
 
 __device__ __forceinline__ void raise_error(unsigned *err, unsigned code) { atomicCAS(err, 0u, code); }
+
+// Nonzero unless the scale's fp32 bits are ones the exponent code represents exactly: +0 (taken as 2^-127) or
+// a positive normal power of two (no sign, no mantissa bits, not Inf / NaN).
+__device__ __forceinline__ uint32_t ue8m0_inexact_bits(uint32_t b) {
+    return (b & 0x807FFFFFu) | (((b >> 23) & 0xFFu) == 0xFFu ? 1u : 0u);
+}
+constexpr uint32_t UE8M0_ZERO_F32_BITS = 0x00400000u;  // 2^-127 (fp32 subnormal): the value of exponent code 0
 
 // Slow path of the bounded mbarrier wait.  false = gave up (this CTA is aborting).
 __device__ __noinline__ bool wait_bounded_slow(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *err,
@@ -832,9 +860,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // ---------------------------------------------------------------- MMA issuer (leader CTA)
         if (C::PROMO && lane == 0 && rank == 0) {
             // fp32 scale promotion: each 128-K block's partial product goes to its own TMEM buffer of the current
-            // partial stage (KPS buffers of BN columns); the epilogue warps release a partial stage once they have
-            // read it, so the MMAs run up to two stages ahead of the promotion
-            constexpr uint32_t IDESC_P = idesc_f8f6f4_e4m3(C::TILE_M, BN);
+            // partial stage (KPS buffers of BN columns; E2M1 B: each 32-K MMA to its own, KPS * PSUB buffers); the
+            // epilogue warps release a partial stage once they have read it, so the MMAs run up to two stages
+            // ahead of the promotion
+            constexpr uint32_t IDESC_P = idesc_f8f6f4_e4m3(C::TILE_M, BN, C::BF4);
             int s = 0;
             uint32_t ph = 0;
             int pb = 0;  // partial stage
@@ -843,8 +872,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int k = 0; k < my_tiles && ok; ++k) {
                 Tile ti;
                 if (!tile_at(k, ti)) continue;
-                for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
-                    const int nk = min(C::KPS, nkb - kb0);
+                // (K-grouped: the group's own K blocks; none: no stage, the epilogue writes zeros or nothing)
+                const int tile_nkb = p.mode == MODE_KGROUPED ? ctl_main.mm[ti.g] : nkb;
+                for (int kb0 = 0; kb0 < tile_nkb; kb0 += C::KPS) {
+                    const int nk = min(C::KPS, tile_nkb - kb0);
                     if (!wait_bounded(&full[s], ph, s_abort, p.err, p.wait_limit_ns)) { ok = false; break; }
                     if (!wait_bounded(&tmem_empty[pb], pb_ph ^ 1u, s_abort, p.err, p.wait_limit_ns)) {
                         ok = false;
@@ -854,12 +885,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint32_t a_stage = smem_u32(sA + s * C::A_BYTES);
                     const uint32_t b_stage = smem_u32(sB + s * C::B_BYTES);
                     for (int i = 0; i < nk; ++i) {
-                        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((pb * C::KPS + i) * BN);
 #pragma unroll
-                        for (int kk = 0; kk < BLOCK_K / MMA_K; ++kk)
-                            tc_mma_f8<CTAS>(d_tmem, sdesc_kmajor_sw128(a_stage + i * C::A_BYTES1 + kk * MMA_K),
+                        for (int kk = 0; kk < BLOCK_K / MMA_K; ++kk) {
+                            // partial (pb * KPS + i) * PSUB + sub: the K block's, or (PSUB = 4) this 32-K slice's
+                            const int part = (pb * C::KPS + i) * C::PSUB + (C::PSUB > 1 ? kk : 0);
+                            tc_mma_f8<CTAS>(tmem_base + static_cast<uint32_t>(part * BN),
+                                            sdesc_kmajor_sw128(a_stage + i * C::A_BYTES1 + kk * MMA_K),
                                             sdesc_kmajor_sw128(b_stage + i * C::B_BYTES1 + kk * MMA_K), IDESC_P,
-                                            kk != 0);
+                                            C::PSUB > 1 ? 0u : static_cast<uint32_t>(kk != 0));
+                        }
                     }
                     tc_commit<CTAS>(&empty[s]);
                     tc_commit<CTAS>(&tmem_full[pb]);
@@ -1000,15 +1034,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
             }
         };
+        // One 32-column fp32 chunk of this lane's row into D [G][M][N] (K-grouped calls): two 16-column halves
+        // (64-byte rows, the swizzled staging of the bf16 chunks), each stored or added by one TMA operation on the
+        // 3-D map, which clips rows past M.
+        auto emit_f32 = [&](const Tile &ti, int c, const uint32_t(&r)[32]) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint8_t *buf = stage_buf + (chunk_count & 1) * EPI_CHUNK_BYTES;
+                if (chunk_count >= 2) {
+                    if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
+                    __syncwarp();
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int sw = j ^ ((lane >> 1) & 3);
+                    *reinterpret_cast<uint4 *>(buf + lane * 64 + sw * 16) =
+                        make_uint4(r[16 * h + 4 * j], r[16 * h + 4 * j + 1], r[16 * h + 4 * j + 2],
+                                   r[16 * h + 4 * j + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const int x = ti.n0 + 32 * c + 16 * h, y = ti.row0 + my_rows + 32 * q;
+                    if (p.out_mode == OUT_F32_ADD)
+                        tma_reduce_add_3d(&tmap_d, buf, x, y, ti.g);
+                    else
+                        tma_store_3d(&tmap_d, buf, x, y, ti.g);
+                    bulk_commit_group();
+                }
+                ++chunk_count;
+            }
+        };
         int pb = 0;  // promotion: the partial stage read next
         uint32_t pb_ph = 0;
-        // fp32 scale promotion of one tile: this lane's row accumulates partial(kb) * sfa[row, kb] * sfb[g, nb, kb]
-        // over the K blocks in registers (BN = 128 columns: one 128-column block of B's scales), then it is
-        // written as bf16.  The scales are read from the caller's arrays one partial stage ahead: the loads go out
-        // right after a stage is released and are used after the next stage's wait.  false = gave up.
+        // this warp's two staging buffers of per-column B scales (promotion with sfb_cols)
+        float *psb = reinterpret_cast<float *>(smem + C::OFF_PSB) + (warp - EPI_WARP0) * 2 * C::PSB_FLOATS;
+        int psb_stage = 0;  // partial stages read with per-column scales (selects the staging buffer)
+        // fp32 scale promotion of one tile: this lane's row accumulates partial * sfa[row, kb] * sfb over the tile's
+        // K blocks in registers, then it is written as bf16 (or, K-grouped, fp32).  B's scale is either one per
+        // 128-column block and K block (BN = 128: one value per partial, read by every lane), or one per column
+        // (K-grouped: per K block; E2M1 B: per 32-K sub-block, one partial each).  Per-column scales are copied
+        // into this warp's staging buffer one partial stage ahead and read back four columns at a time; the
+        // per-row A scales (and the per-block B scale) are loaded into registers one stage ahead.  false = gave up.
         auto promote_tile = [&](const Tile &ti) -> bool {
             const int r_local = my_rows + 32 * q + lane;
             const int row = ti.row0 + r_local;
+            constexpr bool kgrouped = C::PCOL && !C::BF4;  // (the K-grouped calls' configuration)
+            const int tile_nkb = kgrouped ? ctl.mm[ti.g] : nkb;  // K blocks of this tile
+            const int kbase = kgrouped ? ctl.off[ti.g] : 0;      // its first K block in the scale arrays
+            constexpr bool col_scales = C::PCOL;
             bool row_in;          // the row exists in the A scale array (rows past it read no scale)
             long long sa_base;    // element of (row, K block 0); K block kb at sa_base + kb * sfa_ld
             if (p.mode == MODE_MASKED) {
@@ -1020,7 +1094,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 sa_base = row;
             }
             const float *sfb_t = p.sfb32 + static_cast<long long>(ti.g) * p.sfb_sg +
-                                 static_cast<long long>(ti.n0 / 128) * p.sfb_sn;
+                                 (col_scales ? static_cast<long long>(ti.n0)
+                                             : static_cast<long long>(ti.n0 / 128) * p.sfb_sn);
             float acc_r[BN];
 #pragma unroll
             for (int j = 0; j < BN; ++j) acc_r[j] = 0.f;
@@ -1029,35 +1104,107 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                 for (int i = 0; i < C::KPS; ++i) {
                     const int kb = kb0 + i;
-                    const bool in = kb < nkb;
-                    sa_n[i] = (in && row_in) ? __ldg(p.sfa32 + sa_base + static_cast<long long>(kb) * p.sfa_ld) : 0.f;
-                    sb_n[i] = in ? __ldg(sfb_t + static_cast<long long>(kb) * p.sfb_sk) : 0.f;
+                    const bool in = kb < tile_nkb;
+                    const long long kg = kbase + kb;
+                    sa_n[i] = (in && row_in) ? __ldg(p.sfa32 + sa_base + kg * p.sfa_ld) : 0.f;
+                    sb_n[i] = (in && !col_scales) ? __ldg(sfb_t + kg * p.sfb_sk) : 0.f;
+                    if (!col_scales && p.check_scales) {
+                        const uint32_t ba = __float_as_uint(sa_n[i]), bb = __float_as_uint(sb_n[i]);
+                        if (ue8m0_inexact_bits(ba) | ue8m0_inexact_bits(bb)) raise_error(p.err, ERR_BAD_SCALE);
+                        if (ba == 0u) sa_n[i] = __uint_as_float(UE8M0_ZERO_F32_BITS);
+                        if (bb == 0u) sb_n[i] = __uint_as_float(UE8M0_ZERO_F32_BITS);
+                    }
                 }
             };
+            // the per-column scales of the partial stage starting at K block kb0: KPS * PSUB rows of BN columns
+            // (row i = the scale row PSUB * (kbase + kb0) + i), 16 bytes per copy; rows past the tile's K blocks
+            // and columns past N are zero-filled
+            auto fetch_cols = [&](int kb0, int buf) {
+                float *dst = psb + buf * C::PSB_FLOATS;
+                constexpr int Q = BN / 4;                 // 16-byte copies per row
+                constexpr int F4 = C::PSB_FLOATS / 4;     // and per stage
+#pragma unroll
+                for (int u = 0; u < (F4 + 31) / 32; ++u) {
+                    const int f = lane + 32 * u;
+                    if (F4 % 32 != 0 && f >= F4) break;
+                    const int i = f / Q, c4 = f % Q;
+                    const bool in = kb0 + i / C::PSUB < tile_nkb && ti.n0 + 4 * c4 < p.N;
+                    const float *src =
+                        sfb_t + static_cast<long long>(C::PSUB * (kbase + kb0) + i) * p.sfb_sk + 4 * c4;
+                    cp_async_16(dst + 4 * f, in ? src : p.sfb32, in ? 16u : 0u);
+                }
+                cp_async_commit();
+            };
             load_scales(0);
-            for (int kb0 = 0; kb0 < nkb; kb0 += C::KPS) {
-                const int nk = min(C::KPS, nkb - kb0);
-                if (!warp_wait_bounded(&tmem_full[pb], pb_ph, s_abort, p.err, p.wait_limit_ns, lane)) return false;
+            if constexpr (col_scales) {
+                if (tile_nkb > 0) fetch_cols(0, psb_stage & 1);
+            }
+            for (int kb0 = 0; kb0 < tile_nkb; kb0 += C::KPS) {
+                const int nk = min(C::KPS, tile_nkb - kb0);
+                const float *sbs = psb + (psb_stage & 1) * C::PSB_FLOATS;
+                if constexpr (col_scales) {
+                    if (kb0 + C::KPS < tile_nkb) {
+                        __syncwarp();  // every lane is done with the other buffer (read two stages back)
+                        fetch_cols(kb0 + C::KPS, (psb_stage + 1) & 1);
+                        cp_async_wait<1>();
+                    } else {
+                        cp_async_wait<0>();
+                    }
+                    __syncwarp();  // this stage's copies by every lane are visible
+                }
+                if (!warp_wait_bounded(&tmem_full[pb], pb_ph, s_abort, p.err, p.wait_limit_ns, lane)) {
+                    if constexpr (col_scales) cp_async_wait<0>();
+                    return false;
+                }
                 tc_fence_after_sync();
-                float sc[C::KPS];
+                const uint32_t t_part = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                                        static_cast<uint32_t>(pb * C::KPS * C::PSUB * BN);
+                if constexpr (col_scales) {
 #pragma unroll
-                for (int i = 0; i < C::KPS; ++i) sc[i] = sa_n[i] * sb_n[i];
-                const uint32_t t_part =
-                    tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(pb * C::KPS * BN);
+                    for (int i = 0; i < C::KPS * C::PSUB; ++i) {
+                        if (i / C::PSUB < nk) {
+                            const float sa = sa_n[i / C::PSUB];
+                            const float4 *sb4 = reinterpret_cast<const float4 *>(sbs + i * BN);
+                            static_assert(BN == 64, "per-column promotion reads a partial as two 32-column loads");
+                            uint32_t r[2][32];  // both halves of the partial in flight at once
+                            tmem_ld_32x32b_x32(t_part + static_cast<uint32_t>(i * BN), r[0]);
+                            tmem_ld_32x32b_x32(t_part + static_cast<uint32_t>(i * BN + 32), r[1]);
+                            tmem_ld_wait_regs(r[0]);
+                            tmem_ld_wait_regs(r[1]);
 #pragma unroll
-                for (int i = 0; i < C::KPS; ++i) {
-                    if (i < nk) {
+                            for (int c = 0; c < 2; ++c) {
 #pragma unroll
-                        for (int c = 0; c < BN / 32; c += 2) {
-                            uint32_t r0[32], r1[32];
-                            tmem_ld_32x32b_x32(t_part + static_cast<uint32_t>(i * BN + 32 * c), r0);
-                            tmem_ld_32x32b_x32(t_part + static_cast<uint32_t>(i * BN + 32 * c + 32), r1);
-                            tmem_ld_wait_regs(r0);
-                            tmem_ld_wait_regs(r1);
+                                for (int j = 0; j < 8; ++j) {
+                                    const float4 v = lds_f32x4(sb4 + 8 * c + j);  // the same address in every lane
+                                    const int o = 32 * c + 4 * j;
+                                    acc_r[o] = fmaf(__uint_as_float(r[c][4 * j]) * v.x, sa, acc_r[o]);
+                                    acc_r[o + 1] = fmaf(__uint_as_float(r[c][4 * j + 1]) * v.y, sa, acc_r[o + 1]);
+                                    acc_r[o + 2] = fmaf(__uint_as_float(r[c][4 * j + 2]) * v.z, sa, acc_r[o + 2]);
+                                    acc_r[o + 3] = fmaf(__uint_as_float(r[c][4 * j + 3]) * v.w, sa, acc_r[o + 3]);
+                                }
+                            }
+                        }
+                    }
+                } else {
+                    float sc[C::KPS];
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                acc_r[32 * c + j] = fmaf(__uint_as_float(r0[j]), sc[i], acc_r[32 * c + j]);
-                                acc_r[32 * c + 32 + j] = fmaf(__uint_as_float(r1[j]), sc[i], acc_r[32 * c + 32 + j]);
+                    for (int i = 0; i < C::KPS; ++i) sc[i] = sa_n[i] * sb_n[i];
+#pragma unroll
+                    for (int i = 0; i < C::KPS; ++i) {
+                        if (i < nk) {
+#pragma unroll
+                            for (int c = 0; c < BN / 32; c += 2) {
+                                uint32_t r0[32], r1[32];
+                                tmem_ld_32x32b_x32(t_part + static_cast<uint32_t>(i * BN + 32 * c), r0);
+                                tmem_ld_32x32b_x32(t_part + static_cast<uint32_t>(i * BN + 32 * c + 32), r1);
+                                tmem_ld_wait_regs(r0);
+                                tmem_ld_wait_regs(r1);
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) {
+                                    acc_r[32 * c + j] = fmaf(__uint_as_float(r0[j]), sc[i], acc_r[32 * c + j]);
+                                    acc_r[32 * c + 32 + j] =
+                                        fmaf(__uint_as_float(r1[j]), sc[i], acc_r[32 * c + 32 + j]);
+                                }
                             }
                         }
                     }
@@ -1073,19 +1220,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 pb ^= 1;
                 if (pb == 0) pb_ph ^= 1u;
-                if (kb0 + C::KPS < nkb) load_scales(kb0 + C::KPS);
+                if constexpr (col_scales) ++psb_stage;
+                if (kb0 + C::KPS < tile_nkb) load_scales(kb0 + C::KPS);
             }
-            const bool valid = row_owned(ti, row, r_local);
-            const bool tma_ok = p.mode == MODE_DENSE || __all_sync(0xffffffffu, valid);
+            if constexpr (kgrouped) {  // fp32 D
+                const int halves = tile_nkb == 0 && p.out_mode == OUT_F32_ADD ? 0 : BN / 16;  // (adding zeros)
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t h[16];
+                for (int hc = 0; hc < BN / 16; ++hc) {  // 16-column halves, straight from the accumulators
+                    if (hc >= halves) break;
+                    uint8_t *buf = stage_buf + (chunk_count & 1) * EPI_CHUNK_BYTES;
+                    if (chunk_count >= 2) {
+                        if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
+                        __syncwarp();
+                    }
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    __nv_bfloat162 v = __floats2bfloat162_rn(acc_r[32 * c + 2 * j], acc_r[32 * c + 2 * j + 1]);
-                    h[j] = *reinterpret_cast<uint32_t *>(&v);
+                    for (int j = 0; j < 4; ++j) {
+                        const int sw = j ^ ((lane >> 1) & 3);
+                        const float *v = acc_r + 16 * hc + 4 * j;
+                        *reinterpret_cast<float4 *>(buf + lane * 64 + sw * 16) = make_float4(v[0], v[1], v[2], v[3]);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        const int x = ti.n0 + 16 * hc, y = ti.row0 + my_rows + 32 * q;
+                        if (p.out_mode == OUT_F32_ADD)
+                            tma_reduce_add_3d(&tmap_d, buf, x, y, ti.g);
+                        else
+                            tma_store_3d(&tmap_d, buf, x, y, ti.g);
+                        bulk_commit_group();
+                    }
+                    ++chunk_count;
                 }
-                emit_bf16(ti, row, c, h, tma_ok, valid);
+            } else {
+                const bool valid = row_owned(ti, row, r_local);
+                const bool tma_ok = p.mode == MODE_DENSE || __all_sync(0xffffffffu, valid);
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t h[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        __nv_bfloat162 v = __floats2bfloat162_rn(acc_r[32 * c + 2 * j], acc_r[32 * c + 2 * j + 1]);
+                        h[j] = *reinterpret_cast<uint32_t *>(&v);
+                    }
+                    emit_bf16(ti, row, c, h, tma_ok, valid);
+                }
             }
             return true;
         };
@@ -1168,44 +1346,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                 }
             } else if (p.out_mode != OUT_BF16) {
-                // fp32 D [G][M][N] through a 3-D map that clips rows past M: per 32-column TMEM load two 16-column
-                // chunks (64-byte rows, the same swizzled staging), each stored or added by one TMA operation.
+                // fp32 D [G][M][N] (K-grouped): per 32-column TMEM load, two TMA stores or adds of 16 columns
                 const bool no_k = ctl.mm[ti.g] == 0;  // an empty K range: the accumulator holds nothing
+                if (!(no_k && p.out_mode == OUT_F32_ADD)) {  // (adding zeros)
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(t_row + 32 * c, r);
-                    tmem_ld_wait_regs(r);
-                    if (no_k) {
-                        if (p.out_mode == OUT_F32_ADD) continue;  // adding zeros
+                    for (int c = 0; c < BN / 32; ++c) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(t_row + 32 * c, r);
+                        tmem_ld_wait_regs(r);
+                        if (no_k) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) r[j] = 0u;
-                    }
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint8_t *buf = stage_buf + (chunk_count & 1) * EPI_CHUNK_BYTES;
-                        if (chunk_count >= 2) {
-                            if (lane == 0) bulk_wait_group_read<1>();  // the store that last used buf has read it
-                            __syncwarp();
+                            for (int j = 0; j < 32; ++j) r[j] = 0u;
                         }
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int sw = j ^ ((lane >> 1) & 3);
-                            *reinterpret_cast<uint4 *>(buf + lane * 64 + sw * 16) =
-                                make_uint4(r[16 * h + 4 * j], r[16 * h + 4 * j + 1], r[16 * h + 4 * j + 2],
-                                           r[16 * h + 4 * j + 3]);
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            const int x = ti.n0 + 32 * c + 16 * h, y = ti.row0 + my_rows + 32 * q;
-                            if (p.out_mode == OUT_F32_ADD)
-                                tma_reduce_add_3d(&tmap_d, buf, x, y, ti.g);
-                            else
-                                tma_store_3d(&tmap_d, buf, x, y, ti.g);
-                            bulk_commit_group();
-                        }
-                        ++chunk_count;
+                        emit_f32(ti, c, r);
                     }
                 }
             } else {

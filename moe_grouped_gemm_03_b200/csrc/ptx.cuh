@@ -177,6 +177,27 @@ __device__ __forceinline__ void bulk_wait_group_read() {
 // Wait until all of this thread's bulk groups have completed.
 __device__ __forceinline__ void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// 16 bytes from global to shared memory without passing through registers (cp.async, cached in L2 only); both
+// addresses 16-byte aligned.  src_bytes = 0 reads nothing and writes 16 zero bytes.
+__device__ __forceinline__ void cp_async_16(void *dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// 16 bytes of shared memory into registers, kept after the instructions before it (a volatile load)
+__device__ __forceinline__ float4 lds_f32x4(const float4 *p) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(smem_u32(p)));
+    return v;
+}
+// Wait until at most N of this thread's cp.async groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ------------------------------------------------------------------------------------------------
 // Tensor Memory and tcgen05
 // ------------------------------------------------------------------------------------------------
@@ -365,11 +386,11 @@ __host__ __device__ constexpr uint32_t idesc_mxf8_e4m3(int M, int N, bool b_e2m1
            | (static_cast<uint32_t>(M >> 4) << 24);            // M / 16
 }
 
-// Instruction descriptor of kind::f8f6f4 (no block scaling): fp32 accumulator (bits 4-5 = 1), A and B E4M3,
-// both K-major, N / 8 and M / 16 (the bit layout of CUTLASS's UMMA::InstrDescriptor).
-__host__ __device__ constexpr uint32_t idesc_f8f6f4_e4m3(int M, int N) {
+// Instruction descriptor of kind::f8f6f4 (no block scaling): fp32 accumulator (bits 4-5 = 1), A E4M3, B E4M3 or
+// E2M1, both K-major, N / 8 and M / 16 (the bit layout of CUTLASS's UMMA::InstrDescriptor).
+__host__ __device__ constexpr uint32_t idesc_f8f6f4_e4m3(int M, int N, bool b_e2m1 = false) {
     return (1u << 4)                                           // accumulator F32
-           | (0u << 7) | (0u << 10)                            // A and B E4M3
+           | (0u << 7) | ((b_e2m1 ? 5u : 0u) << 10)            // A E4M3, B E4M3 (0) or E2M1 (5)
            | (static_cast<uint32_t>(N >> 3) << 17)              // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);             // M / 16
 }

@@ -53,11 +53,7 @@ struct PackParams {
     long long sfa_words, sfb_words;
 };
 
-// Nonzero unless the scale's fp32 bits are ones the exponent code represents exactly: +0 (taken as 2^-127) or
-// a positive normal power of two (no sign, no mantissa bits, not Inf / NaN).
-__device__ __forceinline__ uint32_t ue8m0_inexact_bits(uint32_t b) {
-    return (b & 0x807FFFFFu) | (((b >> 23) & 0xFFu) == 0xFFu ? 1u : 0u);
-}
+// (ue8m0_inexact_bits, shared with the promotion GEMM's scale check, is in gemm_kernel.cuh)
 constexpr uint32_t ONE_F32_BITS = 0x3F800000u;  // 1.0f: the code 0x7F written for entries past the problem
 
 // Most threads per block of the pre-pass (the host launches at most one block per SM).

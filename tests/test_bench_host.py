@@ -51,8 +51,10 @@ def test_recorded_traffic_is_used_only_for_the_captured_code(tmp_path, monkeypat
 
 def test_launches_per_call():
     dense = synth.make_dense(128, 256, 512)
+    long_k = synth.make_dense(128, 256, 2176)
     nn = synth.make_contiguous_nn([129], 256, 256)
-    assert bench.launches_per_call(dense) == 2  # scale pre-pass + GEMM
+    assert bench.launches_per_call(dense) == 1  # a short call: the promotion GEMM alone
+    assert bench.launches_per_call(long_k) == 2  # scale pre-pass + GEMM
     assert bench.launches_per_call(nn) == 2  # B read in place by the swapped-operand tiles
     assert bench.launches_per_call(nn, promotion=True) == 2  # transpose + the promotion GEMM
     assert bench.launches_per_call(dense, promotion=True) == 1  # the promotion GEMM has no pre-pass

@@ -68,12 +68,19 @@ def test_config1_dense_small():
 
 
 @pytest.mark.parametrize("M,N,K", [
+    # short calls (K <= 2048, 2MNK <= 2^34): one kernel, the promotion GEMM on power-of-two scales
     (1, 16, 128),        # one row, narrowest N
     (128, 128, 128),     # one tile, one K block
     (300, 608, 384),     # ragged M tail, N not a multiple of any tile width
     (129, 4096, 256),    # M tail of one row over many N tiles
     (1000, 2048, 1024),  # several waves of tiles
-    (64, 7168, 512),     # N=7168 (224-wide tiles)
+    (64, 7168, 512),     # N=7168
+    # longer K: the scale pre-pass and the block-scaled GEMM
+    (1, 16, 2176),
+    (300, 608, 2304),
+    (129, 4096, 2560),
+    (1000, 2048, 2176),  # several waves of tiles
+    (64, 7168, 4096),    # N=7168 (224-wide tiles)
 ])
 def test_dense_shapes(M, N, K, policy):
     _full_check(synth.make_dense(M, N, K, seed=M + N + K))

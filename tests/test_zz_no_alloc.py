@@ -47,7 +47,8 @@ def _rescaled(p, ja, jb):
     return p
 
 
-@pytest.mark.parametrize("M,N,K", [(512, 2048, 1024), (300, 7168, 384), (4096, 7168, 7168)])
+# (128, 256, 512) is a short call (one kernel, no buffer); the others pack their scales into the buffer
+@pytest.mark.parametrize("M,N,K", [(512, 2048, 2560), (300, 7168, 2304), (4096, 7168, 7168), (128, 256, 512)])
 def test_noalloc_equals_allocating_entry_point_bit_for_bit_on_two_calls(M, N, K):
     for call, seed in enumerate((M + 1, M + 2)):  # two calls in a row, different inputs and scales
         p = synth.make_dense(M, N, K, seed=seed)
@@ -61,7 +62,7 @@ def test_noalloc_large_then_small_call_matches_oracle():
     big = _rescaled(synth.make_dense(2048, 7168, 4096, seed=31), 2, -3)
     out, ref = _both(big)
     assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), "large call"
-    small = _rescaled(synth.make_dense(300, 640, 384, seed=32), -4, 5)
+    small = _rescaled(synth.make_dense(300, 640, 2560, seed=32), -4, 5)  # (K > 2048: packed into the buffer)
     out, ref = _both(small)
     assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), "small call after the large one"
     assert_close(bf16_to_f64(out), oracle.problem_full(small).reshape(small.M, small.N), "small call vs oracle")
