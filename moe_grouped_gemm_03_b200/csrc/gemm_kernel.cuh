@@ -1177,10 +1177,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                 for (int j = 0; j < 8; ++j) {
                                     const float4 v = lds_f32x4(sb4 + 8 * c + j);  // the same address in every lane
                                     const int o = 32 * c + 4 * j;
-                                    acc_r[o] = fmaf(__uint_as_float(r[c][4 * j]) * v.x, sa, acc_r[o]);
-                                    acc_r[o + 1] = fmaf(__uint_as_float(r[c][4 * j + 1]) * v.y, sa, acc_r[o + 1]);
-                                    acc_r[o + 2] = fmaf(__uint_as_float(r[c][4 * j + 2]) * v.z, sa, acc_r[o + 2]);
-                                    acc_r[o + 3] = fmaf(__uint_as_float(r[c][4 * j + 3]) * v.w, sa, acc_r[o + 3]);
+                                    // acc += (partial * sfb) * sfa, two columns per instruction
+                                    float t0, t1, t2, t3;
+                                    mul_f32x2(t0, t1, __uint_as_float(r[c][4 * j]), __uint_as_float(r[c][4 * j + 1]),
+                                              v.x, v.y);
+                                    mul_f32x2(t2, t3, __uint_as_float(r[c][4 * j + 2]),
+                                              __uint_as_float(r[c][4 * j + 3]), v.z, v.w);
+                                    fma_f32x2(acc_r[o], acc_r[o + 1], t0, t1, sa, sa);
+                                    fma_f32x2(acc_r[o + 2], acc_r[o + 3], t2, t3, sa, sa);
                                 }
                             }
                         }
@@ -1200,10 +1204,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                 tmem_ld_wait_regs(r0);
                                 tmem_ld_wait_regs(r1);
 #pragma unroll
-                                for (int j = 0; j < 32; ++j) {
-                                    acc_r[32 * c + j] = fmaf(__uint_as_float(r0[j]), sc[i], acc_r[32 * c + j]);
-                                    acc_r[32 * c + 32 + j] =
-                                        fmaf(__uint_as_float(r1[j]), sc[i], acc_r[32 * c + 32 + j]);
+                                for (int j = 0; j < 32; j += 2) {  // acc += partial * (sfa * sfb), two columns at once
+                                    fma_f32x2(acc_r[32 * c + j], acc_r[32 * c + j + 1], __uint_as_float(r0[j]),
+                                              __uint_as_float(r0[j + 1]), sc[i], sc[i]);
+                                    fma_f32x2(acc_r[32 * c + 32 + j], acc_r[32 * c + 33 + j], __uint_as_float(r1[j]),
+                                              __uint_as_float(r1[j + 1]), sc[i], sc[i]);
                                 }
                             }
                         }
