@@ -296,11 +296,17 @@ struct ScaleArgs {
     int sfb_ld = 0;       // K-grouped: one scale per row of B, [K/128][sfb_ld]; FP4 B: [G][K/32][sfb_ld]
 };
 
-// Launch of the scale pre-pass: one warp per atom, spread over every SM (one block each), so that every SM is
+// Launch of the scale pre-pass: one warp per work item (an atom, or 32 B-side atoms of the swapped-operand
+// layout), spread over every SM (one block each), so that every SM is
 // free for the GEMM (a programmatic dependent) at about the same time.  An SM running a pre-pass block takes no
 // GEMM CTA until that block is done (the pre-pass keeps the default shared-memory carveout).
 int launch_pack(const dg::PackParams &pk, int device, cudaStream_t stream) {
-    const long long atoms = (pk.sfa_words + pk.sfb_words) / dg::SF_ATOM_WORDS;
+    // warp work items: one per atom, except the B-side atoms of one scale per 128 x 128 block of B (the swapped
+    // layout's, and the others' unless K-grouped or E2M1), built 32 to a warp
+    const long long sfa_atoms = pk.sfa_words / dg::SF_ATOM_WORDS, sfb_atoms = pk.sfb_words / dg::SF_ATOM_WORDS;
+    const bool sfb_batched = !pk.swap && pk.mode != dg::MODE_KGROUPED && !pk.sfb_fp4;
+    const long long atoms = pk.swap ? (sfa_atoms + 31) / 32 + sfb_atoms
+                                    : sfa_atoms + (sfb_batched ? (sfb_atoms + 31) / 32 : sfb_atoms);
     constexpr long long kMaxWarps = dg::PACK_THREADS / 32;
     DeviceInfo info;  // (cached per device)
     const int sms = device_info(info) == DG_OK && info.device == device && info.num_sms > 0 ? info.num_sms : 1;

@@ -60,7 +60,8 @@ constexpr uint32_t ONE_F32_BITS = 0x3F800000u;  // 1.0f: the code 0x7F written f
 constexpr int PACK_THREADS = 1024;
 
 // One warp per atom: lane l builds the words of rows l, l+32, l+64, l+96 (words 4l .. 4l+3) and writes them
-// with one 16-byte store, so an atom is one coalesced 512-byte write.
+// with one 16-byte store, so an atom is one coalesced 512-byte write.  (Swapped operands' B-side atoms, one word
+// repeated in every row, are built 32 to a warp: one round of scale loads for all of them.)
 __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackParams p) {
     grid_launch_dependents();  // the GEMM may start its prologue; it waits for this grid before reading
     // The group tables, as the GEMM derives them.  No padding: clamped row counts, first rows, window prefix.
@@ -129,17 +130,77 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
     const long long num_warps = static_cast<long long>(gridDim.x) * warps_per_block;
     const int nnb128 = (p.N + 127) / 128;
     uint32_t bad_bits = 0;  // nonzero once this lane read a scale the block-scaled MMA cannot represent
-    for (long long atom = static_cast<long long>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5); atom < total;
-         atom += num_warps) {
-        uint32_t word[4] = {0u, 0u, 0u, 0u};
-        uint32_t *dst;
-        if (p.swap) {
-            if (atom < sfa_atoms) {  // B side: the block scales of 128 rows of B, the same word in every row
+    // Work items of the warps.  Swapped operands: first the B-side atoms 32 at a time (each holds one word, the
+    // same in all 128 rows: lane l builds the word of the batch's atom l, then the warp writes the 32 atoms), then
+    // the token-side atoms one each.  Otherwise the A-side atoms one each, then the B-side atoms: 32 at a time when
+    // B has one scale per 128 x 128 block (an atom's 128 rows then hold at most two words, those of the two
+    // blocks it meets), else (K-grouped, E2M1 B: a scale per row) one each.
+    const long long b_batches = p.swap ? (sfa_atoms + 31) / 32 : 0;
+    const bool sfb_batched = !p.swap && !kgrouped && !p.sfb_fp4;
+    const long long sfb_total = total - sfa_atoms;
+    const long long items = p.swap ? b_batches + sfb_total : (sfb_batched ? sfa_atoms + (sfb_total + 31) / 32 : total);
+    for (long long item = static_cast<long long>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5); item < items;
+         item += num_warps) {
+        if (sfb_batched && item >= sfa_atoms) {  // 32 B-side atoms [G][n_tiles][num_sf_groups][sfb_atoms]
+            const long long first_b = (item - sfa_atoms) * 32;
+            const long long b = first_b + lane;  // this lane's atom
+            constexpr uint32_t PAST_N = 0x7F7F7F7Fu;  // rows past N: 2^0 in all four bytes
+            uint32_t w0 = PAST_N, w1 = PAST_N;        // words of the atom's first 128-row block and the next
+            int n_first = 0;                          // the atom's first row of B
+            if (b < sfb_total) {
+                const int a = static_cast<int>(b % p.sfb_atoms);
+                long long rest = b / p.sfb_atoms;
+                const int q = static_cast<int>(rest % p.sfb_kwords);
+                rest /= p.sfb_kwords;
+                const int nt = static_cast<int>(rest % p.n_tiles);
+                const long long g = rest / p.n_tiles;
+                n_first = nt * p.bn + a * 128;
+                const int blk0 = n_first / 128;
+                const int n_end = min(p.N, n_first + 128);  // the atom's rows below N: n_first .. n_end - 1
+                int kb_first, kb_count;
+                k_blocks(q, kb_first, kb_count);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int blk = blk0 + h;
+                    if (blk * 128 >= n_end || (h == 1 && n_first % 128 == 0)) continue;  // no row of the atom in it
+                    // [G][N/128][K/128], or [G][K/128][N/128] for B in the NN orientation
+                    const float *base = p.sfb_kn ? p.sfb + g * p.nkb * nnb128 + blk : p.sfb + (g * nnb128 + blk) * p.nkb;
+                    const size_t stride_kb = p.sfb_kn ? static_cast<size_t>(nnb128) : 1;
+                    uint32_t wv = 0;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int kb = kb_first + i;
+                        const uint32_t bits = i < kb_count ? __float_as_uint(__ldg(base + kb * stride_kb)) : ONE_F32_BITS;
+                        wv |= ((bits >> 23) & 0xFFu) << (8 * i);
+                        bad_bits |= ue8m0_inexact_bits(bits);
+                    }
+                    (h == 0 ? w0 : w1) = wv;
+                }
+            }
+#pragma unroll 2
+            for (int i = 0; i < 32; ++i) {
+                const uint32_t x0 = __shfl_sync(0xffffffffu, w0, i), x1 = __shfl_sync(0xffffffffu, w1, i);
+                const int nf = __shfl_sync(0xffffffffu, n_first, i);
+                if (first_b + i >= sfb_total) break;  // (the same for every lane)
+                uint32_t word[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int n = nf + lane + 32 * j;
+                    word[j] = n >= p.N ? PAST_N : (n / 128 == nf / 128 ? x0 : x1);
+                }
+                *reinterpret_cast<uint4 *>(p.sfb_out + (first_b + i) * SF_ATOM_WORDS + 4 * lane) =
+                    make_uint4(word[0], word[1], word[2], word[3]);
+            }
+            continue;
+        }
+        if (p.swap && item < b_batches) {  // B side: the block scales of 128 rows of B
+            const long long atom = item * 32 + lane;
+            uint32_t wv = 0;
+            if (atom < sfa_atoms) {
                 const int q = static_cast<int>(atom % p.num_sf_groups);
                 const long long rest = atom / p.num_sf_groups;
                 const int blk = static_cast<int>(rest % p.b_blocks);
                 const long long g = rest / p.b_blocks;
-                uint32_t wv = 0;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int kb = SF_GROUP * q + i;
@@ -150,9 +211,22 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
                     wv |= ((bits >> 23) & 0xFFu) << (8 * i);
                     if (in) bad_bits |= ue8m0_inexact_bits(bits);
                 }
-                word[0] = word[1] = word[2] = word[3] = wv;
-                dst = p.sfa_out + atom * SF_ATOM_WORDS;
-            } else {  // token side: the per-row scales of 256 tokens of one chunk of one group
+            }
+            const long long n_here = sfa_atoms - item * 32;  // atoms of this batch (32 except the last)
+#pragma unroll 4
+            for (int i = 0; i < 32; ++i) {
+                const uint32_t w = __shfl_sync(0xffffffffu, wv, i);
+                if (i < n_here)
+                    *reinterpret_cast<uint4 *>(p.sfa_out + (item * 32 + i) * SF_ATOM_WORDS + 4 * lane) =
+                        make_uint4(w, w, w, w);
+            }
+            continue;
+        }
+        const long long atom = p.swap ? sfa_atoms + (item - b_batches) : item;
+        uint32_t word[4] = {0u, 0u, 0u, 0u};
+        uint32_t *dst;
+        if (p.swap) {
+            {  // token side: the per-row scales of 256 tokens of one chunk of one group
                 const long long b = atom - sfa_atoms;
                 const int a = static_cast<int>(b % p.sfb_atoms);
                 const long long rest = b / p.sfb_atoms;
