@@ -139,7 +139,9 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
     const bool sfb_batched = !p.swap && !kgrouped && !p.sfb_fp4;
     const long long sfb_total = total - sfa_atoms;
     const long long items = p.swap ? b_batches + sfb_total : (sfb_batched ? sfa_atoms + (sfb_total + 31) / 32 : total);
-    for (long long item = static_cast<long long>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5); item < items;
+    // (item i goes to warp i / gridDim.x of block i % gridDim.x: the B-side batches, 16 KB of stores each, spread
+    // over all SMs instead of filling the first blocks, and the blocks finish at about the same time)
+    for (long long item = static_cast<long long>(threadIdx.x >> 5) * gridDim.x + blockIdx.x; item < items;
          item += num_warps) {
         if (sfb_batched && item >= sfa_atoms) {  // 32 B-side atoms [G][n_tiles][num_sf_groups][sfb_atoms]
             const long long first_b = (item - sfa_atoms) * 32;
@@ -228,10 +230,11 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
         if (p.swap) {
             {  // token side: the per-row scales of 256 tokens of one chunk of one group
                 const long long b = atom - sfa_atoms;
-                const int a = static_cast<int>(b % p.sfb_atoms);
-                const long long rest = b / p.sfb_atoms;
-                const int q = static_cast<int>(rest % p.num_sf_groups);
-                const int w = static_cast<int>(rest / p.num_sf_groups);  // chunk over all groups (runs)
+                const int b32 = static_cast<int>(b);  // (token-side atoms: chunks x scale groups x 2, far below 2^31)
+                const int a = b32 % p.sfb_atoms;
+                const int rest = b32 / p.sfb_atoms;
+                const int q = rest % p.num_sf_groups;
+                const int w = rest / p.num_sf_groups;  // chunk over all groups (runs)
                 if (w >= s_wpre[ntab]) continue;  // past the last chunk: never read
                 const int g = upper_index(s_wpre, ntab, w);  // group, or run (contiguous)
                 const int m = s_cnt[g];
@@ -240,23 +243,35 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_scales_kernel(const PackPar
                 const long long first = p.mode == MODE_MASKED ? 0 : s_off[g];  // the group's first token row
                 const int gid = swap_contig ? s_rg[g] : g;
                 const float *base = p.sfa + (p.mode == MODE_MASKED ? static_cast<long long>(g) * p.nkb * p.sfa_ld : 0);
+                // all sixteen loads (four rows x four K blocks) first, then the words
+                long long tok[4];
+                bool in[4], check[4];
+                uint32_t bits[4][4];
+                int grp[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int r = a * 128 + lane + 32 * j;
                     const long long local = static_cast<long long>(c) * cs + r;  // token within the group
-                    const long long tok = first + local;
-                    const bool in = tok < p.sfa_ld;
-                    // scales of rows the call owns are checked (contiguous: rows whose m_indices is the group)
-                    const bool check = in && local < m && r < cs &&
-                                       (!swap_contig || __ldg(p.m_indices + tok) == gid);
+                    tok[j] = first + local;
+                    in[j] = tok[j] < p.sfa_ld;
+                    check[j] = in[j] && local < m && r < cs;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int kb = SF_GROUP * q + i;
-                        const uint32_t bits = (in && kb < p.nkb)
-                                                  ? __float_as_uint(__ldg(base + static_cast<size_t>(kb) * p.sfa_ld + tok))
-                                                  : ONE_F32_BITS;
-                        word[j] |= ((bits >> 23) & 0xFFu) << (8 * i);
-                        if (check && kb < p.nkb) bad_bits |= ue8m0_inexact_bits(bits);
+                        bits[j][i] = (in[j] && kb < p.nkb)
+                                         ? __float_as_uint(__ldg(base + static_cast<size_t>(kb) * p.sfa_ld + tok[j]))
+                                         : ONE_F32_BITS;
+                    }
+                    grp[j] = swap_contig && check[j] ? __ldg(p.m_indices + tok[j]) : gid;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    // scales of rows the call owns are checked (contiguous: rows whose m_indices is the group)
+                    const bool chk = check[j] && grp[j] == gid;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        word[j] |= ((bits[j][i] >> 23) & 0xFFu) << (8 * i);
+                        if (chk && SF_GROUP * q + i < p.nkb) bad_bits |= ue8m0_inexact_bits(bits[j][i]);
                     }
                 }
                 dst = p.sfb_out + b * SF_ATOM_WORDS;
