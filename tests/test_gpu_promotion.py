@@ -54,6 +54,11 @@ CASES = {
     "masked": lambda: synth.make_masked(5, 200, 384, 512, masked_m=[0, 1, 128, 200, 77], seed=54, expected_m=100),
     "nopad": lambda: synth.make_nopad([130, 0, 257, 5], 256, 256, seed=55, extra_rows=9),
     "nn": lambda: synth.make_contiguous_nn([129, 300], 400, 384, seed=56),
+    # more than a wave of 128-wide pair tiles (two waves on 74 pairs), every call kind's row tables in play
+    "dense_waves": lambda: synth.make_dense(1200, 2048, 640, seed=71),
+    "contiguous_waves": lambda: synth.make_contiguous([600, 500], 2048, 512, seed=72),
+    "masked_waves": lambda: synth.make_masked(5, 200, 2048, 512, masked_m=[0, 1, 128, 200, 77], seed=73, expected_m=100),
+    "nn_waves": lambda: synth.make_contiguous_nn([600, 500], 2048, 384, seed=74),
 }
 
 

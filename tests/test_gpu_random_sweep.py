@@ -5,7 +5,8 @@ N a multiple of 16 that is seldom a multiple of the tile width, K from one to tw
 counts from 1 to 8, and the CTA-pair policy drawn as well. The single-CTA and pair paths, the window tables and
 the per-CTA tile lists meet combinations that the fixed cases do not. Two larger cases put more row windows in
 the dense and K-grouped launches than one raster group holds (the tile order then has several groups and a
-narrower last one); they are checked on sampled rows from every window.
+narrower last one); they are checked on sampled rows from every window. A second sweep runs random draws with
+fp32 (non-power-of-two) scales through the fp32 promotion path of every call kind.
 """
 import numpy as np
 import pytest
@@ -78,6 +79,30 @@ def test_random_shape(case):
     got = bf16_to_f64(out).reshape(-1, p.N)
     valid = ~np.isnan(ref[:, 0])
     assert_close(got[valid], ref[valid], f"{p.name} policy {policy} swap {swap}")
+    assert untouched_rows_ok(out, valid), f"{p.name}: rows outside the groups were written"
+
+
+@pytest.mark.parametrize("case", range(24))
+def test_random_shape_fp32_promotion(case):
+    """The same draws with every scale given its own fp32 mantissa (no power of two left) and fp32 scale promotion
+    on: each call kind's promotion epilogue -- one B scale per 128-column block, per column and K block (K-grouped,
+    fp32 D), per column and 32-K sub-block (W4A8) -- against the oracle on random shapes and CTA policies."""
+    import moe_grouped_gemm_03_b200 as dg
+
+    p = synth.with_fp32_scales(_draw(100 + case), seed=case)
+    policy = int(np.random.default_rng(500 + case).choice([-1, 0, 1]))
+    dg.set_cta_pair_policy(policy)
+    dg.set_fp32_scale_promotion(True)
+    try:
+        out = run_problem(p)
+        dg.check_device_error()
+    finally:
+        dg.set_cta_pair_policy(-1)
+        dg.set_fp32_scale_promotion(False)
+    ref = oracle.problem_full(p).reshape(-1, p.N)
+    got = bf16_to_f64(out).reshape(-1, p.N)
+    valid = ~np.isnan(ref[:, 0])
+    assert_close(got[valid], ref[valid], f"{p.name} (fp32 scales, promotion) policy {policy}")
     assert untouched_rows_ok(out, valid), f"{p.name}: rows outside the groups were written"
 
 
