@@ -15,8 +15,11 @@
 //
 // Cfg::PROMO (any finite fp32 scales): the promotion runs in the epilogue warps instead.  Plain kind::f8f6f4
 // MMAs write each 128-K block's partial product into its own TMEM buffer (two partial stages of KPS buffers),
-// and the epilogue warps accumulate partial * sfa * sfb in fp32 registers over 128-wide tiles, reading the
-// caller's fp32 scales directly (no pre-pass).
+// and the epilogue warps accumulate partial * sfa * sfb in fp32 registers, reading the caller's fp32 scales
+// directly (no pre-pass): 128-wide tiles with one B scale per 128-column block, or (Cfg::PCOL) 64-wide tiles
+// with one B scale per column -- per K block for the K-grouped call (fp32 D), per 32-K sub-block for E2M1 B,
+// whose four 32-K MMAs per K block then write four partials.  The host also runs short dense calls on power-of-two
+// scales through the 128-wide promotion kernel, with the scale check of the block-scaled path.
 //
 // CTAS = 1: one CTA computes a 128 x BN output tile.  CTAS = 2: a cluster of two CTAs (a CTA pair) computes
 // a 256 x BN tile with tcgen05.mma.cta_group::2: each CTA loads its own 128 rows of A and its own BN/2 rows
