@@ -6,7 +6,9 @@ with power-of-two 1x128 / 128x128 scales, bf16 out; seeded synthetic inputs), th
 headline metric is quoted on.  Other workloads can be timed with --workload for reference (the default line
 is the contract line): 1 dense 128x256x512; 3 and 5 contiguous grouped; 4 masked grouped; 6 no-padding grouped;
 7 contiguous with B in the NN orientation; 8 K-grouped with fp32 output; 9 contiguous W4A8 (B in E2M1);
-10 workload 2 with fp32 (non-power-of-two) scales, through the fp32 scale-promotion path.
+10 workload 2 with fp32 (non-power-of-two) scales, through the fp32 scale-promotion path.  The default line
+also times workloads 3, 4 and 5 (under "grouped", the M-grouped half of the metric) and workload 1 (under
+"latency") in the same process with the same protocol.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 2]
 
@@ -57,6 +59,9 @@ def parse():
     ap.add_argument("--grouped", default="auto",
                     help="comma-separated workloads timed after the main one and reported under 'grouped' "
                          "(auto: 3,4,5 when the main workload is 2 on one GPU; none: skip)")
+    ap.add_argument("--latency", default="auto",
+                    help="comma-separated latency-bound workloads timed after the grouped ones and reported under "
+                         "'latency' (auto: 1 when the main workload is 2 on one GPU; none: skip)")
     ap.add_argument("--ref-seconds", type=float, default=30.0,
                     help="reference arm: wall time of all warm-up and timed oracle steps together")
     return ap.parse_args()
@@ -236,6 +241,7 @@ def call_library(p, t, out):
         dg.m_grouped_fp8_gemm_nt_masked((t["a"], t["sfa"]), (t["b"], t["sfb"]), out, t["masked_m"], p.expected_m)
 
 
+LATENCY_WORKLOADS = (1,)  # the default line's latency-bound workload (the small dense call)
 PROMOTION_WORKLOADS = (10,)  # run with fp32 scale promotion (their scales are not powers of two)
 
 
@@ -549,6 +555,14 @@ def run_ours(args, world, rank, local):
     if workloads:
         del p
         line["grouped"] = run_grouped(workloads, args, world, local, flush, peaks, peak_src, num_sms)
+    latency = args.latency
+    if latency == "auto":
+        latency = ",".join(str(w) for w in LATENCY_WORKLOADS) if args.workload == 2 and world == 1 else ""
+    small = [int(w) for w in latency.split(",") if w.strip() and w.strip() != "none"]
+    if small:
+        # the small dense call: one launch (latency-bound; two CUDA events around one trivial kernel already
+        # measure about 6 us on this protocol)
+        line["latency"] = run_grouped(small, args, world, local, flush, peaks, peak_src, num_sms)
     dg.set_fp32_scale_promotion(False)
     if rank == 0:
         print(json.dumps(line), flush=True)
