@@ -269,7 +269,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
     return wait_bounded_slow(bar, parity, abort, err, limit);
 }
 
-// Whole-warp wait: lane 0 waits, the verdict is broadcast, and the warp leaves converged (the callers
+// Whole-warp wait: lane 0 waits, the outcome is broadcast, and the warp leaves converged (the callers
 // follow with .sync.aligned tcgen05 instructions).
 __device__ __forceinline__ bool warp_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort,
                                                   unsigned *err, uint64_t limit, int lane) {

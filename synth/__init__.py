@@ -412,7 +412,7 @@ def zipf_counts(total: int, G: int, s: float) -> np.ndarray:
 # The five workloads (all seed 0); 6: workload 5's token split in the no-padding layout; 7: workload 3 with B
 # in the NN orientation; 8: workload 3's token counts as the K extents of a K-grouped (weight-gradient) GEMM;
 # 9: workload 3 with B in E2M1 (W4A8).
-CONFIGS = {
+WORKLOAD_NAMES = {
     1: "dense FP8 NT GEMM M=128 N=256 K=512",
     2: "dense FP8 NT GEMM M=4096 N=7168 K=7168",
     3: "M-grouped contiguous FP8 GEMM G=8 N=4096 K=7168, tokens U[1024,8192] per group",
@@ -428,37 +428,37 @@ CONFIGS = {
 
 def make_config(i: int, seed: int = 0) -> Problem:
     if i == 1:
-        return make_dense(128, 256, 512, seed, name=CONFIGS[1])
+        return make_dense(128, 256, 512, seed, name=WORKLOAD_NAMES[1])
     if i == 2:
-        return make_dense(4096, 7168, 7168, seed, name=CONFIGS[2])
+        return make_dense(4096, 7168, 7168, seed, name=WORKLOAD_NAMES[2])
     if i == 3:
         rng = np.random.default_rng(seed)
         counts = rng.integers(1024, 8192, endpoint=True, size=8)
-        return make_contiguous(counts, 4096, 7168, rng=rng, name=CONFIGS[3])
+        return make_contiguous(counts, 4096, 7168, rng=rng, name=WORKLOAD_NAMES[3])
     if i == 4:
-        return make_masked(32, 256, 7168, 2048, seed=seed, expected_m=128, name=CONFIGS[4])
+        return make_masked(32, 256, 7168, 2048, seed=seed, expected_m=128, name=WORKLOAD_NAMES[4])
     if i == 5:
         rng = np.random.default_rng(seed)
-        return make_contiguous(zipf_counts(65536, 64, 1.2), 7168, 2048, rng=rng, name=CONFIGS[5])
+        return make_contiguous(zipf_counts(65536, 64, 1.2), 7168, 2048, rng=rng, name=WORKLOAD_NAMES[5])
     if i == 9:
         rng = np.random.default_rng(seed)
         counts = rng.integers(1024, 8192, endpoint=True, size=8)
-        return make_contiguous_w4a8(counts, 4096, 7168, rng=rng, name=CONFIGS[9])
+        return make_contiguous_w4a8(counts, 4096, 7168, rng=rng, name=WORKLOAD_NAMES[9])
     if i == 8:
         rng = np.random.default_rng(seed)
         counts = rng.integers(1024, 8192, endpoint=True, size=8)
         return make_k_grouped([align_up(int(c), SCALE_BLOCK) for c in counts], 4096, 7168, rng=rng, with_c=False,
-                              name=CONFIGS[8])
+                              name=WORKLOAD_NAMES[8])
     if i == 7:
         rng = np.random.default_rng(seed)
         counts = rng.integers(1024, 8192, endpoint=True, size=8)
-        return make_contiguous_nn(counts, 4096, 7168, rng=rng, name=CONFIGS[7])
+        return make_contiguous_nn(counts, 4096, 7168, rng=rng, name=WORKLOAD_NAMES[7])
     if i == 6:
         rng = np.random.default_rng(seed)
-        return make_nopad(zipf_counts(65536, 64, 1.2), 7168, 2048, rng=rng, name=CONFIGS[6])
+        return make_nopad(zipf_counts(65536, 64, 1.2), 7168, 2048, rng=rng, name=WORKLOAD_NAMES[6])
     if i == 10:
         p = with_fp32_scales(make_dense(4096, 7168, 7168, seed), seed)
-        p.name = CONFIGS[10]
+        p.name = WORKLOAD_NAMES[10]
         return p
     raise ValueError(f"unknown config {i}")
 
