@@ -330,6 +330,70 @@ def test_k_grouped_row_scale_moves_one_column_of_one_group():
     np.testing.assert_allclose(diff[1, :, n], contribution, rtol=1e-12, atol=1e-9)
 
 
+def test_k_grouped_fp32_scales_against_exact_rational_arithmetic():
+    """K-grouped with arbitrary fp32 scales (one per row and K block on both sides) on integer-valued operands:
+    D_g[m][n] equals the exact rational sum over group g's K blocks of sfa(kb, m) * sfb(kb, n) * (integer dot
+    product), to within fp64 rounding of the sum; an empty group gives zero.  (The oracle scales each element
+    before the dot product, so its rounding is bounded by the sum of the elements' magnitudes.)"""
+    from fractions import Fraction
+
+    rng = np.random.default_rng(26)
+    ks = [256, 0, 128]
+    p = synth.make_k_grouped(ks, M=3, N=20, seed=26, with_c=False)
+    ia = rng.integers(-8, 9, size=(p.M, p.K))
+    ib = rng.integers(-8, 9, size=(p.N, p.K))
+    p.a = _codes_for_values(ia.astype(np.float32))
+    p.b = _codes_for_values(ib.astype(np.float32))
+    p.sfa = rng.uniform(0.01, 3.0, size=p.sfa.shape).astype(np.float32)
+    p.sfb = rng.uniform(0.01, 3.0, size=p.sfb.shape).astype(np.float32)
+    got = oracle.problem_full(p)
+    assert (got[1] == 0).all()
+    first = [0, 2, 2]  # each group's first 128-K block
+    for g, k in enumerate(ks):
+        for m in range(p.M):
+            for n in range(p.N):
+                exact, mag = Fraction(0), 0.0
+                for kb in range(first[g], first[g] + k // 128):
+                    blk = slice(128 * kb, 128 * (kb + 1))
+                    dot = int(ia[m, blk] @ ib[n, blk])
+                    scale = Fraction(float(p.sfa[kb, m])) * Fraction(float(p.sfb[kb, n]))
+                    exact += scale * dot
+                    mag += float(scale) * float(np.abs(ia[m, blk] * ib[n, blk]).sum())
+                assert abs(got[g, m, n] - float(exact)) <= 4e-16 * (mag + 1.0), (g, m, n)
+
+
+def test_w4a8_fp32_scales_against_exact_rational_arithmetic():
+    """W4A8 with arbitrary fp32 scales (A per row and 128-K block, B per row and 32-K sub-block) on integer
+    e4m3 A and E2M1-grid B: each owned row equals the exact rational sum over K blocks kb and their four 32-K
+    sub-blocks j of sfa(kb, m) * sfb(g, 4kb + j, n) * (integer dot product of the sub-block), to within fp64
+    rounding of the sum."""
+    from fractions import Fraction
+
+    rng = np.random.default_rng(27)
+    p = synth.make_contiguous_w4a8([2, 130], N=20, K=256, seed=27)
+    grid = np.array([0, 1, 2, 3, 4, 6, -1, -2, -3, -4, -6])
+    codes_of = {0: 0, 1: 2, 2: 4, 3: 5, 4: 6, 6: 7, -1: 10, -2: 12, -3: 13, -4: 14, -6: 15}
+    ia = rng.integers(-8, 9, size=(p.rows, p.K))
+    ib = rng.choice(grid, size=(p.G, p.N, p.K))
+    p.a = _codes_for_values(ia.astype(np.float32))
+    p.b = synth.pack_e2m1(np.vectorize(codes_of.get)(ib).astype(np.uint8))
+    p.sfa = rng.uniform(0.01, 3.0, size=p.sfa.shape).astype(np.float32)
+    p.sfb = rng.uniform(0.01, 3.0, size=p.sfb.shape).astype(np.float32)
+    full = oracle.problem_full(p)
+    for g, start in enumerate([0, 128]):
+        for m in range(start, start + int(p.counts[g])):
+            for n in range(0, p.N, 3):
+                exact, mag = Fraction(0), 0.0
+                for kb in range(p.K // 128):
+                    for j in range(4):
+                        sub = slice(128 * kb + 32 * j, 128 * kb + 32 * (j + 1))
+                        dot = int(ia[m, sub] @ ib[g, n, sub])
+                        term = Fraction(float(p.sfa[kb, m])) * Fraction(float(p.sfb[g, 4 * kb + j, n])) * dot
+                        exact += term
+                        mag += abs(float(term))
+                assert abs(full[m, n] - float(exact)) <= 1e-15 * (mag + 1.0), (g, m, n)
+
+
 def test_e2m1_decode_matches_the_format_table():
     """All 16 E2M1 codes against the element table of the OCP Microscaling (MX) v1.0 specification (FP4 E2M1:
     +-0, 0.5, 1, 1.5, 2, 3, 4, 6 in code order, sign in bit 3)."""
